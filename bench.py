@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Benchmark: K8/V4 quantised-KV decode attention on B200.
+
+One step = one decode step of the workload over all its attention layers:
+per layer, the quantise-and-append of the step's new tokens (when the workload
+appends) followed by split-K decode attention and the LSE combine, all through
+the C ABI.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--kv-format k8v4|bf16] [--impl ours|reference]
+
+Metric: KV tokens/s (each cached key counted once per layer, heads not
+multiplied) and the decode kernel's achieved HBM GB/s against the measured B200
+copy bandwidth.  Inputs are seeded synthetic tensors of the workload's shape,
+resident in HBM before timing; the KV bytes of one step exceed the 126 MB L2,
+so successive steps stream from HBM.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "KV tokens/s and achieved HBM GB/s (% of B200 peak) for K8/V4 decode attn"
+UNIT = "KV tokens/s"
+DEFAULT_WORKLOAD = "ctx32k_append"
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ["long_context_quantized_b200/csrc/nf_decode.cuh",
+                  "long_context_quantized_b200/csrc/nf_common.cuh",
+                  "long_context_quantized_b200/csrc/nf_api.cu"]
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for s in DECODE_SOURCES:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, fmt):
+    """dram bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{workload}:{fmt}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ GPU workload
+class GpuWorkload:
+    """All layers' pools, queries and step inputs resident on the device."""
+
+    def __init__(self, w, fmt_name, device):
+        import long_context_quantized_b200 as nf
+        self.nf = nf
+        self.w = w
+        self.dev = device
+        self.fmt = nf.NF_KV_K8V4 if fmt_name == "k8v4" else nf.NF_KV_BF16
+        bt = workloads.block_table(w)
+        self.bt = torch.as_tensor(bt, dtype=torch.int32, device=device)
+        self.seqlens = torch.as_tensor(w.seqlens, dtype=torch.int32, device=device)
+        self.before = torch.as_tensor(w.cached, dtype=torch.int32, device=device)
+        self.max_seqlen = max(w.seqlens)
+        self.layers, self.q, self.knew, self.vnew, self.out = [], [], [], [], []
+        for layer in range(w.layers):
+            kv = nf.KVLayer.empty(self.fmt, w.pool_blocks, w.num_kv_heads, device=device, fill=0)
+            knew, vnew = [], []
+            for b in range(w.batch):
+                k, v = workloads.layer_kv(w, layer, b, device=device)
+                c = w.cached[b]
+                nf.nf_kv_append_quant(kv, k[None, :c].contiguous(), v[None, :c].contiguous(), self.bt[b:b + 1],
+                                      torch.zeros(1, dtype=torch.int32, device=device))
+                knew.append(k[c:])
+                vnew.append(v[c:])
+                del k, v
+            self.layers.append(kv)
+            if w.n_new:
+                self.knew.append(torch.stack(knew).contiguous())
+                self.vnew.append(torch.stack(vnew).contiguous())
+            self.q.append(workloads.layer_q(w, layer, device=device))
+            self.out.append(torch.empty((w.batch, w.n_q, w.num_q_heads, 128), dtype=torch.float32, device=device))
+        ws = nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, self.max_seqlen)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        torch.cuda.synchronize()
+        assert nf.nf_get_device_error() == 0
+
+    def append(self, layer):
+        if self.w.n_new:
+            self.nf.nf_kv_append_quant(self.layers[layer], self.knew[layer], self.vnew[layer], self.bt, self.before)
+
+    def decode(self, layer):
+        w = self.w
+        self.nf.nf_decode_attn(self.layers[layer], self.q[layer], self.bt, self.seqlens, self.max_seqlen,
+                               w.softmax_scale, w.causal, self.out[layer], None, self.ws)
+
+    def step(self):
+        for layer in range(self.w.layers):
+            self.append(layer)
+            self.decode(layer)
+
+    # --- byte accounting (algorithmic, per decode launch / per step)
+    def kv_bytes_per_layer(self):
+        per = workloads.kv_bytes_per_token_head("k8v4" if self.fmt == self.nf.NF_KV_K8V4 else "bf16")
+        return sum(self.w.seqlens) * self.w.num_kv_heads * per
+
+    def decode_bytes_per_launch(self):
+        w = self.w
+        q = self.q[0].numel() * self.q[0].element_size()
+        out = w.batch * w.n_q * w.num_q_heads * 128 * 4
+        tables = sum(math.ceil(L / 256) for L in w.seqlens) * 4 + 4 * w.batch
+        return self.kv_bytes_per_layer() + q + out + tables
+
+    def step_bytes(self):
+        w = self.w
+        per = workloads.kv_bytes_per_token_head("k8v4" if self.fmt == self.nf.NF_KV_K8V4 else "bf16")
+        app = w.batch * w.n_new * w.num_kv_heads * (per + 2 * 128 * 2)
+        return w.layers * (self.decode_bytes_per_launch() + app)
+
+    def launches_per_step(self):
+        return self.w.layers * ((1 if self.w.n_new else 0) + 2)
+
+
+def time_graph(g, steps, warmup, stream):
+    """Mean ms per replay: events and replays on the same stream."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def time_decode_launches(gw, steps, stream):
+    """Average duration of one nf_decode_attn call (split kernel + combine),
+    from CUDA events recorded around every call inside a captured graph."""
+    L = gw.w.layers
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for layer in range(L):
+            ev[layer][0].record()
+            gw.decode(layer)
+            ev[layer][1].record()
+    tot, n = 0.0, 0
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        for _ in range(steps):
+            g.replay()
+            torch.cuda.synchronize()
+            for a, b in ev:
+                tot += a.elapsed_time(b)
+                n += 1
+    return tot / n
+
+
+# ------------------------------------------------------------ CPU oracle leg
+def oracle_sample(w, fmt_name, budget_s=12.0, device="cpu"):
+    """Time the CPU oracle on a bounded sample of the workload: decode attention
+    of the rows of kv-head 0 of layer 0 (G * n_q rows per sequence), repeated
+    until about budget_s seconds.  Returns (KV tokens/s, threads, description).
+    KV tokens counts each key once per kv-head processed, scaled by 1 / H_kv."""
+    import oracle
+    fmt = oracle.FMT_K8V4 if fmt_name == "k8v4" else oracle.FMT_BF16
+    bt = workloads.block_table(w)
+    pool = oracle.Pool(fmt, w.pool_blocks, 1, 128, poison=0)
+    for b in range(w.batch):
+        k, v = workloads.layer_kv(w, 0, b, device=device)
+        oracle.append(pool, k[:, :1].float().cpu().numpy()[None], v[:, :1].float().cpu().numpy()[None],
+                      bt[b:b + 1], np.zeros(1, np.int32))
+        del k, v
+    q = workloads.layer_q(w, 0, device=device)[:, :, :w.group].float().cpu().numpy()
+    threads = os.cpu_count() or 1
+    sl = np.array(w.seqlens, np.int32)
+    reps, t_tot = 0, 0.0
+    while True:
+        t0 = time.perf_counter()
+        oracle.decode_attn(pool, q, bt, sl, w.softmax_scale, w.causal, nthreads=threads)
+        t_tot += time.perf_counter() - t0
+        reps += 1
+        if t_tot >= budget_s or reps >= 50:
+            break
+    tokens = sum(w.seqlens) * reps / w.num_kv_heads
+    desc = (f"oracle (C, fp64 attention) on {threads} host threads: layer 0, kv-head 0 of "
+            f"{w.num_kv_heads} ({w.group * w.n_q} query rows per sequence), {reps} repetition(s), "
+            f"{t_tot:.1f} s; KV tokens scaled by 1/{w.num_kv_heads}")
+    return tokens / t_tot, threads, desc, t_tot / reps
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.ORDER)
+    ap.add_argument("--kv-format", default="k8v4", choices=["k8v4", "bf16"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="profiling only: run fewer layers than the workload has")
+    args = ap.parse_args()
+    ws, rank, local = dist_env()
+    w = workloads.get(args.workload)
+    if args.layers:
+        import dataclasses
+        w = dataclasses.replace(w, layers=args.layers)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        per_step = []
+        value, threads, desc, t_rep = oracle_sample(w, args.kv_format, budget_s=0.0, device=dev)
+        for _ in range(args.warmup):
+            oracle_sample(w, args.kv_format, budget_s=0.0, device=dev)
+        for _ in range(args.steps):
+            v, threads, desc, t_rep = oracle_sample(w, args.kv_format, budget_s=0.0, device=dev)
+            per_step.append(t_rep)
+        t = sum(per_step) / len(per_step)
+        value = sum(w.seqlens) / w.num_kv_heads / t
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": w.name, "kv_format": args.kv_format, "step": "oracle sample"},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import long_context_quantized_b200 as nf
+    if ws > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    gw = GpuWorkload(w, args.kv_format, device)
+    stream = torch.cuda.Stream(device=device)
+
+    # ---- the step as a CUDA graph
+    with torch.cuda.stream(stream):
+        gw.step()   # eager warm-up, outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        gw.step()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_graph(g, args.steps, 0, stream)
+    clk = clocks.stop()
+    if ws > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+    err = nf.nf_get_device_error()
+    assert err == 0, f"device error {err}"
+
+    tokens = w.kv_tokens_per_step()
+    value = tokens * ws / (ms / 1e3)
+
+    # ---- dominant kernel: per-launch duration from events in the graph
+    dec_ms = time_decode_launches(gw, max(5, min(args.steps, 30)), stream)
+    peak, peak_kind = measured_peaks()
+    dec_bytes = gw.decode_bytes_per_launch()
+    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    traffic = recorded_traffic(w.name, args.kv_format)
+
+    # ---- end to end: pinned host inputs -> device, the step, result -> host
+    n_layers = w.layers
+    h_q = [t.cpu().pin_memory() for t in gw.q]
+    h_k = [t.cpu().pin_memory() for t in gw.knew]
+    h_v = [t.cpu().pin_memory() for t in gw.vnew]
+    h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in gw.out]
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=stream):
+        for layer in range(n_layers):
+            gw.q[layer].copy_(h_q[layer], non_blocking=True)
+            if w.n_new:
+                gw.knew[layer].copy_(h_k[layer], non_blocking=True)
+                gw.vnew[layer].copy_(h_v[layer], non_blocking=True)
+            gw.append(layer)
+            gw.decode(layer)
+            h_out[layer].copy_(gw.out[layer], non_blocking=True)
+    e2e_ms = time_graph(ge, args.steps, max(3, args.warmup), stream)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in h_q + h_k + h_v)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    del ge, g
+    torch.cuda.synchronize()
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cv, threads, desc, _ = oracle_sample(w, args.kv_format, budget_s=12.0, device=device)
+        cpu = {"value": cv, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    l2_note = ("KV bytes per step %.1f MB > 126 MB L2: no flush needed" % (gw.kv_bytes_per_layer() * w.layers / 1e6)
+               if gw.kv_bytes_per_layer() * w.layers > 126e6 else "L2-resident (correctness-size workload)")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8/s4 KV codes, f16 tensor-core products, f32 softmax/accumulate"
+        if args.kv_format == "k8v4" else "bf16 KV, bf16 tensor-core products, f32 softmax/accumulate",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlens": list(w.seqlens), "n_q": w.n_q,
+                   "n_new": w.n_new, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
+                   "layers": w.layers, "kv_format": args.kv_format, "causal": w.causal,
+                   "l2": l2_note, "timing": "CUDA graph of one step, CUDA events, max over ranks"},
+        "step_gbs": gw.step_bytes() / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "nf_decode_attn (split kernel + combine)", "peak_source": peak_kind,
+                     "bytes_per_launch": dec_bytes, "launch_us": dec_ms * 1e3},
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens * ws / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": gw.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * nf.h -- C ABI of the B200 (sm_100a) library for single-request, long-context
+ * decode attention over a K8/V4-quantised, segmented KV cache.
+ *
+ * Sources of the operations (pages of the NInfer write-ups; no page gives
+ * code or a kernel interface, so the interface below is this library's own):
+ *  - KV dtype "rk8v4 (K8/V4)": int8 keys, 4-bit values.  Page "3090 单卡跑
+ *    Qwen3.8-27B：NInfer 上机实测（180K 上下文 / C2 并发 / 4bit KV）", section
+ *    一.3 启动 (--kv-dtype rk8v4; int8 KV reaches 160K where rk8v4 reaches 180K
+ *    at equal speed).  The pages do not define the bits; this header does (see
+ *    nf_kv_layer).
+ *  - A segmented KV cache in a pool of fixed capacity, one segment streamed
+ *    at a time, decode tuned for one long request.  Page "標籤: vLLM", section
+ *    2 "C++/CUDA 層的 kernel fusion 與 KV cache 策略"; page "3090 单卡跑
+ *    Qwen3.8-27B", section 一.3 (--kv-capacity 184320, --max-concurrency 2).
+ *  - MTP draft verification (1 + 3 query tokens with a causal mask among
+ *    them).  Page "3090 单卡跑 Qwen3.8-27B", section 一.3 (--spec mtp
+ *    --draft-tokens 3).
+ *  - Decode is HBM-bandwidth bound and KV bytes per token drive long-context
+ *    decode.  Page "3090 单卡跑 Qwen3.8-27B", section 二 测评 and the replies.
+ *  - Refuse rather than overrun a memory budget.  Same page, section 一.3
+ *    (the engine refuses to start over budget); here: every call validates its
+ *    arguments on the host and returns a status before launching anything.
+ *
+ * Conventions for every call:
+ *  - The caller owns every buffer (pool planes, block tables, lengths, q, out,
+ *    workspace).  The library never allocates, frees or synchronises; all work
+ *    is enqueued on `stream` (NULL = the legacy default stream) of the current
+ *    CUDA device, and all pointers except `kv` itself are device pointers.
+ *  - Arguments are validated on the host first; on any error nothing is
+ *    launched and the status says why (nf_last_error() gives a message).
+ *  - A launch failure or an earlier asynchronous CUDA error is returned as
+ *    NF_ERR_CUDA.
+ *  - Data-dependent problems that only the device sees (a block id outside the
+ *    pool, a length outside [n_q, max_seqlen]) never trap: the kernel skips the
+ *    offending work and records a code that nf_get_device_error() returns.
+ *  - Calls keep no state between them and are safe to call from several host
+ *    threads on different streams.
+ */
+#ifndef NF_H_
+#define NF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same type as cudaStream_t. */
+typedef struct CUstream_st *nf_stream_t;
+
+typedef int32_t nf_status;
+#define NF_OK 0
+#define NF_ERR_INVALID_ARG 1  /* null pointer, negative size, inconsistent shape */
+#define NF_ERR_UNSUPPORTED 2  /* head_dim != 128, block_size != 256, v_group != 32, dtype */
+#define NF_ERR_WORKSPACE 3    /* workspace smaller than nf_decode_attn_workspace_size() */
+#define NF_ERR_CUDA 4         /* a CUDA launch or earlier asynchronous error */
+#define NF_ERR_DEVICE_CHECK 5 /* returned by nf_get_device_error() when a code is set */
+
+/* Device error codes recorded by the kernels (nf_get_device_error). */
+#define NF_DEVERR_NONE 0
+#define NF_DEVERR_BLOCK_ID 1  /* a block-table entry outside [0, num_blocks) */
+#define NF_DEVERR_TABLE 2     /* a position whose block index is >= max_blocks */
+#define NF_DEVERR_SEQLEN 3    /* seqlens[b] < n_q or > max_seqlen */
+
+/* Element types. */
+#define NF_F32 0
+#define NF_BF16 1
+#define NF_F16 2
+
+/* KV cache formats. */
+#define NF_KV_K8V4 0 /* the rk8v4 format defined below */
+#define NF_KV_BF16 1 /* unquantised bf16 K and V (for byte-count comparison) */
+
+/*
+ * One layer's view of the caller-owned KV pool.
+ *
+ * The pool holds `num_blocks` segments of `block_size` = 256 token slots for
+ * each of `num_kv_heads` heads; head_dim is 128.  Token position p of
+ * sequence b lives in block block_table[b * max_blocks + p / 256], slot p % 256.
+ *
+ * fmt NF_KV_K8V4 ("rk8v4"; 202 bytes per token per kv-head):
+ *   k_codes  int8    [num_blocks][num_kv_heads][256][128]  K codes in [-127, 127]
+ *   k_scales fp16    [num_blocks][num_kv_heads][256]       one K scale per token
+ *   v_codes  uint8   [num_blocks][num_kv_heads][256][64]   V codes in [-7, 7] as
+ *            two's-complement nibbles; byte j holds channel 2j in bits 0..3 and
+ *            channel 2j+1 in bits 4..7
+ *   v_scales fp16    [num_blocks][num_kv_heads][256][4]    one V scale per 32
+ *            channels (v_group = 32)
+ *   Quantisation of a vector x (128 K channels, or one 32-channel V group):
+ *     scale = fp16(fp32(max|x| / Q)) rounded half to even, saturated at 65504,
+ *             Q = 127 for K and 7 for V;
+ *     code  = clamp(round_half_even(fp32(x / float(scale))), -Q, Q), or 0 when
+ *             scale is 0.
+ *   Dequantised value = code * scale (exact in fp32).
+ * fmt NF_KV_BF16 (512 bytes per token per kv-head):
+ *   k_codes  bf16 [num_blocks][num_kv_heads][256][128]  (keys)
+ *   v_codes  bf16 [num_blocks][num_kv_heads][256][128]  (values)
+ *   k_scales, v_scales unused (may be NULL); v_group ignored.
+ * Every plane must be 16-byte aligned.
+ */
+typedef struct {
+    int32_t fmt;          /* NF_KV_K8V4 or NF_KV_BF16 */
+    int32_t num_blocks;   /* pool capacity in blocks (>= 1) */
+    int32_t block_size;   /* must be 256 */
+    int32_t num_kv_heads; /* >= 1 */
+    int32_t head_dim;     /* must be 128 */
+    int32_t v_group;      /* must be 32 for NF_KV_K8V4 */
+    void *k_codes;
+    void *k_scales;
+    void *v_codes;
+    void *v_scales;
+} nf_kv_layer;
+
+/*
+ * nf_kv_append_quant -- quantise new K/V tokens and write them into the pool.
+ *
+ * k_new, v_new: [batch][n_new][num_kv_heads][128] of in_dtype (NF_F32 or
+ *   NF_BF16), contiguous.  Token i of sequence b is written at position
+ *   seqlens_before[b] + i (seqlens_before: int32 [batch], device), through
+ *   block_table (int32 [batch][max_blocks], device).  Slots not written keep
+ *   their bytes.  The call does not advance any length: the caller does that
+ *   once per step.  For NF_KV_BF16 pools the values are rounded to bf16
+ *   (half to even) and stored.
+ * A token whose block index is >= max_blocks or whose block id is outside the
+ * pool is skipped and NF_DEVERR_TABLE / NF_DEVERR_BLOCK_ID is recorded.
+ * batch * n_new == 0 launches nothing and returns NF_OK.
+ */
+nf_status nf_kv_append_quant(const nf_kv_layer *kv, const void *k_new, const void *v_new,
+                             int32_t in_dtype, int32_t batch, int32_t n_new,
+                             const int32_t *block_table, int32_t max_blocks,
+                             const int32_t *seqlens_before, nf_stream_t stream);
+
+/*
+ * nf_decode_attn_workspace_size -- bytes of device workspace nf_decode_attn
+ * needs for this shape on a device with `num_sms` streaming multiprocessors
+ * (pass the device's count; nf_decode_attn uses the current device's).  The
+ * workspace holds the split partials and needs no initialisation.
+ * Returns 0 for an invalid shape.
+ */
+size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_heads,
+                                     int32_t num_kv_heads, int32_t max_seqlen, int32_t num_sms);
+
+/*
+ * nf_decode_attn -- split-K decode attention over the pool.
+ *
+ * For every sequence b < batch, query token j < n_q and query head h <
+ * num_q_heads, with G = num_q_heads / num_kv_heads and L = seqlens[b] (keys in
+ * the cache, including tokens appended for this step):
+ *   query j sits at position P = L - n_q + j and sees keys t in [0, P] when
+ *   causal != 0, else all t in [0, L);
+ *   s_t = softmax_scale * (q[b][j][h] . k_hat_t) with k_hat of kv-head h / G;
+ *   out[b][j][h] = sum_t exp(s_t - m) v_hat_t / sum_t exp(s_t - m);
+ *   out_lse[b][j][h] = m + ln sum_t exp(s_t - m)   (natural log; m = max s_t).
+ * q: [batch][n_q][num_q_heads][128] of q_dtype (NF_F32 or NF_BF16), device.
+ * out: fp32 [batch][n_q][num_q_heads][128]; out_lse: fp32 [batch][n_q]
+ *   [num_q_heads] or NULL.
+ * seqlens: int32 [batch], device; each must lie in [n_q, max_seqlen], the host
+ *   bound used to size the split plan (violations: NF_DEVERR_SEQLEN, and that
+ *   sequence's rows come out as o = 0, lse = -inf).
+ * block_table: int32 [batch][max_blocks], device; max_blocks >= ceil(max_seqlen
+ *   / 256).  Only entries for positions < L are read.
+ * workspace: device scratch of at least nf_decode_attn_workspace_size(...)
+ *   bytes (16-byte aligned).  Not retained after the call's kernels finish.
+ * Numerics: dequantised keys are used exactly; the fp32 query is split into two
+ *   fp16 halves (bf16 queries are converted to fp16); each dequantised value
+ *   and each softmax weight is rounded to fp16 before the tensor-core P.V
+ *   product; scores, softmax statistics and accumulators are fp32.
+ */
+nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                         int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                         int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                         float softmax_scale, int32_t causal, float *out, float *out_lse,
+                         void *workspace, size_t workspace_bytes, nf_stream_t stream);
+
+/*
+ * nf_attn_combine -- log-sum-exp merge of split attention results (the
+ * flash-decoding reduction; the pages do not describe it).
+ *
+ * part_o: fp32 [n_splits][rows][head_dim]; part_lse: fp32 [n_splits][rows]
+ * (natural log).  For each row: lse = ln sum_j exp(part_lse[j]) and
+ * out = sum_j exp(part_lse[j] - lse) part_o[j], skipping splits whose lse is
+ * -inf (they saw no key); a row with no finite split gets out = 0, lse = -inf.
+ * out: fp32 [rows][head_dim]; out_lse: fp32 [rows] or NULL.  head_dim must be a
+ * multiple of 4 in [4, 1024].  rows == 0 launches nothing.
+ */
+nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_splits,
+                          int32_t rows, int32_t head_dim, float *out, float *out_lse,
+                          nf_stream_t stream);
+
+/*
+ * nf_get_device_error -- read and clear the device error code of the current
+ * device (NF_DEVERR_*).  Synchronises with the device.  Returns NF_OK when no
+ * code was set, NF_ERR_DEVICE_CHECK when one was (written to *code), or
+ * NF_ERR_CUDA.
+ */
+nf_status nf_get_device_error(int32_t *code);
+
+/* Static text for a status code. */
+const char *nf_status_string(nf_status status);
+
+/* Message describing the last failing call on this host thread ("" if none). */
+const char *nf_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NF_H_ */

@@ -1,0 +1,294 @@
+// nf_api.cu -- the C ABI of libnf: host-side validation, split planning and
+// kernel launches.  The declarations and their contracts are in include/nf.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+
+#include "nf.h"
+#include "nf_append.cuh"
+#include "nf_combine.cuh"
+#include "nf_common.cuh"
+#include "nf_decode.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+nf_status fail(nf_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+nf_status after_launch(const char *what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    g_msg[0] = '\0';
+    return NF_OK;
+}
+
+nf_status check_layer(const nf_kv_layer *kv) {
+    if (!kv) return fail(NF_ERR_INVALID_ARG, "kv is NULL");
+    if (kv->fmt != NF_KV_K8V4 && kv->fmt != NF_KV_BF16)
+        return fail(NF_ERR_UNSUPPORTED, "kv->fmt %d is not NF_KV_K8V4 or NF_KV_BF16", kv->fmt);
+    if (kv->block_size != nf::kBlock)
+        return fail(NF_ERR_UNSUPPORTED, "kv->block_size %d (only 256)", kv->block_size);
+    if (kv->head_dim != nf::kHeadDim)
+        return fail(NF_ERR_UNSUPPORTED, "kv->head_dim %d (only 128)", kv->head_dim);
+    if (kv->fmt == NF_KV_K8V4 && kv->v_group != nf::kVGroup)
+        return fail(NF_ERR_UNSUPPORTED, "kv->v_group %d (only 32)", kv->v_group);
+    if (kv->num_blocks < 1 || kv->num_kv_heads < 1)
+        return fail(NF_ERR_INVALID_ARG, "kv->num_blocks %d / num_kv_heads %d must be >= 1",
+                    kv->num_blocks, kv->num_kv_heads);
+    if (!kv->k_codes || !kv->v_codes) return fail(NF_ERR_INVALID_ARG, "kv code planes are NULL");
+    if (kv->fmt == NF_KV_K8V4 && (!kv->k_scales || !kv->v_scales))
+        return fail(NF_ERR_INVALID_ARG, "kv scale planes are NULL");
+    auto misaligned = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) != 0; };
+    if (misaligned(kv->k_codes) || misaligned(kv->v_codes) ||
+        (kv->fmt == NF_KV_K8V4 && (misaligned(kv->k_scales) || misaligned(kv->v_scales))))
+        return fail(NF_ERR_INVALID_ARG, "kv planes must be 16-byte aligned");
+    return NF_OK;
+}
+
+// ---------------------------------------------------------------- split plan
+// The context of each (sequence, kv-head) is cut into n_splits ranges of
+// split_len keys (a multiple of 64) so that batch * H_kv * row_groups *
+// n_splits CTAs fill the GPU about four times over.  Computed from the host
+// bound max_seqlen only; sequences shorter than that leave their last splits
+// empty (they write lse = -inf and exit).
+struct SplitPlan {
+    int n_splits = 0, split_len = 0, n_row_groups = 0, nt = 0, rows_total = 0;
+    size_t part_o_bytes = 0, part_lse_bytes = 0;
+    size_t bytes() const { return part_o_bytes + part_lse_bytes; }
+};
+
+constexpr int kCtasPerSm = 4;
+constexpr int kSplitQuantum = 64;
+
+bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sms, SplitPlan &sp) {
+    if (batch < 1 || n_q < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0 || max_seqlen < n_q ||
+        num_sms < 1)
+        return false;
+    const long long rows_per_head = (long long)(H_q / H_kv) * n_q;
+    if (rows_per_head > 4096) return false;
+    sp.nt = rows_per_head <= 8 ? 1 : 2;
+    sp.n_row_groups = (int)((rows_per_head + nf::kRowsPerCta - 1) / nf::kRowsPerCta);
+    const long long units = (long long)batch * H_kv * sp.n_row_groups;
+    const long long target = (long long)num_sms * kCtasPerSm;
+    const long long max_splits = (max_seqlen + kSplitQuantum - 1) / kSplitQuantum;
+    long long n = (target + units - 1) / units;
+    if (n < 1) n = 1;
+    if (n > max_splits) n = max_splits;
+    long long len = (max_seqlen + n - 1) / n;
+    len = (len + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
+    n = (max_seqlen + len - 1) / len;
+    if (n * units > 0x7fffffffLL) return false;
+    sp.n_splits = (int)n;
+    sp.split_len = (int)len;
+    sp.rows_total = (int)((long long)batch * n_q * H_q);
+    sp.part_o_bytes = (size_t)n * sp.rows_total * nf::kHeadDim * sizeof(float);
+    sp.part_lse_bytes = ((size_t)n * sp.rows_total * sizeof(float) + 255) / 256 * 256;
+    return true;
+}
+
+int current_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+template <int NT, bool QF32, int FMT>
+void launch_decode(const nf::DecodeParams &p, dim3 grid, cudaStream_t s) {
+    nf::decode_split_kernel<NT, QF32, FMT><<<grid, nf::kDecodeWarps * 32, 0, s>>>(p);
+}
+
+template <int NT>
+void dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, dim3 grid, cudaStream_t s) {
+    if (fmt == NF_KV_K8V4) {
+        if (qf32) launch_decode<NT, true, NF_KV_K8V4>(p, grid, s);
+        else launch_decode<NT, false, NF_KV_K8V4>(p, grid, s);
+    } else {
+        if (qf32) launch_decode<NT, true, NF_KV_BF16>(p, grid, s);
+        else launch_decode<NT, false, NF_KV_BF16>(p, grid, s);
+    }
+}
+
+nf_status launch_combine(const float *part_o, const float *part_lse, int n_splits, int rows,
+                         int head_dim, float *out, float *out_lse, cudaStream_t s) {
+    nf::CombineParams c{part_o, part_lse, n_splits, rows, head_dim, out, out_lse};
+    nf::combine_kernel<<<rows, nf::kCombineWarps * 32, 0, s>>>(c);
+    return after_launch("combine kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+nf_status nf_kv_append_quant(const nf_kv_layer *kv, const void *k_new, const void *v_new,
+                             int32_t in_dtype, int32_t batch, int32_t n_new,
+                             const int32_t *block_table, int32_t max_blocks,
+                             const int32_t *seqlens_before, nf_stream_t stream) {
+    nf_status st = check_layer(kv);
+    if (st != NF_OK) return st;
+    if (batch < 0 || n_new < 0) return fail(NF_ERR_INVALID_ARG, "batch %d / n_new %d < 0", batch, n_new);
+    if (in_dtype != NF_F32 && in_dtype != NF_BF16)
+        return fail(NF_ERR_UNSUPPORTED, "in_dtype %d (NF_F32 or NF_BF16)", in_dtype);
+    if ((long long)batch * n_new == 0) {
+        g_msg[0] = '\0';
+        return NF_OK;
+    }
+    if (!k_new || !v_new || !block_table || !seqlens_before)
+        return fail(NF_ERR_INVALID_ARG, "a device pointer is NULL");
+    if (max_blocks < 1) return fail(NF_ERR_INVALID_ARG, "max_blocks %d < 1", max_blocks);
+    const size_t align = in_dtype == NF_F32 ? 16 : 8;
+    if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & (align - 1))
+        return fail(NF_ERR_INVALID_ARG, "k_new / v_new must be %zu-byte aligned", align);
+    nf::AppendParams p{};
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.in_f32 = in_dtype == NF_F32;
+    p.batch = batch;
+    p.n_new = n_new;
+    p.num_kv_heads = kv->num_kv_heads;
+    p.block_table = block_table;
+    p.max_blocks = max_blocks;
+    p.seqlens_before = seqlens_before;
+    p.num_blocks = kv->num_blocks;
+    p.fmt = kv->fmt;
+    p.k_codes = kv->k_codes;
+    p.k_scales = static_cast<__half *>(kv->k_scales);
+    p.v_codes = kv->v_codes;
+    p.v_scales = static_cast<__half *>(kv->v_scales);
+    const long long items = (long long)batch * n_new * kv->num_kv_heads;
+    const long long blocks = (items + 7) / 8;
+    if (blocks > 0x7fffffffLL) return fail(NF_ERR_INVALID_ARG, "too many tokens in one append");
+    nf::append_quant_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    return after_launch("append kernel launch");
+}
+
+size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_heads,
+                                     int32_t num_kv_heads, int32_t max_seqlen, int32_t num_sms) {
+    SplitPlan sp;
+    if (!make_plan(batch, n_q, num_q_heads, num_kv_heads, max_seqlen, num_sms, sp)) return 0;
+    return sp.bytes();
+}
+
+nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                         int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                         int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                         float softmax_scale, int32_t causal, float *out, float *out_lse,
+                         void *workspace, size_t workspace_bytes, nf_stream_t stream) {
+    nf_status st = check_layer(kv);
+    if (st != NF_OK) return st;
+    if (q_dtype != NF_F32 && q_dtype != NF_BF16)
+        return fail(NF_ERR_UNSUPPORTED, "q_dtype %d (NF_F32 or NF_BF16)", q_dtype);
+    if (batch < 1 || n_q < 1 || num_q_heads < 1)
+        return fail(NF_ERR_INVALID_ARG, "batch %d, n_q %d, num_q_heads %d must be >= 1", batch, n_q,
+                    num_q_heads);
+    if (batch > 65535 || kv->num_kv_heads > 65535)
+        return fail(NF_ERR_UNSUPPORTED, "batch %d / num_kv_heads %d above 65535", batch, kv->num_kv_heads);
+    if (num_q_heads % kv->num_kv_heads != 0)
+        return fail(NF_ERR_INVALID_ARG, "num_q_heads %d not a multiple of num_kv_heads %d",
+                    num_q_heads, kv->num_kv_heads);
+    if (max_seqlen < n_q) return fail(NF_ERR_INVALID_ARG, "max_seqlen %d < n_q %d", max_seqlen, n_q);
+    if ((long long)max_blocks * nf::kBlock < max_seqlen)
+        return fail(NF_ERR_INVALID_ARG, "max_blocks %d cannot hold max_seqlen %d", max_blocks, max_seqlen);
+    if (!q || !block_table || !seqlens || !out) return fail(NF_ERR_INVALID_ARG, "a device pointer is NULL");
+    if (!std::isfinite(softmax_scale)) return fail(NF_ERR_INVALID_ARG, "softmax_scale is not finite");
+    const uintptr_t qa = reinterpret_cast<uintptr_t>(q);
+    if ((q_dtype == NF_F32 && (qa & 15)) || (q_dtype == NF_BF16 && (qa & 7)) ||
+        (reinterpret_cast<uintptr_t>(out) & 15))
+        return fail(NF_ERR_INVALID_ARG, "q / out misaligned");
+    const int sms = current_sm_count();
+    if (sms < 1) return fail(NF_ERR_CUDA, "cannot query the current device");
+    SplitPlan sp;
+    if (!make_plan(batch, n_q, num_q_heads, kv->num_kv_heads, max_seqlen, sms, sp))
+        return fail(NF_ERR_INVALID_ARG, "unsupported shape (n_q * group too large?)");
+    if (workspace_bytes < sp.bytes() || (!workspace && sp.bytes() > 0))
+        return fail(NF_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, sp.bytes());
+    if (reinterpret_cast<uintptr_t>(workspace) & 15)
+        return fail(NF_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+
+    nf::DecodeParams p{};
+    p.k_codes = kv->k_codes;
+    p.k_scales = static_cast<const __half *>(kv->k_scales);
+    p.v_codes = kv->v_codes;
+    p.v_scales = static_cast<const __half *>(kv->v_scales);
+    p.num_blocks = kv->num_blocks;
+    p.num_kv_heads = kv->num_kv_heads;
+    p.q = q;
+    p.batch = batch;
+    p.n_q = n_q;
+    p.num_q_heads = num_q_heads;
+    p.group = num_q_heads / kv->num_kv_heads;
+    p.rows_per_head = p.group * n_q;
+    p.block_table = block_table;
+    p.max_blocks = max_blocks;
+    p.seqlens = seqlens;
+    p.max_seqlen = max_seqlen;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.causal = causal != 0;
+    p.split_len = sp.split_len;
+    p.n_splits = sp.n_splits;
+    p.n_row_groups = sp.n_row_groups;
+    p.part_o = static_cast<float *>(workspace);
+    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + sp.part_o_bytes);
+    p.rows_total = sp.rows_total;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)(sp.n_splits * sp.n_row_groups), (unsigned)kv->num_kv_heads, (unsigned)batch);
+    if (sp.nt == 1) dispatch_decode<1>(p, q_dtype == NF_F32, kv->fmt, grid, s);
+    else dispatch_decode<2>(p, q_dtype == NF_F32, kv->fmt, grid, s);
+    st = after_launch("decode kernel launch");
+    if (st != NF_OK) return st;
+    return launch_combine(p.part_o, p.part_lse, sp.n_splits, sp.rows_total, nf::kHeadDim, out, out_lse, s);
+}
+
+nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_splits,
+                          int32_t rows, int32_t head_dim, float *out, float *out_lse,
+                          nf_stream_t stream) {
+    if (n_splits < 1 || rows < 0) return fail(NF_ERR_INVALID_ARG, "n_splits %d / rows %d", n_splits, rows);
+    if (head_dim < 4 || head_dim > 1024 || head_dim % 4 != 0)
+        return fail(NF_ERR_UNSUPPORTED, "head_dim %d (multiple of 4 in [4, 1024])", head_dim);
+    if (rows == 0) {
+        g_msg[0] = '\0';
+        return NF_OK;
+    }
+    if (!part_o || !part_lse || !out) return fail(NF_ERR_INVALID_ARG, "a device pointer is NULL");
+    if ((reinterpret_cast<uintptr_t>(part_o) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return fail(NF_ERR_INVALID_ARG, "part_o / out must be 16-byte aligned");
+    return launch_combine(part_o, part_lse, n_splits, rows, head_dim, out, out_lse,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+nf_status nf_get_device_error(int32_t *code) {
+    if (!code) return fail(NF_ERR_INVALID_ARG, "code is NULL");
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, nf::g_device_error, sizeof(v));
+    if (e == cudaSuccess) {
+        const int32_t zero = 0;
+        e = cudaMemcpyToSymbol(nf::g_device_error, &zero, sizeof(zero));
+    }
+    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    *code = v;
+    return v ? NF_ERR_DEVICE_CHECK : NF_OK;
+}
+
+const char *nf_status_string(nf_status status) {
+    switch (status) {
+        case NF_OK: return "ok";
+        case NF_ERR_INVALID_ARG: return "invalid argument";
+        case NF_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case NF_ERR_WORKSPACE: return "workspace too small";
+        case NF_ERR_CUDA: return "CUDA error";
+        case NF_ERR_DEVICE_CHECK: return "device-side check failed";
+        default: return "unknown status";
+    }
+}
+
+const char *nf_last_error(void) { return g_msg; }
+
+}  // extern "C"

@@ -1,0 +1,98 @@
+// nf_common.cuh -- device helpers shared by the kernels of libnf (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nf.h"
+
+namespace nf {
+
+constexpr int kHeadDim = 128;
+constexpr int kBlock = 256;   // tokens per KV segment
+constexpr int kVGroup = 32;   // V channels per scale
+
+// First device-side problem seen since the last nf_get_device_error().
+__device__ int32_t g_device_error;
+
+__device__ __forceinline__ void report(int32_t code) { atomicCAS(&g_device_error, 0, code); }
+
+__device__ __forceinline__ uint32_t h2_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 u32_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    return h2_u32(__floats2half2_rn(lo, hi));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// 2^x on the MUFU unit (relative error ~2^-22; -inf gives +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// D = A * B + D, m16n8k16, fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Same with bf16 inputs.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit elements held one row-pair per lane.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Read-only 16-byte global load.
+__device__ __forceinline__ uint4 ldg16(const void *p) {
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+// Four int8 codes (one per byte of w) -> two fp16x2: (c0, c1), (c2, c3).
+// Offset-binary trick: byte u = c + 128 placed under the exponent of 1024
+// gives the fp16 value 1024 + u exactly; subtracting 1152 leaves c exactly.
+__device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    const __half2 bias = u32_h2(0x64806480u);  // 1152, 1152
+    lo = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4140)), bias));
+    hi = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4342)), bias));
+}
+
+// Packed two's-complement nibbles -> fp16x2 codes, exact.  For a word w with
+// nibbles n0..n7 (n_k in bits 4k..4k+3):
+//   nib_even(w) = (n0, n4) as fp16 values in [-8, 7]
+//   nib_odd(w)  = (n1, n5)
+// (apply to w >> 8 for (n2, n6) and (n3, n7)).  The sign bit is flipped to get
+// u = c + 8; u sits under the exponent of 1024 (or 1024 * 16 for the odd
+// nibble) and the bias is removed exactly.
+__device__ __forceinline__ __half2 nib_even(uint32_t w) {
+    const uint32_t x = ((w ^ 0x88888888u) & 0x000F000Fu) | 0x64006400u;  // 1024 + u
+    return __hsub2(u32_h2(x), u32_h2(0x64086408u));                      // - 1032
+}
+__device__ __forceinline__ __half2 nib_odd(uint32_t w) {
+    const uint32_t x = ((w ^ 0x88888888u) & 0x00F000F0u) | 0x64006400u;  // 1024 + 16u
+    return __hfma2(u32_h2(x), u32_h2(0x2C002C00u), u32_h2(0xD480D480u)); // /16 - 72
+}
+
+}  // namespace nf

@@ -1,0 +1,182 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Codes and scales must match bit for bit (every byte of the pool planes,
+untouched slots included); attention outputs within max-abs 2e-3 and
+relative-L2 1e-3 of the oracle's fp64 result, lse within 2e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_quantized_b200 as nf
+import oracle
+import workloads
+from nfcase import ATOL, REL_L2, run_case, gpu_layer, oracle_pool, compare_pool, oracle_attention, \
+    select_heads, check_attention
+
+pytestmark = pytest.mark.gpu
+
+K8, BF = nf.NF_KV_K8V4, nf.NF_KV_BF16
+
+
+@pytest.fixture(autouse=True)
+def _clean_device_error():
+    torch.cuda.synchronize()
+    assert nf.nf_get_device_error() == 0
+    yield
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------- edge-case shapes
+SMALL = [
+    # (id, kwargs for workloads.custom)
+    ("len1", dict(cached=(1,))),
+    ("len15", dict(cached=(15,))),
+    ("len16", dict(cached=(16,))),
+    ("len17", dict(cached=(17,))),
+    ("len255", dict(cached=(255,))),
+    ("len256", dict(cached=(256,))),
+    ("len257", dict(cached=(257,))),
+    ("len1000_gqa8", dict(cached=(1000,), num_q_heads=16, num_kv_heads=2)),
+    ("len700_mha", dict(cached=(700,), num_q_heads=3, num_kv_heads=3)),
+    ("len2049_gqa5", dict(cached=(2049,), num_q_heads=10, num_kv_heads=2)),
+    ("ragged3", dict(cached=(1, 300, 1000), num_q_heads=8, num_kv_heads=2)),
+    ("mtp4_causal", dict(cached=(500,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True)),
+    ("mtp4_noncausal", dict(cached=(500,), n_new=4, n_q=4, num_q_heads=8, num_kv_heads=2, causal=False)),
+    ("mtp3_gqa5", dict(cached=(300, 41), n_new=3, n_q=3, num_q_heads=10, num_kv_heads=2, causal=True)),
+    ("mtp4_short", dict(cached=(0,), n_new=4, n_q=4, num_q_heads=8, num_kv_heads=1, causal=True)),
+    ("append1", dict(cached=(767,), n_new=1, num_q_heads=8, num_kv_heads=1)),
+    ("q_rows_64", dict(cached=(400,), n_new=4, n_q=4, num_q_heads=16, num_kv_heads=1, causal=True)),
+]
+
+
+@pytest.mark.parametrize("fmt", [K8, BF], ids=["k8v4", "bf16"])
+@pytest.mark.parametrize("qdt", [torch.float32, torch.bfloat16], ids=["qf32", "qbf16"])
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_shapes(case, qdt, fmt):
+    w = workloads.custom(case[0], q_dtype=qdt, kv_in_dtype=qdt, **case[1])
+    run_case(w, 0, fmt)
+
+
+def test_max_seqlen_above_actual_lengths():
+    # the split plan is sized for 5000 keys; the sequences are shorter, so the
+    # trailing splits see no key and must not disturb the result
+    w = workloads.custom("slack", cached=(700, 33), num_q_heads=8, num_kv_heads=2)
+    run_case(w, 0, K8, max_seqlen=5000)
+
+
+def test_large_query_scale_and_outlier_keys():
+    # peaked softmax: a large-norm query against outlier channels
+    w = workloads.custom("peaked", cached=(3000,), num_q_heads=8, num_kv_heads=1,
+                         q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, dist="k_outlier_channels")
+    q = workloads.layer_q(w, 0, device="cuda").float() * 6.0
+    run_case(w, 0, K8, q_override=q.to(torch.bfloat16))
+
+
+# ------------------------------------------------------------- combine
+def test_combine_matches_oracle():
+    g = torch.Generator(device="cpu").manual_seed(5)
+    S, rows = 37, 45
+    po = torch.randn((S, rows, 128), generator=g)
+    pl = torch.randn((S, rows), generator=g) * 4
+    pl[3] = -math.inf
+    pl[:, 7] = -math.inf          # a row no split saw
+    out = torch.empty((rows, 128), device="cuda")
+    lse = torch.empty(rows, device="cuda")
+    nf.nf_attn_combine(po.cuda(), pl.cuda(), out, lse)
+    ro, rl = oracle.combine(po.double().numpy(), pl.double().numpy())
+    go = out.cpu().double().numpy()
+    assert np.abs(go - ro).max() <= 1e-5
+    gl = lse.cpu().double().numpy()
+    assert gl[7] == -math.inf and np.all(go[7] == 0)
+    fin = np.isfinite(rl)
+    assert np.abs(gl[fin] - rl[fin]).max() <= 1e-5
+
+
+# ------------------------------------------------ device checks, no faults
+def test_bad_block_id_is_reported_not_faulted():
+    w = workloads.custom("bad", cached=(600,), num_q_heads=4, num_kv_heads=1)
+    bt = workloads.block_table(w).copy()
+    g = gpu_layer(w, 0, K8)                     # a clean run first
+    assert nf.nf_get_device_error() == 0
+    bt_bad = torch.as_tensor(bt, dtype=torch.int32, device="cuda")
+    bt_bad[0, 1] = w.pool_blocks + 7            # the block holding keys 256..511
+    out = torch.empty_like(g["out"])
+    sl = torch.tensor([600], dtype=torch.int32, device="cuda")
+    ws = torch.empty(nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 600), dtype=torch.uint8, device="cuda")
+    nf.nf_decode_attn(g["kv"], g["q"], bt_bad, sl, 600, w.softmax_scale, False, out, None, ws)
+    assert nf.nf_get_device_error() == nf.NF_DEVERR_BLOCK_ID
+    # the context is still usable and a correct call still gives the right answer
+    nf.nf_decode_attn(g["kv"], g["q"], torch.as_tensor(bt, device="cuda"), sl, 600, w.softmax_scale,
+                      False, out, None, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, g["out"])
+    assert nf.nf_get_device_error() == 0
+
+
+def test_append_outside_table_is_reported():
+    kv = nf.KVLayer.empty(K8, 2, 1, fill=0)
+    bt = torch.tensor([[0, 1]], dtype=torch.int32, device="cuda")
+    k = torch.randn((1, 1, 1, 128), device="cuda")
+    nf.nf_kv_append_quant(kv, k, k, bt, torch.tensor([512], dtype=torch.int32, device="cuda"))
+    assert nf.nf_get_device_error() == nf.NF_DEVERR_TABLE
+    bt[0, 1] = 9
+    nf.nf_kv_append_quant(kv, k, k, bt, torch.tensor([256], dtype=torch.int32, device="cuda"))
+    assert nf.nf_get_device_error() == nf.NF_DEVERR_BLOCK_ID
+    assert torch.all(kv.k_codes == 0)
+
+
+def test_seqlen_above_bound_is_reported():
+    w = workloads.custom("sl", cached=(300,), num_q_heads=4, num_kv_heads=1)
+    g = gpu_layer(w, 0, K8)
+    sl = torch.tensor([400], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(g["out"])
+    lse = torch.empty_like(g["lse"])
+    ws = torch.empty(nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 300), dtype=torch.uint8, device="cuda")
+    nf.nf_decode_attn(g["kv"], g["q"], torch.as_tensor(g["bt"], device="cuda"), sl, 300,
+                      w.softmax_scale, False, out, lse, ws)
+    assert nf.nf_get_device_error() == nf.NF_DEVERR_SEQLEN
+    assert torch.all(out == 0) and torch.all(torch.isinf(lse))
+
+
+def test_workspace_too_small_is_refused():
+    w = workloads.custom("ws", cached=(300,), num_q_heads=4, num_kv_heads=1)
+    g = gpu_layer(w, 0, K8)
+    need = nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 300)
+    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(nf.NfError) as e:
+        nf.nf_decode_attn(g["kv"], g["q"], torch.as_tensor(g["bt"], device="cuda"),
+                          torch.tensor([300], dtype=torch.int32, device="cuda"), 300,
+                          w.softmax_scale, False, torch.empty_like(g["out"]), None, ws)
+    assert e.value.status == nf.NF_ERR_WORKSPACE
+
+
+# ------------------------------------------------- the five workloads, full size
+def _full_size(name, fmt, heads, layer=0):
+    w = workloads.get(name)
+    g = gpu_layer(w, layer, fmt)
+    pool, hs = oracle_pool(w, fmt, g["kvin"], g["bt"], heads)
+    compare_pool(g["kv"], pool, hs)
+    ref_o, ref_l = oracle_attention(w, pool, hs, g["q"], g["bt"])
+    return check_attention(select_heads(g["out"], w, hs), select_heads(g["lse"], w, hs), ref_o, ref_l)
+
+
+def test_workload_tiny_all_heads():
+    _full_size("tiny", K8, heads=None)
+
+
+@pytest.mark.parametrize("name,heads,layer", [
+    ("ctx32k_append", [0, 3], 0),
+    ("ctx32k_append", [1], 15),
+    ("ragged_c2", [0, 3], 0),
+    ("mtp_verify", [2], 0),
+    ("longest", [0, 7], 0),
+])
+def test_workload_full_size_sampled_heads(name, heads, layer):
+    _full_size(name, K8, heads=heads, layer=layer)
+
+
+def test_workload_longest_bf16_cache_sampled_head():
+    _full_size("longest", BF, heads=[5])
