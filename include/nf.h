@@ -175,6 +175,36 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
                          void *workspace, size_t workspace_bytes, nf_stream_t stream);
 
 /*
+ * nf_decode_attn_noalloc -- nf_decode_attn for callers that cannot allocate
+ * device memory when they call: for example a host engine that reserves its
+ * whole memory budget at start-up and gives plug-in kernels no allocator, or
+ * a latency-critical loop where cudaMalloc's implicit device synchronisation
+ * is not acceptable.  The pages have no counterpart of this call; it exists
+ * for such callers only.
+ *
+ * Same arguments and results as nf_decode_attn, minus the workspace.  The
+ * split partials go to a scratch array of NF_NOALLOC_SCRATCH_BYTES that lives
+ * in the library's device image: every GPU that loads libnf holds it until the
+ * process exits.  The call allocates nothing (no cudaMalloc, no allocating
+ * library routine).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture on the device.
+ *  - Shapes whose nf_decode_attn_workspace_size() exceeds
+ *    NF_NOALLOC_SCRATCH_BYTES are refused with NF_ERR_WORKSPACE.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents; the call needs nothing in it to start at zero.  Calls that
+ *    overlap on the GPU (concurrent streams, or other host threads) race on
+ *    it: order them on one stream.
+ */
+#define NF_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+nf_status nf_decode_attn_noalloc(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                                 int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                                 int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                                 float softmax_scale, int32_t causal, float *out, float *out_lse,
+                                 nf_stream_t stream);
+
+/*
  * nf_attn_combine -- log-sum-exp merge of split attention results (the
  * flash-decoding reduction; the pages do not describe it).
  *

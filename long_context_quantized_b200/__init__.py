@@ -17,7 +17,8 @@ import torch
 
 __all__ = [
     "NF_OK", "NF_KV_K8V4", "NF_KV_BF16", "NF_F32", "NF_BF16", "NfError", "KVLayer",
-    "nf_kv_append_quant", "nf_decode_attn_workspace_size", "nf_decode_attn", "nf_attn_combine",
+    "nf_kv_append_quant", "nf_decode_attn_workspace_size", "nf_decode_attn", "nf_decode_attn_noalloc",
+    "nf_attn_combine",
     "nf_get_device_error", "nf_status_string", "library_path", "load_library",
 ]
 
@@ -75,6 +76,8 @@ def load_library():
         lib.nf_decode_attn_workspace_size.restype = S
         lib.nf_decode_attn.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, P, P, P, S, P]
         lib.nf_decode_attn.restype = I
+        lib.nf_decode_attn_noalloc.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, P, P, P]
+        lib.nf_decode_attn_noalloc.restype = I
         lib.nf_attn_combine.argtypes = [P, P, I, I, I, P, P, P]
         lib.nf_attn_combine.restype = I
         lib.nf_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32)]
@@ -209,6 +212,27 @@ def nf_decode_attn(kv: KVLayer, q, block_table, seqlens, max_seqlen: int, softma
         block_table.shape[1], _dptr(seqlens), int(max_seqlen), float(softmax_scale), int(bool(causal)),
         _dptr(out), _dptr(out_lse), _dptr(workspace), ws_bytes, _stream(stream))
     _check(st, "nf_decode_attn")
+
+
+NF_NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def nf_decode_attn_noalloc(kv: KVLayer, q, block_table, seqlens, max_seqlen: int, softmax_scale: float,
+                           causal: bool, out, out_lse=None, stream=None):
+    """nf_decode_attn for callers that cannot allocate device memory at call
+    time: the scratch is a fixed array inside libnf's device image (see nf.h).
+    Calls on one device share it, so do not overlap them on the GPU."""
+    _need(q, "q")
+    _need(block_table, "block_table", torch.int32)
+    _need(seqlens, "seqlens", torch.int32)
+    _need(out, "out", torch.float32)
+    _need(out_lse, "out_lse", torch.float32)
+    B, n_q, H_q = q.shape[0], q.shape[1], q.shape[2]
+    st = load_library().nf_decode_attn_noalloc(
+        ctypes.byref(kv.c), _dptr(q), _dtype_code(q.dtype), B, n_q, H_q, _dptr(block_table),
+        block_table.shape[1], _dptr(seqlens), int(max_seqlen), float(softmax_scale), int(bool(causal)),
+        _dptr(out), _dptr(out_lse), _stream(stream))
+    _check(st, "nf_decode_attn_noalloc")
 
 
 def nf_attn_combine(part_o, part_lse, out, out_lse=None, stream=None):

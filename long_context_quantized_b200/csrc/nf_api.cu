@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 
 #include "nf.h"
 #include "nf_append.cuh"
@@ -121,6 +122,36 @@ nf_status launch_combine(const float *part_o, const float *part_lse, int n_split
     nf::CombineParams c{part_o, part_lse, n_splits, rows, head_dim, out, out_lse};
     nf::combine_kernel<<<rows, nf::kCombineWarps * 32, 0, s>>>(c);
     return after_launch("combine kernel launch");
+}
+
+// Scratch of nf_decode_attn_noalloc (for callers that cannot allocate device
+// memory).  It is part of the library's device image, so every GPU that loads
+// libnf holds NF_NOALLOC_SCRATCH_BYTES of it until the process exits.  In host
+// code the name is only a stand-in for the symbol: its device address comes
+// from cudaGetSymbolAddress on each device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NF_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device with that device current.
+nf_status noalloc_scratch(void **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(NF_ERR_UNSUPPORTED, "device %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(NF_ERR_CUDA, "cudaGetSymbolAddress(no-alloc scratch): %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return NF_OK;
 }
 
 }  // namespace
@@ -245,6 +276,27 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
     st = after_launch("decode kernel launch");
     if (st != NF_OK) return st;
     return launch_combine(p.part_o, p.part_lse, sp.n_splits, sp.rows_total, nf::kHeadDim, out, out_lse, s);
+}
+
+nf_status nf_decode_attn_noalloc(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                                 int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                                 int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                                 float softmax_scale, int32_t causal, float *out, float *out_lse,
+                                 nf_stream_t stream) {
+    if (kv && kv->num_kv_heads > 0) {
+        const int sms = current_sm_count();
+        SplitPlan sp;
+        if (sms > 0 && make_plan(batch, n_q, num_q_heads, kv->num_kv_heads, max_seqlen, sms, sp) &&
+            sp.bytes() > NF_NOALLOC_SCRATCH_BYTES)
+            return fail(NF_ERR_WORKSPACE, "shape needs %zu bytes of scratch, above the %zu-byte no-alloc maximum",
+                        sp.bytes(), (size_t)NF_NOALLOC_SCRATCH_BYTES);
+    }
+    void *scratch = nullptr;
+    const nf_status st = noalloc_scratch(&scratch);
+    if (st != NF_OK) return st;
+    return nf_decode_attn(kv, q, q_dtype, batch, n_q, num_q_heads, block_table, max_blocks, seqlens,
+                          max_seqlen, softmax_scale, causal, out, out_lse, scratch,
+                          NF_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_splits,

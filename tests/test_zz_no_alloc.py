@@ -1,0 +1,66 @@
+"""nf_decode_attn_noalloc: the decode-attention entry point for callers that
+cannot allocate device memory at call time (an engine that reserves its whole
+budget at start-up and gives plug-ins no allocator, or a latency-critical loop
+that cannot afford cudaMalloc's implicit synchronisation).  Its scratch is a
+fixed array inside libnf's device image.
+
+Checked through the C ABI against nf_decode_attn (caller-provided workspace)
+on two calls in a row with different queries, within the parity tolerance the
+other GPU tests use.  This file is collected last on purpose."""
+import numpy as np
+import pytest
+import torch
+
+import long_context_quantized_b200 as nf
+import workloads
+from nfcase import ATOL, REL_L2, gpu_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def _close(a, b):
+    a = a.double().cpu().numpy()
+    b = b.double().cpu().numpy()
+    assert np.all(np.isfinite(a))
+    assert np.abs(a - b).max() <= ATOL
+    assert np.linalg.norm(a - b) / np.linalg.norm(b) <= REL_L2
+
+
+def test_noalloc_matches_workspace_entry_point_on_two_calls():
+    w = workloads.custom("noalloc", cached=(3000, 1200), n_new=4, n_q=4, num_q_heads=16, num_kv_heads=2,
+                         q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, causal=True)
+    g = gpu_layer(w, 0, nf.NF_KV_K8V4)
+    bt = torch.as_tensor(g["bt"], device="cuda")
+    sl = torch.as_tensor(w.seqlens, dtype=torch.int32, device="cuda")
+    msl = max(w.seqlens)
+    assert nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, msl) \
+        <= nf.NF_NOALLOC_SCRATCH_BYTES
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, msl),
+                     dtype=torch.uint8, device="cuda")
+    queries = [g["q"], (g["q"].float() * -1.5).to(torch.bfloat16)]
+    for q in queries:  # two calls in a row; the second must not see the first's scratch
+        ref = torch.empty_like(g["out"])
+        ref_lse = torch.empty_like(g["lse"])
+        nf.nf_decode_attn(g["kv"], q, bt, sl, msl, w.softmax_scale, True, ref, ref_lse, ws)
+        out = torch.full_like(g["out"], float("nan"))
+        lse = torch.full_like(g["lse"], float("nan"))
+        nf.nf_decode_attn_noalloc(g["kv"], q, bt, sl, msl, w.softmax_scale, True, out, lse)
+        torch.cuda.synchronize()
+        _close(out, ref)
+        _close(lse, ref_lse)
+    assert nf.nf_get_device_error() == 0
+
+
+def test_noalloc_refuses_shapes_above_its_scratch():
+    # 64 sequences x 8 queries x 64 heads needs far more scratch than the fixed array
+    kv = nf.KVLayer.empty(nf.NF_KV_K8V4, 4, 8, device="cuda", fill=0)
+    B, n_q, H_q, msl = 64, 8, 64, 1 << 20
+    need = nf.nf_decode_attn_workspace_size(B, n_q, H_q, 8, msl)
+    assert need > nf.NF_NOALLOC_SCRATCH_BYTES
+    q = torch.zeros((B, n_q, H_q, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((B, n_q, H_q, 128), dtype=torch.float32, device="cuda")
+    bt = torch.zeros((B, msl // 256), dtype=torch.int32, device="cuda")
+    sl = torch.full((B,), 16, dtype=torch.int32, device="cuda")
+    with pytest.raises(nf.NfError) as e:
+        nf.nf_decode_attn_noalloc(kv, q, bt, sl, msl, 0.1, False, out)
+    assert e.value.status == nf.NF_ERR_WORKSPACE
