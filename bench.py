@@ -172,7 +172,7 @@ class GpuWorkload:
             self.q.append(workloads.layer_q(w, layer, device=device))
             self.out.append(torch.empty((w.batch, w.n_q, w.num_q_heads, 128), dtype=torch.float32, device=device))
         ws = nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, self.max_seqlen)
-        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.ws = torch.zeros(ws, dtype=torch.uint8, device=device)
         torch.cuda.synchronize()
         assert nf.nf_get_device_error() == 0
 

@@ -63,6 +63,7 @@ typedef int32_t nf_status;
 #define NF_DEVERR_BLOCK_ID 1  /* a block-table entry outside [0, num_blocks) */
 #define NF_DEVERR_TABLE 2     /* a position whose block index is >= max_blocks */
 #define NF_DEVERR_SEQLEN 3    /* seqlens[b] < n_q or > max_seqlen */
+#define NF_DEVERR_TIMEOUT 4   /* a bounded wait inside a kernel gave up (the kernel returned) */
 
 /* Element types. */
 #define NF_F32 0
@@ -136,8 +137,11 @@ nf_status nf_kv_append_quant(const nf_kv_layer *kv, const void *k_new, const voi
  * nf_decode_attn_workspace_size -- bytes of device workspace nf_decode_attn
  * needs for this shape on a device with `num_sms` streaming multiprocessors
  * (pass the device's count; nf_decode_attn uses the current device's).  The
- * workspace holds the split partials and needs no initialisation.
- * Returns 0 for an invalid shape.
+ * workspace holds one ticket counter per (sequence, kv-head) and the (o, lse)
+ * partials of the context splits.  Zero-fill it once before its first use
+ * (e.g. cudaMemsetAsync); every call leaves it zero-filled where it must be
+ * when its kernel completes, so it can be reused call after call on one
+ * stream.  Returns 0 for an invalid or unsupported shape.
  */
 size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_heads,
                                      int32_t num_kv_heads, int32_t max_seqlen, int32_t num_sms);
@@ -162,7 +166,10 @@ size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_h
  * block_table: int32 [batch][max_blocks], device; max_blocks >= ceil(max_seqlen
  *   / 256).  Only entries for positions < L are read.
  * workspace: device scratch of at least nf_decode_attn_workspace_size(...)
- *   bytes (16-byte aligned).  Not retained after the call's kernels finish.
+ *   bytes, 256-byte aligned, zero-filled before its first use (see above).
+ *   Calls that share a workspace must not overlap on the GPU.
+ * Supported: batch <= 256, (num_q_heads / num_kv_heads) * n_q <= 64; other
+ *   shapes return NF_ERR_UNSUPPORTED.
  * Numerics: dequantised keys are used exactly; the fp32 query is split into two
  *   fp16 halves (bf16 queries are converted to fp16); each dequantised value
  *   and each softmax weight is rounded to fp16 before the tensor-core P.V
@@ -193,9 +200,10 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
  *  - Shapes whose nf_decode_attn_workspace_size() exceeds
  *    NF_NOALLOC_SCRATCH_BYTES are refused with NF_ERR_WORKSPACE.
  *  - All calls on a device share the one array and it keeps the last call's
- *    contents; the call needs nothing in it to start at zero.  Calls that
- *    overlap on the GPU (concurrent streams, or other host threads) race on
- *    it: order them on one stream.
+ *    contents; each call first clears (cudaMemsetAsync on `stream`) the
+ *    counters that must start at zero.  Calls that overlap on the GPU
+ *    (concurrent streams, or other host threads) race on it: order them on
+ *    one stream.
  */
 #define NF_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 nf_status nf_decode_attn_noalloc(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 
 #include "nf.h"
@@ -53,44 +54,34 @@ nf_status check_layer(const nf_kv_layer *kv) {
     return NF_OK;
 }
 
-// ---------------------------------------------------------------- split plan
-// The context of each (sequence, kv-head) is cut into n_splits ranges of
-// split_len keys (a multiple of 64) so that batch * H_kv * row_groups *
-// n_splits CTAs fill the GPU about four times over.  Computed from the host
-// bound max_seqlen only; sequences shorter than that leave their last splits
-// empty (they write lse = -inf and exit).
-struct SplitPlan {
-    int n_splits = 0, split_len = 0, n_row_groups = 0, nt = 0, rows_total = 0;
-    size_t part_o_bytes = 0, part_lse_bytes = 0;
-    size_t bytes() const { return part_o_bytes + part_lse_bytes; }
+// ---------------------------------------------------------------- plan
+// The decode kernel is persistent: one CTA per SM, each taking an equal share
+// of all (sequence, kv-head) key chunks (computed on the device from seqlens).
+// The workspace holds one ticket counter per (sequence, kv-head) -- zero
+// between calls -- and one (o, lse) partial slot per CTA plus one per segment
+// (a CTA's pieces and a segment's pieces both form contiguous runs, so slot
+// segment + cta is unique).
+struct Plan {
+    int ctas = 0, nt = 0, n_rg = 0, rows = 0, segments = 0, slot_floats = 0;
+    size_t ticket_bytes = 0, partial_bytes = 0;
+    size_t bytes() const { return ticket_bytes + partial_bytes; }
 };
 
-constexpr int kCtasPerSm = 4;
-constexpr int kSplitQuantum = 64;
-
-bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sms, SplitPlan &sp) {
+bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sms, Plan &pl) {
     if (batch < 1 || n_q < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0 || max_seqlen < n_q ||
-        num_sms < 1)
+        num_sms < 1 || batch > nf::kMaxBatch)
         return false;
-    const long long rows_per_head = (long long)(H_q / H_kv) * n_q;
-    if (rows_per_head > 4096) return false;
-    sp.nt = rows_per_head <= 8 ? 1 : 2;
-    sp.n_row_groups = (int)((rows_per_head + nf::kRowsPerCta - 1) / nf::kRowsPerCta);
-    const long long units = (long long)batch * H_kv * sp.n_row_groups;
-    const long long target = (long long)num_sms * kCtasPerSm;
-    const long long max_splits = (max_seqlen + kSplitQuantum - 1) / kSplitQuantum;
-    long long n = (target + units - 1) / units;
-    if (n < 1) n = 1;
-    if (n > max_splits) n = max_splits;
-    long long len = (max_seqlen + n - 1) / n;
-    len = (len + kSplitQuantum - 1) / kSplitQuantum * kSplitQuantum;
-    n = (max_seqlen + len - 1) / len;
-    if (n * units > 0x7fffffffLL) return false;
-    sp.n_splits = (int)n;
-    sp.split_len = (int)len;
-    sp.rows_total = (int)((long long)batch * n_q * H_q);
-    sp.part_o_bytes = (size_t)n * sp.rows_total * nf::kHeadDim * sizeof(float);
-    sp.part_lse_bytes = ((size_t)n * sp.rows_total * sizeof(float) + 255) / 256 * 256;
+    const long long rows = (long long)(H_q / H_kv) * n_q;
+    if (rows > nf::kMaxRows) return false;
+    pl.rows = (int)rows;
+    pl.nt = rows <= 8 ? 1 : 2;
+    pl.n_rg = pl.nt == 1 ? 1 : (int)((rows + 15) / 16);
+    if (pl.n_rg == 3) pl.n_rg = 4;  // 8 consumer warps split evenly over 1, 2 or 4 row groups
+    pl.ctas = num_sms;
+    pl.segments = batch * H_kv;
+    pl.ticket_bytes = ((size_t)pl.segments * 4 + 255) / 256 * 256;
+    pl.slot_floats = (pl.rows * (nf::kHeadDim + 1) + 3) / 4 * 4;
+    pl.partial_bytes = ((size_t)(pl.ctas + pl.segments) * pl.slot_floats * sizeof(float) + 255) / 256 * 256;
     return true;
 }
 
@@ -102,19 +93,28 @@ int current_sm_count() {
 }
 
 template <int NT, bool QF32, int FMT>
-void launch_decode(const nf::DecodeParams &p, dim3 grid, cudaStream_t s) {
-    nf::decode_split_kernel<NT, QF32, FMT><<<grid, nf::kDecodeWarps * 32, 0, s>>>(p);
+cudaError_t launch_decode(const nf::DecodeParams &p, int ctas, cudaStream_t s) {
+    constexpr int smem = nf::DecodeSmem<NT, FMT>::kBytes;
+    // opt in to the large dynamic shared memory, once per device
+    static std::atomic<uint64_t> opted{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+    if (!bit || !(opted.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(nf::decode_kernel<NT, QF32, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        opted.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    nf::decode_kernel<NT, QF32, FMT><<<ctas, nf::kDecodeThreads, smem, s>>>(p);
+    return cudaSuccess;
 }
 
 template <int NT>
-void dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, dim3 grid, cudaStream_t s) {
-    if (fmt == NF_KV_K8V4) {
-        if (qf32) launch_decode<NT, true, NF_KV_K8V4>(p, grid, s);
-        else launch_decode<NT, false, NF_KV_K8V4>(p, grid, s);
-    } else {
-        if (qf32) launch_decode<NT, true, NF_KV_BF16>(p, grid, s);
-        else launch_decode<NT, false, NF_KV_BF16>(p, grid, s);
-    }
+cudaError_t dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, int ctas, cudaStream_t s) {
+    if (fmt == NF_KV_K8V4)
+        return qf32 ? launch_decode<NT, true, NF_KV_K8V4>(p, ctas, s) : launch_decode<NT, false, NF_KV_K8V4>(p, ctas, s);
+    return qf32 ? launch_decode<NT, true, NF_KV_BF16>(p, ctas, s) : launch_decode<NT, false, NF_KV_BF16>(p, ctas, s);
 }
 
 nf_status launch_combine(const float *part_o, const float *part_lse, int n_splits, int rows,
@@ -202,9 +202,9 @@ nf_status nf_kv_append_quant(const nf_kv_layer *kv, const void *k_new, const voi
 
 size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_heads,
                                      int32_t num_kv_heads, int32_t max_seqlen, int32_t num_sms) {
-    SplitPlan sp;
-    if (!make_plan(batch, n_q, num_q_heads, num_kv_heads, max_seqlen, num_sms, sp)) return 0;
-    return sp.bytes();
+    Plan pl;
+    if (!make_plan(batch, n_q, num_q_heads, num_kv_heads, max_seqlen, num_sms, pl)) return 0;
+    return pl.bytes();
 }
 
 nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
@@ -235,13 +235,14 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
         return fail(NF_ERR_INVALID_ARG, "q / out misaligned");
     const int sms = current_sm_count();
     if (sms < 1) return fail(NF_ERR_CUDA, "cannot query the current device");
-    SplitPlan sp;
-    if (!make_plan(batch, n_q, num_q_heads, kv->num_kv_heads, max_seqlen, sms, sp))
-        return fail(NF_ERR_INVALID_ARG, "unsupported shape (n_q * group too large?)");
-    if (workspace_bytes < sp.bytes() || (!workspace && sp.bytes() > 0))
-        return fail(NF_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, sp.bytes());
-    if (reinterpret_cast<uintptr_t>(workspace) & 15)
-        return fail(NF_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    Plan pl;
+    if (!make_plan(batch, n_q, num_q_heads, kv->num_kv_heads, max_seqlen, sms, pl))
+        return fail(NF_ERR_UNSUPPORTED, "unsupported shape (batch <= %d and group * n_q <= %d)", nf::kMaxBatch,
+                    nf::kMaxRows);
+    if (workspace_bytes < pl.bytes() || !workspace)
+        return fail(NF_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, pl.bytes());
+    if (reinterpret_cast<uintptr_t>(workspace) & 255)
+        return fail(NF_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
 
     nf::DecodeParams p{};
     p.k_codes = kv->k_codes;
@@ -255,27 +256,25 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
     p.n_q = n_q;
     p.num_q_heads = num_q_heads;
     p.group = num_q_heads / kv->num_kv_heads;
-    p.rows_per_head = p.group * n_q;
+    p.rows = pl.rows;
+    p.n_rg = pl.n_rg;
     p.block_table = block_table;
     p.max_blocks = max_blocks;
     p.seqlens = seqlens;
     p.max_seqlen = max_seqlen;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.causal = causal != 0;
-    p.split_len = sp.split_len;
-    p.n_splits = sp.n_splits;
-    p.n_row_groups = sp.n_row_groups;
-    p.part_o = static_cast<float *>(workspace);
-    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + sp.part_o_bytes);
-    p.rows_total = sp.rows_total;
+    p.out = out;
+    p.out_lse = out_lse;
+    p.tickets = static_cast<int32_t *>(workspace);
+    p.partials = reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.ticket_bytes);
+    p.slot_floats = pl.slot_floats;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const dim3 grid((unsigned)(sp.n_splits * sp.n_row_groups), (unsigned)kv->num_kv_heads, (unsigned)batch);
-    if (sp.nt == 1) dispatch_decode<1>(p, q_dtype == NF_F32, kv->fmt, grid, s);
-    else dispatch_decode<2>(p, q_dtype == NF_F32, kv->fmt, grid, s);
-    st = after_launch("decode kernel launch");
-    if (st != NF_OK) return st;
-    return launch_combine(p.part_o, p.part_lse, sp.n_splits, sp.rows_total, nf::kHeadDim, out, out_lse, s);
+    const cudaError_t e = pl.nt == 1 ? dispatch_decode<1>(p, q_dtype == NF_F32, kv->fmt, pl.ctas, s)
+                                     : dispatch_decode<2>(p, q_dtype == NF_F32, kv->fmt, pl.ctas, s);
+    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "decode kernel set-up: %s", cudaGetErrorString(e));
+    return after_launch("decode kernel launch");
 }
 
 nf_status nf_decode_attn_noalloc(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
@@ -283,17 +282,25 @@ nf_status nf_decode_attn_noalloc(const nf_kv_layer *kv, const void *q, int32_t q
                                  int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
                                  float softmax_scale, int32_t causal, float *out, float *out_lse,
                                  nf_stream_t stream) {
+    size_t tickets = 0;
     if (kv && kv->num_kv_heads > 0) {
         const int sms = current_sm_count();
-        SplitPlan sp;
-        if (sms > 0 && make_plan(batch, n_q, num_q_heads, kv->num_kv_heads, max_seqlen, sms, sp) &&
-            sp.bytes() > NF_NOALLOC_SCRATCH_BYTES)
-            return fail(NF_ERR_WORKSPACE, "shape needs %zu bytes of scratch, above the %zu-byte no-alloc maximum",
-                        sp.bytes(), (size_t)NF_NOALLOC_SCRATCH_BYTES);
+        Plan pl;
+        if (sms > 0 && make_plan(batch, n_q, num_q_heads, kv->num_kv_heads, max_seqlen, sms, pl)) {
+            if (pl.bytes() > NF_NOALLOC_SCRATCH_BYTES)
+                return fail(NF_ERR_WORKSPACE, "shape needs %zu bytes of scratch, above the %zu-byte no-alloc maximum",
+                            pl.bytes(), (size_t)NF_NOALLOC_SCRATCH_BYTES);
+            tickets = pl.ticket_bytes;
+        }
     }
     void *scratch = nullptr;
     const nf_status st = noalloc_scratch(&scratch);
     if (st != NF_OK) return st;
+    // the ticket counters must start at zero; the array keeps the last call's bytes
+    if (tickets) {
+        const cudaError_t e = cudaMemsetAsync(scratch, 0, tickets, reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return fail(NF_ERR_CUDA, "clearing the no-alloc tickets: %s", cudaGetErrorString(e));
+    }
     return nf_decode_attn(kv, q, q_dtype, batch, n_q, num_q_heads, block_table, max_blocks, seqlens,
                           max_seqlen, softmax_scale, causal, out, out_lse, scratch,
                           NF_NOALLOC_SCRATCH_BYTES, stream);

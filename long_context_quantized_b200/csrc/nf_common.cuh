@@ -64,6 +64,62 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     return y;
 }
 
+// ---------------------------------------------------------------- mbarrier / TMA
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Wait for the phase of `bar` with the given parity to complete, for at most
+// kWaitLimitNs.  Returns false on timeout (the caller records the error).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+// 1-D bulk copy global -> shared on the TMA engine, completing on `bar`
+// (16-byte aligned addresses, size a multiple of 16).  No multicast.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+// Named barrier among `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
+
 // Read-only 16-byte global load.
 __device__ __forceinline__ uint4 ldg16(const void *p) {
     return __ldg(reinterpret_cast<const uint4 *>(p));
@@ -86,12 +142,19 @@ __device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t &lo, uint32_t &
 // (apply to w >> 8 for (n2, n6) and (n3, n7)).  The sign bit is flipped to get
 // u = c + 8; u sits under the exponent of 1024 (or 1024 * 16 for the odd
 // nibble) and the bias is removed exactly.
+// One lop3 does the sign flip, the mask and the exponent insertion: where mask
+// bit b is set the result is w ^ c, elsewhere c (truth table 0x6a).
+__device__ __forceinline__ uint32_t lop3_sel_xor(uint32_t w, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(d) : "r"(w), "r"(b), "r"(c));
+    return d;
+}
 __device__ __forceinline__ __half2 nib_even(uint32_t w) {
-    const uint32_t x = ((w ^ 0x88888888u) & 0x000F000Fu) | 0x64006400u;  // 1024 + u
+    const uint32_t x = lop3_sel_xor(w, 0x000F000Fu, 0x64086408u);      // 1024 + u
     return __hsub2(u32_h2(x), u32_h2(0x64086408u));                      // - 1032
 }
 __device__ __forceinline__ __half2 nib_odd(uint32_t w) {
-    const uint32_t x = ((w ^ 0x88888888u) & 0x00F000F0u) | 0x64006400u;  // 1024 + 16u
+    const uint32_t x = lop3_sel_xor(w, 0x00F000F0u, 0x64806480u);      // 1024 + 16u
     return __hfma2(u32_h2(x), u32_h2(0x2C002C00u), u32_h2(0xD480D480u)); // /16 - 72
 }
 

@@ -1,38 +1,81 @@
-// nf_decode.cuh -- split-K decode attention over the segmented K8/V4 (or bf16)
-// pool.
+// nf_decode.cuh -- persistent split-K decode attention over the segmented
+// K8/V4 (or bf16) KV pool, with the log-sum-exp combine fused in.
 //
-// Work unit: one CTA per (sequence b, kv-head h, context split, row group).
-// The GQA group's G * n_q query rows of kv-head h are served by the same CTA,
-// so each key/value byte of the split is fetched once for all of them (page
-// "標籤: vLLM", section 2: stream one KV segment at a time, decode tuned for a
-// single long request).  A row group is 16 query rows; wider groups (n_q * G >
-// 16, MTP verification) run one CTA per 16 rows over the same split, launched
-// next to each other so the second read of the split is served by L2.
+// The pages' engine streams the KV cache one segment at a time through the SM
+// and tunes decode for a single long request (page "標籤: vLLM", section 2
+// "C++/CUDA 層的 kernel fusion 與 KV cache 策略"); decode is HBM-bound and
+// KV bytes per token drive it (page "3090 单卡跑 Qwen3.8-27B：NInfer 上机实测",
+// section 二 and its replies).  The B200 form of that idea:
 //
-// Inside a CTA each warp takes 16-token tiles of the split in turn and keeps
-// its own online-softmax state; the warps are merged at the end and the CTA
-// writes one (o, lse) partial per row for nf_attn_combine.
-//
-// Tensor-core mapping (mma.sync m16n8k16, "swap AB" so that the 16-token tile
-// is the M dimension and the query rows are N = 8):
-//   S^T[token][row] = K_codes[token][ch] . Q^T[ch][row]   (fp16, exact codes)
-//     lane (g, t) reads bytes 32t..32t+31 of tokens g and g+8, which it feeds
-//     to the 8 k-steps; q is permuted the same way once per CTA.
-//   O^T[ch][row] += V_hat^T[ch][token] . P^T[token][row]  (fp16, fp32 acc)
-//     lane (g, t) reads the 32 channels of V group t for tokens g and g+8,
-//     converts them to fp16 and scales them, and movmatrix transposes them
-//     into the A fragments; P^T comes from the S^T accumulator layout through
-//     movmatrix as well.
-// The K scale is per token and multiplies the rows of S^T after the MMA.
+// Work: every (sequence b, kv-head h) is a segment of ceil(L_b / 32) chunks of
+//   32 keys; the chunks of all segments form one list of W chunks that the
+//   persistent grid (one CTA per SM, at most W CTAs) cuts into equal
+//   contiguous ranges, read from the device-side lengths -- ragged batches
+//   balance by keys, with no host read of the lengths.  A CTA's range covers
+//   pieces of one or more segments; all G * n_q query rows of a kv-head
+//   (GQA group x MTP queries) are served by the CTA that streams the keys, so
+//   each byte is fetched from HBM once.
+// Pipeline: a producer warp cuts each piece into stages of up to 256 keys
+//   (64 for the bf16 cache) inside one 256-key block and moves each stage's K
+//   codes, V nibbles, K scales and V scales into a ring of shared-memory
+//   buffers with 1-D bulk copies on the TMA engine, completing on an mbarrier.
+//   Stages are large because a ring buffer turns over at a roughly fixed rate
+//   per SM (about 2.7 stages per microsecond measured on B200): bandwidth is
+//   stage bytes x that rate, so 32-52 KB stages keep it above the HBM rate.
+//   All consumer warps work on every stage -- each takes units of 32 keys (16
+//   for bf16) -- and release it on an "empty" mbarrier, so stages retire in
+//   order.
+// Math per 16-key m-tile (mma.sync m16n8k16, "swap AB": keys are M, query rows
+//   N = 8): S^T = K_codes . Q^T with int8 codes -> fp16 exactly and the K scale
+//   per key applied to the rows of S^T; O^T += V_hat^T . P^T with nibbles ->
+//   fp16 exactly, times the fp16 V scale of (key, 32-channel group), and
+//   movmatrix transposing V and P into fragment layout.  The running max of a
+//   row is only raised (and O rescaled) when a tile's max exceeds it by more
+//   than 2^8; the cross-lane max is only reduced when some lane asks for that.
+// Merge: at the end of each piece the consumer warps merge through shared
+//   memory.  A segment owned by one CTA is written straight to out; otherwise
+//   each piece writes an (o, lse) partial and takes a ticket of the segment's
+//   counter; the CTA with the last ticket merges the partials into out and
+//   resets the counter (no CTA ever waits for another).
+// Every mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT
+// and the kernel runs to its end without further waits.
 #pragma once
 
 #include "nf_common.cuh"
 
 namespace nf {
 
-constexpr int kDecodeWarps = 4;
-constexpr int kTile = 16;
-constexpr int kRowsPerCta = 16;
+constexpr int kChunk = 32;  // keys per unit of work balance
+constexpr int kConsumerWarps = 8;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxBatch = 256;
+constexpr int kMaxRows = 64;  // G * n_q per kv-head
+
+template <int FMT, int NT>
+struct Stage;
+template <int NT>
+struct Stage<NF_KV_K8V4, NT> {
+    static constexpr int kTok = 256;                  // keys per stage: one block
+    static constexpr int kK = 0;                      // int8  [kTok][128]
+    static constexpr int kV = kTok * 128;             // uint8 [kTok][64]
+    static constexpr int kKs = kV + kTok * 64;        // fp16  [kTok]
+    static constexpr int kVs = kKs + kTok * 2;        // fp16  [kTok][4]
+    static constexpr int kBytesPerTok = 202;
+    static constexpr int kStride = kTok * kBytesPerTok;  // 51712, a 128-byte multiple
+    static constexpr int kStages = 3;
+    static constexpr int kUnitTiles = 2;              // 16-key m-tiles per consumer work unit
+};
+template <int NT>
+struct Stage<NF_KV_BF16, NT> {
+    static constexpr int kTok = 64;
+    static constexpr int kK = 0;                      // bf16 [kTok][128]
+    static constexpr int kV = kTok * 256;             // bf16 [kTok][128]
+    static constexpr int kKs = 0, kVs = 0;
+    static constexpr int kBytesPerTok = 512;
+    static constexpr int kStride = kTok * kBytesPerTok;
+    static constexpr int kStages = 4;
+    static constexpr int kUnitTiles = 1;
+};
 
 struct DecodeParams {
     const void *k_codes;
@@ -41,324 +84,687 @@ struct DecodeParams {
     const __half *v_scales;
     int num_blocks, num_kv_heads;
     const void *q;
-    int batch, n_q, num_q_heads, group, rows_per_head;  // rows_per_head = group * n_q
+    int batch, n_q, num_q_heads, group, rows;  // rows = group * n_q per kv-head
+    int n_rg;                                  // row groups (of 8 * NT rows)
     const int32_t *block_table;
     int max_blocks;
     const int32_t *seqlens;
     int max_seqlen;
     float scale_log2;  // softmax_scale * log2(e)
     int causal;
-    int split_len, n_splits, n_row_groups;
-    float *part_o;    // [n_splits][rows_total][128]
-    float *part_lse;  // [n_splits][rows_total]
-    int rows_total;
+    float *out;      // [batch][n_q][H_q][128]
+    float *out_lse;  // [batch][n_q][H_q] or null
+    int32_t *tickets;  // [batch * H_kv], zero between calls
+    float *partials;   // [gridDim.x + batch * H_kv] slots of slot_floats
+    int slot_floats;   // rows * 128 (o) + rows (lse), rounded up to 4 floats
 };
 
-// Output channel held by row `rho` (0..15) of PV m-tile `m`, for the K8/V4
-// V layout (lane t converts channels 32t..32t+31, pairing nibbles k and k+4).
+template <int NT, int FMT>
+struct DecodeSmem {
+    static constexpr int NR = NT * 8;
+    using ST = Stage<FMT, NT>;
+    static constexpr int kStagesBytes = ST::kStages * ST::kStride;
+    static constexpr int kMergeO = kStagesBytes;                               // float [8][NR][132]
+    static constexpr int kMergeM = kMergeO + kConsumerWarps * NR * 132 * 4;    // float [8][NR]
+    static constexpr int kMergeL = kMergeM + kConsumerWarps * NR * 4;          // float [8][NR]
+    static constexpr int kBars = kMergeL + kConsumerWarps * NR * 4;            // u64 [2][stages]
+    static constexpr int kStageOk = kBars + 2 * ST::kStages * 8;               // int [stages]
+    static constexpr int kSeqC = kStageOk + ST::kStages * 4;                   // int [kMaxBatch]
+    static constexpr int kSeqBase = (kSeqC + kMaxBatch * 4 + 7) / 8 * 8;       // i64 [kMaxBatch + 1]
+    static constexpr int kMisc = kSeqBase + (kMaxBatch + 1) * 8;              // int [4]
+    static constexpr int kBytes = kMisc + 16;
+    static_assert(kBytes <= 232448, "shared memory per CTA");
+    static_assert(ST::kStride % 128 == 0, "stage alignment");
+};
+
+// Output channel of row `rho` (0..15) of PV m-tile `m` (K8/V4: lane t converts
+// channels 32t..32t+31 of V, pairing nibbles k and k + 4 of each word).
 __device__ __forceinline__ int v_channel_k8v4(int m, int rho) {
     const int p = 2 * m + (rho >> 3), jj = rho & 7;
     return 32 * (jj >> 1) + 8 * (p >> 2) + (p & 3) + 4 * (jj & 1);
 }
-// Same for the bf16 cache (lane t holds channel pairs 32t + 2p, 32t + 2p + 1).
+// bf16 cache: lane t's u-th 16-byte load holds channels 32u + 8t .. 32u + 8t + 7.
 __device__ __forceinline__ int v_channel_bf16(int m, int rho) {
     const int p = 2 * m + (rho >> 3), jj = rho & 7;
-    return 32 * (jj >> 1) + 2 * p + (jj & 1);
+    return 32 * (p >> 2) + 8 * (jj >> 1) + 2 * (p & 3) + (jj & 1);
+}
+// Physical K channel of element e (0..3) of k-step ks for lane t.
+__device__ __forceinline__ int k_channel(int fmt, int ks, int t, int e) {
+    return fmt == NF_KV_K8V4 ? 32 * t + 4 * ks + e : 32 * (ks >> 1) + 8 * t + 4 * (ks & 1) + e;
+}
+
+// Walks a CTA's chunk range piece by piece (a piece = the part of one segment
+// that falls in the range).  Producer and consumers walk it identically.
+struct PieceWalker {
+    const int *C;              // chunks per sequence
+    const long long *base;     // first chunk of sequence b's segments
+    int H, batch;
+    long long x, end;          // next chunk, end of the CTA range
+    int b = 0;
+    // current piece
+    int pb, ph;                // sequence, kv-head
+    long long s0, xs, xe;      // segment start chunk, piece [xs, xe)
+    __device__ bool next() {
+        if (x >= end) return false;
+        while (b + 1 <= batch && base[b + 1] <= x) ++b;
+        pb = b;
+        ph = (int)((x - base[b]) / C[b]);
+        s0 = base[b] + (long long)ph * C[b];
+        xs = x;
+        xe = min(s0 + C[b], end);
+        x = xe;
+        return true;
+    }
+};
+
+// End (exclusive, in chunks of the segment) of the stage that starts at chunk
+// cx: at most kTok keys, never crossing a 256-key block.
+template <int FMT, int NT>
+__device__ __forceinline__ int stage_end(int cx, int cx_end) {
+    constexpr int per_blk = kBlock / kChunk, per_stage = Stage<FMT, NT>::kTok / kChunk;
+    return min(cx_end, min((cx / per_blk + 1) * per_blk, cx + per_stage));
+}
+
+__device__ __forceinline__ int owner_cta(long long x, long long W, int P) {
+    return (int)(((x + 1) * P - 1) / W);
 }
 
 template <int NT, bool QF32, int FMT>
-__global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
+    using ST = Stage<FMT, NT>;
+    using SM = DecodeSmem<NT, FMT>;
+    constexpr int MT = ST::kUnitTiles;
     constexpr bool K8 = (FMT == NF_KV_K8V4);
-    constexpr int NR = NT * 8;  // rows held by this CTA
-    __shared__ float sm_m[kDecodeWarps][NR];
-    __shared__ float sm_l[kDecodeWarps][NR];
-    __shared__ float sm_o[kDecodeWarps][NR][kHeadDim + 4];
+    constexpr int NS = ST::kStages;
+    constexpr int NR = SM::NR;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    float *sm_o = reinterpret_cast<float *>(smem + SM::kMergeO);
+    float *sm_m = reinterpret_cast<float *>(smem + SM::kMergeM);
+    float *sm_l = reinterpret_cast<float *>(smem + SM::kMergeL);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::kBars);
+    uint64_t *empty = full + NS;
+    volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + SM::kStageOk);
+    int *seqC = reinterpret_cast<int *>(smem + SM::kSeqC);
+    long long *seqBase = reinterpret_cast<long long *>(smem + SM::kSeqBase);
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + SM::kMisc);  // [0] abort, [1] last-ticket
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int b = blockIdx.z, h = blockIdx.y;
-    const int split = blockIdx.x / p.n_row_groups, rg = blockIdx.x % p.n_row_groups;
-    const int row0 = rg * kRowsPerCta;
+    const int H = p.num_kv_heads;
 
-    int L = p.seqlens[b];
-    if (L < p.n_q || L > p.max_seqlen) {
-        if (threadIdx.x == 0 && split == 0 && rg == 0 && h == 0) report(NF_DEVERR_SEQLEN);
-        L = 0;
+    // ---- set-up: barriers and the chunk list (every CTA computes the same)
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kConsumerWarps);
+            stage_ok[i] = 0;
+        }
+        misc[0] = 0;
+        misc[1] = 0;
+        fence_mbar_init();
     }
-    const int t0 = split * p.split_len;
-    const int t1 = min(t0 + p.split_len, L);
+    if (warp == 0) {
+        for (int b = lane; b < p.batch; b += 32) {
+            const int L = p.seqlens[b];
+            const bool ok = L >= p.n_q && L <= p.max_seqlen;
+            if (!ok && blockIdx.x == 0) report(NF_DEVERR_SEQLEN);
+            seqC[b] = ok ? (L + kChunk - 1) / kChunk : 0;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            long long acc = 0;
+            for (int b = 0; b < p.batch; ++b) {
+                seqBase[b] = acc;
+                acc += (long long)seqC[b] * H;
+            }
+            seqBase[p.batch] = acc;
+        }
+    }
+    __syncthreads();
+    const long long W = seqBase[p.batch];
+    // CTAs taking part: never more than there are chunks, so that every CTA
+    // between a segment's first and last owner holds a piece of it
+    const int P = (int)(W < (long long)gridDim.x ? W : (long long)gridDim.x);
+    const long long c_begin = (int)blockIdx.x < P ? W * blockIdx.x / P : 0;
+    const long long c_end = (int)blockIdx.x < P ? W * (blockIdx.x + 1) / P : 0;
 
-    // ---- query fragments (B operand of S^T = K . Q^T), permuted like the K bytes
+    // segments of sequences with no valid key: o = 0, lse = -inf
+    for (int s = blockIdx.x; s < p.batch * H; s += gridDim.x) {
+        const int b = s / H, h = s % H;
+        if (seqC[b] != 0) continue;
+        for (int idx = threadIdx.x; idx < p.rows * kHeadDim; idx += blockDim.x) {
+            const int r = idx / kHeadDim, ch = idx % kHeadDim;
+            const int j = r / p.group, gq = r % p.group;
+            const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+            p.out[row * kHeadDim + ch] = 0.f;
+            if (ch == 0 && p.out_lse) p.out_lse[row] = -INFINITY;
+        }
+    }
+
+    PieceWalker walk{seqC, seqBase, H, p.batch, c_begin, c_end};
+
+    // =================================================================== producer
+    // The whole warp walks the stages; its lanes hold a window of 32 block-table
+    // entries (one global load per 32 blocks), lane 0 waits for free buffers
+    // and issues the bulk copies.
+    if (warp == kConsumerWarps) {
+        uint32_t kst = 0;  // CTA-wide stage counter
+        bool stop = false;
+        while (!stop && walk.next()) {
+            const int32_t *bt = p.block_table + (size_t)walk.pb * p.max_blocks;
+            const int nblk = (seqC[walk.pb] * kChunk + kBlock - 1) / kBlock;
+            int win = -1000000, my_blk = 0;
+            const int cx1 = (int)(walk.xe - walk.s0);
+            for (int cx = (int)(walk.xs - walk.s0); cx < cx1; ++kst) {
+                const int ce = stage_end<FMT, NT>(cx, cx1);
+                const int tok0 = cx * kChunk, ntok = (ce - cx) * kChunk;
+                cx = ce;
+                const int bi = tok0 >> 8;
+                if (bi >= win + 32) {  // warp-uniform refill of the window
+                    win = bi;
+                    my_blk = win + lane < nblk ? bt[win + lane] : -1;
+                }
+                const int blk = __shfl_sync(0xffffffffu, my_blk, bi - win);
+                if (lane == 0) {
+                    const int stage = (int)(kst % NS);
+                    const uint32_t round = kst / NS;
+                    if (!misc[0] && !mbar_wait(&empty[stage], (round & 1) ^ 1)) {
+                        report(NF_DEVERR_TIMEOUT);
+                        misc[0] = 1;
+                    }
+                    if (!misc[0]) {
+                        unsigned char *st = smem + stage * ST::kStride;
+                        if (blk < 0 || blk >= p.num_blocks) {
+                            report(NF_DEVERR_BLOCK_ID);
+                            stage_ok[stage] = 0;
+                            mbar_arrive(&full[stage]);
+                        } else {
+                            stage_ok[stage] = 1;
+                            const size_t si = ((size_t)blk * H + walk.ph) * kBlock + (tok0 & (kBlock - 1));
+                            mbar_arrive_expect_tx(&full[stage], (uint32_t)(ntok * ST::kBytesPerTok));
+                            if (K8) {
+                                bulk_g2s(st + ST::kK, static_cast<const int8_t *>(p.k_codes) + si * 128, ntok * 128, &full[stage]);
+                                bulk_g2s(st + ST::kV, static_cast<const uint8_t *>(p.v_codes) + si * 64, ntok * 64, &full[stage]);
+                                bulk_g2s(st + ST::kKs, p.k_scales + si, ntok * 2, &full[stage]);
+                                bulk_g2s(st + ST::kVs, p.v_scales + si * 4, ntok * 8, &full[stage]);
+                            } else {
+                                bulk_g2s(st + ST::kK, static_cast<const __nv_bfloat16 *>(p.k_codes) + si * 128, ntok * 256, &full[stage]);
+                                bulk_g2s(st + ST::kV, static_cast<const __nv_bfloat16 *>(p.v_codes) + si * 128, ntok * 256, &full[stage]);
+                            }
+                        }
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, misc[0], 0)) {
+                    stop = true;
+                    break;
+                }
+            }
+        }
+        if (lane == 0) {
+            // before leaving, make sure no copy into this CTA's shared memory is
+            // still in flight: wait for the buffers of the last round issued
+            const uint32_t issued = kst;
+            for (uint32_t kk = issued > (uint32_t)NS ? issued - NS : 0; kk < issued && !misc[0]; ++kk)
+                if (!mbar_wait(&full[kk % NS], (kk / NS) & 1)) {
+                    report(NF_DEVERR_TIMEOUT);
+                    misc[0] = 1;
+                }
+        }
+        return;  // the merge barriers below are among the consumer warps only
+    }
+
+    // =================================================================== consumers
+    const int CW = kConsumerWarps / p.n_rg;  // warps per row group
+    const int rg = warp / CW, slot = warp % CW;
+    const int g = lane >> 2, t = lane & 3;
+    const int row0 = rg * NR;
+
     uint32_t qf[NT][8][2];
     uint32_t ql[QF32 ? NT : 1][8][2];
-    int lim[NT][2];  // last visible key position for rows 8nt+2t+e (-1: row unused)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int r = row0 + nt * 8 + g;
-        const bool rv = r < p.rows_per_head;
-        const int j = rv ? r / p.group : 0, gq = rv ? r % p.group : 0;
-        const size_t qoff = (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const int c = 32 * t + 4 * ks;
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-            if (rv) {
-                if (QF32) {
-                    const float4 v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qoff + c);
-                    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-                } else {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.q) + qoff + c);
-                    x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-                    x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
-                }
-            }
-            if (K8) {
-                qf[nt][ks][0] = pack_f16(x[0], x[1]);
-                qf[nt][ks][1] = pack_f16(x[2], x[3]);
-                if (QF32) {
-                    const float2 h0 = __half22float2(u32_h2(qf[nt][ks][0]));
-                    const float2 h1 = __half22float2(u32_h2(qf[nt][ks][1]));
-                    ql[nt][ks][0] = pack_f16(x[0] - h0.x, x[1] - h0.y);
-                    ql[nt][ks][1] = pack_f16(x[2] - h1.x, x[3] - h1.y);
-                }
-            } else {
-                qf[nt][ks][0] = pack_bf16(x[0], x[1]);
-                qf[nt][ks][1] = pack_bf16(x[2], x[3]);
-                if (QF32) {
-                    const float lo0 = x[0] - __uint_as_float(qf[nt][ks][0] << 16);
-                    const float lo1 = x[1] - __uint_as_float(qf[nt][ks][0] & 0xFFFF0000u);
-                    const float lo2 = x[2] - __uint_as_float(qf[nt][ks][1] << 16);
-                    const float lo3 = x[3] - __uint_as_float(qf[nt][ks][1] & 0xFFFF0000u);
-                    ql[nt][ks][0] = pack_bf16(lo0, lo1);
-                    ql[nt][ks][1] = pack_bf16(lo2, lo3);
-                }
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int rr = row0 + nt * 8 + 2 * t + e;
-            if (rr >= p.rows_per_head) lim[nt][e] = -1;
-            else lim[nt][e] = p.causal ? (L - p.n_q + rr / p.group) : (L - 1);
-        }
-    }
-
     float m_run[NT][2], l_run[NT][2];
     float acc[8][NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        m_run[nt][0] = m_run[nt][1] = -INFINITY;
-        l_run[nt][0] = l_run[nt][1] = 0.f;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) acc[m][nt][0] = acc[m][nt][1] = acc[m][nt][2] = acc[m][nt][3] = 0.f;
-    }
+    int lim[NT][2];
 
-    const int ntiles = t1 > t0 ? (t1 - t0 + kTile - 1) / kTile : 0;
-    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks;
-
-    for (int tile = warp; tile < ntiles; tile += kDecodeWarps) {
-        const int tb = t0 + tile * kTile;
-        const int blk = bt[tb >> 8];
-        if (blk < 0 || blk >= p.num_blocks) {
-            if (lane == 0) report(NF_DEVERR_BLOCK_ID);
-            continue;
-        }
-        const size_t si = ((size_t)blk * p.num_kv_heads + h) * kBlock + (tb & (kBlock - 1));
-        const bool vg0 = tb + g < L, vg1 = tb + g + 8 < L;
-
-        // ---- loads for tokens g and g + 8
-        uint4 kq[2][K8 ? 2 : 4];
-        uint4 vq[2][K8 ? 1 : 4];
-        float sk[2];
-        uint32_t sv[2];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const size_t s = si + g + 8 * hh;
-            if (K8) {
-                const int8_t *kp = static_cast<const int8_t *>(p.k_codes) + s * kHeadDim + 32 * t;
-                kq[hh][0] = ldg16(kp);
-                kq[hh][1] = ldg16(kp + 16);
-                vq[hh][0] = ldg16(static_cast<const uint8_t *>(p.v_codes) + s * (kHeadDim / 2) + 16 * t);
-                sk[hh] = __half2float(p.k_scales[s]);
-                const __half vs = p.v_scales[s * (kHeadDim / kVGroup) + t];
-                sv[hh] = h2_u32(__half2half2(vs));
-            } else {
-                const __nv_bfloat16 *kp = static_cast<const __nv_bfloat16 *>(p.k_codes) + s * kHeadDim + 32 * t;
-                const __nv_bfloat16 *vp = static_cast<const __nv_bfloat16 *>(p.v_codes) + s * kHeadDim + 32 * t;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    kq[hh][u] = ldg16(kp + 8 * u);
-                    vq[hh][u] = ldg16(vp + 8 * u);
-                }
-                sk[hh] = 1.0f;
-            }
-        }
-        // keys past the end of the sequence: their slots hold stale bytes, so
-        // their values are zeroed (not just their weights)
-        if (K8) {
-            if (!vg0) sv[0] = 0u;
-            if (!vg1) sv[1] = 0u;
-        } else {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (!vg0) vq[0][u] = make_uint4(0, 0, 0, 0);
-                if (!vg1) vq[1][u] = make_uint4(0, 0, 0, 0);
-            }
-        }
-
-        // ---- S^T = K . Q^T
-        float s[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            if (K8) {
-                const uint32_t w0 = reinterpret_cast<const uint32_t *>(&kq[0][ks >> 2])[ks & 3];
-                const uint32_t w1 = reinterpret_cast<const uint32_t *>(&kq[1][ks >> 2])[ks & 3];
-                i8x4_to_f16(w0, a0, a2);
-                i8x4_to_f16(w1, a1, a3);
-            } else {
-                // 4 bf16 channels 32t + 4ks .. +3: words 2ks, 2ks+1 of the 32-channel run
-                const uint32_t *k0 = reinterpret_cast<const uint32_t *>(&kq[0][0]);
-                const uint32_t *k1 = reinterpret_cast<const uint32_t *>(&kq[1][0]);
-                a0 = k0[2 * ks]; a2 = k0[2 * ks + 1];
-                a1 = k1[2 * ks]; a3 = k1[2 * ks + 1];
-            }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                if (K8) {
-                    mma_f16(s[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
-                    if (QF32) mma_f16(s[nt], a0, a1, a2, a3, ql[nt][ks][0], ql[nt][ks][1]);
-                } else {
-                    mma_bf16(s[nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
-                    if (QF32) mma_bf16(s[nt], a0, a1, a2, a3, ql[nt][ks][0], ql[nt][ks][1]);
-                }
-            }
-        }
-
-        // ---- online softmax (log2 domain); rows 8nt + 2t + e, tokens g and g + 8
-        uint32_t pb0[NT], pb1[NT], pb0l[NT], pb1l[NT];
-        const float c0 = sk[0] * p.scale_log2, c1 = sk[1] * p.scale_log2;
-        const int pos0 = tb + g, pos1 = tb + g + 8;
+    uint32_t kst = 0;
+    while (walk.next()) {
+        const int b = walk.pb, h = walk.ph;
+        const int L = seqC[b] ? p.seqlens[b] : 0;
+        // query fragments of this (sequence, kv-head), permuted like the K channels
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            float pr[2][2];  // [token half][e]
+            const int r = row0 + nt * 8 + g;
+            const bool rv = r < p.rows;
+            const int j = rv ? r / p.group : 0, gq = rv ? r % p.group : 0;
+            const size_t qoff = (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                float x[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = k_channel(FMT, ks, t, e);
+                    if (!rv) x[e] = 0.f;
+                    else if (QF32) x[e] = static_cast<const float *>(p.q)[qoff + c];
+                    else x[e] = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[qoff + c]);
+                }
+                if (K8) {
+                    qf[nt][ks][0] = pack_f16(x[0], x[1]);
+                    qf[nt][ks][1] = pack_f16(x[2], x[3]);
+                    if (QF32) {
+                        const float2 h0 = __half22float2(u32_h2(qf[nt][ks][0]));
+                        const float2 h1 = __half22float2(u32_h2(qf[nt][ks][1]));
+                        ql[nt][ks][0] = pack_f16(x[0] - h0.x, x[1] - h0.y);
+                        ql[nt][ks][1] = pack_f16(x[2] - h1.x, x[3] - h1.y);
+                    }
+                } else {
+                    qf[nt][ks][0] = pack_bf16(x[0], x[1]);
+                    qf[nt][ks][1] = pack_bf16(x[2], x[3]);
+                    if (QF32) {
+                        ql[nt][ks][0] = pack_bf16(x[0] - __uint_as_float(qf[nt][ks][0] << 16),
+                                                  x[1] - __uint_as_float(qf[nt][ks][0] & 0xFFFF0000u));
+                        ql[nt][ks][1] = pack_bf16(x[2] - __uint_as_float(qf[nt][ks][1] << 16),
+                                                  x[3] - __uint_as_float(qf[nt][ks][1] & 0xFFFF0000u));
+                    }
+                }
+            }
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const float x0 = (vg0 && pos0 <= lim[nt][e]) ? s[nt][e] * c0 : -INFINITY;
-                const float x1 = (vg1 && pos1 <= lim[nt][e]) ? s[nt][2 + e] * c1 : -INFINITY;
-                float mx = fmaxf(x0, x1);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                const float m_new = fmaxf(m_run[nt][e], mx);
-                const float m_use = m_new == -INFINITY ? 0.f : m_new;
-                const float alpha = ex2(m_run[nt][e] - m_use);
-                m_run[nt][e] = m_new;
-                pr[0][e] = ex2(x0 - m_use);
-                pr[1][e] = ex2(x1 - m_use);
-                l_run[nt][e] = l_run[nt][e] * alpha + pr[0][e] + pr[1][e];
+                const int rr = row0 + nt * 8 + 2 * t + e;
+                lim[nt][e] = rr >= p.rows ? -1 : (p.causal ? L - p.n_q + rr / p.group : L - 1);
+                m_run[nt][e] = -INFINITY;
+                l_run[nt][e] = 0.f;
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc[m][nt][0] = acc[m][nt][1] = acc[m][nt][2] = acc[m][nt][3] = 0.f;
+        }
+        // keys every row of the group sees, for the no-mask fast path
+        const int all_see = p.causal ? L - p.n_q + 1 : L;
+
+        const int cx1 = (int)(walk.xe - walk.s0);
+        for (int cx = (int)(walk.xs - walk.s0); cx < cx1; ++kst) {
+            const int ce = stage_end<FMT, NT>(cx, cx1);
+            const int tok0 = cx * kChunk, n_mt = (ce - cx) * (kChunk / 16);
+            cx = ce;
+            const int stage = (int)(kst % NS);
+            if (!misc[0] && !mbar_wait(&full[stage], (kst / NS) & 1)) {
+                report(NF_DEVERR_TIMEOUT);
+                misc[0] = 1;
+            }
+            if (!misc[0] && stage_ok[stage]) {
+                const unsigned char *st = smem + stage * ST::kStride;
+                const int n_units = n_mt / MT;  // stages hold whole 32-key chunks
+                for (int un = slot; un < n_units; un += CW) {
+                    const int ubase = tok0 + 16 * MT * un;                // first key of the unit
+                    const bool fast = ubase + 16 * MT <= all_see;          // every row sees every key
+
+                    // ---- S^T = K . Q^T for the unit's MT m-tiles of 16 keys
+                    float s[MT][NT][4];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int tau0 = 16 * (MT * un + mt) + g;          // key of this lane in the stage
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
+                        if (K8) {
+                            const unsigned char *k0 = st + ST::kK + tau0 * 128 + 32 * t;
+                            const uint4 ka0 = lds128(k0), ka1 = lds128(k0 + 16);
+                            const uint4 kb0 = lds128(k0 + 8 * 128), kb1 = lds128(k0 + 8 * 128 + 16);
+                            const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
+                            const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+#pragma unroll
+                            for (int ks = 0; ks < 8; ++ks) {
+                                uint32_t a0, a1, a2, a3;
+                                i8x4_to_f16(wa[ks], a0, a2);
+                                i8x4_to_f16(wb[ks], a1, a3);
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    mma_f16(s[mt][nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+                                    if (QF32) mma_f16(s[mt][nt], a0, a1, a2, a3, ql[nt][ks][0], ql[nt][ks][1]);
+                                }
+                            }
+                        } else {
+                            const unsigned char *k0 = st + ST::kK + tau0 * 256 + 16 * t;
+                            uint32_t wa[16], wb[16];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const uint4 va = lds128(k0 + 64 * u), vb = lds128(k0 + 8 * 256 + 64 * u);
+                                wa[4 * u] = va.x; wa[4 * u + 1] = va.y; wa[4 * u + 2] = va.z; wa[4 * u + 3] = va.w;
+                                wb[4 * u] = vb.x; wb[4 * u + 1] = vb.y; wb[4 * u + 2] = vb.z; wb[4 * u + 3] = vb.w;
+                            }
+#pragma unroll
+                            for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    mma_bf16(s[mt][nt], wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
+                                             qf[nt][ks][0], qf[nt][ks][1]);
+                                    if (QF32)
+                                        mma_bf16(s[mt][nt], wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
+                                                 ql[nt][ks][0], ql[nt][ks][1]);
+                                }
+                            }
+                        }
+                    }
+
+                    // ---- scores in the log2 domain; rows 8nt + 2t + e, keys tau0 / tau0 + 8 of each m-tile
+                    float xv[MT][NT][4];
+                    bool kv_ok[MT][2];
+                    bool raise = false;
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int tau0 = 16 * (MT * un + mt) + g;
+                        const int pos0 = tok0 + tau0, pos1 = pos0 + 8;
+                        kv_ok[mt][0] = fast || pos0 < L;
+                        kv_ok[mt][1] = fast || pos1 < L;
+                        const float c0 = (K8 ? __half2float(reinterpret_cast<const __half *>(st + ST::kKs)[tau0]) : 1.0f) * p.scale_log2;
+                        const float c1 = (K8 ? __half2float(reinterpret_cast<const __half *>(st + ST::kKs)[tau0 + 8]) : 1.0f) * p.scale_log2;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                float x0 = s[mt][nt][e] * c0, x1 = s[mt][nt][2 + e] * c1;
+                                if (!fast) {
+                                    if (!(kv_ok[mt][0] && pos0 <= lim[nt][e])) x0 = -INFINITY;
+                                    if (!(kv_ok[mt][1] && pos1 <= lim[nt][e])) x1 = -INFINITY;
+                                }
+                                xv[mt][nt][e] = x0;
+                                xv[mt][nt][2 + e] = x1;
+                            }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            float mx = fmaxf(xv[0][nt][e], xv[0][nt][2 + e]);
+#pragma unroll
+                            for (int mt = 1; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(xv[mt][nt][e], xv[mt][nt][2 + e]));
+                            raise |= mx > m_run[nt][e] + 8.0f;  // true when m_run is -inf and mx finite
+                        }
+                    if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                float mx = fmaxf(xv[0][nt][e], xv[0][nt][2 + e]);
+#pragma unroll
+                                for (int mt = 1; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(xv[mt][nt][e], xv[mt][nt][2 + e]));
+                                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                                const float m_new = fmaxf(m_run[nt][e], mx);
+                                const float alpha = m_new == -INFINITY ? 1.f : ex2(m_run[nt][e] - m_new);
+                                m_run[nt][e] = m_new;
+                                l_run[nt][e] *= alpha;
+#pragma unroll
+                                for (int m = 0; m < 8; ++m) {
+                                    acc[m][nt][e] *= alpha;
+                                    acc[m][nt][2 + e] *= alpha;
+                                }
+                            }
+                    }
+                    // weights (P^T) as B fragments of the PV product
+                    uint32_t pb[MT][NT][2], pbl[MT][NT][2];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const float mu0 = m_run[nt][0] == -INFINITY ? 0.f : m_run[nt][0];
+                        const float mu1 = m_run[nt][1] == -INFINITY ? 0.f : m_run[nt][1];
+#pragma unroll
+                        for (int mt = 0; mt < MT; ++mt) {
+                            const float p00 = ex2(xv[mt][nt][0] - mu0), p01 = ex2(xv[mt][nt][1] - mu1);
+                            const float p10 = ex2(xv[mt][nt][2] - mu0), p11 = ex2(xv[mt][nt][3] - mu1);
+                            l_run[nt][0] += p00 + p10;
+                            l_run[nt][1] += p01 + p11;
+                            if (K8) {
+                                pb[mt][nt][0] = movmatrix_t(pack_f16(p00, p01));
+                                pb[mt][nt][1] = movmatrix_t(pack_f16(p10, p11));
+                            } else {
+                                // bf16 weights split into hi + lo so they keep ~16 bits
+                                const uint32_t h0 = pack_bf16(p00, p01), h1 = pack_bf16(p10, p11);
+                                pb[mt][nt][0] = movmatrix_t(h0);
+                                pb[mt][nt][1] = movmatrix_t(h1);
+                                pbl[mt][nt][0] = movmatrix_t(pack_bf16(p00 - __uint_as_float(h0 << 16),
+                                                                       p01 - __uint_as_float(h0 & 0xFFFF0000u)));
+                                pbl[mt][nt][1] = movmatrix_t(pack_bf16(p10 - __uint_as_float(h1 << 16),
+                                                                       p11 - __uint_as_float(h1 & 0xFFFF0000u)));
+                            }
+                        }
+                    }
+
+                    // ---- O^T += V^T . P^T over 8 channel m-tiles, one 16-key k-tile per m-tile of the unit
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const int tau0 = 16 * (MT * un + mt) + g, tau1 = tau0 + 8;
+                        if (K8) {
+                            const uint4 v0 = lds128(st + ST::kV + tau0 * 64 + 16 * t);
+                            const uint4 v1 = lds128(st + ST::kV + tau1 * 64 + 16 * t);
+                            const __half *vs = reinterpret_cast<const __half *>(st + ST::kVs);
+                            // keys past the end hold stale bytes: zero their values, not just their weights
+                            const __half2 s0 = kv_ok[mt][0] ? __half2half2(vs[tau0 * 4 + t]) : __float2half2_rn(0.f);
+                            const __half2 s1 = kv_ok[mt][1] ? __half2half2(vs[tau1 * 4 + t]) : __float2half2_rn(0.f);
+                            const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w};
+                            const uint32_t w1[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                            for (int m = 0; m < 8; ++m) {
+                                const uint32_t x0 = w0[m >> 1] >> ((m & 1) * 8);
+                                const uint32_t x1 = w1[m >> 1] >> ((m & 1) * 8);
+                                const uint32_t a0 = movmatrix_t(h2_u32(__hmul2(nib_even(x0), s0)));
+                                const uint32_t a1 = movmatrix_t(h2_u32(__hmul2(nib_odd(x0), s0)));
+                                const uint32_t a2 = movmatrix_t(h2_u32(__hmul2(nib_even(x1), s1)));
+                                const uint32_t a3 = movmatrix_t(h2_u32(__hmul2(nib_odd(x1), s1)));
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) mma_f16(acc[m][nt], a0, a1, a2, a3, pb[mt][nt][0], pb[mt][nt][1]);
+                            }
+                        } else {
+                            const unsigned char *v0p = st + ST::kV + tau0 * 256 + 16 * t;
+                            uint32_t w0[16], w1[16];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                uint4 va = lds128(v0p + 64 * u), vb = lds128(v0p + 8 * 256 + 64 * u);
+                                if (!kv_ok[mt][0]) va = make_uint4(0, 0, 0, 0);
+                                if (!kv_ok[mt][1]) vb = make_uint4(0, 0, 0, 0);
+                                w0[4 * u] = va.x; w0[4 * u + 1] = va.y; w0[4 * u + 2] = va.z; w0[4 * u + 3] = va.w;
+                                w1[4 * u] = vb.x; w1[4 * u + 1] = vb.y; w1[4 * u + 2] = vb.z; w1[4 * u + 3] = vb.w;
+                            }
+#pragma unroll
+                            for (int m = 0; m < 8; ++m) {
+                                const uint32_t a0 = movmatrix_t(w0[2 * m]), a1 = movmatrix_t(w0[2 * m + 1]);
+                                const uint32_t a2 = movmatrix_t(w1[2 * m]), a3 = movmatrix_t(w1[2 * m + 1]);
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    mma_bf16(acc[m][nt], a0, a1, a2, a3, pb[mt][nt][0], pb[mt][nt][1]);
+                                    mma_bf16(acc[m][nt], a0, a1, a2, a3, pbl[mt][nt][0], pbl[mt][nt][1]);
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+        }
+
+        // ---- merge the consumer warps of each row group (shared memory)
+        const int s_id = b * H + h;
+        const int first = owner_cta(walk.s0, W, P);
+        const int last = owner_cta(walk.s0 + seqC[b] - 1, W, P);
+        const int n_pieces = last - first + 1;
+        const int rows_here = p.rows;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float l = l_run[nt][e];
+                l += __shfl_xor_sync(0xffffffffu, l, 4);
+                l += __shfl_xor_sync(0xffffffffu, l, 8);
+                l += __shfl_xor_sync(0xffffffffu, l, 16);
+                const int rr = nt * 8 + 2 * t + e;
+                if (g == 0) {
+                    sm_m[warp * NR + rr] = m_run[nt][e];
+                    sm_l[warp * NR + rr] = l;
+                }
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
-                    acc[m][nt][e] *= alpha;
-                    acc[m][nt][2 + e] *= alpha;
+                    const int c0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
+                    const int c1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
+                    sm_o[(warp * NR + rr) * 132 + c0] = acc[m][nt][e];
+                    sm_o[(warp * NR + rr) * 132 + c1] = acc[m][nt][2 + e];
                 }
             }
-            if (K8) {
-                pb0[nt] = movmatrix_t(pack_f16(pr[0][0], pr[0][1]));
-                pb1[nt] = movmatrix_t(pack_f16(pr[1][0], pr[1][1]));
-            } else {
-                // bf16 P split into hi + lo so the weights keep ~16 bits
-                const uint32_t h0 = pack_bf16(pr[0][0], pr[0][1]);
-                const uint32_t h1 = pack_bf16(pr[1][0], pr[1][1]);
-                pb0[nt] = movmatrix_t(h0);
-                pb1[nt] = movmatrix_t(h1);
-                pb0l[nt] = movmatrix_t(pack_bf16(pr[0][0] - __uint_as_float(h0 << 16),
-                                                 pr[0][1] - __uint_as_float(h0 & 0xFFFF0000u)));
-                pb1l[nt] = movmatrix_t(pack_bf16(pr[1][0] - __uint_as_float(h1 << 16),
-                                                 pr[1][1] - __uint_as_float(h1 & 0xFFFF0000u)));
+        named_sync(1, kConsumerWarps * 32);
+        {
+            // per-row factors of the row group's warps: f_w = 2^(m_w - M) / L
+            const int tid = slot * 32 + lane, nthr = CW * 32;
+            float *fac = sm_l;  // [warp][rr] factors overwrite the sums they are built from
+            for (int rr = tid; rr < NR; rr += nthr) {
+                float M = -INFINITY;
+                for (int w = 0; w < CW; ++w) M = fmaxf(M, sm_m[(rg * CW + w) * NR + rr]);
+                float ls = 0.f;
+                if (M != -INFINITY)
+                    for (int w = 0; w < CW; ++w) ls += sm_l[(rg * CW + w) * NR + rr] * ex2(sm_m[(rg * CW + w) * NR + rr] - M);
+                const float inv = M == -INFINITY ? 0.f : 1.0f / ls;
+                for (int w = 0; w < CW; ++w) {
+                    const int wi = (rg * CW + w) * NR + rr;
+                    fac[wi] = M == -INFINITY ? 0.f : ex2(sm_m[wi] - M) * inv;
+                }
+                // the row's lse goes where warp 0 of the group kept its max
+                sm_m[(rg * CW) * NR + rr] = M == -INFINITY ? -INFINITY : (M + log2f(ls)) * 0.69314718055994531f;
             }
-        }
-
-        // ---- O^T += V^T . P^T over 8 m-tiles of 16 channels
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            uint32_t xa0, xb0, xa1, xb1;  // 8x8 tiles p = 2m, 2m+1 for token halves 0, 1
-            if (K8) {
-                const int i = m >> 1;
-                const uint32_t w0 = reinterpret_cast<const uint32_t *>(&vq[0][0])[i] >> ((m & 1) * 8);
-                const uint32_t w1 = reinterpret_cast<const uint32_t *>(&vq[1][0])[i] >> ((m & 1) * 8);
-                const __half2 s0 = u32_h2(sv[0]), s1 = u32_h2(sv[1]);
-                xa0 = h2_u32(__hmul2(nib_even(w0), s0));
-                xb0 = h2_u32(__hmul2(nib_odd(w0), s0));
-                xa1 = h2_u32(__hmul2(nib_even(w1), s1));
-                xb1 = h2_u32(__hmul2(nib_odd(w1), s1));
-            } else {
-                const uint32_t *v0 = reinterpret_cast<const uint32_t *>(&vq[0][0]);
-                const uint32_t *v1 = reinterpret_cast<const uint32_t *>(&vq[1][0]);
-                xa0 = v0[2 * m]; xb0 = v0[2 * m + 1];
-                xa1 = v1[2 * m]; xb1 = v1[2 * m + 1];
-            }
-            const uint32_t a0 = movmatrix_t(xa0), a1 = movmatrix_t(xb0);
-            const uint32_t a2 = movmatrix_t(xa1), a3 = movmatrix_t(xb1);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                if (K8) {
-                    mma_f16(acc[m][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+            named_sync(3 + rg, nthr);
+            float *slotp = p.partials + (size_t)(s_id + blockIdx.x) * p.slot_floats;
+            for (int idx = tid; idx < NR * kHeadDim; idx += nthr) {
+                const int rr = idx / kHeadDim, ch = idx % kHeadDim;
+                const int r = row0 + rr;
+                if (r >= rows_here) continue;
+                float o = 0.f;
+#pragma unroll 8
+                for (int w = 0; w < CW; ++w) {
+                    const int wi = (rg * CW + w) * NR + rr;
+                    o += sm_o[wi * 132 + ch] * fac[wi];
+                }
+                const float lse = sm_m[(rg * CW) * NR + rr];
+                if (n_pieces == 1) {
+                    const int j = r / p.group, gq = r % p.group;
+                    const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+                    p.out[row * kHeadDim + ch] = o;
+                    if (ch == 0 && p.out_lse) p.out_lse[row] = lse;
                 } else {
-                    mma_bf16(acc[m][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
-                    mma_bf16(acc[m][nt], a0, a1, a2, a3, pb0l[nt], pb1l[nt]);
+                    slotp[r * kHeadDim + ch] = o;
+                    if (ch == 0) slotp[rows_here * kHeadDim + r] = lse;
                 }
             }
+            if (n_pieces > 1) __threadfence();
         }
-    }
-
-    // ---- merge the warps of the CTA
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            float l = l_run[nt][e];
-            l += __shfl_xor_sync(0xffffffffu, l, 4);
-            l += __shfl_xor_sync(0xffffffffu, l, 8);
-            l += __shfl_xor_sync(0xffffffffu, l, 16);
-            if (g == 0) {
-                sm_m[warp][nt * 8 + 2 * t + e] = m_run[nt][e];
-                sm_l[warp][nt * 8 + 2 * t + e] = l;
-            }
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int ch0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
-                const int ch1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
-                sm_o[warp][nt * 8 + 2 * t + e][ch0] = acc[m][nt][e];
-                sm_o[warp][nt * 8 + 2 * t + e][ch1] = acc[m][nt][2 + e];
-            }
+        named_sync(1, kConsumerWarps * 32);
+        if (threadIdx.x == 0) {
+            int is_last = 0;
+            if (n_pieces > 1) is_last = atomicAdd(&p.tickets[s_id], 1) == n_pieces - 1;
+            misc[1] = is_last;
         }
-    __syncthreads();
-
-    for (int idx = threadIdx.x; idx < NR * kHeadDim; idx += blockDim.x) {
-        const int rr = idx / kHeadDim, ch = idx % kHeadDim;
-        const int r = row0 + rr;
-        if (r >= p.rows_per_head) continue;
-        float M = -INFINITY;
+        named_sync(1, kConsumerWarps * 32);
+        if (misc[1]) {
+            // This CTA holds the last ticket: merge every piece of the segment.
+            // The partials live in L2 (loads bypass L1); the loads are arranged
+            // so that each lane has many independent ones in flight:
+            // step 1: warp w takes rows w, w+8, ...; its lanes load the lse of
+            //   up to 160 pieces at once and reduce max and weight sum;
+            // step 2: warp w takes pieces w, w+8, ...; lane c owns channels
+            //   4c..4c+3 of a batch of rows, loads o and lse of two pieces x
+            //   all rows of the batch at once, and the warps' sums are added in
+            //   shared memory.
+            __threadfence();
+            const int nthr = kConsumerWarps * 32;
+            const int tid = threadIdx.x;
+            const int np = last - first + 1;
+            const float *pbase = p.partials + (size_t)(s_id + first) * p.slot_floats;
+            const int lse_off = rows_here * kHeadDim;
+            constexpr float kLog2e = 1.4426950408889634f;
+            for (int r = warp; r < rows_here; r += kConsumerWarps) {
+                float l[5];
+                float M = -INFINITY;
+                for (int i0 = 0; i0 < np; i0 += 160) {
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm_m[w][rr]);
-        float o = 0.f, lse = -INFINITY;
-        if (M != -INFINITY) {
-            float lsum = 0.f, osum = 0.f;
+                    for (int k = 0; k < 5; ++k) {
+                        const int i = i0 + lane + 32 * k;
+                        l[k] = i < np ? __ldcg(pbase + (size_t)i * p.slot_floats + lse_off + r) : -INFINITY;
+                        M = fmaxf(M, l[k]);
+                    }
+                }
 #pragma unroll
-            for (int w = 0; w < kDecodeWarps; ++w) {
-                const float f = ex2(sm_m[w][rr] - M);
-                lsum += sm_l[w][rr] * f;
-                osum += sm_o[w][rr][ch] * f;
+                for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+                float ws = 0.f;
+                if (M != -INFINITY) {
+                    if (np <= 160) {
+#pragma unroll
+                        for (int k = 0; k < 5; ++k) ws += ex2((l[k] - M) * kLog2e);
+                    } else {
+                        for (int i = lane; i < np; i += 32)
+                            ws += ex2((__ldcg(pbase + (size_t)i * p.slot_floats + lse_off + r) - M) * kLog2e);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+                if (lane == 0) {
+                    sm_m[r] = M;
+                    sm_l[r] = ws;
+                }
             }
-            o = osum / lsum;
-            lse = (M + log2f(lsum)) * 0.69314718055994531f;
+            named_sync(2, nthr);
+            constexpr int RB = 8;                              // rows per batch
+            float4 *red = reinterpret_cast<float4 *>(sm_o);    // [warp][RB][32]
+            for (int r0 = 0; r0 < rows_here; r0 += RB) {
+                float4 a[RB];
+                float Mr[RB];
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    a[rb] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    Mr[rb] = r0 + rb < rows_here ? sm_m[r0 + rb] : -INFINITY;
+                }
+                for (int i = warp; i < np; i += 2 * kConsumerWarps) {
+                    const int i2 = i + kConsumerWarps;
+                    const float *sp = pbase + (size_t)i * p.slot_floats;
+                    const float *sp2 = pbase + (size_t)(i2 < np ? i2 : i) * p.slot_floats;
+                    float4 o1[RB], o2[RB];
+                    float l1[RB], l2[RB];
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+                        const int r = min(r0 + rb, rows_here - 1);
+                        o1[rb] = __ldcg(reinterpret_cast<const float4 *>(sp + r * kHeadDim) + lane);
+                        o2[rb] = __ldcg(reinterpret_cast<const float4 *>(sp2 + r * kHeadDim) + lane);
+                        l1[rb] = __ldcg(sp + lse_off + r);
+                        l2[rb] = __ldcg(sp2 + lse_off + r);
+                    }
+#pragma unroll
+                    for (int rb = 0; rb < RB; ++rb) {
+                        if (Mr[rb] == -INFINITY) continue;
+                        const float w1 = ex2((l1[rb] - Mr[rb]) * kLog2e);
+                        const float w2 = i2 < np ? ex2((l2[rb] - Mr[rb]) * kLog2e) : 0.f;
+                        a[rb].x += w1 * o1[rb].x + w2 * o2[rb].x;
+                        a[rb].y += w1 * o1[rb].y + w2 * o2[rb].y;
+                        a[rb].z += w1 * o1[rb].z + w2 * o2[rb].z;
+                        a[rb].w += w1 * o1[rb].w + w2 * o2[rb].w;
+                    }
+                }
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) red[(warp * RB + rb) * 32 + lane] = a[rb];
+                named_sync(2, nthr);
+                const int nr = min(RB, rows_here - r0);
+                for (int idx = tid; idx < nr * 32; idx += nthr) {
+                    const int rb = idx / 32, c4 = idx % 32, r = r0 + rb;
+                    const float M = sm_m[r], ws = sm_l[r];
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        const float4 x = red[(w * RB + rb) * 32 + c4];
+                        v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+                    }
+                    const float inv = M == -INFINITY ? 0.f : 1.0f / ws;
+                    v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+                    const int j = r / p.group, gq = r % p.group;
+                    const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+                    reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = v;
+                    if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(ws);
+                }
+                named_sync(2, nthr);
+            }
+            if (tid == 0) p.tickets[s_id] = 0;
+            named_sync(1, kConsumerWarps * 32);
         }
-        const int j = r / p.group, gq = r % p.group;
-        const size_t grow = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-        p.part_o[((size_t)split * p.rows_total + grow) * kHeadDim + ch] = o;
-        if (ch == 0) p.part_lse[(size_t)split * p.rows_total + grow] = lse;
     }
 }
 

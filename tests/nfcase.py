@@ -48,7 +48,7 @@ def gpu_layer(w, layer, fmt, q_override=None, max_seqlen=None, bt=None, seqlens=
     q = workloads.layer_q(w, layer, device=dev) if q_override is None else q_override
     sl = torch.as_tensor(w.seqlens if seqlens is None else seqlens, dtype=torch.int32, device=dev)
     msl = max(w.seqlens) if max_seqlen is None else max_seqlen
-    ws = torch.empty(nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, msl),
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, msl),
                      dtype=torch.uint8, device=dev)
     out = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), dtype=torch.float32, device=dev)
     lse = torch.empty((w.batch, w.n_q, w.num_q_heads), dtype=torch.float32, device=dev)

@@ -105,7 +105,7 @@ def test_bad_block_id_is_reported_not_faulted():
     bt_bad[0, 1] = w.pool_blocks + 7            # the block holding keys 256..511
     out = torch.empty_like(g["out"])
     sl = torch.tensor([600], dtype=torch.int32, device="cuda")
-    ws = torch.empty(nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 600), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 600), dtype=torch.uint8, device="cuda")
     nf.nf_decode_attn(g["kv"], g["q"], bt_bad, sl, 600, w.softmax_scale, False, out, None, ws)
     assert nf.nf_get_device_error() == nf.NF_DEVERR_BLOCK_ID
     # the context is still usable and a correct call still gives the right answer
@@ -134,7 +134,7 @@ def test_seqlen_above_bound_is_reported():
     sl = torch.tensor([400], dtype=torch.int32, device="cuda")
     out = torch.empty_like(g["out"])
     lse = torch.empty_like(g["lse"])
-    ws = torch.empty(nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 300), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 300), dtype=torch.uint8, device="cuda")
     nf.nf_decode_attn(g["kv"], g["q"], torch.as_tensor(g["bt"], device="cuda"), sl, 300,
                       w.softmax_scale, False, out, lse, ws)
     assert nf.nf_get_device_error() == nf.NF_DEVERR_SEQLEN
@@ -145,7 +145,7 @@ def test_workspace_too_small_is_refused():
     w = workloads.custom("ws", cached=(300,), num_q_heads=4, num_kv_heads=1)
     g = gpu_layer(w, 0, K8)
     need = nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 300)
-    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
     with pytest.raises(nf.NfError) as e:
         nf.nf_decode_attn(g["kv"], g["q"], torch.as_tensor(g["bt"], device="cuda"),
                           torch.tensor([300], dtype=torch.int32, device="cuda"), 300,
