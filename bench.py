@@ -209,7 +209,9 @@ class GpuWorkload:
         return w.layers * (self.decode_bytes_per_launch() + app)
 
     def launches_per_step(self):
-        return self.w.layers * ((1 if self.w.n_new else 0) + 2)
+        # per layer: the append kernel (when the step appends) and the decode
+        # kernel, whose cross-CTA combine is fused in
+        return self.w.layers * ((1 if self.w.n_new else 0) + 1)
 
 
 def time_graph(g, steps, warmup, stream):
@@ -229,7 +231,7 @@ def time_graph(g, steps, warmup, stream):
 
 
 def time_decode_launches(gw, steps, stream):
-    """Average duration of one nf_decode_attn call (split kernel + combine),
+    """Average duration of one nf_decode_attn call (one fused kernel launch),
     from CUDA events recorded around every call inside a captured graph."""
     L = gw.w.layers
     ev = [(torch.cuda.Event(enable_timing=True, external=True),
@@ -430,7 +432,7 @@ def main():
         "step_gbs": gw.step_bytes() / (ms / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "nf_decode_attn (split kernel + combine)", "peak_source": peak_kind,
+                     "kernel": "decode_kernel (nf_decode_attn: split-K with fused combine)", "peak_source": peak_kind,
                      "bytes_per_launch": dec_bytes, "launch_us": dec_ms * 1e3},
         "cpu_baseline": cpu,
         "e2e": {"value": tokens * ws / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

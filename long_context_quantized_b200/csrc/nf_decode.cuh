@@ -25,11 +25,17 @@
 //   All consumer warps work on every stage -- each takes units of 32 keys (16
 //   for bf16) -- and release it on an "empty" mbarrier, so stages retire in
 //   order.
-// Math per 16-key m-tile (mma.sync m16n8k16, "swap AB": keys are M, query rows
-//   N = 8): S^T = K_codes . Q^T with int8 codes -> fp16 exactly and the K scale
-//   per key applied to the rows of S^T; O^T += V_hat^T . P^T with nibbles ->
-//   fp16 exactly, times the fp16 V scale of (key, 32-channel group), and
-//   movmatrix transposing V and P into fragment layout.  The running max of a
+// Math per 16-key m-tile ("swap AB": keys are the M dimension, query rows N = 8):
+//   S^T = K_codes . Q^T on the integer tensor cores (mma.sync m16n8k32 s8 x s8
+//   -> s32) straight from the int8 codes in shared memory: each query row is
+//   written as three int8 digits, q ~= s (d1 + d2 / 254 + d3 / 254^2) with s =
+//   max|q| / 127 (error below 2^-24 max|q|, fp32 level; two digits, error
+//   below 2^-16 max|q|, when a warp serves 16 rows), the exact int32 dot
+//   products are recombined in fp32, and the K scale of each key multiplies
+//   the rows of S^T.  (The bf16 cache uses bf16 mma.sync instead.)
+//   O^T += V_hat^T . P^T (mma.sync m16n8k16 fp16, fp32 accumulate) with
+//   nibbles -> fp16 exactly, times the fp16 V scale of (key, 32-channel group),
+//   and movmatrix transposing V and P into fragment layout.  The running max of a
 //   row is only raised (and O rescaled) when a tile's max exceeds it by more
 //   than 2^8; the cross-lane max is only reduced when some lane asks for that.
 // Merge: at the end of each piece the consumer warps merge through shared
@@ -63,7 +69,7 @@ struct Stage<NF_KV_K8V4, NT> {
     static constexpr int kBytesPerTok = 202;
     static constexpr int kStride = kTok * kBytesPerTok;  // 51712, a 128-byte multiple
     static constexpr int kStages = 3;
-    static constexpr int kUnitTiles = 2;              // 16-key m-tiles per consumer work unit
+    static constexpr int kUnitTiles = NT == 1 ? 2 : 1;  // 16-key m-tiles per consumer work unit
 };
 template <int NT>
 struct Stage<NF_KV_BF16, NT> {
@@ -104,8 +110,10 @@ struct DecodeSmem {
     static constexpr int NR = NT * 8;
     using ST = Stage<FMT, NT>;
     static constexpr int kStagesBytes = ST::kStages * ST::kStride;
-    static constexpr int kMergeO = kStagesBytes;                               // float [8][NR][132]
-    static constexpr int kMergeM = kMergeO + kConsumerWarps * NR * 132 * 4;    // float [8][NR]
+    // warps' scaled accumulators are summed into kMergeSlots buffers, in rounds
+    static constexpr int kMergeSlots = kConsumerWarps;
+    static constexpr int kMergeO = kStagesBytes;                               // float [slots][NR][132]
+    static constexpr int kMergeM = kMergeO + kMergeSlots * NR * 132 * 4;       // float [8][NR]
     static constexpr int kMergeL = kMergeM + kConsumerWarps * NR * 4;          // float [8][NR]
     static constexpr int kBars = kMergeL + kConsumerWarps * NR * 4;            // u64 [2][stages]
     static constexpr int kStageOk = kBars + 2 * ST::kStages * 8;               // int [stages]
@@ -177,6 +185,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     constexpr bool K8 = (FMT == NF_KV_K8V4);
     constexpr int NS = ST::kStages;
     constexpr int NR = SM::NR;
+    // int8 digits per query element: three for 8 rows; two for 16 rows, where
+    // the third would not fit the register budget (error below 2^-16 max|q|)
+    constexpr int ND = NT == 1 ? 3 : 2;
     extern __shared__ __align__(1024) unsigned char smem[];
     float *sm_o = reinterpret_cast<float *>(smem + SM::kMergeO);
     float *sm_m = reinterpret_cast<float *>(smem + SM::kMergeM);
@@ -318,8 +329,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     const int g = lane >> 2, t = lane & 3;
     const int row0 = rg * NR;
 
-    uint32_t qf[NT][8][2];
-    uint32_t ql[QF32 ? NT : 1][8][2];
+    // bf16 cache: query as bf16 (hi + lo for fp32 q) B fragments.  K8/V4: three
+    // int8 digit words per k word, and the per-row digit weights s/254, s/254^2
+    uint32_t qf[K8 ? 1 : NT][8][2];
+    uint32_t ql[(QF32 && !K8) ? NT : 1][8][2];
+    uint32_t qd[K8 ? NT : 1][ND][8];
+    float qa[K8 ? NT : 1][2], qb[K8 ? NT : 1][2];
     float m_run[NT][2], l_run[NT][2];
     float acc[8][NT][4];
     int lim[NT][2];
@@ -335,26 +350,57 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             const bool rv = r < p.rows;
             const int j = rv ? r / p.group : 0, gq = rv ? r % p.group : 0;
             const size_t qoff = (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim;
+            if (K8) {
+                // lane (g, t) holds channels 32t + 4w + e (w < 8, e < 4) of row g
+                float x[32];
+                float amax = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                float x[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = k_channel(FMT, ks, t, e);
-                    if (!rv) x[e] = 0.f;
-                    else if (QF32) x[e] = static_cast<const float *>(p.q)[qoff + c];
-                    else x[e] = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[qoff + c]);
+                for (int c = 0; c < 32; ++c) {
+                    x[c] = !rv ? 0.f
+                                : QF32 ? static_cast<const float *>(p.q)[qoff + 32 * t + c]
+                                       : __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[qoff + 32 * t + c]);
+                    amax = fmaxf(amax, fabsf(x[c]));
                 }
-                if (K8) {
-                    qf[nt][ks][0] = pack_f16(x[0], x[1]);
-                    qf[nt][ks][1] = pack_f16(x[2], x[3]);
-                    if (QF32) {
-                        const float2 h0 = __half22float2(u32_h2(qf[nt][ks][0]));
-                        const float2 h1 = __half22float2(u32_h2(qf[nt][ks][1]));
-                        ql[nt][ks][0] = pack_f16(x[0] - h0.x, x[1] - h0.y);
-                        ql[nt][ks][1] = pack_f16(x[2] - h1.x, x[3] - h1.y);
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                const float s1 = amax / 127.0f, s2 = s1 / 254.0f, s3 = s2 / 254.0f;
+                const float inv = amax > 0.f ? 127.0f / amax : 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    uint32_t d1w = 0, d2w = 0, d3w = 0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float v = x[4 * w + e];
+                        const float d1 = fminf(fmaxf(rintf(v * inv), -127.f), 127.f);
+                        const float r1 = fmaf(-d1, s1, v);
+                        const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
+                        const float r2 = fmaf(-d2, s2, r1);
+                        const float d3 = fminf(fmaxf(rintf(r2 * inv * 64516.0f), -127.f), 127.f);
+                        d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
+                        d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
+                        d3w |= ((uint32_t)(int)d3 & 0xFFu) << (8 * e);
                     }
-                } else {
+                    qd[nt][0][w] = d1w;
+                    qd[nt][1][w] = d2w;
+                    if (ND == 3) qd[nt][ND - 1][w] = d3w;
+                }
+                // digit weights of the rows 2t + e this lane's accumulators hold
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    qa[nt][e] = __shfl_sync(0xffffffffu, s2, (2 * t + e) * 4);
+                    qb[nt][e] = __shfl_sync(0xffffffffu, s3, (2 * t + e) * 4);
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = k_channel(FMT, ks, t, e);
+                        if (!rv) x[e] = 0.f;
+                        else if (QF32) x[e] = static_cast<const float *>(p.q)[qoff + c];
+                        else x[e] = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[qoff + c]);
+                    }
                     qf[nt][ks][0] = pack_bf16(x[0], x[1]);
                     qf[nt][ks][1] = pack_bf16(x[2], x[3]);
                     if (QF32) {
@@ -409,15 +455,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
                             const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
 #pragma unroll
-                            for (int ks = 0; ks < 8; ++ks) {
-                                uint32_t a0, a1, a2, a3;
-                                i8x4_to_f16(wa[ks], a0, a2);
-                                i8x4_to_f16(wb[ks], a1, a3);
+                            for (int nt = 0; nt < NT; ++nt) {
+                                int dacc[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    mma_f16(s[mt][nt], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
-                                    if (QF32) mma_f16(s[mt][nt], a0, a1, a2, a3, ql[nt][ks][0], ql[nt][ks][1]);
-                                }
+                                for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+                                    for (int dg = 0; dg < ND; ++dg)
+                                        mma_s8(dacc[dg], wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
+                                               qd[nt][dg][2 * ks], qd[nt][dg][2 * ks + 1]);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    s[mt][nt][i] = fmaf(qa[nt][i & 1], (float)(dacc[0][i] * 254 + dacc[1][i]),
+                                                        ND == 3 ? qb[nt][i & 1] * (float)dacc[2][i] : 0.f);
                             }
                         } else {
                             const unsigned char *k0 = st + ST::kK + tau0 * 256 + 16 * t;
@@ -598,13 +647,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                     sm_m[warp * NR + rr] = m_run[nt][e];
                     sm_l[warp * NR + rr] = l;
                 }
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int c0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
-                    const int c1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
-                    sm_o[(warp * NR + rr) * 132 + c0] = acc[m][nt][e];
-                    sm_o[(warp * NR + rr) * 132 + c1] = acc[m][nt][2 + e];
-                }
             }
         named_sync(1, kConsumerWarps * 32);
         {
@@ -625,18 +667,50 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 // the row's lse goes where warp 0 of the group kept its max
                 sm_m[(rg * CW) * NR + rr] = M == -INFINITY ? -INFINITY : (M + log2f(ls)) * 0.69314718055994531f;
             }
-            named_sync(3 + rg, nthr);
+        }
+        named_sync(1, kConsumerWarps * 32);
+        {
+            // each warp adds f_w * acc_w into slot (warp mod slots), one round
+            // of warps after the other
+            constexpr int SLOTS = SM::kMergeSlots;
+#pragma unroll
+            for (int round = 0; round < kConsumerWarps / SLOTS; ++round) {
+                if (warp / SLOTS == round) {
+                    float *buf = sm_o + (warp % SLOTS) * NR * 132;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int rr = nt * 8 + 2 * t + e;
+                            const float f = sm_l[warp * NR + rr];  // this warp's factor for the row
+#pragma unroll
+                            for (int m = 0; m < 8; ++m) {
+                                const int c0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
+                                const int c1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
+                                if (round == 0) {
+                                    buf[rr * 132 + c0] = acc[m][nt][e] * f;
+                                    buf[rr * 132 + c1] = acc[m][nt][2 + e] * f;
+                                } else {
+                                    buf[rr * 132 + c0] += acc[m][nt][e] * f;
+                                    buf[rr * 132 + c1] += acc[m][nt][2 + e] * f;
+                                }
+                            }
+                        }
+                }
+                named_sync(1, kConsumerWarps * 32);
+            }
+        }
+        {
+            const int tid = slot * 32 + lane, nthr = CW * 32;
+            constexpr int SLOTS = SM::kMergeSlots;
+            const int slot0 = (rg * CW) % SLOTS, nslots = CW < SLOTS ? CW : SLOTS;
             float *slotp = p.partials + (size_t)(s_id + blockIdx.x) * p.slot_floats;
             for (int idx = tid; idx < NR * kHeadDim; idx += nthr) {
                 const int rr = idx / kHeadDim, ch = idx % kHeadDim;
                 const int r = row0 + rr;
                 if (r >= rows_here) continue;
                 float o = 0.f;
-#pragma unroll 8
-                for (int w = 0; w < CW; ++w) {
-                    const int wi = (rg * CW + w) * NR + rr;
-                    o += sm_o[wi * 132 + ch] * fac[wi];
-                }
+                for (int sl = 0; sl < nslots; ++sl) o += sm_o[((slot0 + sl) * NR + rr) * 132 + ch];
                 const float lse = sm_m[(rg * CW) * NR + rr];
                 if (n_pieces == 1) {
                     const int j = r / p.group, gq = r % p.group;
@@ -705,7 +779,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 }
             }
             named_sync(2, nthr);
-            constexpr int RB = 8;                              // rows per batch
+            // rows per batch: the warps' float4 sums of a batch must fit the merge buffer
+            constexpr int kRBfit = SM::kMergeSlots * NR * 132 * 4 / (kConsumerWarps * 32 * 16);
+            constexpr int RB = kRBfit < 8 ? kRBfit : 8;
+            static_assert(RB >= 1, "merge buffer too small for the final merge");
             float4 *red = reinterpret_cast<float4 *>(sm_o);    // [warp][RB][32]
             for (int r0 = 0; r0 < rows_here; r0 += RB) {
                 float4 a[RB];
