@@ -138,6 +138,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(x, device=None):
+    """The largest of the ranks' values of x (every rank gets it); x itself
+    when no process group is up.  Timings of the weak-scaled replicas are
+    reduced with it, so the job's time is that of its slowest rank."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world_size, ms_max):
+    """Whole-job KV tokens/s: every rank processes its own replica of the
+    workload, so the job's tokens are world_size times a rank's, over the
+    slowest rank's time."""
+    return tokens_per_rank * world_size / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------ GPU workload
 class GpuWorkload:
     """All layers' pools, queries and step inputs resident on the device."""
@@ -363,16 +382,14 @@ def main():
     time.sleep(0.3)
     ms = time_graph(g, args.steps, 0, stream)
     clk = clocks.stop()
+    ms = max_over_ranks(ms, device)
     if ws > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
         torch.distributed.barrier()
     err = nf.nf_get_device_error()
     assert err == 0, f"device error {err}"
 
     tokens = w.kv_tokens_per_step()
-    value = tokens * ws / (ms / 1e3)
+    value = job_throughput(tokens, ws, ms)
 
     # ---- dominant kernel: per-launch duration from events in the graph
     dec_ms = time_decode_launches(gw, max(5, min(args.steps, 30)), stream)
@@ -398,10 +415,7 @@ def main():
             gw.decode(layer)
             h_out[layer].copy_(gw.out[layer], non_blocking=True)
     e2e_ms = time_graph(ge, args.steps, max(3, args.warmup), stream)
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, device)
     h2d = sum(t.numel() * t.element_size() for t in h_q + h_k + h_v)
     d2h = sum(t.numel() * t.element_size() for t in h_out)
     del ge, g
@@ -435,7 +449,7 @@ def main():
                      "kernel": "decode_kernel (nf_decode_attn: split-K with fused combine)", "peak_source": peak_kind,
                      "bytes_per_launch": dec_bytes, "launch_us": dec_ms * 1e3},
         "cpu_baseline": cpu,
-        "e2e": {"value": tokens * ws / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(tokens, ws, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": gw.launches_per_step() * args.steps,
         "clocks": clk,
