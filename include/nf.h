@@ -64,6 +64,8 @@ typedef int32_t nf_status;
 #define NF_DEVERR_TABLE 2     /* a position whose block index is >= max_blocks */
 #define NF_DEVERR_SEQLEN 3    /* seqlens[b] < n_q or > max_seqlen */
 #define NF_DEVERR_TIMEOUT 4   /* a bounded wait inside a kernel gave up (the kernel returned) */
+#define NF_DEVERR_INTERNAL 5  /* a launch-time invariant of the kernel failed (e.g. shared-memory
+                                 alignment); the call did no work */
 
 /* Element types. */
 #define NF_F32 0

@@ -6,6 +6,9 @@
 #include <atomic>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "nf.h"
 #include "nf_append.cuh"
 #include "nf_combine.cuh"
@@ -85,11 +88,59 @@ bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sm
     return true;
 }
 
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime (no
+// link against libcuda).  It is a host-only function: it packs the tensor map.
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+std::once_flag g_encode_once;
+
+// Tensor map of a K8/V4 layer's V nibbles for the decode kernel: the plane as
+// [num_blocks * H_kv * 256 rows][64 bytes], 32-row boxes, 64-byte swizzle.
+nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map) {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode_tiled) return fail(NF_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t rows = (cuuint64_t)kv->num_blocks * (cuuint64_t)kv->num_kv_heads * nf::kBlock;
+    if (rows > 0x7fffffffull)
+        return fail(NF_ERR_UNSUPPORTED, "pool of %llu token rows per plane (at most 2^31 - 1)", (unsigned long long)rows);
+    const cuuint64_t dims[2] = {64, rows};
+    const cuuint64_t strides[1] = {64};
+    const cuuint32_t box[2] = {64, (cuuint32_t)nf::kChunk};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->v_codes, dims, strides, box, estr,
+                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NF_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return NF_OK;
+}
+
 int current_sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
     return n;
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream finishes; it waits for it (pdl_wait)
+// before touching global memory.
+template <typename Kern, typename Params>
+cudaError_t launch_pdl(Kern kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t s, const Params &p) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 template <int NT, bool QF32, int FMT>
@@ -106,8 +157,7 @@ cudaError_t launch_decode(const nf::DecodeParams &p, int ctas, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         opted.fetch_or(bit, std::memory_order_acq_rel);
     }
-    nf::decode_kernel<NT, QF32, FMT><<<ctas, nf::kDecodeThreads, smem, s>>>(p);
-    return cudaSuccess;
+    return launch_pdl(nf::decode_kernel<NT, QF32, FMT>, (unsigned)ctas, nf::kDecodeThreads, smem, s, p);
 }
 
 template <int NT>
@@ -120,7 +170,8 @@ cudaError_t dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, int c
 nf_status launch_combine(const float *part_o, const float *part_lse, int n_splits, int rows,
                          int head_dim, float *out, float *out_lse, cudaStream_t s) {
     nf::CombineParams c{part_o, part_lse, n_splits, rows, head_dim, out, out_lse};
-    nf::combine_kernel<<<rows, nf::kCombineWarps * 32, 0, s>>>(c);
+    const cudaError_t e = launch_pdl(nf::combine_kernel, (unsigned)rows, nf::kCombineWarps * 32, 0, s, c);
+    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "combine kernel launch: %s", cudaGetErrorString(e));
     return after_launch("combine kernel launch");
 }
 
@@ -196,7 +247,9 @@ nf_status nf_kv_append_quant(const nf_kv_layer *kv, const void *k_new, const voi
     const long long items = (long long)batch * n_new * kv->num_kv_heads;
     const long long blocks = (items + 7) / 8;
     if (blocks > 0x7fffffffLL) return fail(NF_ERR_INVALID_ARG, "too many tokens in one append");
-    nf::append_quant_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    const cudaError_t e = launch_pdl(nf::append_quant_kernel, (unsigned)blocks, 256, 0,
+                                     reinterpret_cast<cudaStream_t>(stream), p);
+    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "append kernel launch: %s", cudaGetErrorString(e));
     return after_launch("append kernel launch");
 }
 
@@ -245,6 +298,10 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
         return fail(NF_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
 
     nf::DecodeParams p{};
+    if (kv->fmt == NF_KV_K8V4) {
+        st = encode_v_map(kv, &p.vmap);
+        if (st != NF_OK) return st;
+    }
     p.k_codes = kv->k_codes;
     p.k_scales = static_cast<const __half *>(kv->k_scales);
     p.v_codes = kv->v_codes;

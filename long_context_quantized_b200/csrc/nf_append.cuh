@@ -60,6 +60,8 @@ __device__ __forceinline__ int make_code(float x, float sigma, int q) {
 }
 
 __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long total = (long long)p.batch * p.n_new * p.num_kv_heads;
@@ -68,6 +70,13 @@ __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p)
     const long long bi = item / p.num_kv_heads;
     const int i = (int)(bi % p.n_new);
     const int b = (int)(bi / p.n_new);
+
+    // the new token's values do not depend on where it goes: load them first,
+    // so their latency overlaps the lengths -> block-table lookups
+    const size_t src = (size_t)item * kHeadDim + 4 * lane;
+    float k[4], v[4];
+    load4(p.k_new, src, p.in_f32 != 0, k);
+    load4(p.v_new, src, p.in_f32 != 0, v);
 
     const int pos = p.seqlens_before[b] + i;
     const int blk_i = pos >> 8;
@@ -81,11 +90,6 @@ __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p)
         return;
     }
     const size_t si = ((size_t)blk * p.num_kv_heads + h) * kBlock + (pos & (kBlock - 1));
-    const size_t src = (size_t)item * kHeadDim + 4 * lane;
-
-    float k[4], v[4];
-    load4(p.k_new, src, p.in_f32 != 0, k);
-    load4(p.v_new, src, p.in_f32 != 0, v);
 
     if (p.fmt == NF_KV_BF16) {
         uint2 kb, vb;

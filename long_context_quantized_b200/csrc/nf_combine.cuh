@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Combi
     __shared__ float red[kCombineWarps];
     __shared__ float4 acc_sm[kCombineWarps][kCombineMaxDim / 4];
     constexpr float kLog2e = 1.4426950408889634f;
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int row = blockIdx.x;
     const float *lse_col = p.part_lse + row;  // stride p.rows

@@ -135,6 +135,34 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
 }
+// 2-D tiled copy global -> shared on the TMA engine through a tensor map (a
+// __grid_constant__ kernel parameter), completing on `bar`.  x is the inner
+// (contiguous) coordinate in elements, y the row.  No multicast.
+__device__ __forceinline__ void tma_load_2d(void *dst, const void *tmap, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+// Four 8x8 matrices of 16-bit elements from shared memory, transposed: lanes
+// 8i..8i+7 give the row addresses of matrix i; lane (g, t) receives elements
+// [2t][g] (low half) and [2t+1][g] (high half) of each matrix.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    return __byte_perm(a, b, sel);
+}
+// Programmatic dependent launch.  pdl_wait: block until the grids this one
+// depends on have completed and their memory operations are visible (at once
+// when the kernel was launched without the attribute); every kernel of libnf
+// calls it before its first global-memory access.  pdl_trigger: let the next
+// kernel in the stream start placing its CTAs (they block in pdl_wait).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 // Named barrier among `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -18,26 +18,33 @@
 // Pipeline: a producer warp cuts each piece into stages of up to 256 keys
 //   (64 for the bf16 cache) inside one 256-key block and moves each stage's K
 //   codes, V nibbles, K scales and V scales into a ring of shared-memory
-//   buffers with 1-D bulk copies on the TMA engine, completing on an mbarrier.
-//   Stages are large because a ring buffer turns over at a roughly fixed rate
-//   per SM (about 2.7 stages per microsecond measured on B200): bandwidth is
-//   stage bytes x that rate, so 32-52 KB stages keep it above the HBM rate.
-//   All consumer warps work on every stage -- each takes units of 32 keys (16
-//   for bf16) -- and release it on an "empty" mbarrier, so stages retire in
-//   order.
+//   buffers on the TMA engine (1-D bulk copies; the V nibbles as 2-D tiles
+//   through a tensor map with the 64-byte swizzle, so that eight keys' rows
+//   of one 16-byte column sit in eight different bank groups), completing on
+//   an mbarrier.  Stages are large because a ring buffer turns over at a
+//   roughly fixed rate per SM (about 2.7 stages per microsecond measured on
+//   B200): bandwidth is stage bytes x that rate, so 32-52 KB stages keep it
+//   above the HBM rate.  All consumer warps work on every stage -- each takes
+//   units of 32 keys (16 for bf16) -- and release it on an "empty" mbarrier,
+//   so stages retire in order.
 // Math per 16-key m-tile ("swap AB": keys are the M dimension, query rows N = 8):
 //   S^T = K_codes . Q^T on the integer tensor cores (mma.sync m16n8k32 s8 x s8
 //   -> s32) straight from the int8 codes in shared memory: each query row is
-//   written as three int8 digits, q ~= s (d1 + d2 / 254 + d3 / 254^2) with s =
-//   max|q| / 127 (error below 2^-24 max|q|, fp32 level; two digits, error
-//   below 2^-16 max|q|, when a warp serves 16 rows), the exact int32 dot
-//   products are recombined in fp32, and the K scale of each key multiplies
-//   the rows of S^T.  (The bf16 cache uses bf16 mma.sync instead.)
-//   O^T += V_hat^T . P^T (mma.sync m16n8k16 fp16, fp32 accumulate) with
-//   nibbles -> fp16 exactly, times the fp16 V scale of (key, 32-channel group),
-//   and movmatrix transposing V and P into fragment layout.  The running max of a
-//   row is only raised (and O rescaled) when a tile's max exceeds it by more
-//   than 2^8; the cross-lane max is only reduced when some lane asks for that.
+//   written as two int8 digits, q ~= s (d1 + d2 / 254) with s = max|q| / 127
+//   (error below 2^-16 max|q| per element), the two exact int32 dot products
+//   are recombined in fp32, and the K scale of each key multiplies the rows of
+//   S^T.  (The bf16 cache uses bf16 mma.sync instead.)
+//   O^T += V_codes^T . (P^T x sigma_V) (mma.sync m16n8k16 fp16, fp32
+//   accumulate): ldmatrix.trans hands each lane the nibbles of one channel for
+//   two consecutive keys, a lop3 and one fp16 op turn a pair into exact fp16
+//   codes -- already in A-fragment layout, with no transpose -- and, since
+//   every 16-channel m-tile lies in one 32-channel scale group, the V scale
+//   of (key, group) multiplies the weights (the B operand) instead of the
+//   values.  The weights are movmatrix-transposed scores.  The running max of
+//   a row is only raised (and O rescaled) when a tile's max exceeds it by more
+//   than 2^4, and the weights are taken relative to max + 4, so they never
+//   exceed 1 and weight x scale stays inside fp16; the cross-lane max is only
+//   reduced when some lane asks for that.
 // Merge: at the end of each piece the consumer warps merge through shared
 //   memory.  A segment owned by one CTA is written straight to out; otherwise
 //   each piece writes an (o, lse) partial and takes a ticket of the segment's
@@ -46,6 +53,8 @@
 // Every mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT
 // and the kernel runs to its end without further waits.
 #pragma once
+
+#include <cuda.h>  // CUtensorMap (a plain struct; no driver call is made here)
 
 #include "nf_common.cuh"
 
@@ -56,6 +65,9 @@ constexpr int kConsumerWarps = 8;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxBatch = 256;
 constexpr int kMaxRows = 64;  // G * n_q per kv-head
+// The running max of a row is raised when a tile's max exceeds it by more than
+// kLazy (log2 units); weights are 2^(x - max - kLazy) <= 1.
+constexpr float kLazy = 4.0f;
 
 template <int FMT, int NT>
 struct Stage;
@@ -67,7 +79,9 @@ struct Stage<NF_KV_K8V4, NT> {
     static constexpr int kKs = kV + kTok * 64;        // fp16  [kTok]
     static constexpr int kVs = kKs + kTok * 2;        // fp16  [kTok][4]
     static constexpr int kBytesPerTok = 202;
-    static constexpr int kStride = kTok * kBytesPerTok;  // 51712, a 128-byte multiple
+    // 51712 bytes of data; buffers start on 1024-byte boundaries, which the
+    // swizzled V tile (a 512-byte pattern) needs
+    static constexpr int kStride = (kTok * kBytesPerTok + 1023) / 1024 * 1024;
     static constexpr int kStages = 3;
     static constexpr int kUnitTiles = NT == 1 ? 2 : 1;  // 16-key m-tiles per consumer work unit
 };
@@ -84,6 +98,7 @@ struct Stage<NF_KV_BF16, NT> {
 };
 
 struct DecodeParams {
+    CUtensorMap vmap;  // K8/V4: v_codes as [num_blocks * H_kv * 256 rows][64 bytes], 32-row boxes, 64-byte swizzle
     const void *k_codes;
     const __half *k_scales;
     const void *v_codes;
@@ -110,12 +125,11 @@ struct DecodeSmem {
     static constexpr int NR = NT * 8;
     using ST = Stage<FMT, NT>;
     static constexpr int kStagesBytes = ST::kStages * ST::kStride;
-    // warps' scaled accumulators are summed into kMergeSlots buffers, in rounds
-    static constexpr int kMergeSlots = kConsumerWarps;
-    static constexpr int kMergeO = kStagesBytes;                               // float [slots][NR][132]
-    static constexpr int kMergeM = kMergeO + kMergeSlots * NR * 132 * 4;       // float [8][NR]
-    static constexpr int kMergeL = kMergeM + kConsumerWarps * NR * 4;          // float [8][NR]
-    static constexpr int kBars = kMergeL + kConsumerWarps * NR * 4;            // u64 [2][stages]
+    static constexpr int kMergeO = kStagesBytes;                               // float [warp][NR][132]
+    static constexpr int kMergeM = kMergeO + kConsumerWarps * NR * 132 * 4;    // float [warp][NR]
+    static constexpr int kMergeL = kMergeM + kConsumerWarps * NR * 4;          // float [warp][NR]
+    static constexpr int kMergeLse = kMergeL + kConsumerWarps * NR * 4;        // float [kMaxRows]
+    static constexpr int kBars = kMergeLse + kMaxRows * 4;                     // u64 [2][stages]
     static constexpr int kStageOk = kBars + 2 * ST::kStages * 8;               // int [stages]
     static constexpr int kSeqC = kStageOk + ST::kStages * 4;                   // int [kMaxBatch]
     static constexpr int kSeqBase = (kSeqC + kMaxBatch * 4 + 7) / 8 * 8;       // i64 [kMaxBatch + 1]
@@ -125,11 +139,13 @@ struct DecodeSmem {
     static_assert(ST::kStride % 128 == 0, "stage alignment");
 };
 
-// Output channel of row `rho` (0..15) of PV m-tile `m` (K8/V4: lane t converts
-// channels 32t..32t+31 of V, pairing nibbles k and k + 4 of each word).
+// Output channel of row `rho` (0..15) of PV m-tile `m` (K8/V4): m-tile m = 2cg
+// + ip covers scale group cg; row rho < 8 is channel 32cg + 4rho + 2ip (the
+// nibble 2ip of b16 column rho of the group's 16-byte column), row rho + 8 the
+// channel after it.
 __device__ __forceinline__ int v_channel_k8v4(int m, int rho) {
-    const int p = 2 * m + (rho >> 3), jj = rho & 7;
-    return 32 * (jj >> 1) + 8 * (p >> 2) + (p & 3) + 4 * (jj & 1);
+    const int cg = m >> 1, ip = m & 1;
+    return 32 * cg + 4 * (rho & 7) + 2 * ip + (rho >> 3);
 }
 // bf16 cache: lane t's u-th 16-byte load holds channels 32u + 8t .. 32u + 8t + 7.
 __device__ __forceinline__ int v_channel_bf16(int m, int rho) {
@@ -185,9 +201,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     constexpr bool K8 = (FMT == NF_KV_K8V4);
     constexpr int NS = ST::kStages;
     constexpr int NR = SM::NR;
-    // int8 digits per query element: three for 8 rows; two for 16 rows, where
-    // the third would not fit the register budget (error below 2^-16 max|q|)
-    constexpr int ND = NT == 1 ? 3 : 2;
     extern __shared__ __align__(1024) unsigned char smem[];
     float *sm_o = reinterpret_cast<float *>(smem + SM::kMergeO);
     float *sm_m = reinterpret_cast<float *>(smem + SM::kMergeM);
@@ -211,8 +224,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         }
         misc[0] = 0;
         misc[1] = 0;
+        // the stage buffers must start on 1024-byte boundaries (swizzled V
+        // tiles); if the shared window ever were not so aligned, do no work
+        if (smem_addr(smem) & 1023u) {
+            if (blockIdx.x == 0) report(NF_DEVERR_INTERNAL);
+            misc[0] = 1;
+        }
         fence_mbar_init();
     }
+    // everything above touched shared memory only; the lengths, tables, query,
+    // pool and workspace may come from the kernels before this one
+    pdl_wait();
+    pdl_trigger();
     if (warp == 0) {
         for (int b = lane; b < p.batch; b += 32) {
             const int L = p.seqlens[b];
@@ -294,7 +317,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             mbar_arrive_expect_tx(&full[stage], (uint32_t)(ntok * ST::kBytesPerTok));
                             if (K8) {
                                 bulk_g2s(st + ST::kK, static_cast<const int8_t *>(p.k_codes) + si * 128, ntok * 128, &full[stage]);
-                                bulk_g2s(st + ST::kV, static_cast<const uint8_t *>(p.v_codes) + si * 64, ntok * 64, &full[stage]);
+                                for (int c = 0; c < ntok; c += kChunk)
+                                    tma_load_2d(st + ST::kV + c * 64, &p.vmap, 0, (int)si + c, &full[stage]);
                                 bulk_g2s(st + ST::kKs, p.k_scales + si, ntok * 2, &full[stage]);
                                 bulk_g2s(st + ST::kVs, p.v_scales + si * 4, ntok * 8, &full[stage]);
                             } else {
@@ -328,13 +352,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     const int rg = warp / CW, slot = warp % CW;
     const int g = lane >> 2, t = lane & 3;
     const int row0 = rg * NR;
+    float *sm_lse = reinterpret_cast<float *>(smem + SM::kMergeLse);
 
-    // bf16 cache: query as bf16 (hi + lo for fp32 q) B fragments.  K8/V4: three
-    // int8 digit words per k word, and the per-row digit weights s/254, s/254^2
+    // bf16 cache: query as bf16 (hi + lo for fp32 q) B fragments.  K8/V4: two
+    // int8 digit words per k word, and the per-row digit weights s, s / 254
     uint32_t qf[K8 ? 1 : NT][8][2];
     uint32_t ql[(QF32 && !K8) ? NT : 1][8][2];
-    uint32_t qd[K8 ? NT : 1][ND][8];
-    float qa[K8 ? NT : 1][2], qb[K8 ? NT : 1][2];
+    uint32_t qd[K8 ? NT : 1][2][8];
+    float qs[K8 ? NT : 1][2];
     float m_run[NT][2], l_run[NT][2];
     float acc[8][NT][4];
     int lim[NT][2];
@@ -363,33 +388,27 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 }
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                const float s1 = amax / 127.0f, s2 = s1 / 254.0f, s3 = s2 / 254.0f;
+                const float s1 = amax / 127.0f;
                 const float inv = amax > 0.f ? 127.0f / amax : 0.f;
 #pragma unroll
                 for (int w = 0; w < 8; ++w) {
-                    uint32_t d1w = 0, d2w = 0, d3w = 0;
+                    uint32_t d1w = 0, d2w = 0;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float v = x[4 * w + e];
                         const float d1 = fminf(fmaxf(rintf(v * inv), -127.f), 127.f);
                         const float r1 = fmaf(-d1, s1, v);
                         const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
-                        const float r2 = fmaf(-d2, s2, r1);
-                        const float d3 = fminf(fmaxf(rintf(r2 * inv * 64516.0f), -127.f), 127.f);
                         d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
                         d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
-                        d3w |= ((uint32_t)(int)d3 & 0xFFu) << (8 * e);
                     }
                     qd[nt][0][w] = d1w;
                     qd[nt][1][w] = d2w;
-                    if (ND == 3) qd[nt][ND - 1][w] = d3w;
                 }
-                // digit weights of the rows 2t + e this lane's accumulators hold
+                // weight of the low digit (s / 254) of the rows 2t + e this lane's
+                // accumulators hold
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    qa[nt][e] = __shfl_sync(0xffffffffu, s2, (2 * t + e) * 4);
-                    qb[nt][e] = __shfl_sync(0xffffffffu, s3, (2 * t + e) * 4);
-                }
+                for (int e = 0; e < 2; ++e) qs[nt][e] = __shfl_sync(0xffffffffu, s1 / 254.0f, (2 * t + e) * 4);
             } else {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
@@ -456,17 +475,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
 #pragma unroll
                             for (int nt = 0; nt < NT; ++nt) {
-                                int dacc[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
+                                int d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
 #pragma unroll
-                                for (int ks = 0; ks < 4; ++ks)
+                                for (int ks = 0; ks < 4; ++ks) {
+                                    mma_s8(d1, wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
+                                           qd[nt][0][2 * ks], qd[nt][0][2 * ks + 1]);
+                                    mma_s8(d2, wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
+                                           qd[nt][1][2 * ks], qd[nt][1][2 * ks + 1]);
+                                }
+                                // |d1 * 254 + d2| < 2^24: exact in fp32
 #pragma unroll
-                                    for (int dg = 0; dg < ND; ++dg)
-                                        mma_s8(dacc[dg], wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
-                                               qd[nt][dg][2 * ks], qd[nt][dg][2 * ks + 1]);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    s[mt][nt][i] = fmaf(qa[nt][i & 1], (float)(dacc[0][i] * 254 + dacc[1][i]),
-                                                        ND == 3 ? qb[nt][i & 1] * (float)dacc[2][i] : 0.f);
+                                for (int i = 0; i < 4; ++i) s[mt][nt][i] = qs[nt][i & 1] * (float)(d1[i] * 254 + d2[i]);
                             }
                         } else {
                             const unsigned char *k0 = st + ST::kK + tau0 * 256 + 16 * t;
@@ -523,7 +542,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             float mx = fmaxf(xv[0][nt][e], xv[0][nt][2 + e]);
 #pragma unroll
                             for (int mt = 1; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(xv[mt][nt][e], xv[mt][nt][2 + e]));
-                            raise |= mx > m_run[nt][e] + 8.0f;  // true when m_run is -inf and mx finite
+                            raise |= mx > m_run[nt][e] + kLazy;  // true when m_run is -inf and mx finite
                         }
                     if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll
@@ -547,12 +566,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                                 }
                             }
                     }
-                    // weights (P^T) as B fragments of the PV product
+                    // weights 2^(x - m - kLazy) <= 1 (P^T) as B fragments of the PV product
                     uint32_t pb[MT][NT][2], pbl[MT][NT][2];
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        const float mu0 = m_run[nt][0] == -INFINITY ? 0.f : m_run[nt][0];
-                        const float mu1 = m_run[nt][1] == -INFINITY ? 0.f : m_run[nt][1];
+                        const float mu0 = (m_run[nt][0] == -INFINITY ? 0.f : m_run[nt][0]) + kLazy;
+                        const float mu1 = (m_run[nt][1] == -INFINITY ? 0.f : m_run[nt][1]) + kLazy;
 #pragma unroll
                         for (int mt = 0; mt < MT; ++mt) {
                             const float p00 = ex2(xv[mt][nt][0] - mu0), p01 = ex2(xv[mt][nt][1] - mu1);
@@ -578,28 +597,52 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                     // ---- O^T += V^T . P^T over 8 channel m-tiles, one 16-key k-tile per m-tile of the unit
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt) {
-                        const int tau0 = 16 * (MT * un + mt) + g, tau1 = tau0 + 8;
+                        const int tb = 16 * (MT * un + mt);  // first key of the m-tile in the stage
                         if (K8) {
-                            const uint4 v0 = lds128(st + ST::kV + tau0 * 64 + 16 * t);
-                            const uint4 v1 = lds128(st + ST::kV + tau1 * 64 + 16 * t);
-                            const __half *vs = reinterpret_cast<const __half *>(st + ST::kVs);
-                            // keys past the end hold stale bytes: zero their values, not just their weights
-                            const __half2 s0 = kv_ok[mt][0] ? __half2half2(vs[tau0 * 4 + t]) : __float2half2_rn(0.f);
-                            const __half2 s1 = kv_ok[mt][1] ? __half2half2(vs[tau1 * 4 + t]) : __float2half2_rn(0.f);
-                            const uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w};
-                            const uint32_t w1[4] = {v1.x, v1.y, v1.z, v1.w};
+                            // nibbles: matrix cg (lanes 8cg..8cg+7 address its rows) = the
+                            // 16-byte column cg (channels 32cg..32cg+31) of 8 keys; the
+                            // column sits at position cg ^ (row address bits 7-8)
+                            uint32_t R[2][4];
+                            const uint32_t vrow = smem_addr(st + ST::kV) + (uint32_t)(tb + (lane & 7)) * 64u;
+                            const uint32_t vaddr = vrow + ((((uint32_t)lane >> 3) ^ ((vrow >> 7) & 3u)) << 4);
+                            ldsm_x4_t(vaddr, R[0][0], R[0][1], R[0][2], R[0][3]);            // keys tb + 0..7
+                            ldsm_x4_t(vaddr + 8 * 64, R[1][0], R[1][1], R[1][2], R[1][3]);   // keys tb + 8..15
+                            // V scales of keys (2t, 2t+1) and (2t+8, 2t+9) per group, as fp16 pairs
+                            uint32_t sp[2][4];
 #pragma unroll
-                            for (int m = 0; m < 8; ++m) {
-                                const uint32_t x0 = w0[m >> 1] >> ((m & 1) * 8);
-                                const uint32_t x1 = w1[m >> 1] >> ((m & 1) * 8);
-                                const uint32_t a0 = movmatrix_t(h2_u32(__hmul2(nib_even(x0), s0)));
-                                const uint32_t a1 = movmatrix_t(h2_u32(__hmul2(nib_odd(x0), s0)));
-                                const uint32_t a2 = movmatrix_t(h2_u32(__hmul2(nib_even(x1), s1)));
-                                const uint32_t a3 = movmatrix_t(h2_u32(__hmul2(nib_odd(x1), s1)));
+                            for (int kh = 0; kh < 2; ++kh) {
+                                const uint4 sv = lds128(st + ST::kVs + (tb + 8 * kh + 2 * t) * 8);
+                                sp[kh][0] = prmt(sv.x, sv.z, 0x5410);
+                                sp[kh][1] = prmt(sv.x, sv.z, 0x7632);
+                                sp[kh][2] = prmt(sv.y, sv.w, 0x5410);
+                                sp[kh][3] = prmt(sv.y, sv.w, 0x7632);
+                                if (!fast) {
+                                    // keys past the end hold stale bytes: zero their scales
+                                    const int pa = tok0 + tb + 8 * kh + 2 * t;
+                                    const uint32_t keep = (pa < L ? 0x0000FFFFu : 0u) | (pa + 1 < L ? 0xFFFF0000u : 0u);
 #pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) mma_f16(acc[m][nt], a0, a1, a2, a3, pb[mt][nt][0], pb[mt][nt][1]);
+                                    for (int cg = 0; cg < 4; ++cg) sp[kh][cg] &= keep;
+                                }
+                            }
+#pragma unroll
+                            for (int cg = 0; cg < 4; ++cg) {
+                                // exact fp16 codes of channel 32cg + 4g + i for the key pairs
+                                const uint32_t lo0 = R[0][cg], hi0 = R[0][cg] >> 8;
+                                const uint32_t lo1 = R[1][cg], hi1 = R[1][cg] >> 8;
+                                const uint32_t a[2][4] = {
+                                    {h2_u32(nib_even(lo0)), h2_u32(nib_odd(lo0)), h2_u32(nib_even(lo1)), h2_u32(nib_odd(lo1))},
+                                    {h2_u32(nib_even(hi0)), h2_u32(nib_odd(hi0)), h2_u32(nib_even(hi1)), h2_u32(nib_odd(hi1))}};
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    const uint32_t b0 = h2_u32(__hmul2(u32_h2(pb[mt][nt][0]), u32_h2(sp[0][cg])));
+                                    const uint32_t b1 = h2_u32(__hmul2(u32_h2(pb[mt][nt][1]), u32_h2(sp[1][cg])));
+#pragma unroll
+                                    for (int ip = 0; ip < 2; ++ip)
+                                        mma_f16(acc[2 * cg + ip][nt], a[ip][0], a[ip][1], a[ip][2], a[ip][3], b0, b1);
+                                }
                             }
                         } else {
+                            const int tau0 = tb + g;
                             const unsigned char *v0p = st + ST::kV + tau0 * 256 + 16 * t;
                             uint32_t w0[16], w1[16];
 #pragma unroll
@@ -649,195 +692,126 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 }
             }
         named_sync(1, kConsumerWarps * 32);
+        // each lane derives its rows' factor f_w = 2^(m_w - M) / sum_v l_v 2^(m_v - M)
+        // from the group's (m, l) and writes f_w * acc_w to its warp's buffer
         {
-            // per-row factors of the row group's warps: f_w = 2^(m_w - M) / L
-            const int tid = slot * 32 + lane, nthr = CW * 32;
-            float *fac = sm_l;  // [warp][rr] factors overwrite the sums they are built from
-            for (int rr = tid; rr < NR; rr += nthr) {
-                float M = -INFINITY;
-                for (int w = 0; w < CW; ++w) M = fmaxf(M, sm_m[(rg * CW + w) * NR + rr]);
-                float ls = 0.f;
-                if (M != -INFINITY)
-                    for (int w = 0; w < CW; ++w) ls += sm_l[(rg * CW + w) * NR + rr] * ex2(sm_m[(rg * CW + w) * NR + rr] - M);
-                const float inv = M == -INFINITY ? 0.f : 1.0f / ls;
-                for (int w = 0; w < CW; ++w) {
-                    const int wi = (rg * CW + w) * NR + rr;
-                    fac[wi] = M == -INFINITY ? 0.f : ex2(sm_m[wi] - M) * inv;
+            float *buf = sm_o + warp * NR * 132;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int rr = nt * 8 + 2 * t + e;
+                    float M = -INFINITY;
+                    for (int w = 0; w < CW; ++w) M = fmaxf(M, sm_m[(rg * CW + w) * NR + rr]);
+                    float f = 0.f;
+                    if (M != -INFINITY) {
+                        float ls = 0.f;
+                        for (int w = 0; w < CW; ++w)
+                            ls += sm_l[(rg * CW + w) * NR + rr] * ex2(sm_m[(rg * CW + w) * NR + rr] - M);
+                        f = ex2(m_run[nt][e] - M) / ls;
+                        // the row's lse: weights were taken relative to m + kLazy
+                        if (slot == 0 && g == 0) sm_lse[row0 + rr] = (M + kLazy + log2f(ls)) * 0.69314718055994531f;
+                    } else if (slot == 0 && g == 0) {
+                        sm_lse[row0 + rr] = -INFINITY;
+                    }
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) {
+                        const int c0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
+                        const int c1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
+                        buf[rr * 132 + c0] = acc[m][nt][e] * f;
+                        buf[rr * 132 + c1] = acc[m][nt][2 + e] * f;
+                    }
                 }
-                // the row's lse goes where warp 0 of the group kept its max
-                sm_m[(rg * CW) * NR + rr] = M == -INFINITY ? -INFINITY : (M + log2f(ls)) * 0.69314718055994531f;
-            }
         }
         named_sync(1, kConsumerWarps * 32);
         {
-            // each warp adds f_w * acc_w into slot (warp mod slots), one round
-            // of warps after the other
-            constexpr int SLOTS = SM::kMergeSlots;
-#pragma unroll
-            for (int round = 0; round < kConsumerWarps / SLOTS; ++round) {
-                if (warp / SLOTS == round) {
-                    float *buf = sm_o + (warp % SLOTS) * NR * 132;
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int rr = nt * 8 + 2 * t + e;
-                            const float f = sm_l[warp * NR + rr];  // this warp's factor for the row
-#pragma unroll
-                            for (int m = 0; m < 8; ++m) {
-                                const int c0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
-                                const int c1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
-                                if (round == 0) {
-                                    buf[rr * 132 + c0] = acc[m][nt][e] * f;
-                                    buf[rr * 132 + c1] = acc[m][nt][2 + e] * f;
-                                } else {
-                                    buf[rr * 132 + c0] += acc[m][nt][e] * f;
-                                    buf[rr * 132 + c1] += acc[m][nt][2 + e] * f;
-                                }
-                            }
-                        }
-                }
-                named_sync(1, kConsumerWarps * 32);
-            }
-        }
-        {
+            // sum the row group's warp buffers, 4 channels per thread
             const int tid = slot * 32 + lane, nthr = CW * 32;
-            constexpr int SLOTS = SM::kMergeSlots;
-            const int slot0 = (rg * CW) % SLOTS, nslots = CW < SLOTS ? CW : SLOTS;
             float *slotp = p.partials + (size_t)(s_id + blockIdx.x) * p.slot_floats;
-            for (int idx = tid; idx < NR * kHeadDim; idx += nthr) {
-                const int rr = idx / kHeadDim, ch = idx % kHeadDim;
+            for (int idx = tid; idx < NR * (kHeadDim / 4); idx += nthr) {
+                const int rr = idx / (kHeadDim / 4), c4 = idx % (kHeadDim / 4);
                 const int r = row0 + rr;
                 if (r >= rows_here) continue;
-                float o = 0.f;
-                for (int sl = 0; sl < nslots; ++sl) o += sm_o[((slot0 + sl) * NR + rr) * 132 + ch];
-                const float lse = sm_m[(rg * CW) * NR + rr];
+                float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int w = 0; w < CW; ++w) {
+                    const float4 x = *reinterpret_cast<const float4 *>(sm_o + ((rg * CW + w) * NR + rr) * 132 + 4 * c4);
+                    o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
+                }
+                const float lse = sm_lse[r];
                 if (n_pieces == 1) {
                     const int j = r / p.group, gq = r % p.group;
                     const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-                    p.out[row * kHeadDim + ch] = o;
-                    if (ch == 0 && p.out_lse) p.out_lse[row] = lse;
+                    reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = o;
+                    if (c4 == 0 && p.out_lse) p.out_lse[row] = lse;
                 } else {
-                    slotp[r * kHeadDim + ch] = o;
-                    if (ch == 0) slotp[rows_here * kHeadDim + r] = lse;
+                    reinterpret_cast<float4 *>(slotp + r * kHeadDim)[c4] = o;
+                    if (c4 == 0) slotp[rows_here * kHeadDim + r] = lse;
                 }
             }
-            if (n_pieces > 1) __threadfence();
         }
         named_sync(1, kConsumerWarps * 32);
         if (threadIdx.x == 0) {
             int is_last = 0;
-            if (n_pieces > 1) is_last = atomicAdd(&p.tickets[s_id], 1) == n_pieces - 1;
+            if (n_pieces > 1) {
+                // release: the CTA's partial writes (ordered before this thread
+                // by the barrier) become visible before the ticket
+                __threadfence();
+                is_last = atomicAdd(&p.tickets[s_id], 1) == n_pieces - 1;
+                if (is_last) __threadfence();  // acquire: the other pieces' partials
+            }
             misc[1] = is_last;
         }
         named_sync(1, kConsumerWarps * 32);
         if (misc[1]) {
             // This CTA holds the last ticket: merge every piece of the segment.
-            // The partials live in L2 (loads bypass L1); the loads are arranged
-            // so that each lane has many independent ones in flight:
-            // step 1: warp w takes rows w, w+8, ...; its lanes load the lse of
-            //   up to 160 pieces at once and reduce max and weight sum;
-            // step 2: warp w takes pieces w, w+8, ...; lane c owns channels
-            //   4c..4c+3 of a batch of rows, loads o and lse of two pieces x
-            //   all rows of the batch at once, and the warps' sums are added in
-            //   shared memory.
-            __threadfence();
-            const int nthr = kConsumerWarps * 32;
-            const int tid = threadIdx.x;
+            // Each thread owns (row, 4 channels) and streams the pieces' o and
+            // lse from L2 (loads bypass L1), kPB pieces' loads in flight at once,
+            // keeping a running max, weight sum and weighted sum.
+            constexpr int kPB = 16;
+            constexpr float kLog2e = 1.4426950408889634f;
+            const int nthr = kConsumerWarps * 32, tid = threadIdx.x;
             const int np = last - first + 1;
             const float *pbase = p.partials + (size_t)(s_id + first) * p.slot_floats;
             const int lse_off = rows_here * kHeadDim;
-            constexpr float kLog2e = 1.4426950408889634f;
-            for (int r = warp; r < rows_here; r += kConsumerWarps) {
-                float l[5];
-                float M = -INFINITY;
-                for (int i0 = 0; i0 < np; i0 += 160) {
+            for (int it = tid; it < rows_here * (kHeadDim / 4); it += nthr) {
+                const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
+                float M = -INFINITY, S = 0.f;
+                float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int i0 = 0; i0 < np; i0 += kPB) {
+                    float4 o[kPB];
+                    float l[kPB];
 #pragma unroll
-                    for (int k = 0; k < 5; ++k) {
-                        const int i = i0 + lane + 32 * k;
-                        l[k] = i < np ? __ldcg(pbase + (size_t)i * p.slot_floats + lse_off + r) : -INFINITY;
-                        M = fmaxf(M, l[k]);
+                    for (int k = 0; k < kPB; ++k) {
+                        const float *sp = pbase + (size_t)(i0 + k) * p.slot_floats;
+                        if (i0 + k < np) {
+                            o[k] = __ldcg(reinterpret_cast<const float4 *>(sp + r * kHeadDim) + c4);
+                            l[k] = __ldcg(sp + lse_off + r);
+                        } else {
+                            o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            l[k] = -INFINITY;
+                        }
+                    }
+                    float Mb = M;
+#pragma unroll
+                    for (int k = 0; k < kPB; ++k) Mb = fmaxf(Mb, l[k]);
+                    if (Mb == -INFINITY) continue;
+                    const float a = M == -INFINITY ? 0.f : ex2((M - Mb) * kLog2e);
+                    S *= a;
+                    A.x *= a; A.y *= a; A.z *= a; A.w *= a;
+                    M = Mb;
+#pragma unroll
+                    for (int k = 0; k < kPB; ++k) {
+                        const float wk = l[k] == -INFINITY ? 0.f : ex2((l[k] - M) * kLog2e);
+                        S += wk;
+                        A.x += wk * o[k].x; A.y += wk * o[k].y; A.z += wk * o[k].z; A.w += wk * o[k].w;
                     }
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-                float ws = 0.f;
-                if (M != -INFINITY) {
-                    if (np <= 160) {
-#pragma unroll
-                        for (int k = 0; k < 5; ++k) ws += ex2((l[k] - M) * kLog2e);
-                    } else {
-                        for (int i = lane; i < np; i += 32)
-                            ws += ex2((__ldcg(pbase + (size_t)i * p.slot_floats + lse_off + r) - M) * kLog2e);
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
-                if (lane == 0) {
-                    sm_m[r] = M;
-                    sm_l[r] = ws;
-                }
-            }
-            named_sync(2, nthr);
-            // rows per batch: the warps' float4 sums of a batch must fit the merge buffer
-            constexpr int kRBfit = SM::kMergeSlots * NR * 132 * 4 / (kConsumerWarps * 32 * 16);
-            constexpr int RB = kRBfit < 8 ? kRBfit : 8;
-            static_assert(RB >= 1, "merge buffer too small for the final merge");
-            float4 *red = reinterpret_cast<float4 *>(sm_o);    // [warp][RB][32]
-            for (int r0 = 0; r0 < rows_here; r0 += RB) {
-                float4 a[RB];
-                float Mr[RB];
-#pragma unroll
-                for (int rb = 0; rb < RB; ++rb) {
-                    a[rb] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    Mr[rb] = r0 + rb < rows_here ? sm_m[r0 + rb] : -INFINITY;
-                }
-                for (int i = warp; i < np; i += 2 * kConsumerWarps) {
-                    const int i2 = i + kConsumerWarps;
-                    const float *sp = pbase + (size_t)i * p.slot_floats;
-                    const float *sp2 = pbase + (size_t)(i2 < np ? i2 : i) * p.slot_floats;
-                    float4 o1[RB], o2[RB];
-                    float l1[RB], l2[RB];
-#pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-                        const int r = min(r0 + rb, rows_here - 1);
-                        o1[rb] = __ldcg(reinterpret_cast<const float4 *>(sp + r * kHeadDim) + lane);
-                        o2[rb] = __ldcg(reinterpret_cast<const float4 *>(sp2 + r * kHeadDim) + lane);
-                        l1[rb] = __ldcg(sp + lse_off + r);
-                        l2[rb] = __ldcg(sp2 + lse_off + r);
-                    }
-#pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-                        if (Mr[rb] == -INFINITY) continue;
-                        const float w1 = ex2((l1[rb] - Mr[rb]) * kLog2e);
-                        const float w2 = i2 < np ? ex2((l2[rb] - Mr[rb]) * kLog2e) : 0.f;
-                        a[rb].x += w1 * o1[rb].x + w2 * o2[rb].x;
-                        a[rb].y += w1 * o1[rb].y + w2 * o2[rb].y;
-                        a[rb].z += w1 * o1[rb].z + w2 * o2[rb].z;
-                        a[rb].w += w1 * o1[rb].w + w2 * o2[rb].w;
-                    }
-                }
-#pragma unroll
-                for (int rb = 0; rb < RB; ++rb) red[(warp * RB + rb) * 32 + lane] = a[rb];
-                named_sync(2, nthr);
-                const int nr = min(RB, rows_here - r0);
-                for (int idx = tid; idx < nr * 32; idx += nthr) {
-                    const int rb = idx / 32, c4 = idx % 32, r = r0 + rb;
-                    const float M = sm_m[r], ws = sm_l[r];
-                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int w = 0; w < kConsumerWarps; ++w) {
-                        const float4 x = red[(w * RB + rb) * 32 + c4];
-                        v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
-                    }
-                    const float inv = M == -INFINITY ? 0.f : 1.0f / ws;
-                    v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
-                    const int j = r / p.group, gq = r % p.group;
-                    const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-                    reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = v;
-                    if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(ws);
-                }
-                named_sync(2, nthr);
+                const float inv = M == -INFINITY ? 0.f : 1.0f / S;
+                A.x *= inv; A.y *= inv; A.z *= inv; A.w *= inv;
+                const int j = r / p.group, gq = r % p.group;
+                const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+                reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = A;
+                if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(S);
             }
             if (tid == 0) p.tickets[s_id] = 0;
             named_sync(1, kConsumerWarps * 32);
