@@ -249,9 +249,25 @@ def time_graph(g, steps, warmup, stream):
     return e0.elapsed_time(e1) / steps
 
 
+def time_decode_stream(gw, steps, stream):
+    """Average duration of one nf_decode_attn launch when the step's decode
+    launches run back to back (as they do inside the step: each may start while
+    the previous one finishes): CUDA events around replays of a graph holding
+    the decode call of every layer, divided by the number of launches."""
+    L = gw.w.layers
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for layer in range(L):
+            gw.decode(layer)
+    ms = time_graph(g, steps, 3, stream)
+    del g
+    return ms / L
+
+
 def time_decode_launches(gw, steps, stream):
-    """Average duration of one nf_decode_attn call (one fused kernel launch),
-    from CUDA events recorded around every call inside a captured graph."""
+    """Average duration of one nf_decode_attn call (one fused kernel launch)
+    timed in isolation: CUDA events recorded around every call inside a
+    captured graph (the events keep consecutive launches from overlapping)."""
     L = gw.w.layers
     ev = [(torch.cuda.Event(enable_timing=True, external=True),
            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
@@ -391,8 +407,9 @@ def main():
     tokens = w.kv_tokens_per_step()
     value = job_throughput(tokens, ws, ms)
 
-    # ---- dominant kernel: per-launch duration from events in the graph
-    dec_ms = time_decode_launches(gw, max(5, min(args.steps, 30)), stream)
+    # ---- dominant kernel: per-launch duration, back to back and in isolation
+    dec_ms = time_decode_stream(gw, max(5, min(args.steps, 30)), stream)
+    dec_iso_ms = time_decode_launches(gw, max(5, min(args.steps, 30)), stream)
     peak, peak_kind = measured_peaks()
     dec_bytes = gw.decode_bytes_per_launch()
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
@@ -447,7 +464,9 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "decode_kernel (nf_decode_attn: split-K with fused combine)", "peak_source": peak_kind,
-                     "bytes_per_launch": dec_bytes, "launch_us": dec_ms * 1e3},
+                     "bytes_per_launch": dec_bytes, "launch_us": dec_ms * 1e3,
+                     "launch_us_isolated": dec_iso_ms * 1e3,
+                     "frac_isolated": dec_bytes / (dec_iso_ms / 1e3) / 1e9 / peak},
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(tokens, ws, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
