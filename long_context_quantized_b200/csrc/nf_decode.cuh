@@ -8,13 +8,13 @@
 // section 二 and its replies).  The B200 form of that idea:
 //
 // Work: every (sequence b, kv-head h) is a segment of ceil(L_b / 32) chunks of
-//   32 keys; the chunks of all segments form one list of W chunks that the
-//   persistent grid (one CTA per SM, at most W CTAs) cuts into equal
-//   contiguous ranges, read from the device-side lengths -- ragged batches
-//   balance by keys, with no host read of the lengths.  A CTA's range covers
-//   pieces of one or more segments; all G * n_q query rows of a kv-head
-//   (GQA group x MTP queries) are served by the CTA that streams the keys, so
-//   each byte is fetched from HBM once.
+//   32 keys; the segments, each counted kSegPad chunks longer (the cost of a
+//   piece's set-up and merge), form one list that the persistent grid (one
+//   CTA per SM) cuts into equal contiguous ranges, read from the device-side
+//   lengths -- ragged batches balance by keys, with no host read of the
+//   lengths.  A CTA's range covers pieces of one or more segments; all G * n_q
+//   query rows of a kv-head (GQA group x MTP queries) are served by the CTA
+//   that streams the keys, so each byte is fetched from HBM once.
 // Pipeline: a producer warp cuts each piece into stages of up to 256 keys
 //   (64 for the bf16 cache) inside one 256-key block and moves each stage's K
 //   codes, V nibbles, K scales and V scales into a ring of shared-memory
@@ -27,29 +27,34 @@
 //   above the HBM rate.  All consumer warps work on every stage -- each takes
 //   units of 32 keys (16 for bf16) -- and release it on an "empty" mbarrier,
 //   so stages retire in order.
-// Math per 16-key m-tile ("swap AB": keys are the M dimension, query rows N = 8):
-//   S^T = K_codes . Q^T on the integer tensor cores (mma.sync m16n8k32 s8 x s8
-//   -> s32) straight from the int8 codes in shared memory: each query row is
-//   written as two int8 digits, q ~= s (d1 + d2 / 254) with s = max|q| / 127
-//   (error below 2^-16 max|q| per element), the two exact int32 dot products
-//   are recombined in fp32, and the K scale of each key multiplies the rows of
-//   S^T.  (The bf16 cache uses bf16 mma.sync instead.)
+// Math per 16-key m-tile, 8 query rows per warp (a second tile for 16 rows):
+//   S = Q . K^T on the integer tensor cores (mma.sync m16n8k32 s8 x s8 -> s32)
+//   straight from the int8 codes in shared memory.  Each query row is written
+//   as two int8 digits, q ~= s (d1 + d2 / 254) with s = max|q| / 127 (error
+//   below 2^-16 max|q| per element); A-fragment rows 0-7 hold the rows' high
+//   digits and rows 8-15 their low digits, so one product gives both, and the
+//   lane's K words land in B-fragment pairs as loaded.  The two int32 sums
+//   are recombined in fp32 and scaled by the key's K scale.  (The bf16 cache
+//   uses bf16 mma.sync the same way, the rows 8-15 holding the low half of an
+//   fp32 query.)
 //   O^T += V_codes^T . (P^T x sigma_V) (mma.sync m16n8k16 fp16, fp32
-//   accumulate): ldmatrix.trans hands each lane the nibbles of one channel for
-//   two consecutive keys, a lop3 and one fp16 op turn a pair into exact fp16
+//   accumulate): the score fragment of S is already the B-fragment layout of
+//   P^T; ldmatrix.trans hands each lane the nibbles of one channel for two
+//   consecutive keys, a lop3 and one fp16 op turn a pair into exact fp16
 //   codes -- already in A-fragment layout, with no transpose -- and, since
-//   every 16-channel m-tile lies in one 32-channel scale group, the V scale
-//   of (key, group) multiplies the weights (the B operand) instead of the
-//   values.  The weights are movmatrix-transposed scores.  The running max of
-//   a row is only raised (and O rescaled) when a tile's max exceeds it by more
-//   than 2^4, and the weights are taken relative to max + 4, so they never
-//   exceed 1 and weight x scale stays inside fp16; the cross-lane max is only
-//   reduced when some lane asks for that.
+//   every 16-channel m-tile lies in one 32-channel scale group, the V scale of
+//   (key, group) multiplies the weights (the B operand) instead of the values.
+//   The running max of a row is only raised (and O rescaled) when a tile's
+//   max exceeds it by more than 2^4, and the weights are taken relative to
+//   max + 4, so they never exceed 1 and weight x scale stays inside fp16; the
+//   cross-lane max is only reduced when some lane asks for that.
 // Merge: at the end of each piece the consumer warps merge through shared
 //   memory.  A segment owned by one CTA is written straight to out; otherwise
 //   each piece writes an (o, lse) partial and takes a ticket of the segment's
 //   counter; the CTA with the last ticket merges the partials into out and
-//   resets the counter (no CTA ever waits for another).
+//   resets the counter (no CTA ever waits for another).  When that was the
+//   CTA's last piece, one bulk copy brings the segment's partials into the
+//   then idle stage ring.
 // Every mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT
 // and the kernel runs to its end without further waits.
 #pragma once
@@ -68,6 +73,10 @@ constexpr int kMaxRows = 64;  // G * n_q per kv-head
 // The running max of a row is raised when a tile's max exceeds it by more than
 // kLazy (log2 units); weights are 2^(x - max - kLazy) <= 1.
 constexpr float kLazy = 4.0f;
+// A CTA whose range crosses into a new segment pays an extra piece set-up and
+// merge; each segment is counted kSegPad chunks longer when the work is cut,
+// so such CTAs get that many fewer keys.
+constexpr int kSegPad = 32;
 
 template <int FMT, int NT>
 struct Stage;
@@ -129,8 +138,8 @@ struct DecodeSmem {
     static constexpr int kMergeM = kMergeO + kConsumerWarps * NR * 132 * 4;    // float [warp][NR]
     static constexpr int kMergeL = kMergeM + kConsumerWarps * NR * 4;          // float [warp][NR]
     static constexpr int kMergeLse = kMergeL + kConsumerWarps * NR * 4;        // float [kMaxRows]
-    static constexpr int kBars = kMergeLse + kMaxRows * 4;                     // u64 [2][stages]
-    static constexpr int kStageOk = kBars + 2 * ST::kStages * 8;               // int [stages]
+    static constexpr int kBars = kMergeLse + kMaxRows * 4;                     // u64 [2][stages] + 1
+    static constexpr int kStageOk = kBars + (2 * ST::kStages + 1) * 8;         // int [stages]
     static constexpr int kSeqC = kStageOk + ST::kStages * 4;                   // int [kMaxBatch]
     static constexpr int kSeqBase = (kSeqC + kMaxBatch * 4 + 7) / 8 * 8;       // i64 [kMaxBatch + 1]
     static constexpr int kMisc = kSeqBase + (kMaxBatch + 1) * 8;              // int [4]
@@ -152,32 +161,35 @@ __device__ __forceinline__ int v_channel_bf16(int m, int rho) {
     const int p = 2 * m + (rho >> 3), jj = rho & 7;
     return 32 * (p >> 2) + 8 * (jj >> 1) + 2 * (p & 3) + (jj & 1);
 }
-// Physical K channel of element e (0..3) of k-step ks for lane t.
-__device__ __forceinline__ int k_channel(int fmt, int ks, int t, int e) {
-    return fmt == NF_KV_K8V4 ? 32 * t + 4 * ks + e : 32 * (ks >> 1) + 8 * t + 4 * (ks & 1) + e;
-}
-
 // Walks a CTA's chunk range piece by piece (a piece = the part of one segment
-// that falls in the range).  Producer and consumers walk it identically.
+// that falls in the range).  Positions are in "cut" units: segment s spans
+// kSegPad padding units and then its C_b chunks; base[b] is the position of
+// sequence b's first segment.  Producer and consumers walk it identically.
 struct PieceWalker {
     const int *C;              // chunks per sequence
-    const long long *base;     // first chunk of sequence b's segments
+    const long long *base;     // position of sequence b's first segment
     int H, batch;
-    long long x, end;          // next chunk, end of the CTA range
+    long long x, end;          // next position, end of the CTA range
     int b = 0;
     // current piece
     int pb, ph;                // sequence, kv-head
-    long long s0, xs, xe;      // segment start chunk, piece [xs, xe)
+    long long s0, xs, xe;      // position of the segment's first chunk, piece [xs, xe)
     __device__ bool next() {
-        if (x >= end) return false;
-        while (b + 1 <= batch && base[b + 1] <= x) ++b;
-        pb = b;
-        ph = (int)((x - base[b]) / C[b]);
-        s0 = base[b] + (long long)ph * C[b];
-        xs = x;
-        xe = min(s0 + C[b], end);
-        x = xe;
-        return true;
+        while (x < end) {
+            while (b + 1 <= batch && base[b + 1] <= x) ++b;
+            const long long span = kSegPad + (long long)C[b];
+            pb = b;
+            ph = (int)((x - base[b]) / span);
+            s0 = base[b] + (long long)ph * span + kSegPad;
+            xs = x > s0 ? x : s0;
+            xe = min(s0 + C[b], end);
+            if (xs < xe) {
+                x = xe;
+                return true;
+            }
+            x = s0 + C[b];  // the range holds only padding of this segment
+        }
+        return false;
     }
 };
 
@@ -191,6 +203,232 @@ __device__ __forceinline__ int stage_end(int cx, int cx_end) {
 
 __device__ __forceinline__ int owner_cta(long long x, long long W, int P) {
     return (int)(((x + 1) * P - 1) / W);
+}
+
+// Per-warp consumer state: the query fragments of the current (sequence,
+// kv-head) and the running softmax of the warp's rows.  In the S = Q . K^T
+// product the query rows are the M dimension: rows 0-7 of an A fragment are
+// the 8 query rows of tile nt (lane row g = query row 8nt + g), rows 8-15 a
+// second operand of the same rows -- the low int8 digit (K8/V4) or the low
+// bf16 half of an fp32 query (bf16 cache; zero for a bf16 query) -- so one
+// product yields both parts.
+template <int NT, bool QF32, int FMT>
+struct WarpState {
+    static constexpr bool K8 = FMT == NF_KV_K8V4;
+    uint32_t qa[NT][K8 ? 4 : 8][4];  // A fragments per k-step (32 channels K8/V4, 16 channels bf16)
+    float qw[NT];                    // K8/V4: s / 254 x softmax scale x log2(e) of row g; bf16: the latter
+    float m_run[NT], l_run[NT];      // running max (log2 units) and weight sum of row g (lane's keys)
+    float acc[8][NT][4];             // O^T fragments: channel rows, query columns 2t, 2t + 1
+    int lim[NT];                     // last key position row g sees (-1: padding row)
+};
+
+// Byte offsets of a lane's data inside a stage buffer, relative to the first
+// key of an m-tile.
+struct LaneOffsets {
+    uint32_t k, ks, v, vs;
+};
+
+// One work unit of a consumer warp: MT m-tiles of 16 keys starting at key ub
+// of the stage buffer st (key tok0 + ub of the segment).  FAST: every row sees
+// every key of the unit, so no mask is applied.
+template <int NT, int MT, bool QF32, int FMT, bool FAST>
+__device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const unsigned char *st, int ub,
+                                            int tok0, int L, int lane, const LaneOffsets &lo) {
+    using ST = Stage<FMT, NT>;
+    constexpr bool K8 = FMT == NF_KV_K8V4;
+    const int g = lane >> 2, t = lane & 3;
+
+    // ---- S = Q . K^T: per m-tile two n-tiles j of 8 keys; the lane's results are
+    // row g x keys tb + 8j + 2t + e (e = 0, 1) -> x[mt][nt][2j + e]
+    float xv[MT][NT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int tb = ub + 16 * mt;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            // K^T B fragments: the lane's column is key tb + 8j + g
+            if (K8) {
+                const unsigned char *k0 = st + ST::kK + (tb + 8 * j) * 128 + lo.k;  // bytes 32t..32t+31
+                const uint4 w0 = lds128(k0), w1 = lds128(k0 + 16);
+                const uint32_t kb[4][2] = {{w0.x, w0.y}, {w0.z, w0.w}, {w1.x, w1.y}, {w1.z, w1.w}};
+                // K scales of the lane's two result keys
+                const float2 sk = __half22float2(
+                    *reinterpret_cast<const __half2 *>(st + ST::kKs + (tb + 8 * j + 2 * t) * 2));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    int d[4] = {0, 0, 0, 0};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_s8(d, ws.qa[nt][ks][0], ws.qa[nt][ks][1], ws.qa[nt][ks][2], ws.qa[nt][ks][3], kb[ks][0],
+                               kb[ks][1]);
+                    // d0, d1: high digit . keys 2t, 2t+1; d2, d3: low digit.  |.| < 2^30,
+                    // the conversion rounds once (relative 2^-24)
+                    xv[mt][nt][2 * j] = (float)(d[0] * 254 + d[2]) * (ws.qw[nt] * sk.x);
+                    xv[mt][nt][2 * j + 1] = (float)(d[1] * 254 + d[3]) * (ws.qw[nt] * sk.y);
+                }
+            } else {
+                const unsigned char *k0 = st + ST::kK + (tb + 8 * j) * 256 + lo.k;  // bytes 64u + 16t .. + 15
+                uint32_t kb[8][2];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint4 w = lds128(k0 + 64 * u);
+                    kb[2 * u][0] = w.x; kb[2 * u][1] = w.y;
+                    kb[2 * u + 1][0] = w.z; kb[2 * u + 1][1] = w.w;
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16(d, ws.qa[nt][ks][0], ws.qa[nt][ks][1], ws.qa[nt][ks][2], ws.qa[nt][ks][3], kb[ks][0],
+                                 kb[ks][1]);
+                    xv[mt][nt][2 * j] = (QF32 ? d[0] + d[2] : d[0]) * ws.qw[nt];
+                    xv[mt][nt][2 * j + 1] = (QF32 ? d[1] + d[3] : d[1]) * ws.qw[nt];
+                }
+            }
+        }
+        if (!FAST) {
+            // keys past the end hold stale bytes; causal rows see keys <= lim
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int pos = tok0 + tb + 8 * (i >> 1) + 2 * t + (i & 1);
+                    if (!(pos < L && pos <= ws.lim[nt])) xv[mt][nt][i] = -INFINITY;
+                }
+        }
+    }
+
+    // ---- lazy running max of row g (the 4 lanes of a row agree on it)
+    bool raise = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        float mx = fmaxf(fmaxf(xv[0][nt][0], xv[0][nt][1]), fmaxf(xv[0][nt][2], xv[0][nt][3]));
+#pragma unroll
+        for (int mt = 1; mt < MT; ++mt)
+            mx = fmaxf(mx, fmaxf(fmaxf(xv[mt][nt][0], xv[mt][nt][1]), fmaxf(xv[mt][nt][2], xv[mt][nt][3])));
+        raise |= mx > ws.m_run[nt] + kLazy;  // true when m_run is -inf and mx finite
+    }
+    if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float mx = fmaxf(fmaxf(xv[0][nt][0], xv[0][nt][1]), fmaxf(xv[0][nt][2], xv[0][nt][3]));
+#pragma unroll
+            for (int mt = 1; mt < MT; ++mt)
+                mx = fmaxf(mx, fmaxf(fmaxf(xv[mt][nt][0], xv[mt][nt][1]), fmaxf(xv[mt][nt][2], xv[mt][nt][3])));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(ws.m_run[nt], mx);
+            const float alpha = m_new == -INFINITY ? 1.f : ex2(ws.m_run[nt] - m_new);
+            ws.m_run[nt] = m_new;
+            ws.l_run[nt] *= alpha;
+            // the accumulators hold query rows 2t and 2t + 1: take their factors
+            const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * t);
+            const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * t + 4);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                ws.acc[m][nt][0] *= a0;
+                ws.acc[m][nt][1] *= a1;
+                ws.acc[m][nt][2] *= a0;
+                ws.acc[m][nt][3] *= a1;
+            }
+        }
+    }
+    // ---- weights 2^(x - m - kLazy) <= 1, already in the B-fragment layout of
+    // the PV product: b0 = keys 2t, 2t+1 of row g, b1 = keys 8 + 2t, 9 + 2t
+    uint32_t pb[MT][NT][2], pbl[MT][NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const float mu = (ws.m_run[nt] == -INFINITY ? 0.f : ws.m_run[nt]) + kLazy;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const float p0 = ex2(xv[mt][nt][0] - mu), p1 = ex2(xv[mt][nt][1] - mu);
+            const float p2 = ex2(xv[mt][nt][2] - mu), p3 = ex2(xv[mt][nt][3] - mu);
+            ws.l_run[nt] += (p0 + p1) + (p2 + p3);
+            if (K8) {
+                pb[mt][nt][0] = pack_f16(p0, p1);
+                pb[mt][nt][1] = pack_f16(p2, p3);
+            } else {
+                // bf16 weights split into hi + lo so they keep ~16 bits
+                const uint32_t h0 = pack_bf16(p0, p1), h1 = pack_bf16(p2, p3);
+                pb[mt][nt][0] = h0;
+                pb[mt][nt][1] = h1;
+                pbl[mt][nt][0] = pack_bf16(p0 - __uint_as_float(h0 << 16), p1 - __uint_as_float(h0 & 0xFFFF0000u));
+                pbl[mt][nt][1] = pack_bf16(p2 - __uint_as_float(h1 << 16), p3 - __uint_as_float(h1 & 0xFFFF0000u));
+            }
+        }
+    }
+
+    // ---- O^T += V^T . P^T over 8 channel m-tiles, one 16-key k-tile per m-tile of the unit
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int tb = ub + 16 * mt;
+        if (K8) {
+            // nibbles: matrix cg (lanes 8cg..8cg+7 address its rows) = the 16-byte
+            // column cg (channels 32cg..32cg+31) of 8 keys, stored at column
+            // position cg ^ (row address bits 7-8) by the swizzled copy
+            uint32_t R[2][4];
+            const uint32_t va = smem_addr(st + ST::kV + tb * 64) + lo.v;
+            ldsm_x4_t(va, R[0][0], R[0][1], R[0][2], R[0][3]);            // keys tb + 0..7
+            ldsm_x4_t(va + 8 * 64, R[1][0], R[1][1], R[1][2], R[1][3]);   // keys tb + 8..15
+            // V scales of keys (2t, 2t+1) and (2t+8, 2t+9) per group, as fp16 pairs
+            uint32_t sp[2][4];
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh) {
+                const uint4 sv = lds128(st + ST::kVs + (tb + 8 * kh) * 8 + lo.vs);
+                sp[kh][0] = prmt(sv.x, sv.z, 0x5410);
+                sp[kh][1] = prmt(sv.x, sv.z, 0x7632);
+                sp[kh][2] = prmt(sv.y, sv.w, 0x5410);
+                sp[kh][3] = prmt(sv.y, sv.w, 0x7632);
+                if (!FAST) {
+                    // keys past the end hold stale bytes: zero their scales
+                    const int pa = tok0 + tb + 8 * kh + 2 * t;
+                    const uint32_t keep = (pa < L ? 0x0000FFFFu : 0u) | (pa + 1 < L ? 0xFFFF0000u : 0u);
+#pragma unroll
+                    for (int cg = 0; cg < 4; ++cg) sp[kh][cg] &= keep;
+                }
+            }
+#pragma unroll
+            for (int cg = 0; cg < 4; ++cg) {
+                // exact fp16 codes of channel 32cg + 4g + i for the key pairs
+                const uint32_t lo0 = R[0][cg], hi0 = R[0][cg] >> 8;
+                const uint32_t lo1 = R[1][cg], hi1 = R[1][cg] >> 8;
+                const uint32_t a[2][4] = {
+                    {h2_u32(nib_even(lo0)), h2_u32(nib_odd(lo0)), h2_u32(nib_even(lo1)), h2_u32(nib_odd(lo1))},
+                    {h2_u32(nib_even(hi0)), h2_u32(nib_odd(hi0)), h2_u32(nib_even(hi1)), h2_u32(nib_odd(hi1))}};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint32_t b0 = h2_u32(__hmul2(u32_h2(pb[mt][nt][0]), u32_h2(sp[0][cg])));
+                    const uint32_t b1 = h2_u32(__hmul2(u32_h2(pb[mt][nt][1]), u32_h2(sp[1][cg])));
+#pragma unroll
+                    for (int ip = 0; ip < 2; ++ip)
+                        mma_f16(ws.acc[2 * cg + ip][nt], a[ip][0], a[ip][1], a[ip][2], a[ip][3], b0, b1);
+                }
+            }
+        } else {
+            const unsigned char *v0p = st + ST::kV + tb * 256 + lo.v;
+            const bool ok0 = FAST || tok0 + tb + g < L, ok1 = FAST || tok0 + tb + g + 8 < L;
+            uint32_t w0[16], w1[16];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                uint4 va = lds128(v0p + 64 * u), vb = lds128(v0p + 8 * 256 + 64 * u);
+                if (!ok0) va = make_uint4(0, 0, 0, 0);  // stale bytes past the end
+                if (!ok1) vb = make_uint4(0, 0, 0, 0);
+                w0[4 * u] = va.x; w0[4 * u + 1] = va.y; w0[4 * u + 2] = va.z; w0[4 * u + 3] = va.w;
+                w1[4 * u] = vb.x; w1[4 * u + 1] = vb.y; w1[4 * u + 2] = vb.z; w1[4 * u + 3] = vb.w;
+            }
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const uint32_t a0 = movmatrix_t(w0[2 * m]), a1 = movmatrix_t(w0[2 * m + 1]);
+                const uint32_t a2 = movmatrix_t(w1[2 * m]), a3 = movmatrix_t(w1[2 * m + 1]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16(ws.acc[m][nt], a0, a1, a2, a3, pb[mt][nt][0], pb[mt][nt][1]);
+                    mma_bf16(ws.acc[m][nt], a0, a1, a2, a3, pbl[mt][nt][0], pbl[mt][nt][1]);
+                }
+            }
+        }
+    }
 }
 
 template <int NT, bool QF32, int FMT>
@@ -207,6 +445,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     float *sm_l = reinterpret_cast<float *>(smem + SM::kMergeL);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::kBars);
     uint64_t *empty = full + NS;
+    uint64_t *fin_bar = full + 2 * NS;  // the final merge's bulk copy
     volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + SM::kStageOk);
     int *seqC = reinterpret_cast<int *>(smem + SM::kSeqC);
     long long *seqBase = reinterpret_cast<long long *>(smem + SM::kSeqBase);
@@ -222,6 +461,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             mbar_init(&empty[i], kConsumerWarps);
             stage_ok[i] = 0;
         }
+        mbar_init(fin_bar, 1);
         misc[0] = 0;
         misc[1] = 0;
         // the stage buffers must start on 1024-byte boundaries (swizzled V
@@ -248,7 +488,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             long long acc = 0;
             for (int b = 0; b < p.batch; ++b) {
                 seqBase[b] = acc;
-                acc += (long long)seqC[b] * H;
+                acc += seqC[b] ? (long long)(seqC[b] + kSegPad) * H : 0;
             }
             seqBase[p.batch] = acc;
         }
@@ -354,40 +594,51 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     const int row0 = rg * NR;
     float *sm_lse = reinterpret_cast<float *>(smem + SM::kMergeLse);
 
-    // bf16 cache: query as bf16 (hi + lo for fp32 q) B fragments.  K8/V4: two
-    // int8 digit words per k word, and the per-row digit weights s, s / 254
-    uint32_t qf[K8 ? 1 : NT][8][2];
-    uint32_t ql[(QF32 && !K8) ? NT : 1][8][2];
-    uint32_t qd[K8 ? NT : 1][2][8];
-    float qs[K8 ? NT : 1][2];
-    float m_run[NT][2], l_run[NT][2];
-    float acc[8][NT][4];
-    int lim[NT][2];
+    WarpState<NT, QF32, FMT> ws;
+    LaneOffsets lo;
+    if (K8) {
+        lo.k = g * 128 + 32 * t;
+        lo.ks = 0;
+        // the swizzled copy puts column c of key row r at position c ^ ((r >> 1) & 3)
+        // (stage buffers and m-tiles start on 1024-byte boundaries of the V plane)
+        lo.v = (lane & 7) * 64 + ((((uint32_t)lane >> 3) ^ (((uint32_t)lane & 7) >> 1)) & 3u) * 16;
+        lo.vs = 16 * t;
+    } else {
+        lo.k = g * 256 + 16 * t;
+        lo.v = lo.k;
+        lo.ks = lo.vs = 0;
+    }
 
-    uint32_t kst = 0;
+    int stage = 0;
+    uint32_t phase = 0;      // parity of the ring's current round
+    uint32_t fin_phase = 0;  // parity of the final-merge copy barrier
     while (walk.next()) {
         const int b = walk.pb, h = walk.ph;
         const int L = seqC[b] ? p.seqlens[b] : 0;
-        // query fragments of this (sequence, kv-head), permuted like the K channels
+        // query fragments of this (sequence, kv-head): lane (g, t) holds row g of
+        // tile nt, channels 32t..32t+31 (K8/V4: k-step ks takes channels 32t + 8ks
+        // + 0..3 and + 4..7) or 32u + 8t + 4h + 0..3 (bf16 cache: k-step 2u + h)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int r = row0 + nt * 8 + g;
             const bool rv = r < p.rows;
             const int j = rv ? r / p.group : 0, gq = rv ? r % p.group : 0;
             const size_t qoff = (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim;
+            float x[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const size_t ch = qoff + (K8 ? 32 * t + c : 32 * (c >> 3) + 8 * t + (c & 7));
+                x[c] = !rv ? 0.f
+                            : QF32 ? static_cast<const float *>(p.q)[ch]
+                                   : __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[ch]);
+            }
             if (K8) {
-                // lane (g, t) holds channels 32t + 4w + e (w < 8, e < 4) of row g
-                float x[32];
                 float amax = 0.f;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    x[c] = !rv ? 0.f
-                                : QF32 ? static_cast<const float *>(p.q)[qoff + 32 * t + c]
-                                       : __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[qoff + 32 * t + c]);
-                    amax = fmaxf(amax, fabsf(x[c]));
-                }
+                for (int c = 0; c < 32; ++c) amax = fmaxf(amax, fabsf(x[c]));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+                // q ~= s (d1 + d2 / 254), s = max|q| / 127, digits in [-127, 127]
                 const float s1 = amax / 127.0f;
                 const float inv = amax > 0.f ? 127.0f / amax : 0.f;
 #pragma unroll
@@ -402,273 +653,58 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                         d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
                         d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
                     }
-                    qd[nt][0][w] = d1w;
-                    qd[nt][1][w] = d2w;
+                    // word w = 2ks + hh: A rows g (digit 1) and g + 8 (digit 2)
+                    ws.qa[nt][w >> 1][2 * (w & 1)] = d1w;
+                    ws.qa[nt][w >> 1][2 * (w & 1) + 1] = d2w;
                 }
-                // weight of the low digit (s / 254) of the rows 2t + e this lane's
-                // accumulators hold
-#pragma unroll
-                for (int e = 0; e < 2; ++e) qs[nt][e] = __shfl_sync(0xffffffffu, s1 / 254.0f, (2 * t + e) * 4);
+                ws.qw[nt] = s1 / 254.0f * p.scale_log2;
             } else {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    float x[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = k_channel(FMT, ks, t, e);
-                        if (!rv) x[e] = 0.f;
-                        else if (QF32) x[e] = static_cast<const float *>(p.q)[qoff + c];
-                        else x[e] = __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[qoff + c]);
-                    }
-                    qf[nt][ks][0] = pack_bf16(x[0], x[1]);
-                    qf[nt][ks][1] = pack_bf16(x[2], x[3]);
-                    if (QF32) {
-                        ql[nt][ks][0] = pack_bf16(x[0] - __uint_as_float(qf[nt][ks][0] << 16),
-                                                  x[1] - __uint_as_float(qf[nt][ks][0] & 0xFFFF0000u));
-                        ql[nt][ks][1] = pack_bf16(x[2] - __uint_as_float(qf[nt][ks][1] << 16),
-                                                  x[3] - __uint_as_float(qf[nt][ks][1] & 0xFFFF0000u));
-                    }
+                for (int w = 0; w < 16; ++w) {
+                    // word w = 2 (2u + hh) + e2 holds channels 32u + 8t + 4hh + 2e2 + 0..1
+                    const uint32_t hi = pack_bf16(x[2 * w], x[2 * w + 1]);
+                    const uint32_t lo_ = QF32 ? pack_bf16(x[2 * w] - __uint_as_float(hi << 16),
+                                                          x[2 * w + 1] - __uint_as_float(hi & 0xFFFF0000u))
+                                              : 0u;
+                    ws.qa[nt][w >> 1][2 * (w & 1)] = hi;
+                    ws.qa[nt][w >> 1][2 * (w & 1) + 1] = lo_;
                 }
+                ws.qw[nt] = p.scale_log2;
             }
+            ws.lim[nt] = !rv ? -1 : (p.causal ? L - p.n_q + r / p.group : L - 1);
+            ws.m_run[nt] = -INFINITY;
+            ws.l_run[nt] = 0.f;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int rr = row0 + nt * 8 + 2 * t + e;
-                lim[nt][e] = rr >= p.rows ? -1 : (p.causal ? L - p.n_q + rr / p.group : L - 1);
-                m_run[nt][e] = -INFINITY;
-                l_run[nt][e] = 0.f;
-            }
-#pragma unroll
-            for (int m = 0; m < 8; ++m) acc[m][nt][0] = acc[m][nt][1] = acc[m][nt][2] = acc[m][nt][3] = 0.f;
+            for (int m = 0; m < 8; ++m) ws.acc[m][nt][0] = ws.acc[m][nt][1] = ws.acc[m][nt][2] = ws.acc[m][nt][3] = 0.f;
         }
         // keys every row of the group sees, for the no-mask fast path
         const int all_see = p.causal ? L - p.n_q + 1 : L;
 
         const int cx1 = (int)(walk.xe - walk.s0);
-        for (int cx = (int)(walk.xs - walk.s0); cx < cx1; ++kst) {
+        for (int cx = (int)(walk.xs - walk.s0); cx < cx1;) {
             const int ce = stage_end<FMT, NT>(cx, cx1);
-            const int tok0 = cx * kChunk, n_mt = (ce - cx) * (kChunk / 16);
+            const int tok0 = cx * kChunk, n_units = (ce - cx) * (kChunk / (16 * MT));
             cx = ce;
-            const int stage = (int)(kst % NS);
-            if (!misc[0] && !mbar_wait(&full[stage], (kst / NS) & 1)) {
+            if (!misc[0] && !mbar_wait(&full[stage], phase)) {
                 report(NF_DEVERR_TIMEOUT);
                 misc[0] = 1;
             }
             if (!misc[0] && stage_ok[stage]) {
                 const unsigned char *st = smem + stage * ST::kStride;
-                const int n_units = n_mt / MT;  // stages hold whole 32-key chunks
                 for (int un = slot; un < n_units; un += CW) {
-                    const int ubase = tok0 + 16 * MT * un;                // first key of the unit
-                    const bool fast = ubase + 16 * MT <= all_see;          // every row sees every key
-
-                    // ---- S^T = K . Q^T for the unit's MT m-tiles of 16 keys
-                    float s[MT][NT][4];
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const int tau0 = 16 * (MT * un + mt) + g;          // key of this lane in the stage
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) s[mt][nt][0] = s[mt][nt][1] = s[mt][nt][2] = s[mt][nt][3] = 0.f;
-                        if (K8) {
-                            const unsigned char *k0 = st + ST::kK + tau0 * 128 + 32 * t;
-                            const uint4 ka0 = lds128(k0), ka1 = lds128(k0 + 16);
-                            const uint4 kb0 = lds128(k0 + 8 * 128), kb1 = lds128(k0 + 8 * 128 + 16);
-                            const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
-                            const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                int d1[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};
-#pragma unroll
-                                for (int ks = 0; ks < 4; ++ks) {
-                                    mma_s8(d1, wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
-                                           qd[nt][0][2 * ks], qd[nt][0][2 * ks + 1]);
-                                    mma_s8(d2, wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
-                                           qd[nt][1][2 * ks], qd[nt][1][2 * ks + 1]);
-                                }
-                                // |d1 * 254 + d2| < 2^24: exact in fp32
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) s[mt][nt][i] = qs[nt][i & 1] * (float)(d1[i] * 254 + d2[i]);
-                            }
-                        } else {
-                            const unsigned char *k0 = st + ST::kK + tau0 * 256 + 16 * t;
-                            uint32_t wa[16], wb[16];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const uint4 va = lds128(k0 + 64 * u), vb = lds128(k0 + 8 * 256 + 64 * u);
-                                wa[4 * u] = va.x; wa[4 * u + 1] = va.y; wa[4 * u + 2] = va.z; wa[4 * u + 3] = va.w;
-                                wb[4 * u] = vb.x; wb[4 * u + 1] = vb.y; wb[4 * u + 2] = vb.z; wb[4 * u + 3] = vb.w;
-                            }
-#pragma unroll
-                            for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    mma_bf16(s[mt][nt], wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
-                                             qf[nt][ks][0], qf[nt][ks][1]);
-                                    if (QF32)
-                                        mma_bf16(s[mt][nt], wa[2 * ks], wb[2 * ks], wa[2 * ks + 1], wb[2 * ks + 1],
-                                                 ql[nt][ks][0], ql[nt][ks][1]);
-                                }
-                            }
-                        }
-                    }
-
-                    // ---- scores in the log2 domain; rows 8nt + 2t + e, keys tau0 / tau0 + 8 of each m-tile
-                    float xv[MT][NT][4];
-                    bool kv_ok[MT][2];
-                    bool raise = false;
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const int tau0 = 16 * (MT * un + mt) + g;
-                        const int pos0 = tok0 + tau0, pos1 = pos0 + 8;
-                        kv_ok[mt][0] = fast || pos0 < L;
-                        kv_ok[mt][1] = fast || pos1 < L;
-                        const float c0 = (K8 ? __half2float(reinterpret_cast<const __half *>(st + ST::kKs)[tau0]) : 1.0f) * p.scale_log2;
-                        const float c1 = (K8 ? __half2float(reinterpret_cast<const __half *>(st + ST::kKs)[tau0 + 8]) : 1.0f) * p.scale_log2;
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                float x0 = s[mt][nt][e] * c0, x1 = s[mt][nt][2 + e] * c1;
-                                if (!fast) {
-                                    if (!(kv_ok[mt][0] && pos0 <= lim[nt][e])) x0 = -INFINITY;
-                                    if (!(kv_ok[mt][1] && pos1 <= lim[nt][e])) x1 = -INFINITY;
-                                }
-                                xv[mt][nt][e] = x0;
-                                xv[mt][nt][2 + e] = x1;
-                            }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            float mx = fmaxf(xv[0][nt][e], xv[0][nt][2 + e]);
-#pragma unroll
-                            for (int mt = 1; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(xv[mt][nt][e], xv[mt][nt][2 + e]));
-                            raise |= mx > m_run[nt][e] + kLazy;  // true when m_run is -inf and mx finite
-                        }
-                    if (__any_sync(0xffffffffu, raise)) {
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                float mx = fmaxf(xv[0][nt][e], xv[0][nt][2 + e]);
-#pragma unroll
-                                for (int mt = 1; mt < MT; ++mt) mx = fmaxf(mx, fmaxf(xv[mt][nt][e], xv[mt][nt][2 + e]));
-                                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                                const float m_new = fmaxf(m_run[nt][e], mx);
-                                const float alpha = m_new == -INFINITY ? 1.f : ex2(m_run[nt][e] - m_new);
-                                m_run[nt][e] = m_new;
-                                l_run[nt][e] *= alpha;
-#pragma unroll
-                                for (int m = 0; m < 8; ++m) {
-                                    acc[m][nt][e] *= alpha;
-                                    acc[m][nt][2 + e] *= alpha;
-                                }
-                            }
-                    }
-                    // weights 2^(x - m - kLazy) <= 1 (P^T) as B fragments of the PV product
-                    uint32_t pb[MT][NT][2], pbl[MT][NT][2];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const float mu0 = (m_run[nt][0] == -INFINITY ? 0.f : m_run[nt][0]) + kLazy;
-                        const float mu1 = (m_run[nt][1] == -INFINITY ? 0.f : m_run[nt][1]) + kLazy;
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt) {
-                            const float p00 = ex2(xv[mt][nt][0] - mu0), p01 = ex2(xv[mt][nt][1] - mu1);
-                            const float p10 = ex2(xv[mt][nt][2] - mu0), p11 = ex2(xv[mt][nt][3] - mu1);
-                            l_run[nt][0] += p00 + p10;
-                            l_run[nt][1] += p01 + p11;
-                            if (K8) {
-                                pb[mt][nt][0] = movmatrix_t(pack_f16(p00, p01));
-                                pb[mt][nt][1] = movmatrix_t(pack_f16(p10, p11));
-                            } else {
-                                // bf16 weights split into hi + lo so they keep ~16 bits
-                                const uint32_t h0 = pack_bf16(p00, p01), h1 = pack_bf16(p10, p11);
-                                pb[mt][nt][0] = movmatrix_t(h0);
-                                pb[mt][nt][1] = movmatrix_t(h1);
-                                pbl[mt][nt][0] = movmatrix_t(pack_bf16(p00 - __uint_as_float(h0 << 16),
-                                                                       p01 - __uint_as_float(h0 & 0xFFFF0000u)));
-                                pbl[mt][nt][1] = movmatrix_t(pack_bf16(p10 - __uint_as_float(h1 << 16),
-                                                                       p11 - __uint_as_float(h1 & 0xFFFF0000u)));
-                            }
-                        }
-                    }
-
-                    // ---- O^T += V^T . P^T over 8 channel m-tiles, one 16-key k-tile per m-tile of the unit
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        const int tb = 16 * (MT * un + mt);  // first key of the m-tile in the stage
-                        if (K8) {
-                            // nibbles: matrix cg (lanes 8cg..8cg+7 address its rows) = the
-                            // 16-byte column cg (channels 32cg..32cg+31) of 8 keys; the
-                            // column sits at position cg ^ (row address bits 7-8)
-                            uint32_t R[2][4];
-                            const uint32_t vrow = smem_addr(st + ST::kV) + (uint32_t)(tb + (lane & 7)) * 64u;
-                            const uint32_t vaddr = vrow + ((((uint32_t)lane >> 3) ^ ((vrow >> 7) & 3u)) << 4);
-                            ldsm_x4_t(vaddr, R[0][0], R[0][1], R[0][2], R[0][3]);            // keys tb + 0..7
-                            ldsm_x4_t(vaddr + 8 * 64, R[1][0], R[1][1], R[1][2], R[1][3]);   // keys tb + 8..15
-                            // V scales of keys (2t, 2t+1) and (2t+8, 2t+9) per group, as fp16 pairs
-                            uint32_t sp[2][4];
-#pragma unroll
-                            for (int kh = 0; kh < 2; ++kh) {
-                                const uint4 sv = lds128(st + ST::kVs + (tb + 8 * kh + 2 * t) * 8);
-                                sp[kh][0] = prmt(sv.x, sv.z, 0x5410);
-                                sp[kh][1] = prmt(sv.x, sv.z, 0x7632);
-                                sp[kh][2] = prmt(sv.y, sv.w, 0x5410);
-                                sp[kh][3] = prmt(sv.y, sv.w, 0x7632);
-                                if (!fast) {
-                                    // keys past the end hold stale bytes: zero their scales
-                                    const int pa = tok0 + tb + 8 * kh + 2 * t;
-                                    const uint32_t keep = (pa < L ? 0x0000FFFFu : 0u) | (pa + 1 < L ? 0xFFFF0000u : 0u);
-#pragma unroll
-                                    for (int cg = 0; cg < 4; ++cg) sp[kh][cg] &= keep;
-                                }
-                            }
-#pragma unroll
-                            for (int cg = 0; cg < 4; ++cg) {
-                                // exact fp16 codes of channel 32cg + 4g + i for the key pairs
-                                const uint32_t lo0 = R[0][cg], hi0 = R[0][cg] >> 8;
-                                const uint32_t lo1 = R[1][cg], hi1 = R[1][cg] >> 8;
-                                const uint32_t a[2][4] = {
-                                    {h2_u32(nib_even(lo0)), h2_u32(nib_odd(lo0)), h2_u32(nib_even(lo1)), h2_u32(nib_odd(lo1))},
-                                    {h2_u32(nib_even(hi0)), h2_u32(nib_odd(hi0)), h2_u32(nib_even(hi1)), h2_u32(nib_odd(hi1))}};
-#pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    const uint32_t b0 = h2_u32(__hmul2(u32_h2(pb[mt][nt][0]), u32_h2(sp[0][cg])));
-                                    const uint32_t b1 = h2_u32(__hmul2(u32_h2(pb[mt][nt][1]), u32_h2(sp[1][cg])));
-#pragma unroll
-                                    for (int ip = 0; ip < 2; ++ip)
-                                        mma_f16(acc[2 * cg + ip][nt], a[ip][0], a[ip][1], a[ip][2], a[ip][3], b0, b1);
-                                }
-                            }
-                        } else {
-                            const int tau0 = tb + g;
-                            const unsigned char *v0p = st + ST::kV + tau0 * 256 + 16 * t;
-                            uint32_t w0[16], w1[16];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                uint4 va = lds128(v0p + 64 * u), vb = lds128(v0p + 8 * 256 + 64 * u);
-                                if (!kv_ok[mt][0]) va = make_uint4(0, 0, 0, 0);
-                                if (!kv_ok[mt][1]) vb = make_uint4(0, 0, 0, 0);
-                                w0[4 * u] = va.x; w0[4 * u + 1] = va.y; w0[4 * u + 2] = va.z; w0[4 * u + 3] = va.w;
-                                w1[4 * u] = vb.x; w1[4 * u + 1] = vb.y; w1[4 * u + 2] = vb.z; w1[4 * u + 3] = vb.w;
-                            }
-#pragma unroll
-                            for (int m = 0; m < 8; ++m) {
-                                const uint32_t a0 = movmatrix_t(w0[2 * m]), a1 = movmatrix_t(w0[2 * m + 1]);
-                                const uint32_t a2 = movmatrix_t(w1[2 * m]), a3 = movmatrix_t(w1[2 * m + 1]);
-#pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    mma_bf16(acc[m][nt], a0, a1, a2, a3, pb[mt][nt][0], pb[mt][nt][1]);
-                                    mma_bf16(acc[m][nt], a0, a1, a2, a3, pbl[mt][nt][0], pbl[mt][nt][1]);
-                                }
-                            }
-                        }
-                    }
+                    const int ub = 16 * MT * un;  // first key of the unit in the stage
+                    if (tok0 + ub + 16 * MT <= all_see)
+                        decode_unit<NT, MT, QF32, FMT, true>(ws, st, ub, tok0, L, lane, lo);
+                    else
+                        decode_unit<NT, MT, QF32, FMT, false>(ws, st, ub, tok0, L, lane, lo);
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == NS) {
+                stage = 0;
+                phase ^= 1u;
+            }
         }
 
         // ---- merge the consumer warps of each row group (shared memory)
@@ -678,19 +714,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         const int n_pieces = last - first + 1;
         const int rows_here = p.rows;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float l = l_run[nt][e];
-                l += __shfl_xor_sync(0xffffffffu, l, 4);
-                l += __shfl_xor_sync(0xffffffffu, l, 8);
-                l += __shfl_xor_sync(0xffffffffu, l, 16);
-                const int rr = nt * 8 + 2 * t + e;
-                if (g == 0) {
-                    sm_m[warp * NR + rr] = m_run[nt][e];
-                    sm_l[warp * NR + rr] = l;
-                }
+        for (int nt = 0; nt < NT; ++nt) {
+            float l = ws.l_run[nt];
+            l += __shfl_xor_sync(0xffffffffu, l, 1);
+            l += __shfl_xor_sync(0xffffffffu, l, 2);
+            if (t == 0) {
+                sm_m[warp * NR + nt * 8 + g] = ws.m_run[nt];
+                sm_l[warp * NR + nt * 8 + g] = l;
             }
+        }
         named_sync(1, kConsumerWarps * 32);
         // each lane derives its rows' factor f_w = 2^(m_w - M) / sum_v l_v 2^(m_v - M)
         // from the group's (m, l) and writes f_w * acc_w to its warp's buffer
@@ -708,7 +740,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                         float ls = 0.f;
                         for (int w = 0; w < CW; ++w)
                             ls += sm_l[(rg * CW + w) * NR + rr] * ex2(sm_m[(rg * CW + w) * NR + rr] - M);
-                        f = ex2(m_run[nt][e] - M) / ls;
+                        f = ex2(sm_m[warp * NR + rr] - M) / ls;
                         // the row's lse: weights were taken relative to m + kLazy
                         if (slot == 0 && g == 0) sm_lse[row0 + rr] = (M + kLazy + log2f(ls)) * 0.69314718055994531f;
                     } else if (slot == 0 && g == 0) {
@@ -718,8 +750,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                     for (int m = 0; m < 8; ++m) {
                         const int c0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
                         const int c1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
-                        buf[rr * 132 + c0] = acc[m][nt][e] * f;
-                        buf[rr * 132 + c1] = acc[m][nt][2 + e] * f;
+                        buf[rr * 132 + c0] = ws.acc[m][nt][e] * f;
+                        buf[rr * 132 + c1] = ws.acc[m][nt][2 + e] * f;
                     }
                 }
         }
@@ -764,15 +796,55 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         named_sync(1, kConsumerWarps * 32);
         if (misc[1]) {
             // This CTA holds the last ticket: merge every piece of the segment.
-            // Each thread owns (row, 4 channels) and streams the pieces' o and
-            // lse from L2 (loads bypass L1), kPB pieces' loads in flight at once,
-            // keeping a running max, weight sum and weighted sum.
+            // Each thread owns (row, 4 channels): weights 2^(lse_i - M) over the
+            // pieces' (o_i, lse_i), normalised.  When this was the CTA's last
+            // piece the stage ring is free: one bulk copy brings all the pieces'
+            // slots (consecutive in the workspace) into it.  Otherwise the
+            // slots stream from L2, kPB pieces' loads in flight at once.
             constexpr int kPB = 16;
             constexpr float kLog2e = 1.4426950408889634f;
             const int nthr = kConsumerWarps * 32, tid = threadIdx.x;
             const int np = last - first + 1;
             const float *pbase = p.partials + (size_t)(s_id + first) * p.slot_floats;
             const int lse_off = rows_here * kHeadDim;
+            const uint32_t fin_bytes = (uint32_t)np * (uint32_t)p.slot_floats * 4u;
+            if (walk.x >= walk.end && fin_bytes <= (uint32_t)(NS * ST::kStride)) {
+                if (tid == 0) {
+                    // the ring's last reads (generic proxy) precede the copy's writes
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_arrive_expect_tx(fin_bar, fin_bytes);
+                    bulk_g2s(smem, pbase, fin_bytes, fin_bar);
+                }
+                if (!misc[0] && !mbar_wait(fin_bar, fin_phase)) {
+                    report(NF_DEVERR_TIMEOUT);
+                    misc[0] = 1;
+                }
+                fin_phase ^= 1u;
+                const float *ps = reinterpret_cast<const float *>(smem);
+                for (int it = tid; it < rows_here * (kHeadDim / 4); it += nthr) {
+                    const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
+                    float M = -INFINITY;
+                    for (int i = 0; i < np; ++i) M = fmaxf(M, ps[(size_t)i * p.slot_floats + lse_off + r]);
+                    float S = 0.f;
+                    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (M != -INFINITY) {
+                        for (int i = 0; i < np; ++i) {
+                            const float *sp = ps + (size_t)i * p.slot_floats;
+                            const float li = sp[lse_off + r];
+                            const float wk = li == -INFINITY ? 0.f : ex2((li - M) * kLog2e);
+                            const float4 o = reinterpret_cast<const float4 *>(sp + r * kHeadDim)[c4];
+                            S += wk;
+                            A.x += wk * o.x; A.y += wk * o.y; A.z += wk * o.z; A.w += wk * o.w;
+                        }
+                    }
+                    const float inv = M == -INFINITY ? 0.f : 1.0f / S;
+                    A.x *= inv; A.y *= inv; A.z *= inv; A.w *= inv;
+                    const int j = r / p.group, gq = r % p.group;
+                    const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+                    reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = A;
+                    if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(S);
+                }
+            } else {
             for (int it = tid; it < rows_here * (kHeadDim / 4); it += nthr) {
                 const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
                 float M = -INFINITY, S = 0.f;
@@ -812,6 +884,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
                 reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = A;
                 if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(S);
+            }
             }
             if (tid == 0) p.tickets[s_id] = 0;
             named_sync(1, kConsumerWarps * 32);
