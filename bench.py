@@ -167,6 +167,8 @@ class GpuWorkload:
         self.w = w
         self.dev = device
         self.fmt = nf.NF_KV_K8V4 if fmt_name == "k8v4" else nf.NF_KV_BF16
+        self.decode_flags = nf.NF_DECODE_EARLY_KV
+        assert w.n_new in (0, w.n_q), "the early-KV guarantee needs n_new == n_q"
         bt = workloads.block_table(w)
         self.bt = torch.as_tensor(bt, dtype=torch.int32, device=device)
         self.seqlens = torch.as_tensor(w.seqlens, dtype=torch.int32, device=device)
@@ -200,9 +202,12 @@ class GpuWorkload:
             self.nf.nf_kv_append_quant(self.layers[layer], self.knew[layer], self.vnew[layer], self.bt, self.before)
 
     def decode(self, layer):
+        # the step appends (when it appends) exactly the n_q newest tokens right
+        # before each decode, and lengths and tables stay fixed: the early-KV
+        # guarantee of nf_decode_attn_ex holds
         w = self.w
-        self.nf.nf_decode_attn(self.layers[layer], self.q[layer], self.bt, self.seqlens, self.max_seqlen,
-                               w.softmax_scale, w.causal, self.out[layer], None, self.ws)
+        self.nf.nf_decode_attn_ex(self.layers[layer], self.q[layer], self.bt, self.seqlens, self.max_seqlen,
+                                  w.softmax_scale, w.causal, self.decode_flags, self.out[layer], None, self.ws)
 
     def step(self):
         for layer in range(self.w.layers):
@@ -459,7 +464,8 @@ def main():
         "config": {"workload": w.name, "batch": w.batch, "seqlens": list(w.seqlens), "n_q": w.n_q,
                    "n_new": w.n_new, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
                    "layers": w.layers, "kv_format": args.kv_format, "causal": w.causal,
-                   "l2": l2_note, "timing": "CUDA graph of one step, CUDA events, max over ranks"},
+                   "l2": l2_note, "timing": "CUDA graph of one step, CUDA events, max over ranks",
+                   "decode_flags": "NF_DECODE_EARLY_KV"},
         "step_gbs": gw.step_bytes() / (ms / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,

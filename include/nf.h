@@ -172,16 +172,46 @@ size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_h
  *   Calls that share a workspace must not overlap on the GPU.
  * Supported: batch <= 256, (num_q_heads / num_kv_heads) * n_q <= 64; other
  *   shapes return NF_ERR_UNSUPPORTED.
- * Numerics: dequantised keys are used exactly; the fp32 query is split into two
- *   fp16 halves (bf16 queries are converted to fp16); each dequantised value
- *   and each softmax weight is rounded to fp16 before the tensor-core P.V
- *   product; scores, softmax statistics and accumulators are fp32.
+ * Numerics (K8/V4): the K codes enter the integer tensor cores exactly and each
+ *   query row as two int8 digits, q ~= s (d1 + d2 / 254) with s = max|q| / 127
+ *   (error below 2^-16 max|q| per element); the V codes are exact in fp16 and
+ *   each softmax weight times its V scale is rounded to fp16 before the
+ *   tensor-core P.V product; scores, softmax statistics and accumulators are
+ *   fp32.  (bf16 cache: bf16 products, the fp32 query and the weights split
+ *   into bf16 high and low parts.)
+ * Launch: the kernel is launched with programmatic dependent launch, so it may
+ *   start while the previous kernel on `stream` finishes; it waits for that
+ *   kernel before reading any argument (see nf_decode_attn_ex for a weaker
+ *   wait).
  */
 nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
                          int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
                          int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
                          float softmax_scale, int32_t causal, float *out, float *out_lse,
                          void *workspace, size_t workspace_bytes, nf_stream_t stream);
+
+/*
+ * nf_decode_attn_ex -- nf_decode_attn with flags.
+ *
+ * NF_DECODE_EARLY_KV: start streaming the cache before the previous kernel on
+ *   `stream` has finished.  The caller guarantees that the kernels still
+ *   running when this call's kernel starts write neither seqlens, nor
+ *   block_table, nor any pool row at a position < seqlens[b] - n_q (they may
+ *   write the rows of the n_q newest positions, as nf_kv_append_quant does for
+ *   the tokens of a decode or verification step).  The kernel then reads the
+ *   lengths, the tables and the older rows at once, and waits for the previous
+ *   kernel before it reads q or the newest rows and before it writes out,
+ *   out_lse or the workspace.  This hides the start-up of each call behind the
+ *   end of the previous one in a sequence of layers.  Without the guarantee
+ *   the results are undefined; nf_decode_attn is this call with flags = 0.
+ * Other bits must be zero (NF_ERR_INVALID_ARG).
+ */
+#define NF_DECODE_EARLY_KV 1u
+nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                            int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                            int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                            float softmax_scale, int32_t causal, uint32_t flags, float *out,
+                            float *out_lse, void *workspace, size_t workspace_bytes, nf_stream_t stream);
 
 /*
  * nf_decode_attn_noalloc -- nf_decode_attn for callers that cannot allocate

@@ -77,6 +77,9 @@ def load_library():
         lib.nf_decode_attn_workspace_size.restype = S
         lib.nf_decode_attn.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, P, P, P, S, P]
         lib.nf_decode_attn.restype = I
+        lib.nf_decode_attn_ex.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, ctypes.c_uint32, P, P,
+                                          P, S, P]
+        lib.nf_decode_attn_ex.restype = I
         lib.nf_decode_attn_noalloc.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, P, P, P]
         lib.nf_decode_attn_noalloc.restype = I
         lib.nf_attn_combine.argtypes = [P, P, I, I, I, P, P, P]
@@ -193,10 +196,22 @@ def nf_decode_attn_workspace_size(batch, n_q, num_q_heads, num_kv_heads, max_seq
                                                             max_seqlen, num_sms))
 
 
+NF_DECODE_EARLY_KV = 1
+
+
 def nf_decode_attn(kv: KVLayer, q, block_table, seqlens, max_seqlen: int, softmax_scale: float,
                    causal: bool, out, out_lse=None, workspace=None, stream=None):
     """Decode attention; q [batch][n_q][H_q][128] (fp32 or bf16), out fp32 of
     the same shape, out_lse fp32 [batch][n_q][H_q] or None (see nf.h)."""
+    nf_decode_attn_ex(kv, q, block_table, seqlens, max_seqlen, softmax_scale, causal, 0, out, out_lse,
+                      workspace, stream, _name="nf_decode_attn")
+
+
+def nf_decode_attn_ex(kv: KVLayer, q, block_table, seqlens, max_seqlen: int, softmax_scale: float,
+                      causal: bool, flags: int, out, out_lse=None, workspace=None, stream=None,
+                      _name="nf_decode_attn_ex"):
+    """nf_decode_attn with flags (NF_DECODE_EARLY_KV: see nf.h for the caller's
+    guarantee)."""
     _need(q, "q")
     _need(block_table, "block_table", torch.int32)
     _need(seqlens, "seqlens", torch.int32)
@@ -205,14 +220,14 @@ def nf_decode_attn(kv: KVLayer, q, block_table, seqlens, max_seqlen: int, softma
     _need(workspace, "workspace")
     B, n_q, H_q = q.shape[0], q.shape[1], q.shape[2]
     if workspace is None:
-        raise NfError(NF_ERR_WORKSPACE, "nf_decode_attn", "workspace tensor required "
+        raise NfError(NF_ERR_WORKSPACE, _name, "workspace tensor required "
                       "(size: nf_decode_attn_workspace_size)")
     ws_bytes = workspace.numel() * workspace.element_size()
-    st = load_library().nf_decode_attn(
+    st = load_library().nf_decode_attn_ex(
         ctypes.byref(kv.c), _dptr(q), _dtype_code(q.dtype), B, n_q, H_q, _dptr(block_table),
         block_table.shape[1], _dptr(seqlens), int(max_seqlen), float(softmax_scale), int(bool(causal)),
-        _dptr(out), _dptr(out_lse), _dptr(workspace), ws_bytes, _stream(stream))
-    _check(st, "nf_decode_attn")
+        int(flags), _dptr(out), _dptr(out_lse), _dptr(workspace), ws_bytes, _stream(stream))
+    _check(st, _name)
 
 
 NF_NOALLOC_SCRATCH_BYTES = 8 << 20

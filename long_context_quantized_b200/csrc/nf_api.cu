@@ -265,6 +265,17 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
                          int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
                          float softmax_scale, int32_t causal, float *out, float *out_lse,
                          void *workspace, size_t workspace_bytes, nf_stream_t stream) {
+    return nf_decode_attn_ex(kv, q, q_dtype, batch, n_q, num_q_heads, block_table, max_blocks, seqlens,
+                             max_seqlen, softmax_scale, causal, 0u, out, out_lse, workspace, workspace_bytes,
+                             stream);
+}
+
+nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                            int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                            int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                            float softmax_scale, int32_t causal, uint32_t flags, float *out,
+                            float *out_lse, void *workspace, size_t workspace_bytes, nf_stream_t stream) {
+    if (flags & ~NF_DECODE_EARLY_KV) return fail(NF_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
     nf_status st = check_layer(kv);
     if (st != NF_OK) return st;
     if (q_dtype != NF_F32 && q_dtype != NF_BF16)
@@ -321,6 +332,7 @@ nf_status nf_decode_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, 
     p.max_seqlen = max_seqlen;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.causal = causal != 0;
+    p.early_kv = (flags & NF_DECODE_EARLY_KV) != 0;
     p.out = out;
     p.out_lse = out_lse;
     p.tickets = static_cast<int32_t *>(workspace);

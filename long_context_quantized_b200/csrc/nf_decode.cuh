@@ -76,7 +76,7 @@ constexpr float kLazy = 4.0f;
 // A CTA whose range crosses into a new segment pays an extra piece set-up and
 // merge; each segment is counted kSegPad chunks longer when the work is cut,
 // so such CTAs get that many fewer keys.
-constexpr int kSegPad = 32;
+constexpr int kSegPad = 64;
 
 template <int FMT, int NT>
 struct Stage;
@@ -122,6 +122,7 @@ struct DecodeParams {
     int max_seqlen;
     float scale_log2;  // softmax_scale * log2(e)
     int causal;
+    int early_kv;      // read lengths, tables and older pool rows before the dependency wait
     float *out;      // [batch][n_q][H_q][128]
     float *out_lse;  // [batch][n_q][H_q] or null
     int32_t *tickets;  // [batch * H_kv], zero between calls
@@ -141,7 +142,8 @@ struct DecodeSmem {
     static constexpr int kBars = kMergeLse + kMaxRows * 4;                     // u64 [2][stages] + 1
     static constexpr int kStageOk = kBars + (2 * ST::kStages + 1) * 8;         // int [stages]
     static constexpr int kSeqC = kStageOk + ST::kStages * 4;                   // int [kMaxBatch]
-    static constexpr int kSeqBase = (kSeqC + kMaxBatch * 4 + 7) / 8 * 8;       // i64 [kMaxBatch + 1]
+    static constexpr int kSeqL = kSeqC + kMaxBatch * 4;                        // int [kMaxBatch]
+    static constexpr int kSeqBase = (kSeqL + kMaxBatch * 4 + 7) / 8 * 8;       // i64 [kMaxBatch + 1]
     static constexpr int kMisc = kSeqBase + (kMaxBatch + 1) * 8;              // int [4]
     static constexpr int kBytes = kMisc + 16;
     static_assert(kBytes <= 232448, "shared memory per CTA");
@@ -431,6 +433,56 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
     }
 }
 
+// Log-sum-exp merge of np pieces' (o, lse) for row r, channels 4c4..4c4+3:
+// M = max lse_i, S = sum_i 2^((lse_i - M) log2 e), A = sum_i that weight x o_i,
+// in piece order.  Pieces are slots of slot_floats floats from `ps`: o at
+// [r][128], lse at lse_off + r.  SMEM: plain loads from shared memory;
+// otherwise loads that bypass L1 (the slots were written by other CTAs), kPB
+// pieces in flight at once.  The arithmetic is the same for both sources.
+template <bool SMEM>
+__device__ __forceinline__ void merge_pieces(const float *ps, int slot_floats, int np, int r, int c4, int lse_off,
+                                             float &M, float &S, float4 &A) {
+    constexpr int kPB = 16;
+    constexpr float kLog2e = 1.4426950408889634f;
+    auto ld1 = [&](const float *a) { return SMEM ? *a : __ldcg(a); };
+    M = -INFINITY;
+    S = 0.f;
+    A = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < np; i0 += kPB) {
+        float l[kPB];
+#pragma unroll
+        for (int k = 0; k < kPB; ++k) l[k] = i0 + k < np ? ld1(ps + (size_t)(i0 + k) * slot_floats + lse_off + r) : -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kPB; ++k) M = fmaxf(M, l[k]);
+    }
+    if (M == -INFINITY) return;
+    for (int i0 = 0; i0 < np; i0 += kPB) {
+        float4 o[kPB];
+        float l[kPB];
+#pragma unroll
+        for (int k = 0; k < kPB; ++k) {
+            const float *sp = ps + (size_t)(i0 + k) * slot_floats;
+            if (i0 + k < np) {
+                const float4 *op = reinterpret_cast<const float4 *>(sp + r * kHeadDim) + c4;
+                o[k] = SMEM ? *op : __ldcg(op);
+                l[k] = ld1(sp + lse_off + r);
+            } else {
+                o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                l[k] = -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kPB; ++k) {
+            const float wk = l[k] == -INFINITY ? 0.f : ex2((l[k] - M) * kLog2e);
+            S += wk;
+            A.x = fmaf(wk, o[k].x, A.x);
+            A.y = fmaf(wk, o[k].y, A.y);
+            A.z = fmaf(wk, o[k].z, A.z);
+            A.w = fmaf(wk, o[k].w, A.w);
+        }
+    }
+}
+
 template <int NT, bool QF32, int FMT>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     using ST = Stage<FMT, NT>;
@@ -448,6 +500,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     uint64_t *fin_bar = full + 2 * NS;  // the final merge's bulk copy
     volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + SM::kStageOk);
     int *seqC = reinterpret_cast<int *>(smem + SM::kSeqC);
+    int *seqL = reinterpret_cast<int *>(smem + SM::kSeqL);
     long long *seqBase = reinterpret_cast<long long *>(smem + SM::kSeqBase);
     volatile int *misc = reinterpret_cast<volatile int *>(smem + SM::kMisc);  // [0] abort, [1] last-ticket
 
@@ -473,8 +526,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         fence_mbar_init();
     }
     // everything above touched shared memory only; the lengths, tables, query,
-    // pool and workspace may come from the kernels before this one
-    pdl_wait();
+    // pool and workspace may come from the kernels before this one.  With
+    // early_kv the caller guarantees that the kernels still running write
+    // neither the lengths, the block tables nor the pool rows older than the
+    // newest n_q positions of each sequence: those are read at once, and the
+    // wait is taken before the query, the newest rows, the outputs and the
+    // workspace are touched.
+    if (!p.early_kv) pdl_wait();
     pdl_trigger();
     if (warp == 0) {
         for (int b = lane; b < p.batch; b += 32) {
@@ -482,6 +540,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             const bool ok = L >= p.n_q && L <= p.max_seqlen;
             if (!ok && blockIdx.x == 0) report(NF_DEVERR_SEQLEN);
             seqC[b] = ok ? (L + kChunk - 1) / kChunk : 0;
+            seqL[b] = ok ? L : 0;
         }
         __syncwarp();
         if (lane == 0) {
@@ -501,19 +560,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     const long long c_begin = (int)blockIdx.x < P ? W * blockIdx.x / P : 0;
     const long long c_end = (int)blockIdx.x < P ? W * (blockIdx.x + 1) / P : 0;
 
-    // segments of sequences with no valid key: o = 0, lse = -inf
-    for (int s = blockIdx.x; s < p.batch * H; s += gridDim.x) {
-        const int b = s / H, h = s % H;
-        if (seqC[b] != 0) continue;
-        for (int idx = threadIdx.x; idx < p.rows * kHeadDim; idx += blockDim.x) {
-            const int r = idx / kHeadDim, ch = idx % kHeadDim;
-            const int j = r / p.group, gq = r % p.group;
-            const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-            p.out[row * kHeadDim + ch] = 0.f;
-            if (ch == 0 && p.out_lse) p.out_lse[row] = -INFINITY;
-        }
-    }
-
     PieceWalker walk{seqC, seqBase, H, p.batch, c_begin, c_end};
 
     // =================================================================== producer
@@ -523,6 +569,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     if (warp == kConsumerWarps) {
         uint32_t kst = 0;  // CTA-wide stage counter
         bool stop = false;
+        bool waited = !p.early_kv;
         while (!stop && walk.next()) {
             const int32_t *bt = p.block_table + (size_t)walk.pb * p.max_blocks;
             const int nblk = (seqC[walk.pb] * kChunk + kBlock - 1) / kBlock;
@@ -532,6 +579,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 const int ce = stage_end<FMT, NT>(cx, cx1);
                 const int tok0 = cx * kChunk, ntok = (ce - cx) * kChunk;
                 cx = ce;
+                if (!waited && tok0 + ntok > seqL[walk.pb] - p.n_q) {
+                    pdl_wait();  // the newest rows may come from the kernels before this one
+                    waited = true;
+                }
                 const int bi = tok0 >> 8;
                 if (bi >= win + 32) {  // warp-uniform refill of the window
                     win = bi;
@@ -588,6 +639,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     }
 
     // =================================================================== consumers
+    if (p.early_kv) pdl_wait();
+    // segments of sequences with no valid key: o = 0, lse = -inf
+    for (int s = blockIdx.x; s < p.batch * H; s += gridDim.x) {
+        const int b = s / H, h = s % H;
+        if (seqC[b] != 0) continue;
+        for (int idx = threadIdx.x; idx < p.rows * kHeadDim; idx += kConsumerWarps * 32) {
+            const int r = idx / kHeadDim, ch = idx % kHeadDim;
+            const int j = r / p.group, gq = r % p.group;
+            const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+            p.out[row * kHeadDim + ch] = 0.f;
+            if (ch == 0 && p.out_lse) p.out_lse[row] = -INFINITY;
+        }
+    }
+
     const int CW = kConsumerWarps / p.n_rg;  // warps per row group
     const int rg = warp / CW, slot = warp % CW;
     const int g = lane >> 2, t = lane & 3;
@@ -786,9 +851,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             int is_last = 0;
             if (n_pieces > 1) {
                 // release: the CTA's partial writes (ordered before this thread
-                // by the barrier) become visible before the ticket
-                __threadfence();
-                is_last = atomicAdd(&p.tickets[s_id], 1) == n_pieces - 1;
+                // by the barrier) become visible no later than the ticket
+                is_last = atomic_add_release(&p.tickets[s_id], 1) == n_pieces - 1;
                 if (is_last) __threadfence();  // acquire: the other pieces' partials
             }
             misc[1] = is_last;
@@ -796,19 +860,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         named_sync(1, kConsumerWarps * 32);
         if (misc[1]) {
             // This CTA holds the last ticket: merge every piece of the segment.
-            // Each thread owns (row, 4 channels): weights 2^(lse_i - M) over the
-            // pieces' (o_i, lse_i), normalised.  When this was the CTA's last
+            // Each thread owns (row, 4 channels).  When this was the CTA's last
             // piece the stage ring is free: one bulk copy brings all the pieces'
             // slots (consecutive in the workspace) into it.  Otherwise the
-            // slots stream from L2, kPB pieces' loads in flight at once.
-            constexpr int kPB = 16;
-            constexpr float kLog2e = 1.4426950408889634f;
+            // slots stream from L2.
             const int nthr = kConsumerWarps * 32, tid = threadIdx.x;
             const int np = last - first + 1;
             const float *pbase = p.partials + (size_t)(s_id + first) * p.slot_floats;
             const int lse_off = rows_here * kHeadDim;
             const uint32_t fin_bytes = (uint32_t)np * (uint32_t)p.slot_floats * 4u;
-            if (walk.x >= walk.end && fin_bytes <= (uint32_t)(NS * ST::kStride)) {
+            const bool in_ring = walk.x >= walk.end && fin_bytes <= (uint32_t)(NS * ST::kStride);
+            if (in_ring) {
                 if (tid == 0) {
                     // the ring's last reads (generic proxy) precede the copy's writes
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -820,71 +882,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                     misc[0] = 1;
                 }
                 fin_phase ^= 1u;
-                const float *ps = reinterpret_cast<const float *>(smem);
-                for (int it = tid; it < rows_here * (kHeadDim / 4); it += nthr) {
-                    const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
-                    float M = -INFINITY;
-                    for (int i = 0; i < np; ++i) M = fmaxf(M, ps[(size_t)i * p.slot_floats + lse_off + r]);
-                    float S = 0.f;
-                    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (M != -INFINITY) {
-                        for (int i = 0; i < np; ++i) {
-                            const float *sp = ps + (size_t)i * p.slot_floats;
-                            const float li = sp[lse_off + r];
-                            const float wk = li == -INFINITY ? 0.f : ex2((li - M) * kLog2e);
-                            const float4 o = reinterpret_cast<const float4 *>(sp + r * kHeadDim)[c4];
-                            S += wk;
-                            A.x += wk * o.x; A.y += wk * o.y; A.z += wk * o.z; A.w += wk * o.w;
-                        }
-                    }
-                    const float inv = M == -INFINITY ? 0.f : 1.0f / S;
-                    A.x *= inv; A.y *= inv; A.z *= inv; A.w *= inv;
-                    const int j = r / p.group, gq = r % p.group;
-                    const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-                    reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = A;
-                    if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(S);
-                }
-            } else {
+            }
             for (int it = tid; it < rows_here * (kHeadDim / 4); it += nthr) {
                 const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
-                float M = -INFINITY, S = 0.f;
-                float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int i0 = 0; i0 < np; i0 += kPB) {
-                    float4 o[kPB];
-                    float l[kPB];
-#pragma unroll
-                    for (int k = 0; k < kPB; ++k) {
-                        const float *sp = pbase + (size_t)(i0 + k) * p.slot_floats;
-                        if (i0 + k < np) {
-                            o[k] = __ldcg(reinterpret_cast<const float4 *>(sp + r * kHeadDim) + c4);
-                            l[k] = __ldcg(sp + lse_off + r);
-                        } else {
-                            o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            l[k] = -INFINITY;
-                        }
-                    }
-                    float Mb = M;
-#pragma unroll
-                    for (int k = 0; k < kPB; ++k) Mb = fmaxf(Mb, l[k]);
-                    if (Mb == -INFINITY) continue;
-                    const float a = M == -INFINITY ? 0.f : ex2((M - Mb) * kLog2e);
-                    S *= a;
-                    A.x *= a; A.y *= a; A.z *= a; A.w *= a;
-                    M = Mb;
-#pragma unroll
-                    for (int k = 0; k < kPB; ++k) {
-                        const float wk = l[k] == -INFINITY ? 0.f : ex2((l[k] - M) * kLog2e);
-                        S += wk;
-                        A.x += wk * o[k].x; A.y += wk * o[k].y; A.z += wk * o[k].z; A.w += wk * o[k].w;
-                    }
-                }
+                float M, S;
+                float4 A;
+                // both sources give the same sums in the same order
+                if (in_ring)
+                    merge_pieces<true>(reinterpret_cast<const float *>(smem), p.slot_floats, np, r, c4, lse_off, M, S, A);
+                else
+                    merge_pieces<false>(pbase, p.slot_floats, np, r, c4, lse_off, M, S, A);
                 const float inv = M == -INFINITY ? 0.f : 1.0f / S;
                 A.x *= inv; A.y *= inv; A.z *= inv; A.w *= inv;
                 const int j = r / p.group, gq = r % p.group;
                 const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
                 reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = A;
                 if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(S);
-            }
             }
             if (tid == 0) p.tickets[s_id] = 0;
             named_sync(1, kConsumerWarps * 32);

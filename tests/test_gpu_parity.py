@@ -180,3 +180,72 @@ def test_workload_full_size_sampled_heads(name, heads, layer):
 
 def test_workload_longest_bf16_cache_sampled_head():
     _full_size("longest", BF, heads=[5])
+
+
+# ------------------------------------------- early KV streaming (flag path)
+@pytest.mark.parametrize("name,kw", [
+    ("mtp", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True)),
+    ("ragged", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2)),
+])
+def test_early_kv_back_to_back_layers(name, kw):
+    # several layers of (append the step's tokens, decode) queued on one stream
+    # without host syncs, so each decode kernel starts while the append before
+    # it runs; with NF_DECODE_EARLY_KV the decode streams the older rows before
+    # the append has finished.  Results must equal the plain call bit for bit
+    # and match the oracle.
+    w = workloads.custom("early_" + name, q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, layers=3, **kw)
+    dev = "cuda"
+    bt_np = workloads.block_table(w)
+    bt = torch.as_tensor(bt_np, device=dev)
+    before = torch.as_tensor(w.cached, dtype=torch.int32, device=dev)
+    sl = torch.as_tensor(w.seqlens, dtype=torch.int32, device=dev)
+    msl = max(w.seqlens)
+    res = {}
+    for flags in (0, nf.NF_DECODE_EARLY_KV):
+        kvs, news, qs = [], [], []
+        for layer in range(w.layers):
+            kv = nf.KVLayer.empty(K8, w.pool_blocks, w.num_kv_heads, device=dev, fill=0xA5)
+            kn, vn = [], []
+            for b in range(w.batch):
+                k, v = workloads.layer_kv(w, layer, b, device=dev)
+                c = w.cached[b]
+                nf.nf_kv_append_quant(kv, k[None, :c].contiguous(), v[None, :c].contiguous(), bt[b:b + 1],
+                                      torch.zeros(1, dtype=torch.int32, device=dev))
+                kn.append(k[c:])
+                vn.append(v[c:])
+            kvs.append(kv)
+            news.append((torch.stack(kn).contiguous(), torch.stack(vn).contiguous()))
+            qs.append(workloads.layer_q(w, layer, device=dev))
+        ws = torch.zeros(nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, msl),
+                         dtype=torch.uint8, device=dev)
+        outs = [torch.empty((w.batch, w.n_q, w.num_q_heads, 128), device=dev) for _ in range(w.layers)]
+        lses = [torch.empty((w.batch, w.n_q, w.num_q_heads), device=dev) for _ in range(w.layers)]
+        torch.cuda.synchronize()
+        for layer in range(w.layers):
+            nf.nf_kv_append_quant(kvs[layer], news[layer][0], news[layer][1], bt, before)
+            nf.nf_decode_attn_ex(kvs[layer], qs[layer], bt, sl, msl, w.softmax_scale, w.causal, flags,
+                                 outs[layer], lses[layer], ws)
+        torch.cuda.synchronize()
+        assert nf.nf_get_device_error() == 0
+        res[flags] = (outs, lses, kvs, qs)
+    for layer in range(w.layers):
+        assert torch.equal(res[0][0][layer], res[1][0][layer])
+        assert torch.equal(res[0][1][layer], res[1][1][layer])
+    # the last layer against the oracle
+    layer = w.layers - 1
+    kvin = [workloads.layer_kv(w, layer, b, device=dev) for b in range(w.batch)]
+    pool, hs = oracle_pool(w, K8, kvin, bt_np)
+    compare_pool(res[1][2][layer], pool, hs)
+    ref_o, ref_l = oracle_attention(w, pool, hs, res[1][3][layer], bt_np)
+    check_attention(res[1][0][layer], res[1][1][layer], ref_o, ref_l)
+
+
+def test_decode_flags_rejects_unknown_bits():
+    w = workloads.custom("flags", cached=(300,), num_q_heads=4, num_kv_heads=1)
+    g = gpu_layer(w, 0, K8)
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(1, 1, 4, 1, 300), dtype=torch.uint8, device="cuda")
+    with pytest.raises(nf.NfError) as e:
+        nf.nf_decode_attn_ex(g["kv"], g["q"], torch.as_tensor(g["bt"], device="cuda"),
+                             torch.tensor([300], dtype=torch.int32, device="cuda"), 300, w.softmax_scale, False,
+                             0x2, torch.empty_like(g["out"]), None, ws)
+    assert e.value.status == nf.NF_ERR_INVALID_ARG
