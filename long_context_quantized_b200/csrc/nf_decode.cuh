@@ -683,47 +683,76 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         // query fragments of this (sequence, kv-head): lane (g, t) holds row g of
         // tile nt, channels 32t..32t+31 (K8/V4: k-step ks takes channels 32t + 8ks
         // + 0..3 and + 4..7) or 32u + 8t + 4h + 0..3 (bf16 cache: k-step 2u + h)
+        if (K8) {
+            // The digits are computed once per CTA into the (idle) merge buffer:
+            // warp w encodes rows w, w + 8, ...; lane l takes channels 4l..4l+3 =
+            // 32t + 8ks + 4hh + e (t = l / 8, ks = l / 2 % 4, hh = l % 2).  Layout
+            // [row][t][ks][d1 word hh=0, d2 word hh=0, d1 word hh=1, d2 word hh=1].
+            uint32_t *qsm = reinterpret_cast<uint32_t *>(sm_o);
+            float *qwsm = reinterpret_cast<float *>(sm_o) + kMaxRows * 64;
+            for (int r = warp; r < p.rows; r += kConsumerWarps) {
+                const int j = r / p.group, gq = r % p.group;
+                const size_t qoff =
+                    (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim + 4 * lane;
+                float x[4];
+                if (QF32) {
+                    const float4 v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qoff);
+                    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.q) + qoff);
+                    x[0] = __uint_as_float(v.x << 16);
+                    x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+                    x[2] = __uint_as_float(v.y << 16);
+                    x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+                }
+                float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                // q ~= s (d1 + d2 / 254), s = max|q| / 127, digits in [-127, 127]
+                const float s1 = amax / 127.0f;
+                const float inv = amax > 0.f ? 127.0f / amax : 0.f;
+                uint32_t d1w = 0, d2w = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float d1 = fminf(fmaxf(rintf(x[e] * inv), -127.f), 127.f);
+                    const float r1 = fmaf(-d1, s1, x[e]);
+                    const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
+                    d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
+                    d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
+                }
+                uint32_t *dst = qsm + (r * 4 + (lane >> 3)) * 16 + ((lane >> 1) & 3) * 4 + 2 * (lane & 1);
+                dst[0] = d1w;
+                dst[1] = d2w;
+                if (lane == 0) qwsm[r] = s1 / 254.0f * p.scale_log2;
+            }
+            named_sync(1, kConsumerWarps * 32);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int r = row0 + nt * 8 + g;
+                const bool rv = r < p.rows;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint4 v = rv ? lds128(qsm + (r * 4 + t) * 16 + ks * 4) : make_uint4(0, 0, 0, 0);
+                    ws.qa[nt][ks][0] = v.x; ws.qa[nt][ks][1] = v.y; ws.qa[nt][ks][2] = v.z; ws.qa[nt][ks][3] = v.w;
+                }
+                ws.qw[nt] = rv ? qwsm[r] : 0.f;
+            }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int r = row0 + nt * 8 + g;
             const bool rv = r < p.rows;
-            const int j = rv ? r / p.group : 0, gq = rv ? r % p.group : 0;
-            const size_t qoff = (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim;
-            float x[32];
+            if (!K8) {
+                const int j = rv ? r / p.group : 0, gq = rv ? r % p.group : 0;
+                const size_t qoff = (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim;
+                float x[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const size_t ch = qoff + (K8 ? 32 * t + c : 32 * (c >> 3) + 8 * t + (c & 7));
-                x[c] = !rv ? 0.f
-                            : QF32 ? static_cast<const float *>(p.q)[ch]
-                                   : __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[ch]);
-            }
-            if (K8) {
-                float amax = 0.f;
-#pragma unroll
-                for (int c = 0; c < 32; ++c) amax = fmaxf(amax, fabsf(x[c]));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                // q ~= s (d1 + d2 / 254), s = max|q| / 127, digits in [-127, 127]
-                const float s1 = amax / 127.0f;
-                const float inv = amax > 0.f ? 127.0f / amax : 0.f;
-#pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    uint32_t d1w = 0, d2w = 0;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float v = x[4 * w + e];
-                        const float d1 = fminf(fmaxf(rintf(v * inv), -127.f), 127.f);
-                        const float r1 = fmaf(-d1, s1, v);
-                        const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
-                        d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
-                        d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
-                    }
-                    // word w = 2ks + hh: A rows g (digit 1) and g + 8 (digit 2)
-                    ws.qa[nt][w >> 1][2 * (w & 1)] = d1w;
-                    ws.qa[nt][w >> 1][2 * (w & 1) + 1] = d2w;
+                for (int c = 0; c < 32; ++c) {
+                    const size_t ch = qoff + 32 * (c >> 3) + 8 * t + (c & 7);
+                    x[c] = !rv ? 0.f
+                                : QF32 ? static_cast<const float *>(p.q)[ch]
+                                       : __bfloat162float(static_cast<const __nv_bfloat16 *>(p.q)[ch]);
                 }
-                ws.qw[nt] = s1 / 254.0f * p.scale_log2;
-            } else {
 #pragma unroll
                 for (int w = 0; w < 16; ++w) {
                     // word w = 2 (2u + hh) + e2 holds channels 32u + 8t + 4hh + 2e2 + 0..1
