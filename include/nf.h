@@ -139,8 +139,8 @@ nf_status nf_kv_append_quant(const nf_kv_layer *kv, const void *k_new, const voi
  * nf_decode_attn_workspace_size -- bytes of device workspace nf_decode_attn
  * needs for this shape on a device with `num_sms` streaming multiprocessors
  * (pass the device's count; nf_decode_attn uses the current device's).  The
- * workspace holds one ticket counter per (sequence, kv-head) and the (o, lse)
- * partials of the context splits.  Zero-fill it once before its first use
+ * workspace holds ticket counters (per (sequence, kv-head) and per split) and
+ * the (o, lse) partials of the context splits.  Zero-fill it once before its first use
  * (e.g. cudaMemsetAsync); every call leaves it zero-filled where it must be
  * when its kernel completes, so it can be reused call after call on one
  * stream.  Returns 0 for an invalid or unsupported shape.

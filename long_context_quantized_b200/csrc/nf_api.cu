@@ -60,10 +60,10 @@ nf_status check_layer(const nf_kv_layer *kv) {
 // ---------------------------------------------------------------- plan
 // The decode kernel is persistent: one CTA per SM, each taking an equal share
 // of all (sequence, kv-head) key chunks (computed on the device from seqlens).
-// The workspace holds one ticket counter per (sequence, kv-head) -- zero
-// between calls -- and one (o, lse) partial slot per CTA plus one per segment
-// (a CTA's pieces and a segment's pieces both form contiguous runs, so slot
-// segment + cta is unique).
+// The workspace holds ticket counters -- one per (sequence, kv-head) and one
+// per partial slot, zero between calls -- and one (o, lse) partial slot per
+// CTA plus one per segment (a CTA's pieces and a segment's pieces both form
+// contiguous runs, so slot segment + cta is unique).
 struct Plan {
     int ctas = 0, nt = 0, n_rg = 0, rows = 0, segments = 0, slot_floats = 0;
     size_t ticket_bytes = 0, partial_bytes = 0;
@@ -82,7 +82,9 @@ bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sm
     if (pl.n_rg == 3) pl.n_rg = 4;  // 8 consumer warps split evenly over 1, 2 or 4 row groups
     pl.ctas = num_sms;
     pl.segments = batch * H_kv;
-    pl.ticket_bytes = ((size_t)pl.segments * 4 + 255) / 256 * 256;
+    // one counter per segment, then one per partial slot (group counters of
+    // the two-step merge, indexed like the slots)
+    pl.ticket_bytes = ((size_t)(pl.segments + pl.ctas + pl.segments) * 4 + 255) / 256 * 256;
     pl.slot_floats = (pl.rows * (nf::kHeadDim + 1) + 3) / 4 * 4;
     pl.partial_bytes = ((size_t)(pl.ctas + pl.segments) * pl.slot_floats * sizeof(float) + 255) / 256 * 256;
     return true;
@@ -336,6 +338,7 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
     p.out = out;
     p.out_lse = out_lse;
     p.tickets = static_cast<int32_t *>(workspace);
+    p.gtickets = p.tickets + pl.segments;
     p.partials = reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.ticket_bytes);
     p.slot_floats = pl.slot_floats;
 

@@ -126,6 +126,7 @@ struct DecodeParams {
     float *out;      // [batch][n_q][H_q][128]
     float *out_lse;  // [batch][n_q][H_q] or null
     int32_t *tickets;  // [batch * H_kv], zero between calls
+    int32_t *gtickets; // [gridDim.x + batch * H_kv], indexed like partial slots; zero between calls
     float *partials;   // [gridDim.x + batch * H_kv] slots of slot_floats
     int slot_floats;   // rows * 128 (o) + rows (lse), rounded up to 4 floats
 };
@@ -147,6 +148,9 @@ struct DecodeSmem {
     static constexpr int kMisc = kSeqBase + (kMaxBatch + 1) * 8;              // int [4]
     static constexpr int kBytes = kMisc + 16;
     static_assert(kBytes <= 232448, "shared memory per CTA");
+    // final merge: (row, 4 channels) items of at most 8 rows (NT = 1) or kMaxRows
+    static constexpr int kMaxItems = (NT == 1 ? 8 : kMaxRows) * (kHeadDim / 4);
+    static_assert(kMergeM - kMergeO >= kMaxItems * 24, "final-merge state in the merge buffer");
     static_assert(ST::kStride % 128 == 0, "stage alignment");
 };
 
@@ -433,36 +437,42 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
     }
 }
 
-// Log-sum-exp merge of np pieces' (o, lse) for row r, channels 4c4..4c4+3:
-// M = max lse_i, S = sum_i 2^((lse_i - M) log2 e), A = sum_i that weight x o_i,
-// in piece order.  Pieces are slots of slot_floats floats from `ps`: o at
-// [r][128], lse at lse_off + r.  SMEM: plain loads from shared memory;
-// otherwise loads that bypass L1 (the slots were written by other CTAs), kPB
-// pieces in flight at once.  The arithmetic is the same for both sources.
+// One round of the log-sum-exp merge for row r, channels 4c4..4c4+3: folds n
+// pieces' (o, lse) into the running (M, S, A) -- M the max lse so far, S the
+// sum of weights 2^((lse_i - M) log2 e), A the weighted sum of the o_i -- in
+// piece order, first raising M to the round's max (and rescaling S and A).
+// Piece i is the slot at ps + i * slot_floats: o at [r][128], lse at
+// lse_off + r.  SMEM: plain loads from shared memory; otherwise loads that
+// bypass L1 (the slots were written by other CTAs), kPB in flight at once.
+// The arithmetic is the same for both sources.
 template <bool SMEM>
-__device__ __forceinline__ void merge_pieces(const float *ps, int slot_floats, int np, int r, int c4, int lse_off,
-                                             float &M, float &S, float4 &A) {
+__device__ __forceinline__ void merge_round(const float *ps, size_t slot_floats, int n, int r, int c4, int lse_off,
+                                            float &M, float &S, float4 &A) {
     constexpr int kPB = 16;
     constexpr float kLog2e = 1.4426950408889634f;
     auto ld1 = [&](const float *a) { return SMEM ? *a : __ldcg(a); };
-    M = -INFINITY;
-    S = 0.f;
-    A = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i0 = 0; i0 < np; i0 += kPB) {
+    float Mr = M;
+    for (int i0 = 0; i0 < n; i0 += kPB) {
         float l[kPB];
 #pragma unroll
-        for (int k = 0; k < kPB; ++k) l[k] = i0 + k < np ? ld1(ps + (size_t)(i0 + k) * slot_floats + lse_off + r) : -INFINITY;
+        for (int k = 0; k < kPB; ++k) l[k] = i0 + k < n ? ld1(ps + (size_t)(i0 + k) * slot_floats + lse_off + r) : -INFINITY;
 #pragma unroll
-        for (int k = 0; k < kPB; ++k) M = fmaxf(M, l[k]);
+        for (int k = 0; k < kPB; ++k) Mr = fmaxf(Mr, l[k]);
     }
-    if (M == -INFINITY) return;
-    for (int i0 = 0; i0 < np; i0 += kPB) {
+    if (Mr == -INFINITY) return;
+    if (Mr > M && M != -INFINITY) {
+        const float a = ex2((M - Mr) * kLog2e);
+        S *= a;
+        A.x *= a; A.y *= a; A.z *= a; A.w *= a;
+    }
+    M = Mr;
+    for (int i0 = 0; i0 < n; i0 += kPB) {
         float4 o[kPB];
         float l[kPB];
 #pragma unroll
         for (int k = 0; k < kPB; ++k) {
             const float *sp = ps + (size_t)(i0 + k) * slot_floats;
-            if (i0 + k < np) {
+            if (i0 + k < n) {
                 const float4 *op = reinterpret_cast<const float4 *>(sp + r * kHeadDim) + c4;
                 o[k] = SMEM ? *op : __ldcg(op);
                 l[k] = ld1(sp + lse_off + r);
@@ -479,6 +489,85 @@ __device__ __forceinline__ void merge_pieces(const float *ps, int slot_floats, i
             A.y = fmaf(wk, o[k].y, A.y);
             A.z = fmaf(wk, o[k].z, A.z);
             A.w = fmaf(wk, o[k].w, A.w);
+        }
+    }
+}
+
+// Merges n partial slots -- slot i at src + i * stride floats -- of `rows`
+// rows, in rounds of `per_round` slots: into the slot dst (normalised o and
+// lse, the format of a piece's partial) when dst is not null, else into the
+// output rows of (sequence b, kv-head h).  Run by all consumer threads of the
+// CTA.  in_ring: the stage ring is idle, and each round's slots come into it
+// with bulk copies (one per slot unless the slots are consecutive); else they
+// stream from L2.  The rounds, and so the sums, are the same either way.
+// `state` holds the items' running (M, S, A) between rounds (24 bytes per
+// (row, 4 channels) item).
+__device__ __forceinline__ void merge_slots(const DecodeParams &p, const float *src, size_t stride, int n, int rows,
+                                         int per_round, bool in_ring, unsigned char *smem, float *state,
+                                         int item_cap, uint64_t *fin_bar, uint32_t &fin_phase, volatile int *misc,
+                                         float *dst, int b, int h) {
+    const int nthr = kConsumerWarps * 32, tid = threadIdx.x;
+    const int lse_off = rows * kHeadDim;
+    const uint32_t slot_bytes = (uint32_t)p.slot_floats * 4u;
+    const int n_items = rows * (kHeadDim / 4);
+    float4 *stA = reinterpret_cast<float4 *>(state);
+    float *stM = reinterpret_cast<float *>(stA + item_cap);
+    float *stS = stM + item_cap;
+    for (int it = tid; it < n_items; it += nthr) {
+        stA[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        stM[it] = -INFINITY;
+        stS[it] = 0.f;
+    }
+    for (int i0 = 0; i0 < n; i0 += per_round) {
+        const int nr = min(per_round, n - i0);
+        const float *rsrc = src + (size_t)i0 * stride;
+        if (in_ring) {
+            if (tid == 0) {
+                // the ring's last reads (generic proxy) precede the copies' writes
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive_expect_tx(fin_bar, (uint32_t)nr * slot_bytes);
+                if (stride == (size_t)p.slot_floats)
+                    bulk_g2s(smem, rsrc, (uint32_t)nr * slot_bytes, fin_bar);
+                else
+                    for (int i = 0; i < nr; ++i) bulk_g2s(smem + (size_t)i * slot_bytes, rsrc + (size_t)i * stride, slot_bytes, fin_bar);
+            }
+            if (!misc[0] && !mbar_wait(fin_bar, fin_phase)) {
+                report(NF_DEVERR_TIMEOUT);
+                misc[0] = 1;
+            }
+            fin_phase ^= 1u;
+        }
+        for (int it = tid; it < n_items; it += nthr) {
+            const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
+            float M = stM[it], S = stS[it];
+            float4 A = stA[it];
+            if (in_ring)
+                merge_round<true>(reinterpret_cast<const float *>(smem), p.slot_floats, nr, r, c4, lse_off, M, S, A);
+            else
+                merge_round<false>(rsrc, stride, nr, r, c4, lse_off, M, S, A);
+            stM[it] = M;
+            stS[it] = S;
+            stA[it] = A;
+        }
+        if (in_ring) named_sync(1, kConsumerWarps * 32);  // the ring is read before the next round's copy
+    }
+    // every read of the sources precedes the writes (dst may be the first source)
+    if (!in_ring) named_sync(1, kConsumerWarps * 32);
+    for (int it = tid; it < n_items; it += nthr) {
+        const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
+        const float M = stM[it], S = stS[it];
+        float4 a = stA[it];
+        const float inv = M == -INFINITY ? 0.f : 1.0f / S;
+        a.x *= inv; a.y *= inv; a.z *= inv; a.w *= inv;
+        const float lse = M == -INFINITY ? -INFINITY : M + logf(S);
+        if (dst) {
+            reinterpret_cast<float4 *>(dst + r * kHeadDim)[c4] = a;
+            if (c4 == 0) dst[lse_off + r] = lse;
+        } else {
+            const int j = r / p.group, gq = r % p.group;
+            const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+            reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = a;
+            if (c4 == 0 && p.out_lse) p.out_lse[row] = lse;
         }
     }
 }
@@ -876,59 +965,53 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             }
         }
         named_sync(1, kConsumerWarps * 32);
+        // ---- tickets.  The partials of a segment merge in one step when they fit
+        // one ring round; else in two: the last piece of each group of gp
+        // consecutive pieces merges its group into the group's first slot, and
+        // the last group merges the groups.  The grouping is fixed, so the sums
+        // do not depend on which CTA finishes last.
+        const uint32_t slot_bytes = (uint32_t)p.slot_floats * 4u;
+        const int gp = (int)((uint32_t)(NS * ST::kStride) / slot_bytes);  // slots per ring round
+        const bool two_level = n_pieces > gp;
+        const int pi = (int)blockIdx.x - first;  // this piece's index in the segment
+        const int g0 = two_level ? pi / gp * gp : 0;
+        const int gn = two_level ? min(gp, n_pieces - g0) : n_pieces;
+        int *tk = two_level ? &p.gtickets[s_id + first + g0] : &p.tickets[s_id];
         if (threadIdx.x == 0) {
             int is_last = 0;
             if (n_pieces > 1) {
                 // release: the CTA's partial writes (ordered before this thread
                 // by the barrier) become visible no later than the ticket
-                is_last = atomic_add_release(&p.tickets[s_id], 1) == n_pieces - 1;
+                is_last = atomic_add_release(tk, 1) == gn - 1;
                 if (is_last) __threadfence();  // acquire: the other pieces' partials
             }
             misc[1] = is_last;
         }
         named_sync(1, kConsumerWarps * 32);
         if (misc[1]) {
-            // This CTA holds the last ticket: merge every piece of the segment.
-            // Each thread owns (row, 4 channels).  When this was the CTA's last
-            // piece the stage ring is free: one bulk copy brings all the pieces'
-            // slots (consecutive in the workspace) into it.  Otherwise the
-            // slots stream from L2.
-            const int nthr = kConsumerWarps * 32, tid = threadIdx.x;
-            const int np = last - first + 1;
-            const float *pbase = p.partials + (size_t)(s_id + first) * p.slot_floats;
-            const int lse_off = rows_here * kHeadDim;
-            const uint32_t fin_bytes = (uint32_t)np * (uint32_t)p.slot_floats * 4u;
-            const bool in_ring = walk.x >= walk.end && fin_bytes <= (uint32_t)(NS * ST::kStride);
-            if (in_ring) {
-                if (tid == 0) {
-                    // the ring's last reads (generic proxy) precede the copy's writes
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    mbar_arrive_expect_tx(fin_bar, fin_bytes);
-                    bulk_g2s(smem, pbase, fin_bytes, fin_bar);
+            // This CTA holds the last ticket of the segment (or of a group).  When
+            // this was the CTA's last piece the stage ring is idle.
+            const bool in_ring = walk.x >= walk.end;
+            float *slot0 = p.partials + (size_t)(s_id + first) * p.slot_floats;
+            merge_slots(p, slot0 + (size_t)g0 * p.slot_floats, p.slot_floats, gn, rows_here, gp, in_ring, smem, sm_o,
+                        SM::kMaxItems, fin_bar, fin_phase, misc, two_level ? slot0 + (size_t)g0 * p.slot_floats : nullptr,
+                        b, h);
+            if (threadIdx.x == 0) *tk = 0;
+            if (two_level) {
+                const int ng = (n_pieces + gp - 1) / gp;
+                named_sync(1, kConsumerWarps * 32);
+                if (threadIdx.x == 0) {
+                    const int is_last = atomic_add_release(&p.tickets[s_id], 1) == ng - 1;
+                    if (is_last) __threadfence();
+                    misc[1] = is_last;
                 }
-                if (!misc[0] && !mbar_wait(fin_bar, fin_phase)) {
-                    report(NF_DEVERR_TIMEOUT);
-                    misc[0] = 1;
+                named_sync(1, kConsumerWarps * 32);
+                if (misc[1]) {
+                    merge_slots(p, slot0, (size_t)gp * p.slot_floats, ng, rows_here, gp, in_ring, smem, sm_o,
+                                SM::kMaxItems, fin_bar, fin_phase, misc, nullptr, b, h);
+                    if (threadIdx.x == 0) p.tickets[s_id] = 0;
                 }
-                fin_phase ^= 1u;
             }
-            for (int it = tid; it < rows_here * (kHeadDim / 4); it += nthr) {
-                const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
-                float M, S;
-                float4 A;
-                // both sources give the same sums in the same order
-                if (in_ring)
-                    merge_pieces<true>(reinterpret_cast<const float *>(smem), p.slot_floats, np, r, c4, lse_off, M, S, A);
-                else
-                    merge_pieces<false>(pbase, p.slot_floats, np, r, c4, lse_off, M, S, A);
-                const float inv = M == -INFINITY ? 0.f : 1.0f / S;
-                A.x *= inv; A.y *= inv; A.z *= inv; A.w *= inv;
-                const int j = r / p.group, gq = r % p.group;
-                const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-                reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = A;
-                if (c4 == 0 && p.out_lse) p.out_lse[row] = M == -INFINITY ? -INFINITY : M + logf(S);
-            }
-            if (tid == 0) p.tickets[s_id] = 0;
             named_sync(1, kConsumerWarps * 32);
         }
     }
