@@ -249,3 +249,31 @@ def test_decode_flags_rejects_unknown_bits():
                              torch.tensor([300], dtype=torch.int32, device="cuda"), 300, w.softmax_scale, False,
                              0x2, torch.empty_like(g["out"]), None, ws)
     assert e.value.status == nf.NF_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,kw", [
+    # 8 rows per kv-head, several segments per CTA and many pieces per segment
+    ("rows8", dict(cached=(20000, 3000, 9000), num_q_heads=16, num_kv_heads=2)),
+    # 32 rows per kv-head: partials larger than one ring round -> two-step merge
+    ("rows32", dict(cached=(60000,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True)),
+])
+def test_repeated_calls_are_bitwise_identical(name, kw):
+    # which CTA takes a segment's last ticket changes from run to run; the
+    # merges must not depend on it
+    w = workloads.custom("rep_" + name, q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, **kw)
+    g = gpu_layer(w, 0, K8)
+    bt = torch.as_tensor(g["bt"], device="cuda")
+    sl = torch.as_tensor(w.seqlens, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads,
+                                                      max(w.seqlens)), dtype=torch.uint8, device="cuda")
+    for _ in range(5):
+        out = torch.empty_like(g["out"])
+        lse = torch.empty_like(g["lse"])
+        nf.nf_decode_attn(g["kv"], g["q"], bt, sl, max(w.seqlens), w.softmax_scale, w.causal, out, lse, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out, g["out"]) and torch.equal(lse, g["lse"])
+    assert nf.nf_get_device_error() == 0
+    hs = [0]
+    pool, hs = oracle_pool(w, K8, g["kvin"], g["bt"], hs)
+    ref_o, ref_l = oracle_attention(w, pool, hs, g["q"], g["bt"])
+    check_attention(select_heads(g["out"], w, hs), select_heads(g["lse"], w, hs), ref_o, ref_l)
