@@ -191,7 +191,17 @@ class GpuWorkload:
                 self.knew.append(torch.stack(knew).contiguous())
                 self.vnew.append(torch.stack(vnew).contiguous())
             self.q.append(workloads.layer_q(w, layer, device=device))
-            self.out.append(torch.empty((w.batch, w.n_q, w.num_q_heads, 128), dtype=torch.float32, device=device))
+        # every layer's inputs and outputs live in one tensor per kind (the layers'
+        # tensors are views), so a step's host copies are one transfer each
+        self.q_all = torch.stack(self.q).contiguous()
+        self.q = [self.q_all[i] for i in range(w.layers)]
+        if w.n_new:
+            self.knew_all = torch.stack(self.knew).contiguous()
+            self.vnew_all = torch.stack(self.vnew).contiguous()
+            self.knew = [self.knew_all[i] for i in range(w.layers)]
+            self.vnew = [self.vnew_all[i] for i in range(w.layers)]
+        self.out_all = torch.empty((w.layers, w.batch, w.n_q, w.num_q_heads, 128), dtype=torch.float32, device=device)
+        self.out = [self.out_all[i] for i in range(w.layers)]
         ws = nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, self.max_seqlen)
         self.ws = torch.zeros(ws, dtype=torch.uint8, device=device)
         torch.cuda.synchronize()
@@ -420,26 +430,24 @@ def main():
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     traffic = recorded_traffic(w.name, args.kv_format)
 
-    # ---- end to end: pinned host inputs -> device, the step, result -> host
-    n_layers = w.layers
-    h_q = [t.cpu().pin_memory() for t in gw.q]
-    h_k = [t.cpu().pin_memory() for t in gw.knew]
-    h_v = [t.cpu().pin_memory() for t in gw.vnew]
-    h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in gw.out]
+    # ---- end to end: the step's inputs (every layer's q and new K/V) copied
+    # from pinned host memory, the step, every layer's output copied back
+    h_in = [gw.q_all.cpu().pin_memory()]
+    d_in = [gw.q_all]
+    if w.n_new:
+        h_in += [gw.knew_all.cpu().pin_memory(), gw.vnew_all.cpu().pin_memory()]
+        d_in += [gw.knew_all, gw.vnew_all]
+    h_out = torch.empty_like(gw.out_all, device="cpu").pin_memory()
     ge = torch.cuda.CUDAGraph()
     with torch.cuda.graph(ge, stream=stream):
-        for layer in range(n_layers):
-            gw.q[layer].copy_(h_q[layer], non_blocking=True)
-            if w.n_new:
-                gw.knew[layer].copy_(h_k[layer], non_blocking=True)
-                gw.vnew[layer].copy_(h_v[layer], non_blocking=True)
-            gw.append(layer)
-            gw.decode(layer)
-            h_out[layer].copy_(gw.out[layer], non_blocking=True)
+        for d, hsrc in zip(d_in, h_in):
+            d.copy_(hsrc, non_blocking=True)
+        gw.step()
+        h_out.copy_(gw.out_all, non_blocking=True)
     e2e_ms = time_graph(ge, args.steps, max(3, args.warmup), stream)
     e2e_ms = max_over_ranks(e2e_ms, device)
-    h2d = sum(t.numel() * t.element_size() for t in h_q + h_k + h_v)
-    d2h = sum(t.numel() * t.element_size() for t in h_out)
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
     del ge, g
     torch.cuda.synchronize()
 

@@ -268,6 +268,17 @@ nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_
 nf_status nf_get_device_error(int32_t *code);
 
 /* Static text for a status code. */
+/*
+ * nf_selftest_bounded_wait -- diagnostics: launch one thread that waits on an
+ * mbarrier nothing ever arrives on, for at most limit_us microseconds (1 ..
+ * 1000000), through the same bounded wait every wait of the decode kernel uses.
+ * The wait gives up, records NF_DEVERR_TIMEOUT in the device error word and
+ * the kernel returns; the context stays usable.  Read the word with
+ * nf_get_device_error.  The pages have no counterpart: this checks the
+ * library's stall detection without faulting or hanging the GPU.
+ */
+nf_status nf_selftest_bounded_wait(uint32_t limit_us, nf_stream_t stream);
+
 const char *nf_status_string(nf_status status);
 
 /* Message describing the last failing call on this host thread ("" if none). */

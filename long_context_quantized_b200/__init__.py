@@ -82,6 +82,8 @@ def load_library():
         lib.nf_decode_attn_ex.restype = I
         lib.nf_decode_attn_noalloc.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, P, P, P]
         lib.nf_decode_attn_noalloc.restype = I
+        lib.nf_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
+        lib.nf_selftest_bounded_wait.restype = I
         lib.nf_attn_combine.argtypes = [P, P, I, I, I, P, P, P]
         lib.nf_attn_combine.restype = I
         lib.nf_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32)]
@@ -274,3 +276,9 @@ def nf_get_device_error() -> int:
 
 def nf_status_string(status: int) -> str:
     return load_library().nf_status_string(int(status)).decode()
+
+
+def nf_selftest_bounded_wait(limit_us: int, stream=None):
+    """Run the bounded-wait self-test (see nf.h); afterwards
+    nf_get_device_error() returns NF_DEVERR_TIMEOUT."""
+    _check(load_library().nf_selftest_bounded_wait(int(limit_us), _stream(stream)), "nf_selftest_bounded_wait")

@@ -15,6 +15,20 @@
 #include "nf_common.cuh"
 #include "nf_decode.cuh"
 
+namespace nf {
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// arrives on, for at most limit_ns, and records NF_DEVERR_TIMEOUT when the
+// wait gives up (the path every wait of the decode kernel takes on a stall).
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_limit(&bar, 0, limit_ns)) report(NF_DEVERR_TIMEOUT);
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_addr(&bar)) : "memory");
+}
+}  // namespace nf
+
 namespace {
 
 thread_local char g_msg[512] = "";
@@ -406,6 +420,14 @@ nf_status nf_get_device_error(int32_t *code) {
     if (e != cudaSuccess) return fail(NF_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
     *code = v;
     return v ? NF_ERR_DEVICE_CHECK : NF_OK;
+}
+
+nf_status nf_selftest_bounded_wait(uint32_t limit_us, nf_stream_t stream) {
+    if (limit_us == 0 || limit_us > 1000000u)
+        return fail(NF_ERR_INVALID_ARG, "limit_us %u (1 .. 1000000)", limit_us);
+    nf::bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (uint64_t)limit_us * 1000u);
+    return after_launch("bounded-wait self-test launch");
 }
 
 const char *nf_status_string(nf_status status) {

@@ -141,6 +141,17 @@ def test_seqlen_above_bound_is_reported():
     assert torch.all(out == 0) and torch.all(torch.isinf(lse))
 
 
+def test_bounded_wait_times_out_and_context_survives():
+    # a wait that nothing ends gives up after its limit and reports, instead of
+    # hanging the GPU; the context stays usable
+    nf.nf_selftest_bounded_wait(20000)  # 20 ms
+    torch.cuda.synchronize()
+    assert nf.nf_get_device_error() == nf.NF_DEVERR_TIMEOUT
+    w = workloads.custom("after_timeout", cached=(500,), num_q_heads=8, num_kv_heads=1)
+    run_case(w, 0, K8)
+    assert nf.nf_get_device_error() == 0
+
+
 def test_workspace_too_small_is_refused():
     w = workloads.custom("ws", cached=(300,), num_q_heads=4, num_kv_heads=1)
     g = gpu_layer(w, 0, K8)
