@@ -1,4 +1,4 @@
-"""CPU oracle for K8/V4 quantised-KV decode attention (test infrastructure).
+"""CPU oracle for K8/V4 (and int8 / bf16) KV-cache decode attention (test infrastructure).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
 ``--impl reference`` legs of ``bench.py`` may import this package.  The product
@@ -30,6 +30,7 @@ _lib = None
 
 FMT_K8V4 = 0
 FMT_BF16 = 1
+FMT_K8V8 = 2
 BLOCK = 256
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
@@ -151,6 +152,11 @@ class Pool:
             self.k_scale = np.zeros((num_blocks, num_kv_heads, BLOCK), np.uint16)
             self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 2), np.uint8)
             self.v_scale = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 32), np.uint16)
+        elif fmt == FMT_K8V8:
+            self.k = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), np.int8)
+            self.k_scale = np.zeros((num_blocks, num_kv_heads, BLOCK), np.uint16)
+            self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), np.int8)
+            self.v_scale = np.zeros((num_blocks, num_kv_heads, BLOCK), np.uint16)
         else:
             self.k = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), np.uint16)
             self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), np.uint16)

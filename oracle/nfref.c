@@ -212,6 +212,9 @@ void nfref_quant_v(const float *x, int d, int group, uint16_t *scales, uint8_t *
  *   v_plane  uint8  [num_blocks][H][256][d/2]
  *   v_scale  fp16   [num_blocks][H][256][d/32]
  * fmt 1 (BF16 cache): k_plane, v_plane bf16 [num_blocks][H][256][d]; no scales.
+ * fmt 2 (K8V8, int8 KV): k_plane, v_plane int8 [num_blocks][H][256][d]; k_scale,
+ *   v_scale fp16 [num_blocks][H][256]; V quantised by the K rule (absmax/127
+ *   per token and kv-head).
  * Token position p of sequence b lives in block block_table[b][p / 256],
  * slot p % 256.
  */
@@ -234,6 +237,8 @@ static double v_hat(int fmt, const void *v_plane, const uint16_t *v_scale, size_
 {
     if (fmt == 1)
         return (double)nfref_bf16_to_f32(((const uint16_t *)v_plane)[si * d + c]);
+    if (fmt == 2)
+        return (double)((const int8_t *)v_plane)[si * d + c] * (double)nfref_f16_to_f32(v_scale[si]);
     uint8_t byte = ((const uint8_t *)v_plane)[si * (size_t)(d / 2) + (size_t)(c / 2)];
     int nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
     int code = nib >= 8 ? nib - 16 : nib;
@@ -278,6 +283,9 @@ int nfref_append(int fmt, int num_blocks, int H, int d,
                         ((uint16_t *)k_plane)[si * d + c] = nfref_f32_to_bf16(kx[c]);
                         ((uint16_t *)v_plane)[si * d + c] = nfref_f32_to_bf16(vx[c]);
                     }
+                } else if (fmt == 2) {
+                    nfref_quant_k(kx, d, &k_scale[si], (int8_t *)k_plane + si * d);
+                    nfref_quant_k(vx, d, &v_scale[si], (int8_t *)v_plane + si * d);
                 } else {
                     nfref_quant_k(kx, d, &k_scale[si], (int8_t *)k_plane + si * d);
                     nfref_quant_v(vx, d, 32, &v_scale[si * (size_t)(d / 32)],

@@ -67,6 +67,8 @@ def np_dequant_pool(pool):
     ks = pool.k_scale.view(np.float16).astype(np.float64)
     vs = pool.v_scale.view(np.float16).astype(np.float64)
     k = pool.k.astype(np.float64) * ks[..., None]
+    if pool.fmt == oracle.FMT_K8V8:
+        return k, pool.v.astype(np.float64) * vs[..., None]
     vc = np_unpack_v(pool.v).astype(np.float64)
     v = vc * np.repeat(vs, 32, axis=-1)
     return k, v
@@ -291,6 +293,30 @@ def test_append_places_tokens_through_block_table():
         assert np.array_equal(now[~touched], old[~touched])
 
 
+def test_append_k8v8_quantises_v_by_the_k_rule():
+    # int8 KV: V codes and scales equal the numpy statement of the quantiser
+    # with the K limit (127), one scale per (token, kv-head), int8 codes
+    rng = np.random.default_rng(23)
+    H, d, L = 2, 128, 300
+    pool = oracle.Pool(oracle.FMT_K8V8, 3, H, d, poison=0x5A)
+    bt = np.array([[2, 0]], np.int32)
+    k = rng.standard_normal((1, L, H, d)).astype(np.float32)
+    v = (rng.standard_normal((1, L, H, d)) * rng.uniform(0.01, 40, (1, L, H, 1))).astype(np.float32)
+    v[0, 7, 1] = 0.0                        # a zero vector: scale 0, codes 0
+    assert oracle.append(pool, k, v, bt, np.array([0], np.int32)) == 0
+    for p_ in range(L):
+        blk, slot = bt[0, p_ // 256], p_ % 256
+        for h in range(H):
+            s16, codes = np_quant(v[0, p_, h], 127)
+            assert pool.v_scale[blk, h, slot] == s16
+            assert np.array_equal(pool.v[blk, h, slot].astype(np.int64), codes)
+            s16k, ck = np_quant(k[0, p_, h], 127)
+            assert pool.k_scale[blk, h, slot] == s16k
+            assert np.array_equal(pool.k[blk, h, slot].astype(np.int64), ck)
+    # untouched slots keep the poison
+    assert np.all(pool.v[1].view(np.uint8) == 0x5A) and np.all(pool.v[0, :, 300 - 256:].view(np.uint8) == 0x5A)
+
+
 def test_append_rejects_out_of_range():
     pool = oracle.Pool(oracle.FMT_K8V4, 2, 1, 128)
     k = np.zeros((1, 1, 1, 128), np.float32)
@@ -302,7 +328,7 @@ def test_append_rejects_out_of_range():
 SCALE = float(np.float32(1 / math.sqrt(128)))
 
 
-@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16])
+@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8])
 def test_attention_zero_query_is_mean_of_visible_values(fmt):
     # q = 0 -> all scores 0 -> o = mean of visible v_hat, lse = log(#visible).
     # Causal with n_q = 4: query j sees L - 4 + j + 1 keys.
@@ -401,7 +427,7 @@ def test_attention_split_and_combine_equals_whole():
     assert lse[0] == pytest.approx(lse_w, abs=1e-12)
 
 
-@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16])
+@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8])
 @pytest.mark.parametrize("causal", [False, True])
 def test_attention_matches_numpy_brute_force(fmt, causal):
     cached = [300, 513]
