@@ -7,7 +7,7 @@ appends) followed by split-K decode attention and the LSE combine, all through
 the C ABI.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                  [--kv-format k8v4|bf16] [--impl ours|reference]
+                  [--kv-format k8v4|k8v8|bf16] [--impl ours|reference]
 
 Metric: KV tokens/s (each cached key counted once per layer, heads not
 multiplied) and the decode kernel's achieved HBM GB/s against the measured B200
@@ -166,7 +166,8 @@ class GpuWorkload:
         self.nf = nf
         self.w = w
         self.dev = device
-        self.fmt = nf.NF_KV_K8V4 if fmt_name == "k8v4" else nf.NF_KV_BF16
+        self.fmt_name = fmt_name
+        self.fmt = {"k8v4": nf.NF_KV_K8V4, "k8v8": nf.NF_KV_K8V8, "bf16": nf.NF_KV_BF16}[fmt_name]
         self.decode_flags = nf.NF_DECODE_EARLY_KV
         assert w.n_new in (0, w.n_q), "the early-KV guarantee needs n_new == n_q"
         bt = workloads.block_table(w)
@@ -226,7 +227,7 @@ class GpuWorkload:
 
     # --- byte accounting (algorithmic, per decode launch / per step)
     def kv_bytes_per_layer(self):
-        per = workloads.kv_bytes_per_token_head("k8v4" if self.fmt == self.nf.NF_KV_K8V4 else "bf16")
+        per = workloads.kv_bytes_per_token_head(self.fmt_name)
         return sum(self.w.seqlens) * self.w.num_kv_heads * per
 
     def decode_bytes_per_launch(self):
@@ -238,7 +239,7 @@ class GpuWorkload:
 
     def step_bytes(self):
         w = self.w
-        per = workloads.kv_bytes_per_token_head("k8v4" if self.fmt == self.nf.NF_KV_K8V4 else "bf16")
+        per = workloads.kv_bytes_per_token_head(self.fmt_name)
         app = w.batch * w.n_new * w.num_kv_heads * (per + 2 * 128 * 2)
         return w.layers * (self.decode_bytes_per_launch() + app)
 
@@ -313,7 +314,7 @@ def oracle_sample(w, fmt_name, budget_s=12.0, device="cpu"):
     until about budget_s seconds.  Returns (KV tokens/s, threads, description).
     KV tokens counts each key once per kv-head processed, scaled by 1 / H_kv."""
     import oracle
-    fmt = oracle.FMT_K8V4 if fmt_name == "k8v4" else oracle.FMT_BF16
+    fmt = {"k8v4": oracle.FMT_K8V4, "k8v8": oracle.FMT_K8V8, "bf16": oracle.FMT_BF16}[fmt_name]
     bt = workloads.block_table(w)
     pool = oracle.Pool(fmt, w.pool_blocks, 1, 128, poison=0)
     for b in range(w.batch):
@@ -340,13 +341,20 @@ def oracle_sample(w, fmt_name, budget_s=12.0, device="cpu"):
 
 
 # --------------------------------------------------------------------- main
+DTYPES = {
+    "k8v4": "s8/s4 KV codes, f16 tensor-core products, f32 softmax/accumulate",
+    "k8v8": "s8/s8 KV codes, f16 tensor-core products, f32 softmax/accumulate",
+    "bf16": "bf16 KV, bf16 tensor-core products, f32 softmax/accumulate",
+}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.ORDER)
-    ap.add_argument("--kv-format", default="k8v4", choices=["k8v4", "bf16"])
+    ap.add_argument("--kv-format", default="k8v4", choices=["k8v4", "k8v8", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
@@ -466,8 +474,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "s8/s4 KV codes, f16 tensor-core products, f32 softmax/accumulate"
-        if args.kv_format == "k8v4" else "bf16 KV, bf16 tensor-core products, f32 softmax/accumulate",
+        "vs_baseline": None, "dtype": DTYPES[args.kv_format],
         "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seqlens": list(w.seqlens), "n_q": w.n_q,
                    "n_new": w.n_new, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,

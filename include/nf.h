@@ -8,7 +8,8 @@
  *    Qwen3.8-27B：NInfer 上机实测（180K 上下文 / C2 并发 / 4bit KV）", section
  *    一.3 启动 (--kv-dtype rk8v4; int8 KV reaches 160K where rk8v4 reaches 180K
  *    at equal speed).  The pages do not define the bits; this header does (see
- *    nf_kv_layer).
+ *    nf_kv_layer).  The int8 KV dtype of the same section (--kv-dtype int8)
+ *    is NF_KV_K8V8.
  *  - A segmented KV cache in a pool of fixed capacity, one segment streamed
  *    at a time, decode tuned for one long request.  Page "標籤: vLLM", section
  *    2 "C++/CUDA 層的 kernel fusion 與 KV cache 策略"; page "3090 单卡跑
@@ -75,6 +76,7 @@ typedef int32_t nf_status;
 /* KV cache formats. */
 #define NF_KV_K8V4 0 /* the rk8v4 format defined below */
 #define NF_KV_BF16 1 /* unquantised bf16 K and V (for byte-count comparison) */
+#define NF_KV_K8V8 2 /* the int8 KV dtype defined below (K and V both int8) */
 
 /*
  * One layer's view of the caller-owned KV pool.
@@ -97,6 +99,13 @@ typedef int32_t nf_status;
  *     code  = clamp(round_half_even(fp32(x / float(scale))), -Q, Q), or 0 when
  *             scale is 0.
  *   Dequantised value = code * scale (exact in fp32).
+ * fmt NF_KV_K8V8 (the pages' int8 KV dtype; 260 bytes per token per kv-head):
+ *   k_codes  int8    [num_blocks][num_kv_heads][256][128]  K codes in [-127, 127]
+ *   k_scales fp16    [num_blocks][num_kv_heads][256]       one K scale per token
+ *   v_codes  int8    [num_blocks][num_kv_heads][256][128]  V codes in [-127, 127]
+ *   v_scales fp16    [num_blocks][num_kv_heads][256]       one V scale per token
+ *   K and V are both quantised by the K rule above (Q = 127, one scale per
+ *   token and kv-head); v_group is ignored.
  * fmt NF_KV_BF16 (512 bytes per token per kv-head):
  *   k_codes  bf16 [num_blocks][num_kv_heads][256][128]  (keys)
  *   v_codes  bf16 [num_blocks][num_kv_heads][256][128]  (values)
@@ -104,7 +113,7 @@ typedef int32_t nf_status;
  * Every plane must be 16-byte aligned.
  */
 typedef struct {
-    int32_t fmt;          /* NF_KV_K8V4 or NF_KV_BF16 */
+    int32_t fmt;          /* NF_KV_K8V4, NF_KV_K8V8 or NF_KV_BF16 */
     int32_t num_blocks;   /* pool capacity in blocks (>= 1) */
     int32_t block_size;   /* must be 256 */
     int32_t num_kv_heads; /* >= 1 */
@@ -177,8 +186,9 @@ size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_h
  *   (error below 2^-16 max|q| per element); the V codes are exact in fp16 and
  *   each softmax weight times its V scale is rounded to fp16 before the
  *   tensor-core P.V product; scores, softmax statistics and accumulators are
- *   fp32.  (bf16 cache: bf16 products, the fp32 query and the weights split
- *   into bf16 high and low parts.)
+ *   fp32.  (K8V8: the same, the int8 V codes exact in fp16 likewise; bf16
+ *   cache: bf16 products, the fp32 query and the weights split into bf16 high
+ *   and low parts.)
  * Launch: the kernel is launched with programmatic dependent launch, so it may
  *   start while the previous kernel on `stream` finishes; it waits for that
  *   kernel before reading any argument (see nf_decode_attn_ex for a weaker

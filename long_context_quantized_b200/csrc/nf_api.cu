@@ -50,8 +50,9 @@ nf_status after_launch(const char *what) {
 
 nf_status check_layer(const nf_kv_layer *kv) {
     if (!kv) return fail(NF_ERR_INVALID_ARG, "kv is NULL");
-    if (kv->fmt != NF_KV_K8V4 && kv->fmt != NF_KV_BF16)
-        return fail(NF_ERR_UNSUPPORTED, "kv->fmt %d is not NF_KV_K8V4 or NF_KV_BF16", kv->fmt);
+    if (kv->fmt != NF_KV_K8V4 && kv->fmt != NF_KV_K8V8 && kv->fmt != NF_KV_BF16)
+        return fail(NF_ERR_UNSUPPORTED, "kv->fmt %d is not NF_KV_K8V4, NF_KV_K8V8 or NF_KV_BF16", kv->fmt);
+    const bool scaled = kv->fmt != NF_KV_BF16;
     if (kv->block_size != nf::kBlock)
         return fail(NF_ERR_UNSUPPORTED, "kv->block_size %d (only 256)", kv->block_size);
     if (kv->head_dim != nf::kHeadDim)
@@ -62,11 +63,11 @@ nf_status check_layer(const nf_kv_layer *kv) {
         return fail(NF_ERR_INVALID_ARG, "kv->num_blocks %d / num_kv_heads %d must be >= 1",
                     kv->num_blocks, kv->num_kv_heads);
     if (!kv->k_codes || !kv->v_codes) return fail(NF_ERR_INVALID_ARG, "kv code planes are NULL");
-    if (kv->fmt == NF_KV_K8V4 && (!kv->k_scales || !kv->v_scales))
+    if (scaled && (!kv->k_scales || !kv->v_scales))
         return fail(NF_ERR_INVALID_ARG, "kv scale planes are NULL");
     auto misaligned = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) != 0; };
     if (misaligned(kv->k_codes) || misaligned(kv->v_codes) ||
-        (kv->fmt == NF_KV_K8V4 && (misaligned(kv->k_scales) || misaligned(kv->v_scales))))
+        (scaled && (misaligned(kv->k_scales) || misaligned(kv->v_scales))))
         return fail(NF_ERR_INVALID_ARG, "kv planes must be 16-byte aligned");
     return NF_OK;
 }
@@ -109,8 +110,10 @@ bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sm
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 std::once_flag g_encode_once;
 
-// Tensor map of a K8/V4 layer's V nibbles for the decode kernel: the plane as
-// [num_blocks * H_kv * 256 rows][64 bytes], 32-row boxes, 64-byte swizzle.
+// Tensor map of a quantised layer's V codes for the decode kernel: the plane as
+// [num_blocks * H_kv * 256 rows][row bytes], 32-row boxes, the swizzle as wide
+// as a row -- K8/V4 nibbles 64 bytes (64-byte swizzle), K8V8 codes 128 bytes
+// (128-byte swizzle).
 nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
@@ -123,12 +126,15 @@ nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map) {
     const cuuint64_t rows = (cuuint64_t)kv->num_blocks * (cuuint64_t)kv->num_kv_heads * nf::kBlock;
     if (rows > 0x7fffffffull)
         return fail(NF_ERR_UNSUPPORTED, "pool of %llu token rows per plane (at most 2^31 - 1)", (unsigned long long)rows);
-    const cuuint64_t dims[2] = {64, rows};
-    const cuuint64_t strides[1] = {64};
-    const cuuint32_t box[2] = {64, (cuuint32_t)nf::kChunk};
+    const bool v8 = kv->fmt == NF_KV_K8V8;
+    const cuuint64_t row_bytes = v8 ? 128 : 64;
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)nf::kChunk};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->v_codes, dims, strides, box, estr,
-                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                      CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                      v8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(NF_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
     return NF_OK;
@@ -180,6 +186,8 @@ template <int NT>
 cudaError_t dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, int ctas, cudaStream_t s) {
     if (fmt == NF_KV_K8V4)
         return qf32 ? launch_decode<NT, true, NF_KV_K8V4>(p, ctas, s) : launch_decode<NT, false, NF_KV_K8V4>(p, ctas, s);
+    if (fmt == NF_KV_K8V8)
+        return qf32 ? launch_decode<NT, true, NF_KV_K8V8>(p, ctas, s) : launch_decode<NT, false, NF_KV_K8V8>(p, ctas, s);
     return qf32 ? launch_decode<NT, true, NF_KV_BF16>(p, ctas, s) : launch_decode<NT, false, NF_KV_BF16>(p, ctas, s);
 }
 
@@ -325,7 +333,7 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
         return fail(NF_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
 
     nf::DecodeParams p{};
-    if (kv->fmt == NF_KV_K8V4) {
+    if (kv->fmt != NF_KV_BF16) {
         st = encode_v_map(kv, &p.vmap);
         if (st != NF_OK) return st;
     }

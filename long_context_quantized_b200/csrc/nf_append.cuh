@@ -5,7 +5,8 @@
 // One warp per (sequence, new token, kv-head); lane l owns channels 4l..4l+3.
 // K: absmax over the warp -> fp16 scale absmax/127 -> int8 codes (4 bytes per
 // lane, a coalesced 128-byte row).  V: absmax over each 8-lane group of 32
-// channels -> fp16 scale absmax/7 -> 4 nibbles per lane packed into 2 bytes.
+// channels -> fp16 scale absmax/7 -> 4 nibbles per lane packed into 2 bytes;
+// for the int8 KV dtype (same section, --kv-dtype int8) V takes the K rule.
 // Division and rounding are the IEEE fp32 ones (__fdiv_rn, round half to even),
 // subnormals kept, so the codes are bit-identical to the format definition.
 #pragma once
@@ -59,6 +60,21 @@ __device__ __forceinline__ int make_code(float x, float sigma, int q) {
     return min(max(c, -q), q);
 }
 
+// One 128-channel row held 4 channels per lane -> int8 codes (absmax / 127
+// scale, a coalesced 128-byte row) and its fp16 scale.
+__device__ __forceinline__ void quant_row8(const float (&x)[4], int lane, int8_t *codes, __half *scale) {
+    float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    float sigma;
+    const __half h = make_scale(a, 127.0f, sigma);
+    uint32_t c8 = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) c8 |= (uint32_t)(make_code(x[c], sigma, 127) & 0xFF) << (8 * c);
+    *reinterpret_cast<uint32_t *>(codes + 4 * lane) = c8;
+    if (lane == 0) *scale = h;
+}
+
 __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p) {
     pdl_wait();
     pdl_trigger();
@@ -101,16 +117,12 @@ __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p)
     }
 
     // ---- K: one scale per (token, kv-head)
-    float ak = fmaxf(fmaxf(fabsf(k[0]), fabsf(k[1])), fmaxf(fabsf(k[2]), fabsf(k[3])));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ak = fmaxf(ak, __shfl_xor_sync(0xffffffffu, ak, o));
-    float sk;
-    const __half hk = make_scale(ak, 127.0f, sk);
-    uint32_t kc = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) kc |= (uint32_t)(make_code(k[c], sk, 127) & 0xFF) << (8 * c);
-    *reinterpret_cast<uint32_t *>(static_cast<int8_t *>(p.k_codes) + si * kHeadDim + 4 * lane) = kc;
-    if (lane == 0) p.k_scales[si] = hk;
+    quant_row8(k, lane, static_cast<int8_t *>(p.k_codes) + si * kHeadDim, p.k_scales + si);
+    if (p.fmt == NF_KV_K8V8) {
+        // int8 KV: V by the same rule
+        quant_row8(v, lane, static_cast<int8_t *>(p.v_codes) + si * kHeadDim, p.v_scales + si);
+        return;
+    }
 
     // ---- V: one scale per 32 channels = 8 lanes
     float av = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));

@@ -183,14 +183,15 @@ __device__ __forceinline__ uint4 ldg16(const void *p) {
     return __ldg(reinterpret_cast<const uint4 *>(p));
 }
 
-// Four int8 codes (one per byte of w) -> two fp16x2: (c0, c1), (c2, c3).
-// Offset-binary trick: byte u = c + 128 placed under the exponent of 1024
-// gives the fp16 value 1024 + u exactly; subtracting 1152 leaves c exactly.
-__device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+// Four int8 codes (one per byte of w) -> two fp16x2: even = (c0, c2), odd =
+// (c1, c3).  Offset-binary trick: byte u = c + 128 placed under the exponent
+// of 1024 gives the fp16 value 1024 + u exactly; subtracting 1152 leaves c
+// exactly.
+__device__ __forceinline__ void i8x4_to_f16_eo(uint32_t w, uint32_t &even, uint32_t &odd) {
     const uint32_t u = w ^ 0x80808080u;
     const __half2 bias = u32_h2(0x64806480u);  // 1152, 1152
-    lo = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4140)), bias));
-    hi = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4342)), bias));
+    even = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4240)), bias));
+    odd = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4341)), bias));
 }
 
 // Packed two's-complement nibbles -> fp16x2 codes, exact.  For a word w with

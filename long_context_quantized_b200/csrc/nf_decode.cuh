@@ -1,5 +1,5 @@
 // nf_decode.cuh -- persistent split-K decode attention over the segmented
-// K8/V4 (or bf16) KV pool, with the log-sum-exp combine fused in.
+// K8/V4 (or int8, or bf16) KV pool, with the log-sum-exp combine fused in.
 //
 // The pages' engine streams the KV cache one segment at a time through the SM
 // and tunes decode for a single long request (page "標籤: vLLM", section 2
@@ -16,7 +16,7 @@
 //   query rows of a kv-head (GQA group x MTP queries) are served by the CTA
 //   that streams the keys, so each byte is fetched from HBM once.
 // Pipeline: a producer warp cuts each piece into stages of up to 256 keys
-//   (64 for the bf16 cache) inside one 256-key block and moves each stage's K
+//   (128 for the int8 cache, 64 for bf16) inside one 256-key block and moves each stage's K
 //   codes, V nibbles, K scales and V scales into a ring of shared-memory
 //   buffers on the TMA engine (1-D bulk copies; the V nibbles as 2-D tiles
 //   through a tensor map with the 64-byte swizzle, so that eight keys' rows
@@ -94,6 +94,20 @@ struct Stage<NF_KV_K8V4, NT> {
     static constexpr int kStages = 3;
     static constexpr int kUnitTiles = NT == 1 ? 2 : 1;  // 16-key m-tiles per consumer work unit
 };
+// int8 KV (K8V8): 260 bytes per key; 128-key stages, so that four fit beside
+// the merge buffer.  The V rows are 128 bytes, copied with the 128-byte swizzle.
+template <int NT>
+struct Stage<NF_KV_K8V8, NT> {
+    static constexpr int kTok = 128;
+    static constexpr int kK = 0;                      // int8 [kTok][128]
+    static constexpr int kV = kTok * 128;             // int8 [kTok][128] (swizzled)
+    static constexpr int kKs = kV + kTok * 128;       // fp16 [kTok]
+    static constexpr int kVs = kKs + kTok * 2;        // fp16 [kTok]
+    static constexpr int kBytesPerTok = 260;
+    static constexpr int kStride = (kTok * kBytesPerTok + 1023) / 1024 * 1024;
+    static constexpr int kStages = 4;
+    static constexpr int kUnitTiles = 1;  // 8 units of 16 keys per stage: one per consumer warp
+};
 template <int NT>
 struct Stage<NF_KV_BF16, NT> {
     static constexpr int kTok = 64;
@@ -107,7 +121,8 @@ struct Stage<NF_KV_BF16, NT> {
 };
 
 struct DecodeParams {
-    CUtensorMap vmap;  // K8/V4: v_codes as [num_blocks * H_kv * 256 rows][64 bytes], 32-row boxes, 64-byte swizzle
+    CUtensorMap vmap;  // v_codes as [num_blocks * H_kv * 256 rows][64 (K8/V4) or 128 (K8V8) bytes],
+                       // 32-row boxes, swizzle as wide as a row (unused for bf16)
     const void *k_codes;
     const __half *k_scales;
     const void *v_codes;
@@ -162,6 +177,10 @@ __device__ __forceinline__ int v_channel_k8v4(int m, int rho) {
     const int cg = m >> 1, ip = m & 1;
     return 32 * cg + 4 * (rho & 7) + 2 * ip + (rho >> 3);
 }
+// K8V8: m-tile m is the 16-byte column m (channels 16m..16m+15); row rho < 8
+// is channel 16m + 2rho (the low byte of b16 column rho), row rho + 8 the
+// channel after it.
+__device__ __forceinline__ int v_channel_k8v8(int m, int rho) { return 16 * m + 2 * (rho & 7) + (rho >> 3); }
 // bf16 cache: lane t's u-th 16-byte load holds channels 32u + 8t .. 32u + 8t + 7.
 __device__ __forceinline__ int v_channel_bf16(int m, int rho) {
     const int p = 2 * m + (rho >> 3), jj = rho & 7;
@@ -215,14 +234,14 @@ __device__ __forceinline__ int owner_cta(long long x, long long W, int P) {
 // kv-head) and the running softmax of the warp's rows.  In the S = Q . K^T
 // product the query rows are the M dimension: rows 0-7 of an A fragment are
 // the 8 query rows of tile nt (lane row g = query row 8nt + g), rows 8-15 a
-// second operand of the same rows -- the low int8 digit (K8/V4) or the low
+// second operand of the same rows -- the low int8 digit (int8 K) or the low
 // bf16 half of an fp32 query (bf16 cache; zero for a bf16 query) -- so one
 // product yields both parts.
 template <int NT, bool QF32, int FMT>
 struct WarpState {
-    static constexpr bool K8 = FMT == NF_KV_K8V4;
-    uint32_t qa[NT][K8 ? 4 : 8][4];  // A fragments per k-step (32 channels K8/V4, 16 channels bf16)
-    float qw[NT];                    // K8/V4: s / 254 x softmax scale x log2(e) of row g; bf16: the latter
+    static constexpr bool K8 = FMT != NF_KV_BF16;  // int8 K (K8/V4, K8V8)
+    uint32_t qa[NT][K8 ? 4 : 8][4];  // A fragments per k-step (32 channels int8 K, 16 channels bf16)
+    float qw[NT];                    // int8 K: s / 254 x softmax scale x log2(e) of row g; bf16: the latter
     float m_run[NT], l_run[NT];      // running max (log2 units) and weight sum of row g (lane's keys)
     float acc[8][NT][4];             // O^T fragments: channel rows, query columns 2t, 2t + 1
     int lim[NT];                     // last key position row g sees (-1: padding row)
@@ -241,7 +260,7 @@ template <int NT, int MT, bool QF32, int FMT, bool FAST>
 __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const unsigned char *st, int ub,
                                             int tok0, int L, int lane, const LaneOffsets &lo) {
     using ST = Stage<FMT, NT>;
-    constexpr bool K8 = FMT == NF_KV_K8V4;
+    constexpr bool K8 = FMT != NF_KV_BF16;  // int8 K codes
     const int g = lane >> 2, t = lane & 3;
 
     // ---- S = Q . K^T: per m-tile two n-tiles j of 8 keys; the lane's results are
@@ -369,7 +388,43 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
         const int tb = ub + 16 * mt;
-        if (K8) {
+        if (FMT == NF_KV_K8V8) {
+            // V scales of keys (2t, 2t+1) and (2t+8, 2t+9) as fp16 pairs: one
+            // scale per key serves all channels, so each B fragment takes it once
+            uint32_t sp0 = *reinterpret_cast<const uint32_t *>(st + ST::kVs + (tb + 2 * t) * 2);
+            uint32_t sp1 = *reinterpret_cast<const uint32_t *>(st + ST::kVs + (tb + 8 + 2 * t) * 2);
+            if (!FAST) {
+                // keys past the end hold stale bytes: zero their scales
+                const int pa = tok0 + tb + 2 * t;
+                sp0 &= (pa < L ? 0x0000FFFFu : 0u) | (pa + 1 < L ? 0xFFFF0000u : 0u);
+                sp1 &= (pa + 8 < L ? 0x0000FFFFu : 0u) | (pa + 9 < L ? 0xFFFF0000u : 0u);
+            }
+            uint32_t b0[NT], b1[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                b0[nt] = h2_u32(__hmul2(u32_h2(pb[mt][nt][0]), u32_h2(sp0)));
+                b1[nt] = h2_u32(__hmul2(u32_h2(pb[mt][nt][1]), u32_h2(sp1)));
+            }
+            // codes: matrix i of a load (lanes 8i..8i+7 address its rows) = keys
+            // tb + 8 (i & 1) + 0..7 of the 16-byte column 2cp + (i >> 1), which
+            // the swizzled copy stores at column position column ^ (key & 7); the
+            // lane receives channels 16 column + 2g, + 1 of keys 2t, 2t + 1
+            const uint32_t va = smem_addr(st + ST::kV + tb * 128) + lo.v;
+#pragma unroll
+            for (int cp = 0; cp < 4; ++cp) {
+                uint32_t R[4];
+                ldsm_x4_t(va ^ (32u * cp), R[0], R[1], R[2], R[3]);
+#pragma unroll
+                for (int jc = 0; jc < 2; ++jc) {
+                    uint32_t a[4];
+                    i8x4_to_f16_eo(R[2 * jc], a[0], a[1]);      // keys 2t, 2t+1: rows g, g + 8
+                    i8x4_to_f16_eo(R[2 * jc + 1], a[2], a[3]);  // keys 2t+8, 2t+9
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                        mma_f16(ws.acc[2 * cp + jc][nt], a[0], a[1], a[2], a[3], b0[nt], b1[nt]);
+                }
+            }
+        } else if (K8) {
             // nibbles: matrix cg (lanes 8cg..8cg+7 address its rows) = the 16-byte
             // column cg (channels 32cg..32cg+31) of 8 keys, stored at column
             // position cg ^ (row address bits 7-8) by the swizzled copy
@@ -577,7 +632,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     using ST = Stage<FMT, NT>;
     using SM = DecodeSmem<NT, FMT>;
     constexpr int MT = ST::kUnitTiles;
-    constexpr bool K8 = (FMT == NF_KV_K8V4);
+    constexpr bool K8 = (FMT != NF_KV_BF16);  // int8 K codes (K8/V4, K8V8)
+    constexpr bool V8 = (FMT == NF_KV_K8V8);  // int8 V codes, one V scale per key
     constexpr int NS = ST::kStages;
     constexpr int NR = SM::NR;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -696,11 +752,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             const size_t si = ((size_t)blk * H + walk.ph) * kBlock + (tok0 & (kBlock - 1));
                             mbar_arrive_expect_tx(&full[stage], (uint32_t)(ntok * ST::kBytesPerTok));
                             if (K8) {
+                                constexpr int vrow = V8 ? 128 : 64, vsc = V8 ? 1 : 4;  // V bytes, V scales per key
                                 bulk_g2s(st + ST::kK, static_cast<const int8_t *>(p.k_codes) + si * 128, ntok * 128, &full[stage]);
                                 for (int c = 0; c < ntok; c += kChunk)
-                                    tma_load_2d(st + ST::kV + c * 64, &p.vmap, 0, (int)si + c, &full[stage]);
+                                    tma_load_2d(st + ST::kV + c * vrow, &p.vmap, 0, (int)si + c, &full[stage]);
                                 bulk_g2s(st + ST::kKs, p.k_scales + si, ntok * 2, &full[stage]);
-                                bulk_g2s(st + ST::kVs, p.v_scales + si * 4, ntok * 8, &full[stage]);
+                                bulk_g2s(st + ST::kVs, p.v_scales + si * vsc, ntok * 2 * vsc, &full[stage]);
                             } else {
                                 bulk_g2s(st + ST::kK, static_cast<const __nv_bfloat16 *>(p.k_codes) + si * 128, ntok * 256, &full[stage]);
                                 bulk_g2s(st + ST::kV, static_cast<const __nv_bfloat16 *>(p.v_codes) + si * 128, ntok * 256, &full[stage]);
@@ -750,7 +807,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
 
     WarpState<NT, QF32, FMT> ws;
     LaneOffsets lo;
-    if (K8) {
+    if (V8) {
+        lo.k = g * 128 + 32 * t;
+        lo.ks = lo.vs = 0;
+        // ldmatrix row address of lane l: key 8 ((l >> 3) & 1) + (l & 7) of the
+        // m-tile, 16-byte column (l >> 4) stored at position (l >> 4) ^ (l & 7)
+        // (128-byte swizzle; m-tiles start on 2048-byte boundaries)
+        lo.v = (8 * (((uint32_t)lane >> 3) & 1u) + ((uint32_t)lane & 7u)) * 128 +
+               ((((uint32_t)lane >> 4) ^ ((uint32_t)lane & 7u)) * 16);
+    } else if (K8) {
         lo.k = g * 128 + 32 * t;
         lo.ks = 0;
         // the swizzled copy puts column c of key row r at position c ^ ((r >> 1) & 3)
@@ -931,8 +996,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                     }
 #pragma unroll
                     for (int m = 0; m < 8; ++m) {
-                        const int c0 = K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
-                        const int c1 = K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
+                        const int c0 = V8 ? v_channel_k8v8(m, g) : K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
+                        const int c1 = V8 ? v_channel_k8v8(m, g + 8)
+                                          : K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
                         buf[rr * 132 + c0] = ws.acc[m][nt][e] * f;
                         buf[rr * 132 + c1] = ws.acc[m][nt][2 + e] * f;
                     }

@@ -72,7 +72,7 @@ def oracle_pool(w, fmt, kvin, bt, heads=None):
 def compare_pool(kv, pool, heads):
     """Bit-exact comparison of every byte of the planes (for the listed heads)."""
     gpu = [t[:, heads].contiguous().view(torch.uint8).cpu().numpy() for t in kv.planes()]
-    ref = [a for a in pool.planes()] if kv.fmt == nf.NF_KV_K8V4 else [pool.k, pool.v]
+    ref = [a for a in pool.planes()] if kv.fmt != nf.NF_KV_BF16 else [pool.k, pool.v]
     for gp, rp in zip(gpu, ref):
         g8 = np.ascontiguousarray(gp).view(np.uint8).reshape(-1)
         r8 = np.ascontiguousarray(rp).view(np.uint8).reshape(-1)

@@ -18,7 +18,7 @@ from nfcase import ATOL, REL_L2, run_case, gpu_layer, oracle_pool, compare_pool,
 
 pytestmark = pytest.mark.gpu
 
-K8, BF = nf.NF_KV_K8V4, nf.NF_KV_BF16
+K8, BF, I8 = nf.NF_KV_K8V4, nf.NF_KV_BF16, nf.NF_KV_K8V8
 
 
 @pytest.fixture(autouse=True)
@@ -52,7 +52,7 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("fmt", [K8, BF], ids=["k8v4", "bf16"])
+@pytest.mark.parametrize("fmt", [K8, BF, I8], ids=["k8v4", "bf16", "k8v8"])
 @pytest.mark.parametrize("qdt", [torch.float32, torch.bfloat16], ids=["qf32", "qbf16"])
 @pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
 def test_small_shapes(case, qdt, fmt):
@@ -193,12 +193,18 @@ def test_workload_longest_bf16_cache_sampled_head():
     _full_size("longest", BF, heads=[5])
 
 
+@pytest.mark.parametrize("name,heads", [("ctx32k_append", [2]), ("mtp_verify", [1]), ("longest", [3])])
+def test_workload_int8_cache_sampled_heads(name, heads):
+    _full_size(name, I8, heads=heads)
+
+
 # ------------------------------------------- early KV streaming (flag path)
-@pytest.mark.parametrize("name,kw", [
-    ("mtp", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True)),
-    ("ragged", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2)),
+@pytest.mark.parametrize("name,kw,fmt", [
+    ("mtp", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True), K8),
+    ("ragged", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2), K8),
+    ("mtp_int8", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True), I8),
 ])
-def test_early_kv_back_to_back_layers(name, kw):
+def test_early_kv_back_to_back_layers(name, kw, fmt):
     # several layers of (append the step's tokens, decode) queued on one stream
     # without host syncs, so each decode kernel starts while the append before
     # it runs; with NF_DECODE_EARLY_KV the decode streams the older rows before
@@ -215,7 +221,7 @@ def test_early_kv_back_to_back_layers(name, kw):
     for flags in (0, nf.NF_DECODE_EARLY_KV):
         kvs, news, qs = [], [], []
         for layer in range(w.layers):
-            kv = nf.KVLayer.empty(K8, w.pool_blocks, w.num_kv_heads, device=dev, fill=0xA5)
+            kv = nf.KVLayer.empty(fmt, w.pool_blocks, w.num_kv_heads, device=dev, fill=0xA5)
             kn, vn = [], []
             for b in range(w.batch):
                 k, v = workloads.layer_kv(w, layer, b, device=dev)
@@ -245,7 +251,7 @@ def test_early_kv_back_to_back_layers(name, kw):
     # the last layer against the oracle
     layer = w.layers - 1
     kvin = [workloads.layer_kv(w, layer, b, device=dev) for b in range(w.batch)]
-    pool, hs = oracle_pool(w, K8, kvin, bt_np)
+    pool, hs = oracle_pool(w, fmt, kvin, bt_np)
     compare_pool(res[1][2][layer], pool, hs)
     ref_o, ref_l = oracle_attention(w, pool, hs, res[1][3][layer], bt_np)
     check_attention(res[1][0][layer], res[1][1][layer], ref_o, ref_l)
