@@ -1,4 +1,4 @@
-"""CPU oracle for K8/V4 (and int8 / bf16) KV-cache decode attention (test infrastructure).
+"""CPU oracle for K8/V4 (and int8 / fp8 / bf16) KV-cache decode attention (test infrastructure).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
 ``--impl reference`` legs of ``bench.py`` may import this package.  The product
@@ -31,6 +31,7 @@ _lib = None
 FMT_K8V4 = 0
 FMT_BF16 = 1
 FMT_K8V8 = 2
+FMT_F8 = 3
 BLOCK = 256
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
@@ -66,8 +67,14 @@ def _load():
                        "nfref_f32_to_bf16_n", "nfref_bf16_to_f32_n"):
                 getattr(lib, fn).argtypes = [P, P, ctypes.c_int64]
                 getattr(lib, fn).restype = None
+            lib.nfref_e4m3_encode_n.argtypes = [P, P, ctypes.c_int64]
+            lib.nfref_e4m3_encode_n.restype = None
+            lib.nfref_e4m3_decode_n.argtypes = [P, P, ctypes.c_int64]
+            lib.nfref_e4m3_decode_n.restype = None
             lib.nfref_quant_k.argtypes = [P, I, P, P]
             lib.nfref_quant_k.restype = None
+            lib.nfref_quant_f8.argtypes = [P, I, P, P]
+            lib.nfref_quant_f8.restype = None
             lib.nfref_quant_v.argtypes = [P, I, I, P, P]
             lib.nfref_quant_v.restype = None
             lib.nfref_append.argtypes = [I, I, I, I, P, P, P, P, P, P, I, I, P, I, P]
@@ -118,6 +125,15 @@ def bf16_bits_to_f32(h) -> np.ndarray:
     return _convert("nfref_bf16_to_f32_n", h, np.uint16, np.float32)
 
 
+def f32_to_e4m3_bits(x) -> np.ndarray:
+    """fp32 -> fp8 e4m3 bits, round half to even, saturating at +-448."""
+    return _convert("nfref_e4m3_encode_n", x, np.float32, np.uint8)
+
+
+def e4m3_bits_to_f64(b) -> np.ndarray:
+    return _convert("nfref_e4m3_decode_n", b, np.uint8, np.float64)
+
+
 # --------------------------------------------------------------- quantisation
 def quant_k(x):
     """One key vector (fp32, d values) -> (fp16 scale bits, int8 codes[d])."""
@@ -140,6 +156,17 @@ def quant_v(x, group: int = 32):
     return scales, packed
 
 
+def quant_f8(x):
+    """One key or value vector of the fp8 cache (fp32, d values) -> (fp16 scale
+    bits, e4m3 codes uint8[d])."""
+    lib = _load()
+    x = _c(x, np.float32)
+    codes = np.zeros(x.shape[-1], np.uint8)
+    scale = np.zeros(1, np.uint16)
+    lib.nfref_quant_f8(_ptr(x), x.shape[-1], _ptr(scale), _ptr(codes))
+    return scale[0], codes
+
+
 # ----------------------------------------------------------------------- pool
 class Pool:
     """One layer's host-side pool (planes laid out as in nfref.c)."""
@@ -152,10 +179,11 @@ class Pool:
             self.k_scale = np.zeros((num_blocks, num_kv_heads, BLOCK), np.uint16)
             self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 2), np.uint8)
             self.v_scale = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 32), np.uint16)
-        elif fmt == FMT_K8V8:
-            self.k = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), np.int8)
+        elif fmt in (FMT_K8V8, FMT_F8):
+            code = np.int8 if fmt == FMT_K8V8 else np.uint8
+            self.k = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), code)
             self.k_scale = np.zeros((num_blocks, num_kv_heads, BLOCK), np.uint16)
-            self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), np.int8)
+            self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), code)
             self.v_scale = np.zeros((num_blocks, num_kv_heads, BLOCK), np.uint16)
         else:
             self.k = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), np.uint16)

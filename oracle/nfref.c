@@ -180,6 +180,70 @@ static uint16_t quant_symmetric(const float *x, int n, float qmax, int *codes)
     return s16;
 }
 
+/* ------------------------------------------------------------------ */
+/* fp8 e4m3 (OCP "E4M3FN": 1 sign, 4 exponent bits with bias 7, 3      */
+/* mantissa bits; subnormals m * 2^-9; no infinities; 0x7F / 0xFF NaN; */
+/* largest finite 448), written from that definition.                 */
+/* ------------------------------------------------------------------ */
+
+/* fp32 -> e4m3, round half to even, saturating at +-448 (values beyond the
+ * largest finite one become it), the sign kept for zero results. */
+uint8_t nfref_e4m3_encode(float t)
+{
+    uint8_t sign = signbit(t) ? 0x80 : 0x00;
+    double a = fabs((double)t);
+    if (a > 448.0)
+        a = 448.0;
+    double v = round_to_grid(a, 4, -6);  /* 4 significant bits, emin = -6 */
+    if (v == 0.0)
+        return sign;
+    int e;
+    frexp(v, &e);
+    int E = e - 1;                        /* v in [2^E, 2^(E+1)) */
+    if (E < -6)
+        return (uint8_t)(sign | (uint8_t)(v / ldexp(1.0, -9)));
+    return (uint8_t)(sign | (uint8_t)(((E + 7) << 3) | (int)(v / ldexp(1.0, E - 3) - 8.0)));
+}
+
+double nfref_e4m3_decode(uint8_t b)
+{
+    if ((b & 0x7F) == 0x7F)
+        return NAN;
+    int E = (b >> 3) & 15, m = b & 7;
+    double v = E == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), E - 10);
+    return (b & 0x80) ? -v : v;
+}
+
+void nfref_e4m3_encode_n(const float *x, uint8_t *y, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        y[i] = nfref_e4m3_encode(x[i]);
+}
+void nfref_e4m3_decode_n(const uint8_t *x, double *y, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        y[i] = nfref_e4m3_decode(x[i]);
+}
+
+/* fp8 KV: d values -> one fp16 scale absmax/448 and d e4m3 codes of
+ * x / scale (fp32 division by the stored scale); all codes 0 when the scale
+ * is 0. */
+void nfref_quant_f8(const float *x, int d, uint16_t *scale, uint8_t *codes)
+{
+    float a = 0.0f;
+    for (int c = 0; c < d; ++c) {
+        float v = fabsf(x[c]);
+        if (v > a)
+            a = v;
+    }
+    float s32 = a / 448.0f;
+    uint16_t s16 = nfref_f32_to_f16(s32);
+    float sigma = nfref_f16_to_f32(s16);
+    for (int c = 0; c < d; ++c)
+        codes[c] = sigma == 0.0f ? 0 : nfref_e4m3_encode(x[c] / sigma);
+    *scale = s16;
+}
+
 /* K: d values -> one fp16 scale and d int8 codes. */
 void nfref_quant_k(const float *x, int d, uint16_t *scale, int8_t *codes)
 {
@@ -215,6 +279,8 @@ void nfref_quant_v(const float *x, int d, int group, uint16_t *scales, uint8_t *
  * fmt 2 (K8V8, int8 KV): k_plane, v_plane int8 [num_blocks][H][256][d]; k_scale,
  *   v_scale fp16 [num_blocks][H][256]; V quantised by the K rule (absmax/127
  *   per token and kv-head).
+ * fmt 3 (fp8 KV): k_plane, v_plane e4m3 bytes [num_blocks][H][256][d]; k_scale,
+ *   v_scale fp16 [num_blocks][H][256] (absmax/448 per token and kv-head).
  * Token position p of sequence b lives in block block_table[b][p / 256],
  * slot p % 256.
  */
@@ -229,6 +295,8 @@ static double k_hat(int fmt, const void *k_plane, const uint16_t *k_scale, size_
 {
     if (fmt == 1)
         return (double)nfref_bf16_to_f32(((const uint16_t *)k_plane)[si * d + c]);
+    if (fmt == 3)
+        return nfref_e4m3_decode(((const uint8_t *)k_plane)[si * d + c]) * (double)nfref_f16_to_f32(k_scale[si]);
     double code = (double)((const int8_t *)k_plane)[si * d + c];
     return code * (double)nfref_f16_to_f32(k_scale[si]);
 }
@@ -239,6 +307,8 @@ static double v_hat(int fmt, const void *v_plane, const uint16_t *v_scale, size_
         return (double)nfref_bf16_to_f32(((const uint16_t *)v_plane)[si * d + c]);
     if (fmt == 2)
         return (double)((const int8_t *)v_plane)[si * d + c] * (double)nfref_f16_to_f32(v_scale[si]);
+    if (fmt == 3)
+        return nfref_e4m3_decode(((const uint8_t *)v_plane)[si * d + c]) * (double)nfref_f16_to_f32(v_scale[si]);
     uint8_t byte = ((const uint8_t *)v_plane)[si * (size_t)(d / 2) + (size_t)(c / 2)];
     int nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
     int code = nib >= 8 ? nib - 16 : nib;
@@ -286,6 +356,9 @@ int nfref_append(int fmt, int num_blocks, int H, int d,
                 } else if (fmt == 2) {
                     nfref_quant_k(kx, d, &k_scale[si], (int8_t *)k_plane + si * d);
                     nfref_quant_k(vx, d, &v_scale[si], (int8_t *)v_plane + si * d);
+                } else if (fmt == 3) {
+                    nfref_quant_f8(kx, d, &k_scale[si], (uint8_t *)k_plane + si * d);
+                    nfref_quant_f8(vx, d, &v_scale[si], (uint8_t *)v_plane + si * d);
                 } else {
                     nfref_quant_k(kx, d, &k_scale[si], (int8_t *)k_plane + si * d);
                     nfref_quant_v(vx, d, 32, &v_scale[si * (size_t)(d / 32)],

@@ -1,6 +1,8 @@
 """Pins for the CPU oracle: it is checked against things other than itself.
 
-- IEEE conversions against numpy's / torch's own float16 and bfloat16 casts.
+- IEEE conversions against numpy's / torch's own float16 and bfloat16 casts;
+  the fp8 e4m3 conversions against torch's float8_e4m3fn type and a search
+  over all 254 finite codes.
 - The quantiser against a numpy re-derivation (numpy float32 division, float16
   cast, rint) and against hand-derived cases (tests/golden/).
 - Attention against closed forms (q = 0 gives the mean of the visible values,
@@ -47,6 +49,38 @@ def np_quant(x, qmax):
     return s16.view(np.uint16), np.clip(c, -qmax, qmax).astype(np.int64)
 
 
+def torch_e4m3(codes):
+    """fp64 values of e4m3 bytes through torch's own float8_e4m3fn type."""
+    t = torch.from_numpy(np.ascontiguousarray(codes, np.uint8))
+    return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def e4m3_table():
+    """The finite e4m3 codes and their values (torch's decoding)."""
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    return codes, torch_e4m3(codes)
+
+
+def brute_e4m3(x):
+    """Nearest finite e4m3 code of each fp32 value by search over all codes:
+    ties go to the code with the even mantissa, magnitudes past 448 to +-448,
+    a zero result keeps the sign of x."""
+    codes, vals = e4m3_table()
+    x = np.asarray(x, np.float32).astype(np.float64)
+    out = np.empty(x.shape, np.uint8)
+    for i, xv in enumerate(x.ravel()):
+        d = np.abs(vals - np.clip(xv, -448.0, 448.0))
+        best = np.flatnonzero(d == d.min())
+        if best.size > 1:
+            best = best[(codes[best] & 1) == 0]
+        c = codes[best]
+        if vals[best[0]] == 0.0:  # +0 and -0 tie: the sign of x decides
+            c = np.array([0x80 if np.signbit(xv) else 0x00])
+        assert c.size == 1
+        out.ravel()[i] = c[0]
+    return out
+
+
 def np_unpack_v(packed):
     p = np.asarray(packed, np.uint8).astype(np.int64)
     lo, hi = p & 0xF, p >> 4
@@ -69,6 +103,8 @@ def np_dequant_pool(pool):
     k = pool.k.astype(np.float64) * ks[..., None]
     if pool.fmt == oracle.FMT_K8V8:
         return k, pool.v.astype(np.float64) * vs[..., None]
+    if pool.fmt == oracle.FMT_F8:
+        return (torch_e4m3(pool.k) * ks[..., None], torch_e4m3(pool.v) * vs[..., None])
     vc = np_unpack_v(pool.v).astype(np.float64)
     v = vc * np.repeat(vs, 32, axis=-1)
     return k, v
@@ -317,6 +353,90 @@ def test_append_k8v8_quantises_v_by_the_k_rule():
     assert np.all(pool.v[1].view(np.uint8) == 0x5A) and np.all(pool.v[0, :, 300 - 256:].view(np.uint8) == 0x5A)
 
 
+def test_e4m3_decode_matches_torch_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_bits_to_f64(codes)
+    ref = torch_e4m3(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin])
+    assert np.array_equal(np.signbit(got[fin]), np.signbit(ref[fin]))
+    # the largest finite value and the smallest subnormal
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0xFE] == -448.0
+
+
+def test_e4m3_encode_is_the_nearest_code():
+    codes, vals = e4m3_table()
+    pos = np.unique(vals[vals > 0])
+    mids = (pos[:-1] + pos[1:]) / 2                     # exact ties (representable in fp32)
+    nudge = np.concatenate([np.nextafter(mids.astype(np.float32), np.float32(0)),
+                            np.nextafter(mids.astype(np.float32), np.float32(1e9))])
+    rnd = np.exp(RNG.uniform(np.log(1e-4), np.log(600.0), 4000)).astype(np.float32)
+    x = np.concatenate([mids.astype(np.float32), nudge, rnd, pos.astype(np.float32),
+                        np.float32([0.0, 1e-6, 2.0 ** -10, 448.0, 449.0, 463.9, 464.0, 500.0, 1e30])])
+    x = np.concatenate([x, -x, np.float32([-0.0, -1e-7])])
+    got = oracle.f32_to_e4m3_bits(x)
+    ref = brute_e4m3(x)
+    bad = np.flatnonzero(got != ref)
+    assert bad.size == 0, f"{bad.size} mismatches, e.g. x={x[bad[:4]]} got={got[bad[:4]]} ref={ref[bad[:4]]}"
+
+
+def test_e4m3_encode_matches_torch_cast_in_range():
+    # torch's own fp32 -> float8_e4m3fn cast (round half to even) inside +-448
+    x = np.concatenate([RNG.uniform(-448, 448, 20000), RNG.standard_normal(20000) * 0.01]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.f32_to_e4m3_bits(x), ref)
+
+
+def test_quant_f8_matches_numpy_statement_and_error_bound():
+    for trial in range(200):
+        mag = 10.0 ** RNG.uniform(-6, 4)
+        x = (RNG.standard_normal(128) * mag).astype(np.float32)
+        if trial % 7 == 0:
+            x[RNG.integers(128)] *= 50.0                    # an outlier channel
+        if trial == 3:
+            x[:] = 0.0
+        s16, codes = oracle.quant_f8(x)
+        a = np.max(np.abs(x)).astype(np.float32)
+        ref_s = np_f16_sat(np.float32(a) / np.float32(448.0))
+        assert s16 == ref_s.view(np.uint16)
+        sig = np.float32(ref_s)
+        if sig == 0:
+            assert np.all(codes == 0)
+            continue
+        assert np.array_equal(codes, brute_e4m3(np.clip(x / sig, -448, 448)))
+        # dequantised error of the values x / scale does not clamp: half a step
+        # of 3 mantissa bits, or half the subnormal spacing 2^-9, times the
+        # scale; clamped values (a scale rounded below absmax / 448, e.g. in the
+        # fp16 subnormal range) err by their excess over 448 scales
+        err = np.abs(torch_e4m3(codes) * np.float64(sig) - x.astype(np.float64))
+        t = np.abs(x.astype(np.float64)) / np.float64(sig)
+        unclamped = t <= 448.0
+        bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * np.float64(sig)) * (1 + 1e-6)
+        assert np.all(err[unclamped] <= bound[unclamped])
+        assert np.all(err[~unclamped] <= (t[~unclamped] - 448.0) * np.float64(sig) * (1 + 1e-6) + 1e-30)
+        if 2.0 ** -14 <= a / 448:                           # a normal fp16 scale: nothing clamps
+            assert unclamped.all() or np.max(t) < 448.0 * (1 + 2.0 ** -11)
+
+
+def test_append_f8_quantises_k_and_v():
+    rng = np.random.default_rng(29)
+    H, d, L = 2, 128, 260
+    pool = oracle.Pool(oracle.FMT_F8, 2, H, d, poison=0x5A)
+    bt = np.array([[1, 0]], np.int32)
+    k = (rng.standard_normal((1, L, H, d)) * rng.uniform(0.001, 30, (1, L, H, 1))).astype(np.float32)
+    v = (rng.standard_normal((1, L, H, d)) * rng.uniform(0.001, 30, (1, L, H, 1))).astype(np.float32)
+    v[0, 5, 0] = 0.0
+    assert oracle.append(pool, k, v, bt, np.array([0], np.int32)) == 0
+    for p_ in range(L):
+        blk, slot = bt[0, p_ // 256], p_ % 256
+        for h in range(H):
+            for src, codes, scales in ((k, pool.k, pool.k_scale), (v, pool.v, pool.v_scale)):
+                s16, c = oracle.quant_f8(src[0, p_, h])
+                assert scales[blk, h, slot] == s16 and np.array_equal(codes[blk, h, slot], c)
+    assert np.all(pool.v[0, :, L - 256:].view(np.uint8) == 0x5A)
+
+
 def test_append_rejects_out_of_range():
     pool = oracle.Pool(oracle.FMT_K8V4, 2, 1, 128)
     k = np.zeros((1, 1, 1, 128), np.float32)
@@ -328,7 +448,7 @@ def test_append_rejects_out_of_range():
 SCALE = float(np.float32(1 / math.sqrt(128)))
 
 
-@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8])
+@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8, oracle.FMT_F8])
 def test_attention_zero_query_is_mean_of_visible_values(fmt):
     # q = 0 -> all scores 0 -> o = mean of visible v_hat, lse = log(#visible).
     # Causal with n_q = 4: query j sees L - 4 + j + 1 keys.
@@ -427,7 +547,7 @@ def test_attention_split_and_combine_equals_whole():
     assert lse[0] == pytest.approx(lse_w, abs=1e-12)
 
 
-@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8])
+@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8, oracle.FMT_F8])
 @pytest.mark.parametrize("causal", [False, True])
 def test_attention_matches_numpy_brute_force(fmt, causal):
     cached = [300, 513]
