@@ -8,8 +8,8 @@
  *    Qwen3.8-27B：NInfer 上机实测（180K 上下文 / C2 并发 / 4bit KV）", section
  *    一.3 启动 (--kv-dtype rk8v4; int8 KV reaches 160K where rk8v4 reaches 180K
  *    at equal speed).  The pages do not define the bits; this header does (see
- *    nf_kv_layer).  The int8 KV dtype of the same section (--kv-dtype int8)
- *    is NF_KV_K8V8.
+ *    nf_kv_layer).  The int8 and fp8 KV dtypes of the same section
+ *    (--kv-dtype int8 / fp8) are NF_KV_K8V8 and NF_KV_F8.
  *  - A segmented KV cache in a pool of fixed capacity, one segment streamed
  *    at a time, decode tuned for one long request.  Page "標籤: vLLM", section
  *    2 "C++/CUDA 層的 kernel fusion 與 KV cache 策略"; page "3090 单卡跑
@@ -77,6 +77,7 @@ typedef int32_t nf_status;
 #define NF_KV_K8V4 0 /* the rk8v4 format defined below */
 #define NF_KV_BF16 1 /* unquantised bf16 K and V (for byte-count comparison) */
 #define NF_KV_K8V8 2 /* the int8 KV dtype defined below (K and V both int8) */
+#define NF_KV_F8 3   /* the fp8 KV dtype defined below (K and V both e4m3) */
 
 /*
  * One layer's view of the caller-owned KV pool.
@@ -106,6 +107,13 @@ typedef int32_t nf_status;
  *   v_scales fp16    [num_blocks][num_kv_heads][256]       one V scale per token
  *   K and V are both quantised by the K rule above (Q = 127, one scale per
  *   token and kv-head); v_group is ignored.
+ * fmt NF_KV_F8 (the pages' fp8 KV dtype; 260 bytes per token per kv-head):
+ *   k_codes, v_codes uint8 [num_blocks][num_kv_heads][256][128]  fp8 e4m3
+ *            codes (OCP E4M3FN: bias 7, 3 mantissa bits, largest finite 448)
+ *   k_scales, v_scales fp16 [num_blocks][num_kv_heads][256]  one scale per token
+ *   scale = fp16(fp32(max|x| / 448)) as above; code = e4m3(fp32(x / float(scale)))
+ *   rounded half to even and saturated at +-448 (a zero result keeps the sign
+ *   of x), or 0x00 when scale is 0.  Dequantised value = e4m3 value * scale.
  * fmt NF_KV_BF16 (512 bytes per token per kv-head):
  *   k_codes  bf16 [num_blocks][num_kv_heads][256][128]  (keys)
  *   v_codes  bf16 [num_blocks][num_kv_heads][256][128]  (values)
@@ -113,7 +121,7 @@ typedef int32_t nf_status;
  * Every plane must be 16-byte aligned.
  */
 typedef struct {
-    int32_t fmt;          /* NF_KV_K8V4, NF_KV_K8V8 or NF_KV_BF16 */
+    int32_t fmt;          /* NF_KV_K8V4, NF_KV_K8V8, NF_KV_F8 or NF_KV_BF16 */
     int32_t num_blocks;   /* pool capacity in blocks (>= 1) */
     int32_t block_size;   /* must be 256 */
     int32_t num_kv_heads; /* >= 1 */
@@ -186,7 +194,9 @@ size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_h
  *   (error below 2^-16 max|q| per element); the V codes are exact in fp16 and
  *   each softmax weight times its V scale is rounded to fp16 before the
  *   tensor-core P.V product; scores, softmax statistics and accumulators are
- *   fp32.  (K8V8: the same, the int8 V codes exact in fp16 likewise; bf16
+ *   fp32.  (K8V8: the same, the int8 V codes exact in fp16 likewise.  fp8:
+ *   the e4m3 codes are exact in fp16; S = Q . K^T uses fp16 products with each
+ *   query row split as q = s (hi + lo), s = max|q|, hi and lo fp16.  bf16
  *   cache: bf16 products, the fp32 query and the weights split into bf16 high
  *   and low parts.)
  * Launch: the kernel is launched with programmatic dependent launch, so it may

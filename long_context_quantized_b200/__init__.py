@@ -16,7 +16,7 @@ import threading
 import torch
 
 __all__ = [
-    "NF_OK", "NF_KV_K8V4", "NF_KV_BF16", "NF_KV_K8V8", "NF_F32", "NF_BF16", "NfError", "KVLayer",
+    "NF_OK", "NF_KV_K8V4", "NF_KV_BF16", "NF_KV_K8V8", "NF_KV_F8", "NF_F32", "NF_BF16", "NfError", "KVLayer",
     "nf_kv_append_quant", "nf_decode_attn_workspace_size", "nf_decode_attn", "nf_decode_attn_noalloc",
     "nf_attn_combine",
     "nf_get_device_error", "nf_status_string", "library_path", "load_library",
@@ -32,7 +32,7 @@ NF_ERR_INVALID_ARG, NF_ERR_UNSUPPORTED, NF_ERR_WORKSPACE, NF_ERR_CUDA, NF_ERR_DE
 NF_DEVERR_NONE, NF_DEVERR_BLOCK_ID, NF_DEVERR_TABLE, NF_DEVERR_SEQLEN = 0, 1, 2, 3
 NF_DEVERR_TIMEOUT, NF_DEVERR_INTERNAL = 4, 5
 NF_F32, NF_BF16, NF_F16 = 0, 1, 2
-NF_KV_K8V4, NF_KV_BF16, NF_KV_K8V8 = 0, 1, 2
+NF_KV_K8V4, NF_KV_BF16, NF_KV_K8V8, NF_KV_F8 = 0, 1, 2, 3
 BLOCK = 256
 HEAD_DIM = 128
 
@@ -158,10 +158,11 @@ class KVLayer:
             ks = torch.empty((num_blocks, num_kv_heads, BLOCK), dtype=torch.float16, **kw)
             v = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 2), dtype=torch.uint8, **kw)
             vs = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 32), dtype=torch.float16, **kw)
-        elif fmt == NF_KV_K8V8:
-            k = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM), dtype=torch.int8, **kw)
+        elif fmt in (NF_KV_K8V8, NF_KV_F8):
+            code = torch.int8 if fmt == NF_KV_K8V8 else torch.uint8  # fp8: e4m3 bytes
+            k = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM), dtype=code, **kw)
             ks = torch.empty((num_blocks, num_kv_heads, BLOCK), dtype=torch.float16, **kw)
-            v = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM), dtype=torch.int8, **kw)
+            v = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM), dtype=code, **kw)
             vs = torch.empty((num_blocks, num_kv_heads, BLOCK), dtype=torch.float16, **kw)
         elif fmt == NF_KV_BF16:
             k = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM), dtype=torch.bfloat16, **kw)

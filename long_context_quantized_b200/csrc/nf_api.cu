@@ -50,8 +50,9 @@ nf_status after_launch(const char *what) {
 
 nf_status check_layer(const nf_kv_layer *kv) {
     if (!kv) return fail(NF_ERR_INVALID_ARG, "kv is NULL");
-    if (kv->fmt != NF_KV_K8V4 && kv->fmt != NF_KV_K8V8 && kv->fmt != NF_KV_BF16)
-        return fail(NF_ERR_UNSUPPORTED, "kv->fmt %d is not NF_KV_K8V4, NF_KV_K8V8 or NF_KV_BF16", kv->fmt);
+    if (kv->fmt != NF_KV_K8V4 && kv->fmt != NF_KV_K8V8 && kv->fmt != NF_KV_F8 && kv->fmt != NF_KV_BF16)
+        return fail(NF_ERR_UNSUPPORTED, "kv->fmt %d is not NF_KV_K8V4, NF_KV_K8V8, NF_KV_F8 or NF_KV_BF16",
+                    kv->fmt);
     const bool scaled = kv->fmt != NF_KV_BF16;
     if (kv->block_size != nf::kBlock)
         return fail(NF_ERR_UNSUPPORTED, "kv->block_size %d (only 256)", kv->block_size);
@@ -112,8 +113,8 @@ std::once_flag g_encode_once;
 
 // Tensor map of a quantised layer's V codes for the decode kernel: the plane as
 // [num_blocks * H_kv * 256 rows][row bytes], 32-row boxes, the swizzle as wide
-// as a row -- K8/V4 nibbles 64 bytes (64-byte swizzle), K8V8 codes 128 bytes
-// (128-byte swizzle).
+// as a row -- K8/V4 nibbles 64 bytes (64-byte swizzle), K8V8 and fp8 codes
+// 128 bytes (128-byte swizzle).
 nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
@@ -126,7 +127,7 @@ nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map) {
     const cuuint64_t rows = (cuuint64_t)kv->num_blocks * (cuuint64_t)kv->num_kv_heads * nf::kBlock;
     if (rows > 0x7fffffffull)
         return fail(NF_ERR_UNSUPPORTED, "pool of %llu token rows per plane (at most 2^31 - 1)", (unsigned long long)rows);
-    const bool v8 = kv->fmt == NF_KV_K8V8;
+    const bool v8 = kv->fmt == NF_KV_K8V8 || kv->fmt == NF_KV_F8;
     const cuuint64_t row_bytes = v8 ? 128 : 64;
     const cuuint64_t dims[2] = {row_bytes, rows};
     const cuuint64_t strides[1] = {row_bytes};
@@ -188,6 +189,8 @@ cudaError_t dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, int c
         return qf32 ? launch_decode<NT, true, NF_KV_K8V4>(p, ctas, s) : launch_decode<NT, false, NF_KV_K8V4>(p, ctas, s);
     if (fmt == NF_KV_K8V8)
         return qf32 ? launch_decode<NT, true, NF_KV_K8V8>(p, ctas, s) : launch_decode<NT, false, NF_KV_K8V8>(p, ctas, s);
+    if (fmt == NF_KV_F8)
+        return qf32 ? launch_decode<NT, true, NF_KV_F8>(p, ctas, s) : launch_decode<NT, false, NF_KV_F8>(p, ctas, s);
     return qf32 ? launch_decode<NT, true, NF_KV_BF16>(p, ctas, s) : launch_decode<NT, false, NF_KV_BF16>(p, ctas, s);
 }
 

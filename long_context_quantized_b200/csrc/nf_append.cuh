@@ -6,7 +6,8 @@
 // K: absmax over the warp -> fp16 scale absmax/127 -> int8 codes (4 bytes per
 // lane, a coalesced 128-byte row).  V: absmax over each 8-lane group of 32
 // channels -> fp16 scale absmax/7 -> 4 nibbles per lane packed into 2 bytes;
-// for the int8 KV dtype (same section, --kv-dtype int8) V takes the K rule.
+// for the int8 KV dtype (same section, --kv-dtype int8) V takes the K rule; the
+// fp8 dtype (--kv-dtype fp8) stores e4m3 codes of x / (absmax / 448) for both.
 // Division and rounding are the IEEE fp32 ones (__fdiv_rn, round half to even),
 // subnormals kept, so the codes are bit-identical to the format definition.
 #pragma once
@@ -75,6 +76,21 @@ __device__ __forceinline__ void quant_row8(const float (&x)[4], int lane, int8_t
     if (lane == 0) *scale = h;
 }
 
+// The same row -> e4m3 codes of x / scale (scale absmax / 448), 0 when the
+// scale is 0.
+__device__ __forceinline__ void quant_row_f8(const float (&x)[4], int lane, uint8_t *codes, __half *scale) {
+    float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    float sigma;
+    const __half h = make_scale(a, 448.0f, sigma);
+    float t[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) t[c] = sigma == 0.0f ? 0.0f : __fdiv_rn(x[c], sigma);
+    *reinterpret_cast<uint32_t *>(codes + 4 * lane) = f32x4_to_e4m3(t[0], t[1], t[2], t[3]);
+    if (lane == 0) *scale = h;
+}
+
 __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p) {
     pdl_wait();
     pdl_trigger();
@@ -113,6 +129,12 @@ __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p)
         vb.x = pack_bf16(v[0], v[1]); vb.y = pack_bf16(v[2], v[3]);
         *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.k_codes) + si * kHeadDim + 4 * lane) = kb;
         *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.v_codes) + si * kHeadDim + 4 * lane) = vb;
+        return;
+    }
+
+    if (p.fmt == NF_KV_F8) {
+        quant_row_f8(k, lane, static_cast<uint8_t *>(p.k_codes) + si * kHeadDim, p.k_scales + si);
+        quant_row_f8(v, lane, static_cast<uint8_t *>(p.v_codes) + si * kHeadDim, p.v_scales + si);
         return;
     }
 

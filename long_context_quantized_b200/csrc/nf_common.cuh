@@ -194,6 +194,27 @@ __device__ __forceinline__ void i8x4_to_f16_eo(uint32_t w, uint32_t &even, uint3
     odd = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4341)), bias));
 }
 
+// fp8 e4m3 <-> fp16 / fp32 with the hardware conversions (sm_89 and later).
+// e4m3x4_to_f16: the four e4m3 bytes of w -> (b0, b1) and (b2, b3) as fp16x2,
+// exact (every e4m3 value is an fp16 value).
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+// Four fp32 values -> four e4m3 bytes (x0 in the low byte), each rounded half
+// to even and saturated at +-448.
+__device__ __forceinline__ uint32_t f32x4_to_e4m3(float x0, float x1, float x2, float x3) {
+    uint32_t d;
+    // cvt ... d16, a, b puts a in the upper byte and b in the lower one
+    asm("{\n\t.reg .b16 l, h;\n\tcvt.rn.satfinite.e4m3x2.f32 l, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;\n\tmov.b32 %0, {l, h};\n\t}"
+        : "=r"(d)
+        : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+    return d;
+}
+
 // Packed two's-complement nibbles -> fp16x2 codes, exact.  For a word w with
 // nibbles n0..n7 (n_k in bits 4k..4k+3):
 //   nib_even(w) = (n0, n4) as fp16 values in [-8, 7]

@@ -1,5 +1,5 @@
 // nf_decode.cuh -- persistent split-K decode attention over the segmented
-// K8/V4 (or int8, or bf16) KV pool, with the log-sum-exp combine fused in.
+// K8/V4 (or int8, fp8 or bf16) KV pool, with the log-sum-exp combine fused in.
 //
 // The pages' engine streams the KV cache one segment at a time through the SM
 // and tunes decode for a single long request (page "標籤: vLLM", section 2
@@ -36,7 +36,10 @@
 //   lane's K words land in B-fragment pairs as loaded.  The two int32 sums
 //   are recombined in fp32 and scaled by the key's K scale.  (The bf16 cache
 //   uses bf16 mma.sync the same way, the rows 8-15 holding the low half of an
-//   fp32 query.)
+//   fp32 query; the fp8 cache converts its e4m3 codes to fp16 with the
+//   hardware conversion and uses fp16 mma.sync, the query row scaled to
+//   max |q| = 1 and split into fp16 high and low parts.  The int8 and fp8 V
+//   codes become fp16 pairs the same way, one V scale per key.)
 //   O^T += V_codes^T . (P^T x sigma_V) (mma.sync m16n8k16 fp16, fp32
 //   accumulate): the score fragment of S is already the B-fragment layout of
 //   P^T; ldmatrix.trans hands each lane the nibbles of one channel for two
@@ -108,6 +111,9 @@ struct Stage<NF_KV_K8V8, NT> {
     static constexpr int kStages = 4;
     static constexpr int kUnitTiles = 1;  // 8 units of 16 keys per stage: one per consumer warp
 };
+// fp8 KV: the same bytes per key and layout as K8V8 (e4m3 codes for int8 ones).
+template <int NT>
+struct Stage<NF_KV_F8, NT> : Stage<NF_KV_K8V8, NT> {};
 template <int NT>
 struct Stage<NF_KV_BF16, NT> {
     static constexpr int kTok = 64;
@@ -177,7 +183,7 @@ __device__ __forceinline__ int v_channel_k8v4(int m, int rho) {
     const int cg = m >> 1, ip = m & 1;
     return 32 * cg + 4 * (rho & 7) + 2 * ip + (rho >> 3);
 }
-// K8V8: m-tile m is the 16-byte column m (channels 16m..16m+15); row rho < 8
+// K8V8 and fp8: m-tile m is the 16-byte column m (channels 16m..16m+15); row rho < 8
 // is channel 16m + 2rho (the low byte of b16 column rho), row rho + 8 the
 // channel after it.
 __device__ __forceinline__ int v_channel_k8v8(int m, int rho) { return 16 * m + 2 * (rho & 7) + (rho >> 3); }
@@ -239,9 +245,9 @@ __device__ __forceinline__ int owner_cta(long long x, long long W, int P) {
 // product yields both parts.
 template <int NT, bool QF32, int FMT>
 struct WarpState {
-    static constexpr bool K8 = FMT != NF_KV_BF16;  // int8 K (K8/V4, K8V8)
-    uint32_t qa[NT][K8 ? 4 : 8][4];  // A fragments per k-step (32 channels int8 K, 16 channels bf16)
-    float qw[NT];                    // int8 K: s / 254 x softmax scale x log2(e) of row g; bf16: the latter
+    static constexpr bool K8 = FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8;  // int8 K
+    uint32_t qa[NT][K8 ? 4 : 8][4];  // A fragments per k-step (32 channels int8 K, 16 channels fp16 / bf16)
+    float qw[NT];                    // int8 K: s / 254, fp8 K: s, bf16: 1; times softmax scale x log2(e)
     float m_run[NT], l_run[NT];      // running max (log2 units) and weight sum of row g (lane's keys)
     float acc[8][NT][4];             // O^T fragments: channel rows, query columns 2t, 2t + 1
     int lim[NT];                     // last key position row g sees (-1: padding row)
@@ -260,7 +266,9 @@ template <int NT, int MT, bool QF32, int FMT, bool FAST>
 __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const unsigned char *st, int ub,
                                             int tok0, int L, int lane, const LaneOffsets &lo) {
     using ST = Stage<FMT, NT>;
-    constexpr bool K8 = FMT != NF_KV_BF16;  // int8 K codes
+    constexpr bool K8 = FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8;  // int8 K codes
+    constexpr bool F8 = FMT == NF_KV_F8;                           // e4m3 K and V codes
+    constexpr bool PF16 = FMT != NF_KV_BF16;                       // fp16 weights and V codes
     const int g = lane >> 2, t = lane & 3;
 
     // ---- S = Q . K^T: per m-tile two n-tiles j of 8 keys; the lane's results are
@@ -272,7 +280,30 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             // K^T B fragments: the lane's column is key tb + 8j + g
-            if (K8) {
+            if (F8) {
+                // e4m3 bytes 32t..32t+31 of the key -> fp16 pairs; k-step ks takes
+                // channels 32t + 4ks + 0, 1 (b0) and + 2, 3 (b1), the order the
+                // query fragments were written in
+                const unsigned char *k0 = st + ST::kK + (tb + 8 * j) * 128 + lo.k;
+                const uint4 w0 = lds128(k0), w1 = lds128(k0 + 16);
+                const uint32_t kw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint32_t kb[8][2];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) e4m3x4_to_f16(kw[u], kb[u][0], kb[u][1]);
+                const float2 sk = __half22float2(
+                    *reinterpret_cast<const __half2 *>(st + ST::kKs + (tb + 8 * j + 2 * t) * 2));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(d, ws.qa[nt][ks][0], ws.qa[nt][ks][1], ws.qa[nt][ks][2], ws.qa[nt][ks][3], kb[ks][0],
+                                kb[ks][1]);
+                    // d0, d1: the high fp16 part of the row . keys 2t, 2t+1; d2, d3: the low part
+                    xv[mt][nt][2 * j] = (d[0] + d[2]) * (ws.qw[nt] * sk.x);
+                    xv[mt][nt][2 * j + 1] = (d[1] + d[3]) * (ws.qw[nt] * sk.y);
+                }
+            } else if (K8) {
                 const unsigned char *k0 = st + ST::kK + (tb + 8 * j) * 128 + lo.k;  // bytes 32t..32t+31
                 const uint4 w0 = lds128(k0), w1 = lds128(k0 + 16);
                 const uint32_t kb[4][2] = {{w0.x, w0.y}, {w0.z, w0.w}, {w1.x, w1.y}, {w1.z, w1.w}};
@@ -370,7 +401,7 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
             const float p0 = ex2(xv[mt][nt][0] - mu), p1 = ex2(xv[mt][nt][1] - mu);
             const float p2 = ex2(xv[mt][nt][2] - mu), p3 = ex2(xv[mt][nt][3] - mu);
             ws.l_run[nt] += (p0 + p1) + (p2 + p3);
-            if (K8) {
+            if (PF16) {
                 pb[mt][nt][0] = pack_f16(p0, p1);
                 pb[mt][nt][1] = pack_f16(p2, p3);
             } else {
@@ -388,16 +419,22 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
         const int tb = ub + 16 * mt;
-        if (FMT == NF_KV_K8V8) {
+        if (FMT == NF_KV_K8V8 || F8) {
             // V scales of keys (2t, 2t+1) and (2t+8, 2t+9) as fp16 pairs: one
             // scale per key serves all channels, so each B fragment takes it once
             uint32_t sp0 = *reinterpret_cast<const uint32_t *>(st + ST::kVs + (tb + 2 * t) * 2);
             uint32_t sp1 = *reinterpret_cast<const uint32_t *>(st + ST::kVs + (tb + 8 + 2 * t) * 2);
+            // keys past the end hold stale bytes: zero their scales (and, for
+            // e4m3, whose stale bytes may be NaN, their codes: the lane's code
+            // word holds key 2t in bytes 0-1 and key 2t+1 in bytes 2-3, the
+            // layout of a scale pair)
+            uint32_t keep0 = 0xFFFFFFFFu, keep1 = 0xFFFFFFFFu;
             if (!FAST) {
-                // keys past the end hold stale bytes: zero their scales
                 const int pa = tok0 + tb + 2 * t;
-                sp0 &= (pa < L ? 0x0000FFFFu : 0u) | (pa + 1 < L ? 0xFFFF0000u : 0u);
-                sp1 &= (pa + 8 < L ? 0x0000FFFFu : 0u) | (pa + 9 < L ? 0xFFFF0000u : 0u);
+                keep0 = (pa < L ? 0x0000FFFFu : 0u) | (pa + 1 < L ? 0xFFFF0000u : 0u);
+                keep1 = (pa + 8 < L ? 0x0000FFFFu : 0u) | (pa + 9 < L ? 0xFFFF0000u : 0u);
+                sp0 &= keep0;
+                sp1 &= keep1;
             }
             uint32_t b0[NT], b1[NT];
 #pragma unroll
@@ -417,8 +454,16 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
 #pragma unroll
                 for (int jc = 0; jc < 2; ++jc) {
                     uint32_t a[4];
-                    i8x4_to_f16_eo(R[2 * jc], a[0], a[1]);      // keys 2t, 2t+1: rows g, g + 8
-                    i8x4_to_f16_eo(R[2 * jc + 1], a[2], a[3]);  // keys 2t+8, 2t+9
+                    if (F8) {
+                        // bytes (0, 2) and (1, 3) -> fp16 pairs: rows g and g + 8
+                        const uint32_t r0 = prmt(FAST ? R[2 * jc] : R[2 * jc] & keep0, 0u, 0x3120);
+                        const uint32_t r1 = prmt(FAST ? R[2 * jc + 1] : R[2 * jc + 1] & keep1, 0u, 0x3120);
+                        e4m3x4_to_f16(r0, a[0], a[1]);
+                        e4m3x4_to_f16(r1, a[2], a[3]);
+                    } else {
+                        i8x4_to_f16_eo(R[2 * jc], a[0], a[1]);      // keys 2t, 2t+1: rows g, g + 8
+                        i8x4_to_f16_eo(R[2 * jc + 1], a[2], a[3]);  // keys 2t+8, 2t+9
+                    }
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
                         mma_f16(ws.acc[2 * cp + jc][nt], a[0], a[1], a[2], a[3], b0[nt], b1[nt]);
@@ -632,8 +677,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     using ST = Stage<FMT, NT>;
     using SM = DecodeSmem<NT, FMT>;
     constexpr int MT = ST::kUnitTiles;
-    constexpr bool K8 = (FMT != NF_KV_BF16);  // int8 K codes (K8/V4, K8V8)
-    constexpr bool V8 = (FMT == NF_KV_K8V8);  // int8 V codes, one V scale per key
+    constexpr bool K8 = (FMT != NF_KV_BF16);  // scaled codes through the bulk/tensor-map copies
+    constexpr bool V8 = (FMT == NF_KV_K8V8 || FMT == NF_KV_F8);  // 128-byte V rows, one V scale per key
+    constexpr bool F8 = (FMT == NF_KV_F8);
+    static_assert(SM::kMergeM - SM::kMergeO >= (kMaxRows * 128 + (NT == 1 ? 8 : kMaxRows)) * 4,
+                  "fp8 query fragments and factors in the merge buffer");
     constexpr int NS = ST::kStages;
     constexpr int NR = SM::NR;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -835,15 +883,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         const int b = walk.pb, h = walk.ph;
         const int L = seqC[b] ? p.seqlens[b] : 0;
         // query fragments of this (sequence, kv-head): lane (g, t) holds row g of
-        // tile nt, channels 32t..32t+31 (K8/V4: k-step ks takes channels 32t + 8ks
-        // + 0..3 and + 4..7) or 32u + 8t + 4h + 0..3 (bf16 cache: k-step 2u + h)
+        // tile nt, channels 32t..32t+31 (int8 K: k-step ks takes channels 32t + 8ks
+        // + 0..3 and + 4..7; fp8 K: 32t + 4ks + 0..3) or 32u + 8t + 4h + 0..3
+        // (bf16 cache: k-step 2u + h)
         if (K8) {
-            // The digits are computed once per CTA into the (idle) merge buffer:
-            // warp w encodes rows w, w + 8, ...; lane l takes channels 4l..4l+3 =
-            // 32t + 8ks + 4hh + e (t = l / 8, ks = l / 2 % 4, hh = l % 2).  Layout
-            // [row][t][ks][d1 word hh=0, d2 word hh=0, d1 word hh=1, d2 word hh=1].
+            // The fragments are computed once per CTA into the (idle) merge buffer:
+            // warp w encodes rows w, w + 8, ...; lane l takes channels 4l..4l+3.
+            // int8 K: 4l..4l+3 = 32t + 8ks + 4hh + e (t = l / 8, ks = l / 2 % 4,
+            // hh = l % 2); layout [row][t][ks][d1 word hh=0, d2 word hh=0, d1 word
+            // hh=1, d2 word hh=1].  fp8 K: 4l..4l+3 = 32t + 4ks + e (t = l / 8,
+            // ks = l % 8); layout [row][t][ks][hi e=0,1; lo e=0,1; hi e=2,3; lo
+            // e=2,3] (an f16 A fragment: rows g hold hi, rows g + 8 lo).
             uint32_t *qsm = reinterpret_cast<uint32_t *>(sm_o);
-            float *qwsm = reinterpret_cast<float *>(sm_o) + kMaxRows * 64;
+            float *qwsm = reinterpret_cast<float *>(sm_o) + kMaxRows * (F8 ? 128 : 64);
             for (int r = warp; r < p.rows; r += kConsumerWarps) {
                 const int j = r / p.group, gq = r % p.group;
                 const size_t qoff =
@@ -862,6 +914,23 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                if (F8) {
+                    // q = s (hi + lo), s = max|q|: |q / s| <= 1 stays inside fp16,
+                    // hi = fp16(q / s), lo = fp16(q / s - hi)
+                    const float inv = amax > 0.f ? 1.0f / amax : 0.f;
+                    float y[4], hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        y[e] = x[e] * inv;
+                        hi[e] = __half2float(__float2half_rn(y[e]));
+                        lo[e] = y[e] - hi[e];
+                    }
+                    const uint4 frag = make_uint4(pack_f16(hi[0], hi[1]), pack_f16(lo[0], lo[1]), pack_f16(hi[2], hi[3]),
+                                                  pack_f16(lo[2], lo[3]));
+                    *reinterpret_cast<uint4 *>(qsm + (r * 4 + (lane >> 3)) * 32 + (lane & 7) * 4) = frag;
+                    if (lane == 0) qwsm[r] = amax * p.scale_log2;
+                    continue;
+                }
                 // q ~= s (d1 + d2 / 254), s = max|q| / 127, digits in [-127, 127]
                 const float s1 = amax / 127.0f;
                 const float inv = amax > 0.f ? 127.0f / amax : 0.f;
@@ -884,9 +953,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             for (int nt = 0; nt < NT; ++nt) {
                 const int r = row0 + nt * 8 + g;
                 const bool rv = r < p.rows;
+                constexpr int KS = F8 ? 8 : 4;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint4 v = rv ? lds128(qsm + (r * 4 + t) * 16 + ks * 4) : make_uint4(0, 0, 0, 0);
+                for (int ks = 0; ks < KS; ++ks) {
+                    const uint4 v = rv ? lds128(qsm + (r * 4 + t) * (4 * KS) + ks * 4) : make_uint4(0, 0, 0, 0);
                     ws.qa[nt][ks][0] = v.x; ws.qa[nt][ks][1] = v.y; ws.qa[nt][ks][2] = v.z; ws.qa[nt][ks][3] = v.w;
                 }
                 ws.qw[nt] = rv ? qwsm[r] : 0.f;

@@ -18,7 +18,7 @@ from nfcase import ATOL, REL_L2, run_case, gpu_layer, oracle_pool, compare_pool,
 
 pytestmark = pytest.mark.gpu
 
-K8, BF, I8 = nf.NF_KV_K8V4, nf.NF_KV_BF16, nf.NF_KV_K8V8
+K8, BF, I8, F8 = nf.NF_KV_K8V4, nf.NF_KV_BF16, nf.NF_KV_K8V8, nf.NF_KV_F8
 
 
 @pytest.fixture(autouse=True)
@@ -52,7 +52,7 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("fmt", [K8, BF, I8], ids=["k8v4", "bf16", "k8v8"])
+@pytest.mark.parametrize("fmt", [K8, BF, I8, F8], ids=["k8v4", "bf16", "k8v8", "f8"])
 @pytest.mark.parametrize("qdt", [torch.float32, torch.bfloat16], ids=["qf32", "qbf16"])
 @pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
 def test_small_shapes(case, qdt, fmt):
@@ -198,11 +198,17 @@ def test_workload_int8_cache_sampled_heads(name, heads):
     _full_size(name, I8, heads=heads)
 
 
+@pytest.mark.parametrize("name,heads", [("ctx32k_append", [1]), ("mtp_verify", [3]), ("longest", [6])])
+def test_workload_fp8_cache_sampled_heads(name, heads):
+    _full_size(name, F8, heads=heads)
+
+
 # ------------------------------------------- early KV streaming (flag path)
 @pytest.mark.parametrize("name,kw,fmt", [
     ("mtp", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True), K8),
     ("ragged", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2), K8),
     ("mtp_int8", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True), I8),
+    ("ragged_fp8", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2), F8),
 ])
 def test_early_kv_back_to_back_layers(name, kw, fmt):
     # several layers of (append the step's tokens, decode) queued on one stream
