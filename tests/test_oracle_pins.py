@@ -564,6 +564,28 @@ def test_attention_matches_numpy_brute_force(fmt, causal):
     assert np.array_equal(o2, out[rows]) and np.array_equal(l2, lse[rows])
 
 
+@pytest.mark.parametrize("n_q", [160, 37])
+def test_attention_prefill_chunk_matches_torch_sdpa(n_q):
+    # a prefill chunk (many causal queries, the last n_q positions; n_q = L is
+    # a whole prompt) against torch's own scaled_dot_product_attention in fp64
+    # over the numpy-dequantised pool, the causal mask stated as positions
+    L = 160
+    pool, bt, _, _ = make_pool(oracle.FMT_K8V4, [L], H=2, seed=31)
+    q = RNG.standard_normal((1, n_q, 4, 128)).astype(np.float32)
+    out, lse = oracle.decode_attn(pool, q, bt, [L], SCALE, True, nthreads=2)
+    kh, vh = np_dequant_pool(pool)
+    pos = np.arange(L)
+    K = torch.from_numpy(kh[bt[0, pos // 256], :, pos % 256].transpose(1, 0, 2).copy())   # [H_kv][L][d]
+    V = torch.from_numpy(vh[bt[0, pos // 256], :, pos % 256].transpose(1, 0, 2).copy())
+    K, V = K.repeat_interleave(2, dim=0), V.repeat_interleave(2, dim=0)                    # GQA 2
+    Q = torch.from_numpy(q[0].astype(np.float64)).transpose(0, 1)                          # [H_q][n_q][d]
+    qpos = torch.arange(L - n_q, L)[:, None]
+    mask = torch.arange(L)[None, :] <= qpos                                                # True = attend
+    ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask,
+                                                           scale=float(np.float32(SCALE)))
+    assert np.allclose(out.reshape(n_q, 4, 128), ref.transpose(0, 1).numpy(), rtol=1e-10, atol=1e-12)
+
+
 def test_attention_softmax_scale_is_used():
     # doubling q and halving the scale leaves every score, hence o, unchanged;
     # a different scale changes o
