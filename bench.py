@@ -9,6 +9,10 @@ the C ABI.  Prints ONE JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--kv-format k8v4|k8v8|f8|bf16] [--impl ours|reference]
 
+--workload prefill_chunk measures chunked-prefill attention instead: per layer
+the 1024-token chunk's append and nf_prefill_attn, reported as chunk tokens/s
+and the prefill kernel's TFLOP/s against the measured tensor-core peak.
+
 Metric: KV tokens/s (each cached key counted once per layer, heads not
 multiplied) and the decode kernel's achieved HBM GB/s against the measured B200
 copy bandwidth.  Inputs are seeded synthetic tensors of the workload's shape,
@@ -307,6 +311,191 @@ def time_decode_launches(gw, steps, stream):
     return tot / n
 
 
+def measure_e2e(gw, args, stream, device):
+    """End to end: the step's inputs (every layer's q and new K/V) copied from
+    pinned host memory, the step, every layer's output copied back; returns
+    (ms per step, max over ranks; H2D bytes; D2H bytes)."""
+    h_in = [gw.q_all.cpu().pin_memory()]
+    d_in = [gw.q_all]
+    if gw.w.n_new:
+        h_in += [gw.knew_all.cpu().pin_memory(), gw.vnew_all.cpu().pin_memory()]
+        d_in += [gw.knew_all, gw.vnew_all]
+    h_out = torch.empty_like(gw.out_all, device="cpu").pin_memory()
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=stream):
+        for d, hsrc in zip(d_in, h_in):
+            d.copy_(hsrc, non_blocking=True)
+        gw.step()
+        h_out.copy_(gw.out_all, non_blocking=True)
+    e2e_ms = time_graph(ge, args.steps, max(3, args.warmup), stream)
+    e2e_ms = max_over_ranks(e2e_ms, device)
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+    del ge
+    torch.cuda.synchronize()
+    return e2e_ms, h2d, d2h
+
+
+# ------------------------------------------------------- chunked prefill leg
+PREFILL_METRIC = "prefill chunk tokens/s through chunked-prefill attention over the K8/V4 cache (all layers)"
+PREFILL_UNIT = "tokens/s"
+
+
+class PrefillWorkload(GpuWorkload):
+    """The last chunk of a prompt: per layer the chunk's K/V appended, then
+    nf_prefill_attn of its n_q queries against the whole cache."""
+
+    def decode(self, layer):
+        w = self.w
+        self.nf.nf_prefill_attn(self.layers[layer], self.q[layer], self.bt, self.seqlens, self.max_seqlen,
+                                w.softmax_scale, w.causal, self.out[layer], None)
+
+    def flops_per_launch(self):
+        """2 x 2 x d per (query row, visible key): S = Q . K^T and O = P . V."""
+        w = self.w
+        keys = 0
+        for L in w.seqlens:
+            if w.causal:
+                keys += sum(L - w.n_q + j + 1 for j in range(w.n_q))
+            else:
+                keys += L * w.n_q
+        return 4 * w.head_dim * w.num_q_heads * keys
+
+
+def prefill_oracle_sample(w, budget_s=12.0, device="cpu"):
+    """Time the oracle on rows of the chunk (layer 0, kv-head 0, positions
+    spread over the chunk, all G heads), about budget_s seconds.  Returns
+    (chunk tokens/s for the whole step, threads, description, s per rep)."""
+    import oracle
+    bt = workloads.block_table(w)
+    pool = oracle.Pool(oracle.FMT_K8V4, w.pool_blocks, 1, 128, poison=0)
+    for b in range(w.batch):
+        k, v = workloads.layer_kv(w, 0, b, device=device)
+        oracle.append(pool, k[:, :1].float().cpu().numpy()[None], v[:, :1].float().cpu().numpy()[None],
+                      bt[b:b + 1], np.zeros(1, np.int32))
+        del k, v
+    q = workloads.layer_q(w, 0, device=device)[:, :, :w.group].float().cpu().numpy()
+    threads = os.cpu_count() or 1
+    sl = np.array(w.seqlens, np.int32)
+    pos = np.linspace(0, w.n_q - 1, max(1, min(w.n_q, 2 * threads))).round().astype(np.int64)
+    rows = np.array([j * w.group + gh for j in pos for gh in range(w.group)], np.int64)
+    reps, t_tot = 0, 0.0
+    while True:
+        t0 = time.perf_counter()
+        oracle.decode_attn(pool, q, bt, sl, w.softmax_scale, w.causal, rows=rows, nthreads=threads)
+        t_tot += time.perf_counter() - t0
+        reps += 1
+        if t_tot >= budget_s or reps >= 50:
+            break
+    rows_per_s = len(rows) * reps / t_tot
+    value = rows_per_s / (w.num_q_heads * w.layers)  # a chunk token is H_q rows in each layer
+    desc = (f"oracle (C, fp64 attention) on {threads} host threads: {len(rows)} query rows (positions "
+            f"spread over the {w.n_q}-token chunk, all {w.group} heads of kv-head 0, layer 0), {reps} "
+            f"repetition(s), {t_tot:.1f} s; tokens = rows / (H_q x layers)")
+    return value, threads, desc, t_tot / reps
+
+
+def prefill_main(args, w, ws, rank, local):
+    import long_context_quantized_b200 as nf
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        value, threads, desc, _ = prefill_oracle_sample(w, budget_s=min(12.0, 3.0 * max(1, args.steps)),
+                                                        device=dev)
+        line = {"metric": PREFILL_METRIC, "value": value, "unit": PREFILL_UNIT, "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.n_q * w.batch / value * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": w.name, "kv_format": "k8v4", "step": "oracle sample"},
+                "cpu_baseline": {"value": value, "unit": PREFILL_UNIT, "cores": threads, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": value, "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    gw = PrefillWorkload(w, "k8v4", device)
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        gw.step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        gw.step()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_graph(g, args.steps, 0, stream)
+    clk = clocks.stop()
+    ms = max_over_ranks(ms, device)
+    if ws > 1:
+        torch.distributed.barrier()
+    err = nf.nf_get_device_error()
+    assert err == 0, f"device error {err}"
+    tokens = w.n_q * w.batch
+    value = job_throughput(tokens, ws, ms)
+
+    pf_ms = time_decode_stream(gw, max(3, min(args.steps, 10)), stream)
+    pf_iso_ms = time_decode_launches(gw, max(3, min(args.steps, 10)), stream)
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) if os.path.exists(
+            os.path.join(ROOT, "MEASURED_PEAKS.json")) else open(os.devnull) as f:
+        txt = f.read()
+    peaks = json.loads(txt) if txt else {}
+    # fp16 and bf16 run at the same tensor-core rate; the launches run back to
+    # back for seconds, so the sustained figure applies
+    peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    peak_kind = "measured bf16 sustained (fp16 at the same rate)" if peaks else "fallback"
+    flops = gw.flops_per_launch()
+    achieved = flops / (pf_ms / 1e3) / 1e12
+
+    e2e_ms, h2d, d2h = measure_e2e(gw, args, stream, device)
+    del g
+    torch.cuda.synchronize()
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cv, threads, desc, _ = prefill_oracle_sample(w, budget_s=12.0, device=device)
+        cpu = {"value": cv, "unit": PREFILL_UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": PREFILL_METRIC, "value": value, "unit": PREFILL_UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8/s4 KV codes, f16 tensor-core products (mma.sync), f32 softmax/accumulate",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlens": list(w.seqlens), "n_q": w.n_q,
+                   "n_new": w.n_new, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
+                   "layers": w.layers, "kv_format": "k8v4", "causal": w.causal,
+                   "l2": "KV bytes per step %.0f MB > 126 MB L2" % (gw.kv_bytes_per_layer() * w.layers / 1e6),
+                   "timing": "CUDA graph of one step, CUDA events, max over ranks"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "prefill_kernel (nf_prefill_attn)", "peak_source": peak_kind,
+                     "flops_per_launch": flops, "launch_us": pf_ms * 1e3, "launch_us_isolated": pf_iso_ms * 1e3},
+        "cpu_baseline": cpu,
+        "e2e": {"value": job_throughput(tokens, ws, e2e_ms), "unit": PREFILL_UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": gw.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------ CPU oracle leg
 def oracle_sample(w, fmt_name, budget_s=12.0, device="cpu"):
     """Time the CPU oracle on a bounded sample of the workload: decode attention
@@ -354,7 +543,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.ORDER)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.ORDER + list(workloads.PREFILL))
     ap.add_argument("--kv-format", default="k8v4", choices=["k8v4", "k8v8", "f8", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -366,6 +555,9 @@ def main():
     if args.layers:
         import dataclasses
         w = dataclasses.replace(w, layers=args.layers)
+
+    if w.name in workloads.PREFILL:
+        return prefill_main(args, w, ws, rank, local)
 
     if args.impl == "reference":
         if rank != 0:
@@ -439,25 +631,8 @@ def main():
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     traffic = recorded_traffic(w.name, args.kv_format)
 
-    # ---- end to end: the step's inputs (every layer's q and new K/V) copied
-    # from pinned host memory, the step, every layer's output copied back
-    h_in = [gw.q_all.cpu().pin_memory()]
-    d_in = [gw.q_all]
-    if w.n_new:
-        h_in += [gw.knew_all.cpu().pin_memory(), gw.vnew_all.cpu().pin_memory()]
-        d_in += [gw.knew_all, gw.vnew_all]
-    h_out = torch.empty_like(gw.out_all, device="cpu").pin_memory()
-    ge = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(ge, stream=stream):
-        for d, hsrc in zip(d_in, h_in):
-            d.copy_(hsrc, non_blocking=True)
-        gw.step()
-        h_out.copy_(gw.out_all, non_blocking=True)
-    e2e_ms = time_graph(ge, args.steps, max(3, args.warmup), stream)
-    e2e_ms = max_over_ranks(e2e_ms, device)
-    h2d = sum(t.numel() * t.element_size() for t in h_in)
-    d2h = h_out.numel() * h_out.element_size()
-    del ge, g
+    e2e_ms, h2d, d2h = measure_e2e(gw, args, stream, device)
+    del g
     torch.cuda.synchronize()
 
     cpu = None

@@ -280,6 +280,37 @@ nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_
                           nf_stream_t stream);
 
 /*
+ * nf_prefill_attn -- chunked-prefill attention over a K8/V4 pool (page "3090
+ * 单卡跑 Qwen3.8-27B：NInfer 上机实测", section 一.3: prompts are prefilled in
+ * chunks of --prefill-chunk 1024 tokens; section 二: prefill runs on a
+ * dequantise -> fp16 tensor-core path).
+ *
+ * The operation is nf_decode_attn's for a large n_q: query j of sequence b
+ * sits at position L_b - n_q + j (the chunk's K/V already appended with
+ * nf_kv_append_quant) and, with causal != 0, sees keys 0 .. L_b - n_q + j;
+ * otherwise all L_b keys.  Arguments, layouts and outputs as for
+ * nf_decode_attn, with these differences:
+ *   kv->fmt must be NF_KV_K8V4 and q_dtype NF_BF16 (else NF_ERR_UNSUPPORTED);
+ *   any n_q >= 1 and any GQA group; no workspace (nothing is split across
+ *   CTAs); batch <= 65535, num_kv_heads <= 65535.
+ *   The dequantised V values (code x scale) must lie inside the fp16 range,
+ *   that is every V group's scale <= 65504 / 7: the kernel holds them as fp16.
+ * Numerics: each query row is scaled to max |q| = 1 and rounded to fp16 once;
+ *   K codes are exact in fp16 and the K scale multiplies the fp32 scores; V is
+ *   dequantised to fp16 (one rounding); the softmax weights are rounded to
+ *   fp16; products accumulate in fp32 (mma.sync m16n8k16).
+ * Device errors: NF_DEVERR_SEQLEN (the sequence's rows come out o = 0,
+ *   lse = -inf), NF_DEVERR_BLOCK_ID (that tile's keys read as zeros).
+ * Launch: programmatic dependent launch, as nf_decode_attn; the kernel waits
+ *   for the previous kernel on `stream` before reading any argument.
+ */
+nf_status nf_prefill_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                          int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                          int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                          float softmax_scale, int32_t causal, float *out, float *out_lse,
+                          nf_stream_t stream);
+
+/*
  * nf_get_device_error -- read and clear the device error code of the current
  * device (NF_DEVERR_*).  Synchronises with the device.  Returns NF_OK when no
  * code was set, NF_ERR_DEVICE_CHECK when one was (written to *code), or

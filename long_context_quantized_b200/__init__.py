@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "NF_OK", "NF_KV_K8V4", "NF_KV_BF16", "NF_KV_K8V8", "NF_KV_F8", "NF_F32", "NF_BF16", "NfError", "KVLayer",
     "nf_kv_append_quant", "nf_decode_attn_workspace_size", "nf_decode_attn", "nf_decode_attn_noalloc",
-    "nf_attn_combine",
+    "nf_attn_combine", "nf_prefill_attn",
     "nf_get_device_error", "nf_status_string", "library_path", "load_library",
 ]
 
@@ -82,6 +82,8 @@ def load_library():
         lib.nf_decode_attn_ex.restype = I
         lib.nf_decode_attn_noalloc.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, P, P, P]
         lib.nf_decode_attn_noalloc.restype = I
+        lib.nf_prefill_attn.argtypes = [P, P, I, I, I, I, P, I, P, I, ctypes.c_float, I, P, P, P]
+        lib.nf_prefill_attn.restype = I
         lib.nf_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
         lib.nf_selftest_bounded_wait.restype = I
         lib.nf_attn_combine.argtypes = [P, P, I, I, I, P, P, P]
@@ -236,6 +238,24 @@ def nf_decode_attn_ex(kv: KVLayer, q, block_table, seqlens, max_seqlen: int, sof
         block_table.shape[1], _dptr(seqlens), int(max_seqlen), float(softmax_scale), int(bool(causal)),
         int(flags), _dptr(out), _dptr(out_lse), _dptr(workspace), ws_bytes, _stream(stream))
     _check(st, _name)
+
+
+def nf_prefill_attn(kv: KVLayer, q, block_table, seqlens, max_seqlen: int, softmax_scale: float,
+                    causal: bool, out, out_lse=None, stream=None):
+    """Chunked-prefill attention (see nf.h): the n_q queries of each sequence
+    at positions L - n_q .. L - 1 against its K8/V4 cache; q bf16
+    [batch][n_q][H_q][128], out fp32 of the same shape."""
+    _need(q, "q")
+    _need(block_table, "block_table", torch.int32)
+    _need(seqlens, "seqlens", torch.int32)
+    _need(out, "out", torch.float32)
+    _need(out_lse, "out_lse", torch.float32)
+    B, n_q, H_q = q.shape[0], q.shape[1], q.shape[2]
+    st = load_library().nf_prefill_attn(
+        ctypes.byref(kv.c), _dptr(q), _dtype_code(q.dtype), B, n_q, H_q, _dptr(block_table),
+        block_table.shape[1], _dptr(seqlens), int(max_seqlen), float(softmax_scale), int(bool(causal)),
+        _dptr(out), _dptr(out_lse), _stream(stream))
+    _check(st, "nf_prefill_attn")
 
 
 NF_NOALLOC_SCRATCH_BYTES = 8 << 20

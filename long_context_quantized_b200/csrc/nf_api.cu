@@ -14,6 +14,7 @@
 #include "nf_combine.cuh"
 #include "nf_common.cuh"
 #include "nf_decode.cuh"
+#include "nf_prefill.cuh"
 
 namespace nf {
 // Self-test of the bounded wait: one thread waits on an mbarrier that nothing
@@ -456,3 +457,79 @@ const char *nf_status_string(nf_status status) {
 const char *nf_last_error(void) { return g_msg; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- prefill
+extern "C" nf_status nf_prefill_attn(const nf_kv_layer *kv, const void *q, int32_t q_dtype, int32_t batch,
+                                     int32_t n_q, int32_t num_q_heads, const int32_t *block_table,
+                                     int32_t max_blocks, const int32_t *seqlens, int32_t max_seqlen,
+                                     float softmax_scale, int32_t causal, float *out, float *out_lse,
+                                     nf_stream_t stream) {
+    nf_status st = check_layer(kv);
+    if (st != NF_OK) return st;
+    if (kv->fmt != NF_KV_K8V4) return fail(NF_ERR_UNSUPPORTED, "prefill: kv->fmt %d (only NF_KV_K8V4)", kv->fmt);
+    if (q_dtype != NF_BF16) return fail(NF_ERR_UNSUPPORTED, "prefill: q_dtype %d (only NF_BF16)", q_dtype);
+    if (batch < 1 || n_q < 1 || num_q_heads < 1)
+        return fail(NF_ERR_INVALID_ARG, "batch %d, n_q %d, num_q_heads %d must be >= 1", batch, n_q,
+                    num_q_heads);
+    if (batch > 65535 || kv->num_kv_heads > 65535)
+        return fail(NF_ERR_UNSUPPORTED, "batch %d / num_kv_heads %d above 65535", batch, kv->num_kv_heads);
+    if (num_q_heads % kv->num_kv_heads != 0)
+        return fail(NF_ERR_INVALID_ARG, "num_q_heads %d not a multiple of num_kv_heads %d",
+                    num_q_heads, kv->num_kv_heads);
+    if (max_seqlen < n_q) return fail(NF_ERR_INVALID_ARG, "max_seqlen %d < n_q %d", max_seqlen, n_q);
+    if ((long long)max_blocks * nf::kBlock < max_seqlen)
+        return fail(NF_ERR_INVALID_ARG, "max_blocks %d cannot hold max_seqlen %d", max_blocks, max_seqlen);
+    if (!q || !block_table || !seqlens || !out) return fail(NF_ERR_INVALID_ARG, "a device pointer is NULL");
+    if (!std::isfinite(softmax_scale)) return fail(NF_ERR_INVALID_ARG, "softmax_scale is not finite");
+    if ((reinterpret_cast<uintptr_t>(q) & 7) || (reinterpret_cast<uintptr_t>(out) & 3))
+        return fail(NF_ERR_INVALID_ARG, "q / out misaligned");
+    const long long rows = (long long)(num_q_heads / kv->num_kv_heads) * n_q;
+    const long long row_tiles = (rows + nf::kPfRows - 1) / nf::kPfRows;
+    if (rows > 0x7fffffffLL || row_tiles > 0x7fffffffLL)
+        return fail(NF_ERR_UNSUPPORTED, "prefill: %lld query rows per kv-head", rows);
+
+    nf::PrefillParams p{};
+    p.k_codes = static_cast<const int8_t *>(kv->k_codes);
+    p.k_scales = static_cast<const __half *>(kv->k_scales);
+    p.v_codes = static_cast<const uint8_t *>(kv->v_codes);
+    p.v_scales = static_cast<const __half *>(kv->v_scales);
+    p.num_blocks = kv->num_blocks;
+    p.num_kv_heads = kv->num_kv_heads;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.batch = batch;
+    p.n_q = n_q;
+    p.num_q_heads = num_q_heads;
+    p.group = num_q_heads / kv->num_kv_heads;
+    p.rows = (int)rows;
+    p.row_tiles = (int)row_tiles;
+    p.block_table = block_table;
+    p.max_blocks = max_blocks;
+    p.seqlens = seqlens;
+    p.max_seqlen = max_seqlen;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.causal = causal != 0;
+    p.out = out;
+    p.out_lse = out_lse;
+
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(nf::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        nf::PfSmem::kBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(NF_ERR_CUDA, "prefill kernel attribute: %s", cudaGetErrorString(attr_err));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)row_tiles, (unsigned)kv->num_kv_heads, (unsigned)batch);
+    cfg.blockDim = dim3(nf::kPfThreads);
+    cfg.dynamicSmemBytes = nf::PfSmem::kBytes;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, nf::prefill_kernel, p);
+    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "prefill kernel launch: %s", cudaGetErrorString(e));
+    return after_launch("prefill kernel launch");
+}

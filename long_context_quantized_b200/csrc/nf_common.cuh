@@ -156,6 +156,11 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
 }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return __byte_perm(a, b, sel);
 }
@@ -192,6 +197,13 @@ __device__ __forceinline__ void i8x4_to_f16_eo(uint32_t w, uint32_t &even, uint3
     const __half2 bias = u32_h2(0x64806480u);  // 1152, 1152
     even = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4240)), bias));
     odd = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4341)), bias));
+}
+// The same in byte order: lo = (c0, c1), hi = (c2, c3).
+__device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    const __half2 bias = u32_h2(0x64806480u);
+    lo = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4140)), bias));
+    hi = h2_u32(__hsub2(u32_h2(__byte_perm(u, 0x64646464u, 0x4342)), bias));
 }
 
 // fp8 e4m3 <-> fp16 / fp32 with the hardware conversions (sm_89 and later).

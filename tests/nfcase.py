@@ -22,9 +22,10 @@ LSE_ATOL = 2e-3
 POISON = 0xA5
 
 
-def gpu_layer(w, layer, fmt, q_override=None, max_seqlen=None, bt=None, seqlens=None):
+def gpu_layer(w, layer, fmt, q_override=None, max_seqlen=None, bt=None, seqlens=None, attn="decode"):
     """Fill one layer's pool on the GPU (bulk append of the cached keys, then
-    the step's appended keys), run decode attention.  Returns dict of tensors."""
+    the step's appended keys), run decode (or chunked-prefill) attention.
+    Returns dict of tensors."""
     dev = "cuda"
     bt_np = workloads.block_table(w) if bt is None else bt
     if max_seqlen is not None and bt_np.shape[1] * 256 < max_seqlen:
@@ -48,11 +49,14 @@ def gpu_layer(w, layer, fmt, q_override=None, max_seqlen=None, bt=None, seqlens=
     q = workloads.layer_q(w, layer, device=dev) if q_override is None else q_override
     sl = torch.as_tensor(w.seqlens if seqlens is None else seqlens, dtype=torch.int32, device=dev)
     msl = max(w.seqlens) if max_seqlen is None else max_seqlen
-    ws = torch.zeros(nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, msl),
-                     dtype=torch.uint8, device=dev)
     out = torch.empty((w.batch, w.n_q, w.num_q_heads, 128), dtype=torch.float32, device=dev)
     lse = torch.empty((w.batch, w.n_q, w.num_q_heads), dtype=torch.float32, device=dev)
-    nf.nf_decode_attn(kv, q, bt_t, sl, msl, w.softmax_scale, w.causal, out, lse, ws)
+    if attn == "prefill":
+        nf.nf_prefill_attn(kv, q, bt_t, sl, msl, w.softmax_scale, w.causal, out, lse)
+    else:
+        ws = torch.zeros(nf.nf_decode_attn_workspace_size(w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, msl),
+                         dtype=torch.uint8, device=dev)
+        nf.nf_decode_attn(kv, q, bt_t, sl, msl, w.softmax_scale, w.causal, out, lse, ws)
     torch.cuda.synchronize()
     return dict(kv=kv, q=q, out=out, lse=lse, bt=bt_np, kvin=kvin)
 

@@ -89,3 +89,28 @@ def test_append_and_combine_host_paths(lib):
     assert lib.nf_attn_combine(256, 256, 0, 4, 128, 256, None, None) == nf.NF_ERR_INVALID_ARG
     assert lib.nf_attn_combine(256, 256, 2, 4, 130, 256, None, None) == nf.NF_ERR_UNSUPPORTED
     assert lib.nf_attn_combine(None, 256, 2, 4, 128, 256, None, None) == nf.NF_ERR_INVALID_ARG
+
+
+def _prefill(lib, kv, **over):
+    args = dict(q=256, q_dtype=nf.NF_BF16, batch=1, n_q=64, H_q=4, bt=256, max_blocks=4, seqlens=256,
+                max_seqlen=1000, scale=0.088, causal=1, out=256, lse=None)
+    args.update(over)
+    return lib.nf_prefill_attn(None if kv is None else ctypes.byref(kv), args["q"], args["q_dtype"],
+                               args["batch"], args["n_q"], args["H_q"], args["bt"], args["max_blocks"],
+                               args["seqlens"], args["max_seqlen"], args["scale"], args["causal"],
+                               args["out"], args["lse"], None)
+
+
+def test_prefill_rejects_bad_arguments_before_launch(lib):
+    assert _prefill(lib, None) == nf.NF_ERR_INVALID_ARG
+    assert _prefill(lib, _layer(fmt=nf.NF_KV_K8V8)) == nf.NF_ERR_UNSUPPORTED   # K8/V4 only
+    assert _prefill(lib, _layer(fmt=nf.NF_KV_BF16)) == nf.NF_ERR_UNSUPPORTED
+    assert _prefill(lib, _layer(), q_dtype=nf.NF_F32) == nf.NF_ERR_UNSUPPORTED  # bf16 queries only
+    assert _prefill(lib, _layer(), H_q=3) == nf.NF_ERR_INVALID_ARG
+    assert _prefill(lib, _layer(), n_q=0) == nf.NF_ERR_INVALID_ARG
+    assert _prefill(lib, _layer(), max_seqlen=32) == nf.NF_ERR_INVALID_ARG     # below n_q
+    assert _prefill(lib, _layer(), max_seqlen=2000) == nf.NF_ERR_INVALID_ARG   # table too short
+    assert _prefill(lib, _layer(), q=None) == nf.NF_ERR_INVALID_ARG
+    assert _prefill(lib, _layer(), q=260) == nf.NF_ERR_INVALID_ARG            # misaligned
+    assert _prefill(lib, _layer(), scale=float("nan")) == nf.NF_ERR_INVALID_ARG
+    assert _prefill(lib, _layer(), batch=70000) == nf.NF_ERR_UNSUPPORTED

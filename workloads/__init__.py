@@ -88,6 +88,16 @@ WORKLOADS = {
 
 ORDER = ["tiny", "ctx32k_append", "ragged_c2", "mtp_verify", "longest"]
 
+# Chunked prefill (the pages' --prefill-chunk 1024): the last 1024-token chunk
+# of a 180224-token prompt, appended and then attended causally, 32/4 heads,
+# 16 layers, in the MTP workload's 720-block pool.  A workload of the
+# chunked-prefill attention call, not of the decode step.
+PREFILL = {
+    "prefill_chunk": Workload("prefill_chunk", 6, (179200,), 1024, 1024, 32, 4, 16, torch.bfloat16,
+                              torch.bfloat16, 720, True, "normal", "shuffled"),
+}
+WORKLOADS.update(PREFILL)
+
 
 def get(name: str) -> Workload:
     return WORKLOADS[name]
