@@ -481,10 +481,10 @@ extern "C" nf_status nf_prefill_attn(const nf_kv_layer *kv, const void *q, int32
         return fail(NF_ERR_INVALID_ARG, "max_blocks %d cannot hold max_seqlen %d", max_blocks, max_seqlen);
     if (!q || !block_table || !seqlens || !out) return fail(NF_ERR_INVALID_ARG, "a device pointer is NULL");
     if (!std::isfinite(softmax_scale)) return fail(NF_ERR_INVALID_ARG, "softmax_scale is not finite");
-    if ((reinterpret_cast<uintptr_t>(q) & 7) || (reinterpret_cast<uintptr_t>(out) & 3))
-        return fail(NF_ERR_INVALID_ARG, "q / out misaligned");
+    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
+        return fail(NF_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
     const long long rows = (long long)(num_q_heads / kv->num_kv_heads) * n_q;
-    const long long row_tiles = (rows + nf::kPfRows - 1) / nf::kPfRows;
+    const long long row_tiles = (rows + nf::kTcRows - 1) / nf::kTcRows;
     if (rows > 0x7fffffffLL || row_tiles > 0x7fffffffLL)
         return fail(NF_ERR_UNSUPPORTED, "prefill: %lld query rows per kv-head", rows);
 
@@ -514,22 +514,22 @@ extern "C" nf_status nf_prefill_attn(const nf_kv_layer *kv, const void *q, int32
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(nf::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        nf::PfSmem::kBytes);
+        attr_err = cudaFuncSetAttribute(nf::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        nf::TcSmem::kBytes);
     });
     if (attr_err != cudaSuccess)
         return fail(NF_ERR_CUDA, "prefill kernel attribute: %s", cudaGetErrorString(attr_err));
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)row_tiles, (unsigned)kv->num_kv_heads, (unsigned)batch);
-    cfg.blockDim = dim3(nf::kPfThreads);
-    cfg.dynamicSmemBytes = nf::PfSmem::kBytes;
+    cfg.blockDim = dim3(nf::kTcThreads);
+    cfg.dynamicSmemBytes = nf::TcSmem::kBytes;
     cfg.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, nf::prefill_kernel, p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, nf::prefill_tc_kernel, p);
     if (e != cudaSuccess) return fail(NF_ERR_CUDA, "prefill kernel launch: %s", cudaGetErrorString(e));
     return after_launch("prefill kernel launch");
 }

@@ -1,4 +1,5 @@
-// nf_prefill.cuh -- chunked-prefill attention over the segmented K8/V4 pool.
+// nf_prefill.cuh -- chunked-prefill attention over the segmented K8/V4 pool,
+// on the 5th-generation tensor cores (tcgen05).
 //
 // The pages' engine prefills a prompt in chunks of 1024 tokens (page "3090 单卡跑
 // Qwen3.8-27B：NInfer 上机实测", section 一.3, --prefill-chunk 1024) on a
@@ -10,36 +11,16 @@
 //
 // Work: one CTA per (sequence, kv-head, tile of 128 query rows).  The rows of a
 //   kv-head are its G * n_q (position, q-head) pairs in position-major order,
-//   so the G heads of a position sit in one tile and share its K/V reads (GQA
+//   so the G heads of a position sit in one tile and share its K/V (GQA
 //   packing), and a tile spans 128 / G positions, whose causal limits differ
 //   by that much.  Tiles of late positions, which see the most keys, start
 //   first.
-// Pipeline: each thread holds its share of the next 64-key tile's codes and
-//   scales in registers (read while the warps compute on the current tile) and
-//   then converts them into the other of two shared-memory buffers:
-//     K codes -> exact fp16 codes [key][channel]; the K scale stays per key
-//       and multiplies the scores;
-//     V nibbles x V scale -> fp16 values [key][channel, permuted inside each
-//       8-channel chunk as the nibble unpacking delivers them];
-//   rows of 256 bytes whose 16-byte chunks are XOR-swizzled by key & 7, so
-//   that the ldmatrix reads of 8 keys hit 8 different bank groups.
-// Math per warp (16 query rows): S = Q . K^T on mma.sync m16n8k16 (fp16 in,
-//   fp32 accumulate), each query row scaled to max |q| = 1 and rounded to fp16
-//   once; the online softmax in the log2 domain with a lazy running max (the
-//   max is raised and O rescaled only when a tile exceeds it by more than 4,
-//   the weights 2^(x - max - 4) <= 1); O += P . V with P taken as fp16 straight
-//   from the score registers (the score layout of S is the A layout of P).
 #pragma once
 
 #include "nf_common.cuh"
+#include "nf_tc.cuh"
 
 namespace nf {
-
-constexpr int kPfWarps = 8;
-constexpr int kPfThreads = kPfWarps * 32;
-constexpr int kPfRows = 16 * kPfWarps;  // query rows per CTA
-constexpr int kPfKeys = 64;             // keys per tile
-constexpr float kPfLazy = 4.0f;
 
 struct PrefillParams {
     const int8_t *k_codes;
@@ -50,7 +31,7 @@ struct PrefillParams {
     const __nv_bfloat16 *q;
     int batch, n_q, num_q_heads, group;
     int rows;       // group * n_q per (sequence, kv-head)
-    int row_tiles;  // ceil(rows / kPfRows)
+    int row_tiles;  // ceil(rows / 128)
     const int32_t *block_table;
     int max_blocks;
     const int32_t *seqlens;
@@ -61,285 +42,419 @@ struct PrefillParams {
     float *out_lse;  // [batch][n_q][H_q] or null
 };
 
-struct PfSmem {
-    static constexpr int kTile = kPfKeys * kHeadDim * 2;  // one fp16 [64][128] tile
-    static constexpr int kK = 0;                          // K codes  [2][64][128]
-    static constexpr int kV = 2 * kTile;                  // V values [2][64][128]
-    static constexpr int kSk = 4 * kTile;                 // K scales float [2][64]
-    static constexpr int kBytes = kSk + 2 * kPfKeys * 4;
-    // at start-up the query tile [128][128] fp16 is staged in the K buffers
-    static_assert(kPfRows * kHeadDim * 2 <= 2 * kTile, "query staging");
+// ============================================================================
+// CTA = 128 query rows (the MMA's M) and three roles:
+//   warps 0-3  softmax: thread r owns query row r; reads its row of S from
+//              tensor memory (tcgen05.ld), runs the online softmax, writes
+//              its row of P (fp16) to shared memory, rescales its row of O in
+//              tensor memory when its running max rises, and at the end
+//              reads O, normalises and writes the output;
+//   warps 4-7  converters: thread t stages query row t (scaled to max |q| = 1,
+//              fp16) once, then for every 128-key tile loads key t's K8/V4
+//              codes and scales (prefetched a tile ahead in registers) and
+//              writes the dequantised fp16 K row and V row into a two-stage
+//              ring;
+//   warp 8     tensor memory allocation and, on one thread, the MMAs:
+//              S_j = Q . K_j^T into one of two S buffers, then
+//              O += P_{j-1} . V_{j-1}, each group of 8 MMAs (K = 16) committed
+//              to an mbarrier.
+// Tensor memory (512 columns x 128 lanes): S buffers at columns 0 and 128,
+// O at 256.  Shared operands use the 128-byte-swizzled canonical layouts:
+//   Q, P   A operands, K-major: [2 blocks of 64 columns][128 rows][128 bytes];
+//   K      B operand of S, K-major: [2 blocks of 64 channels][128 keys][128 bytes];
+//   V      B operand of O, MN-major: [2 blocks of 64 channels][128 keys][128 bytes],
+//          channels inside each 8-channel chunk in the nibble-unpacking order.
+// Weights are 2^(x - m - 8) with the lazy max of the decode kernel (threshold
+// 8), so P <= 1 and O is rescaled only when a row's max rises by more than 8.
+// Every mbarrier wait is bounded; a timeout records NF_DEVERR_TIMEOUT and
+// every role leaves its loop.
+// ============================================================================
+constexpr int kTcThreads = 288;
+constexpr int kTcRows = 128;   // query rows per CTA (M of both MMAs)
+constexpr int kTcKeys = 128;   // keys per tile (N of S = Q.K^T, K of O += P.V)
+constexpr float kTcLazy = 8.0f;
+constexpr uint32_t kTcIdescQK = umma_idesc_f16(128, 128, false);  // B = K rows, K-major
+constexpr uint32_t kTcIdescPV = umma_idesc_f16(128, 128, true);   // B = V rows, MN-major
+
+struct TcSmem {
+    static constexpr int kBlk = 16384;                // one 64-column block of 128 rows x 128 bytes
+    static constexpr int kQ = 0;                      // 2 blocks
+    static constexpr int kK = 2 * kBlk;               // [2 stages][2 blocks]
+    static constexpr int kV = 6 * kBlk;               // [2 stages][2 blocks]
+    static constexpr int kP = 10 * kBlk;              // [2 buffers][2 blocks]
+    static constexpr int kBars = 14 * kBlk;           // 11 mbarriers
+    static constexpr int kQf = kBars + 128;           // float [128]
+    static constexpr int kMisc = kQf + 128 * 4;       // tmem base, abort flag
+    static constexpr int kBytes = kMisc + 16;
+    static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
-// Byte offset of 16-byte chunk c of row r in a [rows][256 bytes] swizzled tile.
-__device__ __forceinline__ uint32_t pf_swz(int r, int c) {
-    return (uint32_t)r * 256u + (uint32_t)(((c ^ r) & 7) | (c & 8)) * 16u;
+// byte offset of row r, 16-byte chunk c (0..15 over 128 columns of fp16) in a
+// two-block 128-byte-swizzled operand
+__device__ __forceinline__ uint32_t tc_swz(int r, int c) {
+    return (uint32_t)(c >> 3) * TcSmem::kBlk + (uint32_t)r * 128u + (uint32_t)(((c ^ r) & 7) * 16);
 }
 
-// One thread's share of a tile: key tid / 4, quarter q = tid % 4 (channels
-// 32q .. 32q + 31, one V scale group).
-struct PfRaw {
-    uint4 k0, k1;  // K codes
-    uint4 v;       // V nibbles
-    __half vs;     // the group's V scale
-    __half ks;     // the key's K scale
-    bool ok;       // the key lies inside the sequence
+struct TcRaw {
+    uint4 k[8];  // K codes of the key
+    uint4 v[4];  // V nibbles
+    uint2 vs;    // 4 V scales
+    uint32_t ks; // K scale (low half)
+    int ok;      // key inside the sequence
 };
 
-__device__ __forceinline__ void pf_load(const PrefillParams &p, const int32_t *bt, int L, int h, int tile,
-                                        PfRaw &r) {
-    const int key = threadIdx.x >> 2, qtr = threadIdx.x & 3;
-    const int pos = tile * kPfKeys + key;
-    // a tile lies in one 256-key block, and its first key is < L, so the table
-    // entry of that block exists
-    const int blk = bt[(tile * kPfKeys) >> 8];
+__device__ __forceinline__ void tc_load(const PrefillParams &p, const int32_t *bt, int L, int h, int tile, int t,
+                                        TcRaw &r) {
+    const int pos = tile * kTcKeys + t;
+    const int blk = bt[(tile * kTcKeys) >> 8];  // a tile lies in one block whose entry exists
     r.ok = pos < L;
     if (blk < 0 || blk >= p.num_blocks) {
-        if (threadIdx.x == 0) report(NF_DEVERR_BLOCK_ID);
-        r.k0 = r.k1 = r.v = make_uint4(0, 0, 0, 0);
-        r.vs = r.ks = __float2half(0.f);
-        r.ok = false;
+        if (t == 0) report(NF_DEVERR_BLOCK_ID);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r.k[u] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) r.v[u] = make_uint4(0, 0, 0, 0);
+        r.vs = make_uint2(0, 0);
+        r.ks = 0;
+        r.ok = 0;
         return;
     }
     const size_t si = ((size_t)blk * p.num_kv_heads + h) * kBlock + (pos & (kBlock - 1));
-    r.k0 = ldg16(p.k_codes + si * kHeadDim + 32 * qtr);
-    r.k1 = ldg16(p.k_codes + si * kHeadDim + 32 * qtr + 16);
-    r.v = ldg16(p.v_codes + si * (kHeadDim / 2) + 16 * qtr);
-    r.vs = p.v_scales[si * (kHeadDim / kVGroup) + qtr];
-    r.ks = p.k_scales[si];
+    const unsigned char *kp = reinterpret_cast<const unsigned char *>(p.k_codes) + si * kHeadDim;
+    const unsigned char *vp = p.v_codes + si * (kHeadDim / 2);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) r.k[u] = ldg16(kp + 16 * u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) r.v[u] = ldg16(vp + 16 * u);
+    r.vs = __ldg(reinterpret_cast<const uint2 *>(p.v_scales + si * (kHeadDim / kVGroup)));
+    r.ks = __ldg(reinterpret_cast<const unsigned short *>(p.k_scales + si));
 }
 
-__device__ __forceinline__ void pf_convert(const PfRaw &r, unsigned char *kbuf, unsigned char *vbuf, float *skbuf) {
-    const int key = threadIdx.x >> 2, qtr = threadIdx.x & 3;
-    // K: 32 int8 codes -> 4 chunks of 8 exact fp16 codes, in channel order
-    const uint32_t w[8] = {r.k0.x, r.k0.y, r.k0.z, r.k0.w, r.k1.x, r.k1.y, r.k1.z, r.k1.w};
+// key t's dequantised fp16 K row (code x K scale) and V row (code x V scale;
+// 0 past the end) into stage buffers kb, vb
+__device__ __forceinline__ void tc_convert(const TcRaw &r, int t, unsigned char *kb, unsigned char *vb) {
+    const uint32_t ks2 = r.ok ? (r.ks & 0xFFFFu) * 0x10001u : 0u;
+    const __half2 sk = u32_h2(ks2);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint4 o;
-        i8x4_to_f16(w[2 * c], o.x, o.y);
-        i8x4_to_f16(w[2 * c + 1], o.z, o.w);
-        *reinterpret_cast<uint4 *>(kbuf + pf_swz(key, 4 * qtr + c)) = o;
+    for (int u = 0; u < 8; ++u) {
+        uint4 a, c;
+        i8x4_to_f16(r.k[u].x, a.x, a.y);
+        i8x4_to_f16(r.k[u].y, a.z, a.w);
+        i8x4_to_f16(r.k[u].z, c.x, c.y);
+        i8x4_to_f16(r.k[u].w, c.z, c.w);
+        a.x = h2_u32(__hmul2(u32_h2(a.x), sk)); a.y = h2_u32(__hmul2(u32_h2(a.y), sk));
+        a.z = h2_u32(__hmul2(u32_h2(a.z), sk)); a.w = h2_u32(__hmul2(u32_h2(a.w), sk));
+        c.x = h2_u32(__hmul2(u32_h2(c.x), sk)); c.y = h2_u32(__hmul2(u32_h2(c.y), sk));
+        c.z = h2_u32(__hmul2(u32_h2(c.z), sk)); c.w = h2_u32(__hmul2(u32_h2(c.w), sk));
+        *reinterpret_cast<uint4 *>(kb + tc_swz(t, 2 * u)) = a;
+        *reinterpret_cast<uint4 *>(kb + tc_swz(t, 2 * u + 1)) = c;
     }
-    // V: word u holds channels 32q + 8u + 0..7 (nibble i = channel 8u + i); the
-    // chunk stores them as (0, 4, 1, 5, 2, 6, 3, 7), each times the V scale.
-    // Keys past the end get scale 0 (their stale scale may be anything).
-    const __half2 s2 = r.ok ? __half2half2(r.vs) : __float2half2_rn(0.f);
-    const uint32_t vw[4] = {r.v.x, r.v.y, r.v.z, r.v.w};
+    const uint32_t vsw[2] = {r.vs.x, r.vs.y};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t w = (i & 3) == 0 ? r.v[i >> 2].x : (i & 3) == 1 ? r.v[i >> 2].y
+                         : (i & 3) == 2 ? r.v[i >> 2].z : r.v[i >> 2].w;
+        const int grp = i >> 2;  // 32-channel scale group
+        const uint32_t s16 = (vsw[grp >> 1] >> (16 * (grp & 1))) & 0xFFFFu;
+        const __half2 sv = u32_h2(r.ok ? s16 * 0x10001u : 0u);
         uint4 o;
-        o.x = h2_u32(__hmul2(nib_even(vw[u]), s2));
-        o.y = h2_u32(__hmul2(nib_odd(vw[u]), s2));
-        o.z = h2_u32(__hmul2(nib_even(vw[u] >> 8), s2));
-        o.w = h2_u32(__hmul2(nib_odd(vw[u] >> 8), s2));
-        *reinterpret_cast<uint4 *>(vbuf + pf_swz(key, 4 * qtr + u)) = o;
+        o.x = h2_u32(__hmul2(nib_even(w), sv));
+        o.y = h2_u32(__hmul2(nib_odd(w), sv));
+        o.z = h2_u32(__hmul2(nib_even(w >> 8), sv));
+        o.w = h2_u32(__hmul2(nib_odd(w >> 8), sv));
+        *reinterpret_cast<uint4 *>(vb + tc_swz(t, i)) = o;
     }
-    if (qtr == 0) skbuf[key] = r.ok ? __half2float(r.ks) : 0.f;
 }
 
-__global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
+// bounded wait that also gives up once another role has aborted
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            report(NF_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TcSmem::kBars);
+    uint64_t *q_full = bars + 0, *kv_full = bars + 1, *s_full = bars + 3, *p_full = bars + 5, *pv_done = bars + 7,
+             *o_full = bars + 9, *drain = bars + 10;
+    float *qfs = reinterpret_cast<float *>(smem + TcSmem::kQf);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + TcSmem::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcSmem::kMisc + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.z, h = blockIdx.y;
     const int rt = p.row_tiles - 1 - (int)blockIdx.x;  // late positions first
-    const int r0 = rt * kPfRows;
+    const int r0 = rt * 128;
     const int G = p.group;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], 128);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&pv_done[i], 1);
+        }
+        mbar_init(o_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        // the swizzled operands need 1024-byte alignment of the window
+        if (smem_addr(smem) & 1023u) {
+            if (blockIdx.x == 0 && h == 0 && b == 0) report(NF_DEVERR_INTERNAL);
+            *abort_flag = 1;
+        }
+        fence_mbar_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
 
     pdl_wait();
     pdl_trigger();
     const int L = p.seqlens[b];
-    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks;
     auto out_row = [&](int r) {
         const int j = r / G, gq = r % G;
         return ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * G + gq;
     };
-    if (L < p.n_q || L > p.max_seqlen) {
+    const bool bad_len = L < p.n_q || L > p.max_seqlen;
+    const int last_row = min(r0 + 128, p.rows) - 1;
+    const int n_keys = bad_len ? 0 : (p.causal ? L - p.n_q + last_row / G + 1 : L);
+    const int T = (n_keys + kTcKeys - 1) / kTcKeys;
+    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks;
+
+    if (bad_len) {
         if (threadIdx.x == 0 && rt == p.row_tiles - 1 && h == 0) report(NF_DEVERR_SEQLEN);
-        for (int idx = threadIdx.x; idx < kPfRows * kHeadDim; idx += kPfThreads) {
+        for (int idx = threadIdx.x; idx < 128 * kHeadDim; idx += kTcThreads) {
             const int r = r0 + idx / kHeadDim, ch = idx % kHeadDim;
             if (r >= p.rows) continue;
             p.out[out_row(r) * kHeadDim + ch] = 0.f;
             if (ch == 0 && p.out_lse) p.out_lse[out_row(r)] = -INFINITY;
         }
-        return;
-    }
-    const int last_row = min(r0 + kPfRows, p.rows) - 1;
-    const int n_keys = p.causal ? L - p.n_q + last_row / G + 1 : L;
-    const int tiles = (n_keys + kPfKeys - 1) / kPfKeys;
-
-    PfRaw raw;
-    pf_load(p, bt, L, h, 0, raw);  // in flight while the query is staged
-
-    // ---- query: warp w stages its rows 16w..16w+15 (scaled to max |q| = 1,
-    // fp16) into the K buffers, then loads its A fragments
-    const int rw0 = r0 + 16 * warp;
-    float qf[2] = {0.f, 0.f};  // max |q| x softmax scale x log2(e) of rows g, g + 8
-    {
-        unsigned char *qs = smem + PfSmem::kK;
-        for (int i = 0; i < 16; ++i) {
-            const int r = rw0 + i;
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
+    } else if (warp >= 4 && warp < 8 && !*abort_flag) {
+        // ================================================== converters
+        const int t = threadIdx.x - 128;
+        {
+            const int r = r0 + t;
+            float x[kHeadDim];
             if (r < p.rows) {
-                const uint2 v = *reinterpret_cast<const uint2 *>(p.q + out_row(r) * kHeadDim + 4 * lane);
-                x[0] = __uint_as_float(v.x << 16);
-                x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-                x[2] = __uint_as_float(v.y << 16);
-                x[3] = __uint_as_float(v.y & 0xFFFF0000u);
-            }
-            float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+                const uint4 *qp = reinterpret_cast<const uint4 *>(p.q + out_row(r) * kHeadDim);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                for (int u = 0; u < 16; ++u) {
+                    const uint4 w = __ldg(qp + u);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        x[8 * u + 2 * e] = __uint_as_float(ww[e] << 16);
+                        x[8 * u + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < kHeadDim; ++i) x[i] = 0.f;
+            }
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < kHeadDim; ++i) amax = fmaxf(amax, fabsf(x[i]));
             const float inv = amax > 0.f ? 1.0f / amax : 0.f;
-            uint2 hv;
-            hv.x = pack_f16(x[0] * inv, x[1] * inv);
-            hv.y = pack_f16(x[2] * inv, x[3] * inv);
-            *reinterpret_cast<uint2 *>(qs + pf_swz(16 * warp + i, lane >> 1) + (lane & 1) * 8) = hv;
-            if (i == g) qf[0] = amax * p.scale_log2;
-            if (i == g + 8) qf[1] = amax * p.scale_log2;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                uint4 o;
+                o.x = pack_f16(x[8 * c] * inv, x[8 * c + 1] * inv);
+                o.y = pack_f16(x[8 * c + 2] * inv, x[8 * c + 3] * inv);
+                o.z = pack_f16(x[8 * c + 4] * inv, x[8 * c + 5] * inv);
+                o.w = pack_f16(x[8 * c + 6] * inv, x[8 * c + 7] * inv);
+                *reinterpret_cast<uint4 *>(smem + TcSmem::kQ + tc_swz(t, c)) = o;
+            }
+            qfs[t] = amax * p.scale_log2;
+            fence_async_smem();
+            mbar_arrive(q_full);
         }
-    }
-    __syncwarp();
-    uint32_t qa[8][4];
-    {
-        const uint32_t qb = smem_addr(smem + PfSmem::kK);
-        const int i = lane >> 3, rr = lane & 7;
+        TcRaw ra, rb;
+        if (T > 0) tc_load(p, bt, L, h, 0, t, ra);
+        auto stage_tile = [&](int j, TcRaw &cur, TcRaw &nxt) -> bool {
+            if (j + 1 < T) tc_load(p, bt, L, h, j + 1, t, nxt);
+            const int s = j & 1;
+            if (j >= 2 && !tc_wait(&pv_done[s], ((j - 2) >> 1) & 1, abort_flag)) return false;
+            tc_convert(cur, t, smem + TcSmem::kK + s * 2 * TcSmem::kBlk, smem + TcSmem::kV + s * 2 * TcSmem::kBlk);
+            fence_async_smem();
+            mbar_arrive(&kv_full[s]);
+            return true;
+        };
+        for (int j = 0; j < T; j += 2) {
+            if (!stage_tile(j, ra, rb)) break;
+            if (j + 1 < T && !stage_tile(j + 1, rb, ra)) break;
+        }
+    } else if (warp < 4 && !*abort_flag) {
+        // ================================================== softmax
+        const int r = threadIdx.x;
+        const int row = r0 + r;
+        const int lim = row < p.rows ? (p.causal ? L - p.n_q + row / G : L - 1) : -1;
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
+        float m_run = -INFINITY, l_run = 0.f;
+        // every wait's outcome is made warp-uniform: the tcgen05 loads and
+        // stores below are warp-collective
+        bool ok = __all_sync(0xffffffffu, tc_wait(q_full, 0, abort_flag));
+        const float qf = ok ? qfs[r] : 0.f;
+        for (int j = 0; ok && j < T; ++j) {
+            const int sb = j & 1;
+            if (!__all_sync(0xffffffffu, tc_wait(&s_full[sb], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sv[kTcKeys];
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-            ldsm_x4(qb + pf_swz(16 * warp + 8 * (i & 1) + rr, 2 * ks + (i >> 1)), qa[ks][0], qa[ks][1], qa[ks][2],
-                    qa[ks][3]);
-    }
-    __syncthreads();  // every warp holds its query before the buffers are overwritten
-
-    // ---- per-row limits
-    int lim[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const int r = rw0 + g + 8 * e;
-        lim[e] = r >= p.rows ? -1 : (p.causal ? L - p.n_q + r / G : L - 1);
-    }
-    const bool warp_on = rw0 < p.rows;
-    const int wmin = p.causal ? L - p.n_q + rw0 / G : L - 1;                        // smallest limit of the warp
-    const int wmax = p.causal ? L - p.n_q + min(rw0 + 15, p.rows - 1) / G : L - 1;  // largest
-
-    float o[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-
-    if (tiles > 0) pf_convert(raw, smem + PfSmem::kK, smem + PfSmem::kV, reinterpret_cast<float *>(smem + PfSmem::kSk));
-    __syncthreads();
-
-    const int li = lane >> 3, lr = lane & 7;  // ldmatrix: matrix and row of this lane's address
-    for (int it = 0; it < tiles; ++it) {
-        const int cur = it & 1;
-        if (it + 1 < tiles) pf_load(p, bt, L, h, it + 1, raw);
-        const int key0 = it * kPfKeys;
-        if (warp_on && key0 <= wmax) {
-            const uint32_t kb = smem_addr(smem + PfSmem::kK + cur * PfSmem::kTile);
-            const uint32_t vb = smem_addr(smem + PfSmem::kV + cur * PfSmem::kTile);
-            const float *sk = reinterpret_cast<const float *>(smem + PfSmem::kSk) + cur * kPfKeys;
-            // ---- S = Q . K^T: n-tile n = keys 8n..8n+7; lane: rows g, g + 8 x keys 8n + 2t, +1
-            float s[8][4];
-#pragma unroll
-            for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-                for (int np = 0; np < 4; ++np) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kb + pf_swz(16 * np + 8 * (li >> 1) + lr, 2 * ks + (li & 1)), b0, b1, b2, b3);
-                    mma_f16(s[2 * np], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-                    mma_f16(s[2 * np + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
-                }
-            const bool fast = key0 + kPfKeys - 1 <= wmin;
-#pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const float2 kk = *reinterpret_cast<const float2 *>(sk + 8 * n + 2 * t);
-                s[n][0] *= qf[0] * kk.x;
-                s[n][1] *= qf[0] * kk.y;
-                s[n][2] *= qf[1] * kk.x;
-                s[n][3] *= qf[1] * kk.y;
-                if (!fast) {
-                    const int kp = key0 + 8 * n + 2 * t;
-                    if (kp > lim[0]) s[n][0] = -INFINITY;
-                    if (kp + 1 > lim[0]) s[n][1] = -INFINITY;
-                    if (kp > lim[1]) s[n][2] = -INFINITY;
-                    if (kp + 1 > lim[1]) s[n][3] = -INFINITY;
-                }
+            for (int c = 0; c < 4; ++c) {
+                uint32_t (&part)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]);
+                tmem_ld32(t_lane + (uint32_t)(sb * 128 + 32 * c), part);
             }
-            // ---- lazy running max (the 4 lanes of a row agree on it)
-            float mx[2] = {-INFINITY, -INFINITY};
+            tmem_wait_ld();
+            const int key0 = j * kTcKeys;
+            const int nvis = min(kTcKeys, lim - key0 + 1);  // keys of the tile this row sees (may be <= 0)
+            float mx = -INFINITY;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                mx[0] = fmaxf(mx[0], fmaxf(s[n][0], s[n][1]));
-                mx[1] = fmaxf(mx[1], fmaxf(s[n][2], s[n][3]));
-            }
-            const bool raise = mx[0] > m_run[0] + kPfLazy || mx[1] > m_run[1] + kPfLazy;
+            for (int i = 0; i < kTcKeys; ++i)
+                if (i < nvis) mx = fmaxf(mx, __uint_as_float(sv[i]));
+            const float tmax = mx == -INFINITY ? -INFINITY : mx * qf;
+            const bool raise = tmax > m_run + kTcLazy;
             if (__any_sync(0xffffffffu, raise)) {
+                const float m_new = raise ? tmax : m_run;
+                const float alpha = raise ? ex2(m_run - m_new) : 1.f;  // 0 when m_run was -inf
+                if (j >= 1) {
+                    // O holds P_{j-1} . V_{j-1} once that MMA group has completed
+                    if (!__all_sync(0xffffffffu, tc_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float m = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 1));
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                    const float m_new = fmaxf(m_run[e], m);
-                    const float alpha = m_new == -INFINITY ? 1.f : ex2(m_run[e] - m_new);
-                    m_run[e] = m_new;
-                    l_run[e] *= alpha;
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(t_lane + 256u + 32u * c, o);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int n = 0; n < 16; ++n) {
-                        o[n][2 * e] *= alpha;
-                        o[n][2 * e + 1] *= alpha;
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(t_lane + 256u + 32u * c, o);
+                    }
+                    tmem_wait_st();
+                }
+                l_run *= alpha;
+                m_run = m_new;
+            }
+            const float mu = (m_run == -INFINITY ? 0.f : m_run) + kTcLazy;
+            // the P buffer was last read by P_{j-2} . V_{j-2}
+            if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(&pv_done[sb], ((j - 2) >> 1) & 1, abort_flag))) {
+                ok = false;
+                break;
+            }
+            unsigned char *pb = smem + TcSmem::kP + sb * 2 * TcSmem::kBlk;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                float pv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * c + e;
+                    pv[e] = i < nvis ? ex2(fmaf(__uint_as_float(sv[i]), qf, -mu)) : 0.f;
+                    l_run += pv[e];
+                }
+                uint4 o;
+                o.x = pack_f16(pv[0], pv[1]);
+                o.y = pack_f16(pv[2], pv[3]);
+                o.z = pack_f16(pv[4], pv[5]);
+                o.w = pack_f16(pv[6], pv[7]);
+                *reinterpret_cast<uint4 *>(pb + tc_swz(r, c)) = o;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&p_full[sb]);
+        }
+        if (ok && __all_sync(0xffffffffu, tc_wait(o_full, 0, abort_flag))) {
+            tc_fence_after();
+            const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
+            float *dst = row < p.rows ? p.out + out_row(row) * kHeadDim : nullptr;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(t_lane + 256u + 32u * c, o);
+                tmem_wait_ld();
+                if (dst) {
+                    // column 8g + e holds channel 8g + (0, 4, 1, 5, 2, 6, 3, 7)[e]
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        const uint32_t *q8 = o + 8 * g8;
+                        float4 lo4 = make_float4(__uint_as_float(q8[0]) * inv, __uint_as_float(q8[2]) * inv,
+                                                 __uint_as_float(q8[4]) * inv, __uint_as_float(q8[6]) * inv);
+                        float4 hi4 = make_float4(__uint_as_float(q8[1]) * inv, __uint_as_float(q8[3]) * inv,
+                                                 __uint_as_float(q8[5]) * inv, __uint_as_float(q8[7]) * inv);
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * c + 8 * g8);
+                        d4[0] = lo4;
+                        d4[1] = hi4;
                     }
                 }
             }
-            // ---- P = 2^(x - m - 4) as fp16 A fragments: k-step kk = keys 16kk..16kk+15
-            const float mu0 = (m_run[0] == -INFINITY ? 0.f : m_run[0]) + kPfLazy;
-            const float mu1 = (m_run[1] == -INFINITY ? 0.f : m_run[1]) + kPfLazy;
-            uint32_t pa[4][4];
+            if (dst && p.out_lse)
+                p.out_lse[out_row(row)] =
+                    l_run > 0.f ? (m_run + kTcLazy + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        }
+    } else if (warp == 8 && lane == 0 && !*abort_flag) {
+        // ================================================== MMA issue
+        const uint32_t sQ = smem_addr(smem + TcSmem::kQ), sK = smem_addr(smem + TcSmem::kK);
+        const uint32_t sV = smem_addr(smem + TcSmem::kV), sP = smem_addr(smem + TcSmem::kP);
+        auto pv = [&](int i) -> bool {
+            const int s = i & 1;
+            if (!tc_wait(&p_full[s], (i >> 1) & 1, abort_flag)) return false;
+            tc_fence_after();
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const float p0 = ex2(s[n][0] - mu0), p1 = ex2(s[n][1] - mu0);
-                const float p2 = ex2(s[n][2] - mu1), p3 = ex2(s[n][3] - mu1);
-                l_run[0] += p0 + p1;
-                l_run[1] += p2 + p3;
-                pa[n >> 1][2 * (n & 1)] = pack_f16(p0, p1);
-                pa[n >> 1][2 * (n & 1) + 1] = pack_f16(p2, p3);
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t ad = umma_desc_sw128(sP + s * 2 * TcSmem::kBlk + (kk >> 2) * TcSmem::kBlk + (kk & 3) * 32,
+                                                    16, 1024);
+                const uint64_t bd = umma_desc_sw128(sV + s * 2 * TcSmem::kBlk + kk * 2048, TcSmem::kBlk, 1024);
+                umma_f16(tmem + 256u, ad, bd, kTcIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
             }
-            // ---- O += P . V: n-tile n = stored channel positions 8n..8n+7
+            umma_commit(&pv_done[s]);
+            return true;
+        };
+        bool ok = tc_wait(q_full, 0, abort_flag);
+        for (int j = 0; ok && j < T; ++j) {
+            const int s = j & 1;
+            if (!tc_wait(&kv_full[s], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                for (int cp = 0; cp < 8; ++cp) {
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(vb + pf_swz(16 * kk + 8 * (li & 1) + lr, 2 * cp + (li >> 1)), b0, b1, b2, b3);
-                    mma_f16(o[2 * cp], pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3], b0, b1);
-                    mma_f16(o[2 * cp + 1], pa[kk][0], pa[kk][1], pa[kk][2], pa[kk][3], b2, b3);
-                }
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t ad = umma_desc_sw128(sQ + (ks >> 2) * TcSmem::kBlk + (ks & 3) * 32, 16, 1024);
+                const uint64_t bd =
+                    umma_desc_sw128(sK + s * 2 * TcSmem::kBlk + (ks >> 2) * TcSmem::kBlk + (ks & 3) * 32, 16, 1024);
+                umma_f16(tmem + (uint32_t)(s * 128), ad, bd, kTcIdescQK, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[s]);
+            if (j >= 1 && !pv(j - 1)) { ok = false; break; }
         }
-        if (it + 1 < tiles)
-            pf_convert(raw, smem + PfSmem::kK + (cur ^ 1) * PfSmem::kTile, smem + PfSmem::kV + (cur ^ 1) * PfSmem::kTile,
-                       reinterpret_cast<float *>(smem + PfSmem::kSk) + (cur ^ 1) * kPfKeys);
-        __syncthreads();
+        if (ok && T > 0) ok = pv(T - 1);
+        if (ok) umma_commit(o_full);
+        // every MMA this thread issued has completed before tensor memory is freed
+        umma_commit(drain);
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait_sleep(drain, 0, 20000u))
+            if (global_ns() - t0 > kWaitLimitNs) {
+                report(NF_DEVERR_TIMEOUT);
+                break;
+            }
     }
-
-    // ---- normalise and write: accumulator (n, 2t + e) is channel 8n + t + 4e
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        float l = l_run[e];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        const int r = rw0 + g + 8 * e;
-        if (r >= p.rows) continue;
-        const float inv = l > 0.f ? 1.0f / l : 0.f;
-        float *dst = p.out + out_row(r) * kHeadDim;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            dst[8 * n + t] = o[n][2 * e] * inv;
-            dst[8 * n + t + 4] = o[n][2 * e + 1] * inv;
-        }
-        if (t == 0 && p.out_lse)
-            p.out_lse[out_row(r)] =
-                l > 0.f ? (m_run[e] + kPfLazy + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 

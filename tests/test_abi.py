@@ -111,6 +111,6 @@ def test_prefill_rejects_bad_arguments_before_launch(lib):
     assert _prefill(lib, _layer(), max_seqlen=32) == nf.NF_ERR_INVALID_ARG     # below n_q
     assert _prefill(lib, _layer(), max_seqlen=2000) == nf.NF_ERR_INVALID_ARG   # table too short
     assert _prefill(lib, _layer(), q=None) == nf.NF_ERR_INVALID_ARG
-    assert _prefill(lib, _layer(), q=260) == nf.NF_ERR_INVALID_ARG            # misaligned
+    assert _prefill(lib, _layer(), q=264) == nf.NF_ERR_INVALID_ARG            # not 16-byte aligned
     assert _prefill(lib, _layer(), scale=float("nan")) == nf.NF_ERR_INVALID_ARG
     assert _prefill(lib, _layer(), batch=70000) == nf.NF_ERR_UNSUPPORTED
