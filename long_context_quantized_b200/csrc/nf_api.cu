@@ -371,7 +371,10 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = pl.nt == 1 ? dispatch_decode<1>(p, q_dtype == NF_F32, kv->fmt, pl.ctas, s)
                                      : dispatch_decode<2>(p, q_dtype == NF_F32, kv->fmt, pl.ctas, s);
-    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "decode kernel set-up: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(NF_ERR_CUDA, "decode kernel set-up: %s", cudaGetErrorString(e));
+    }
     return after_launch("decode kernel launch");
 }
 
@@ -530,6 +533,9 @@ extern "C" nf_status nf_prefill_attn(const nf_kv_layer *kv, const void *q, int32
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, nf::prefill_tc_kernel, p);
-    if (e != cudaSuccess) return fail(NF_ERR_CUDA, "prefill kernel launch: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();  // a refused launch leaves no sticky state for the next call
+        return fail(NF_ERR_CUDA, "prefill kernel launch: %s", cudaGetErrorString(e));
+    }
     return after_launch("prefill kernel launch");
 }

@@ -30,6 +30,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Two 2^x at once on the MUFU unit, fp16 in and out (-inf gives +0).
+__device__ __forceinline__ uint32_t ex2_h2(uint32_t x) {
+    uint32_t y;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
 // 2^x on the MUFU unit (relative error ~2^-22; -inf gives +0).
 __device__ __forceinline__ float ex2(float x) {
     float y;

@@ -64,8 +64,8 @@ struct PrefillParams {
 //   K      B operand of S, K-major: [2 blocks of 64 channels][128 keys][128 bytes];
 //   V      B operand of O, MN-major: [2 blocks of 64 channels][128 keys][128 bytes],
 //          channels inside each 8-channel chunk in the nibble-unpacking order.
-// Weights are 2^(x - m - 8) with the lazy max of the decode kernel (threshold
-// 8), so P <= 1 and O is rescaled only when a row's max rises by more than 8.
+// Weights are 2^(x - m) with a lazy running max m: it is raised (and O
+// rescaled) only when a tile's max exceeds it by more than 8, so P <= 2^8.
 // Every mbarrier wait is bounded; a timeout records NF_DEVERR_TIMEOUT and
 // every role leaves its loop.
 // ============================================================================
@@ -149,14 +149,15 @@ __device__ __forceinline__ void tc_convert(const TcRaw &r, int t, unsigned char 
         *reinterpret_cast<uint4 *>(kb + tc_swz(t, 2 * u)) = a;
         *reinterpret_cast<uint4 *>(kb + tc_swz(t, 2 * u + 1)) = c;
     }
-    const uint32_t vsw[2] = {r.vs.x, r.vs.y};
+    // the 4 V scales (one per 32-channel group) as fp16 pairs; 0 past the end
+    const uint32_t keep = r.ok ? 0xFFFFFFFFu : 0u;
+    const uint32_t vsg[4] = {prmt(r.vs.x, 0, 0x1010) & keep, prmt(r.vs.x, 0, 0x3232) & keep,
+                             prmt(r.vs.y, 0, 0x1010) & keep, prmt(r.vs.y, 0, 0x3232) & keep};
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const uint32_t w = (i & 3) == 0 ? r.v[i >> 2].x : (i & 3) == 1 ? r.v[i >> 2].y
                          : (i & 3) == 2 ? r.v[i >> 2].z : r.v[i >> 2].w;
-        const int grp = i >> 2;  // 32-channel scale group
-        const uint32_t s16 = (vsw[grp >> 1] >> (16 * (grp & 1))) & 0xFFFFu;
-        const __half2 sv = u32_h2(r.ok ? s16 * 0x10001u : 0u);
+        const __half2 sv = u32_h2(vsg[i >> 2]);  // 32-channel scale group i / 4
         uint4 o;
         o.x = h2_u32(__hmul2(nib_even(w), sv));
         o.y = h2_u32(__hmul2(nib_odd(w), sv));
@@ -248,35 +249,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         const int t = threadIdx.x - 128;
         {
             const int r = r0 + t;
-            float x[kHeadDim];
+            uint4 qw[16];  // the row as packed bf16
             if (r < p.rows) {
                 const uint4 *qp = reinterpret_cast<const uint4 *>(p.q + out_row(r) * kHeadDim);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const uint4 w = __ldg(qp + u);
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        x[8 * u + 2 * e] = __uint_as_float(ww[e] << 16);
-                        x[8 * u + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
-                    }
-                }
+                for (int u = 0; u < 16; ++u) qw[u] = __ldg(qp + u);
             } else {
 #pragma unroll
-                for (int i = 0; i < kHeadDim; ++i) x[i] = 0.f;
+                for (int u = 0; u < 16; ++u) qw[u] = make_uint4(0, 0, 0, 0);
             }
-            float amax = 0.f;
+            // max |q| straight from the bf16 bits (sign cleared)
+            uint32_t am = 0;
 #pragma unroll
-            for (int i = 0; i < kHeadDim; ++i) amax = fmaxf(amax, fabsf(x[i]));
+            for (int u = 0; u < 16; ++u) {
+                const uint32_t ww[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) am = max(am, max((ww[e] << 16) & 0x7FFFFFFFu, ww[e] & 0x7FFF0000u));
+            }
+            const float amax = __uint_as_float(am);
             const float inv = amax > 0.f ? 1.0f / amax : 0.f;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                uint4 o;
-                o.x = pack_f16(x[8 * c] * inv, x[8 * c + 1] * inv);
-                o.y = pack_f16(x[8 * c + 2] * inv, x[8 * c + 3] * inv);
-                o.z = pack_f16(x[8 * c + 4] * inv, x[8 * c + 5] * inv);
-                o.w = pack_f16(x[8 * c + 6] * inv, x[8 * c + 7] * inv);
-                *reinterpret_cast<uint4 *>(smem + TcSmem::kQ + tc_swz(t, c)) = o;
+                const uint32_t ww[4] = {qw[c].x, qw[c].y, qw[c].z, qw[c].w};
+                uint32_t o4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    o4[e] = pack_f16(__uint_as_float(ww[e] << 16) * inv, __uint_as_float(ww[e] & 0xFFFF0000u) * inv);
+                *reinterpret_cast<uint4 *>(smem + TcSmem::kQ + tc_swz(t, c)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
             qfs[t] = amax * p.scale_log2;
             fence_async_smem();
@@ -312,67 +311,86 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             const int sb = j & 1;
             if (!__all_sync(0xffffffffu, tc_wait(&s_full[sb], (j >> 1) & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
-            uint32_t sv[kTcKeys];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t (&part)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]);
-                tmem_ld32(t_lane + (uint32_t)(sb * 128 + 32 * c), part);
-            }
+            uint32_t sa[32], sbv[32], sc[32], sd[32];
+            tmem_ld32(t_lane + (uint32_t)(sb * 128), sa);
+            tmem_ld32(t_lane + (uint32_t)(sb * 128 + 32), sbv);
+            tmem_ld32(t_lane + (uint32_t)(sb * 128 + 64), sc);
+            tmem_ld32(t_lane + (uint32_t)(sb * 128 + 96), sd);
             tmem_wait_ld();
+#define SV(i) ((i) < 32 ? sa[(i)] : (i) < 64 ? sbv[(i) - 32] : (i) < 96 ? sc[(i) - 64] : sd[(i) - 96])
             const int key0 = j * kTcKeys;
             const int nvis = min(kTcKeys, lim - key0 + 1);  // keys of the tile this row sees (may be <= 0)
-            float mx = -INFINITY;
+            const bool full = nvis >= kTcKeys;  // the row sees the whole tile: no mask
+            if (!full) {
 #pragma unroll
-            for (int i = 0; i < kTcKeys; ++i)
-                if (i < nvis) mx = fmaxf(mx, __uint_as_float(sv[i]));
+                for (int i = 0; i < kTcKeys; ++i)
+                    if (i >= nvis) SV(i) = __float_as_uint(-INFINITY);
+            }
+            // row max over 8 independent partial maxima (short dependency chains)
+            float m8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(SV(e));
+#pragma unroll
+            for (int i = 8; i < kTcKeys; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(SV(i)));
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             const float tmax = mx == -INFINITY ? -INFINITY : mx * qf;
             const bool raise = tmax > m_run + kTcLazy;
-            if (__any_sync(0xffffffffu, raise)) {
-                const float m_new = raise ? tmax : m_run;
-                const float alpha = raise ? ex2(m_run - m_new) : 1.f;  // 0 when m_run was -inf
-                if (j >= 1) {
-                    // O holds P_{j-1} . V_{j-1} once that MMA group has completed
-                    if (!__all_sync(0xffffffffu, tc_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(t_lane + 256u + 32u * c, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(t_lane + 256u + 32u * c, o);
-                    }
-                    tmem_wait_st();
-                }
+            // the warp rescales its rows of O (below, once S is no longer
+            // held) when any of its rows raises its max
+            const bool rescale_o = __any_sync(0xffffffffu, raise) && j >= 1;
+            const float alpha = raise ? ex2(m_run - tmax) : 1.f;  // 0 when m_run was -inf
+            if (raise) {
                 l_run *= alpha;
-                m_run = m_new;
+                m_run = tmax;
             }
-            const float mu = (m_run == -INFINITY ? 0.f : m_run) + kTcLazy;
+            // weights 2^(x - m) <= 2^kTcLazy: inside fp16, and the flat-attention
+            // bulk (a few units below the max) stays in its normal range
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
             // the P buffer was last read by P_{j-2} . V_{j-2}
             if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(&pv_done[sb], ((j - 2) >> 1) & 1, abort_flag))) {
                 ok = false;
                 break;
             }
             unsigned char *pb = smem + TcSmem::kP + sb * 2 * TcSmem::kBlk;
+            // P = 2^(s qf - m), two at a time in fp16 (masked keys hold -inf: 0)
+            float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                float pv[8];
+                uint32_t ph[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = 8 * c + e;
-                    pv[e] = i < nvis ? ex2(fmaf(__uint_as_float(sv[i]), qf, -mu)) : 0.f;
-                    l_run += pv[e];
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = fmaf(__uint_as_float(SV(8 * c + 2 * e)), qf, -mu);
+                    const float x1 = fmaf(__uint_as_float(SV(8 * c + 2 * e + 1)), qf, -mu);
+                    ph[e] = ex2_h2(pack_f16(x0, x1));
                 }
-                uint4 o;
-                o.x = pack_f16(pv[0], pv[1]);
-                o.y = pack_f16(pv[2], pv[3]);
-                o.z = pack_f16(pv[4], pv[5]);
-                o.w = pack_f16(pv[6], pv[7]);
-                *reinterpret_cast<uint4 *>(pb + tc_swz(r, c)) = o;
+                *reinterpret_cast<uint4 *>(pb + tc_swz(r, c)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+                // the row sum from the stored fp16 weights, in fp32
+                const __half2 s01 = __hadd2(u32_h2(ph[0]), u32_h2(ph[1]));
+                const __half2 s23 = __hadd2(u32_h2(ph[2]), u32_h2(ph[3]));
+                const float2 f01 = __half22float2(s01), f23 = __half22float2(s23);
+                lsum[c & 3] += (f01.x + f01.y) + (f23.x + f23.y);
+            }
+            l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+#undef SV
+            if (rescale_o) {
+                // O holds P_{j-1} . V_{j-1} once that MMA group has completed;
+                // P_j . V_j is issued only after this thread's arrival below
+                if (!__all_sync(0xffffffffu, tc_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(t_lane + 256u + 32u * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(t_lane + 256u + 32u * c, o);
+                }
+                tmem_wait_st();
             }
             fence_async_smem();
             tc_fence_before();
@@ -404,7 +422,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             }
             if (dst && p.out_lse)
                 p.out_lse[out_row(row)] =
-                    l_run > 0.f ? (m_run + kTcLazy + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                    l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
         }
     } else if (warp == 8 && lane == 0 && !*abort_flag) {
         // ================================================== MMA issue
