@@ -43,98 +43,124 @@ struct PrefillParams {
 };
 
 // ============================================================================
-// CTA = 128 query rows (the MMA's M) and three roles:
-//   warps 0-3  softmax: thread r owns query row r; reads its row of S from
-//              tensor memory (tcgen05.ld), runs the online softmax, writes
-//              its row of P (fp16) to shared memory, rescales its row of O in
-//              tensor memory when its running max rises, and at the end
-//              reads O, normalises and writes the output;
-//   warps 4-7  converters: thread t stages query row t (scaled to max |q| = 1,
-//              fp16) once, then for every 128-key tile loads key t's K8/V4
-//              codes and scales (prefetched a tile ahead in registers) and
-//              writes the dequantised fp16 K row and V row into a two-stage
-//              ring;
-//   warp 8     tensor memory allocation and, on one thread, the MMAs:
-//              S_j = Q . K_j^T into one of two S buffers, then
-//              O += P_{j-1} . V_{j-1}, each group of 8 MMAs (K = 16) committed
-//              to an mbarrier.
-// Tensor memory (512 columns x 128 lanes): S buffers at columns 0 and 128,
-// O at 256.  Shared operands use the 128-byte-swizzled canonical layouts:
-//   Q, P   A operands, K-major: [2 blocks of 64 columns][128 rows][128 bytes];
-//   K      B operand of S, K-major: [2 blocks of 64 channels][128 keys][128 bytes];
-//   V      B operand of O, MN-major: [2 blocks of 64 channels][128 keys][128 bytes],
+// CTA = 256 query rows: two tiles a, b of 128 rows (each the M of its own
+// MMAs) that share every K/V tile, and four roles:
+//   warps 0-3, 4-7  softmax of tile a, of tile b: thread r owns row r of its
+//              tile; reads its row of S from tensor memory (tcgen05.ld), runs
+//              the online softmax, writes its row of P (fp16) to shared memory,
+//              rescales its row of O in tensor memory when its running max
+//              rises, and at the end reads O, normalises and writes the output;
+//   warps 8-11 converters: they stage both tiles' query rows (scaled to
+//              max |q| = 1, fp16) once; then for every 64-key tile thread t
+//              loads key t's K codes (t < 64) or key t - 64's V nibbles and
+//              scales (prefetched a tile ahead in registers) and writes that
+//              dequantised fp16 row into a two-stage ring;
+//   warp 12    tensor memory allocation and, on one thread, the MMAs: per K/V
+//              tile j, S_x = Q_x . K_j^T (x = a, b) into one of two S buffers
+//              of tile x, then O_x += P_x . V for tile j - 1, each group
+//              committed to an mbarrier.
+// The K/V ring is converted once for 256 rows, and each SM sub-partition runs
+// two softmax warps, one of each tile.
+// Tensor memory (512 columns x 128 lanes): S of tile x, buffer b at columns
+// 128x + 64b (64 keys), O of tile x at 256 + 128x.  Shared operands use the
+// 128-byte-swizzled canonical layouts (rows of 128 bytes = 64 fp16, 8-row
+// groups of 1024 bytes):
+//   Q_x    A of S, K-major: [2 blocks of 64 channels][128 rows][128 bytes];
+//   K      B of S, K-major: [2 blocks of 64 channels][64 keys][128 bytes];
+//   P_x    A of O, K-major: [128 rows][64 keys x 2 bytes];
+//   V      B of O, MN-major: [2 blocks of 64 channels][64 keys][128 bytes],
 //          channels inside each 8-channel chunk in the nibble-unpacking order.
 // Weights are 2^(x - m) with a lazy running max m: it is raised (and O
 // rescaled) only when a tile's max exceeds it by more than 8, so P <= 2^8.
 // Every mbarrier wait is bounded; a timeout records NF_DEVERR_TIMEOUT and
 // every role leaves its loop.
 // ============================================================================
-constexpr int kTcThreads = 288;
-constexpr int kTcRows = 128;   // query rows per CTA (M of both MMAs)
-constexpr int kTcKeys = 128;   // keys per tile (N of S = Q.K^T, K of O += P.V)
+constexpr int kTcThreads = 416;
+constexpr int kTcRows = 256;   // query rows per CTA (two MMA tiles of 128)
+constexpr int kTcKeys = 64;    // keys per K/V tile (N of S = Q.K^T, K of O += P.V)
 constexpr float kTcLazy = 8.0f;
-constexpr uint32_t kTcIdescQK = umma_idesc_f16(128, 128, false);  // B = K rows, K-major
+constexpr uint32_t kTcIdescQK = umma_idesc_f16(128, 64, false);   // B = K rows, K-major
 constexpr uint32_t kTcIdescPV = umma_idesc_f16(128, 128, true);   // B = V rows, MN-major
 
 struct TcSmem {
-    static constexpr int kBlk = 16384;                // one 64-column block of 128 rows x 128 bytes
-    static constexpr int kQ = 0;                      // 2 blocks
-    static constexpr int kK = 2 * kBlk;               // [2 stages][2 blocks]
-    static constexpr int kV = 6 * kBlk;               // [2 stages][2 blocks]
-    static constexpr int kP = 10 * kBlk;              // [2 buffers][2 blocks]
-    static constexpr int kBars = 14 * kBlk;           // 11 mbarriers
-    static constexpr int kQf = kBars + 128;           // float [128]
-    static constexpr int kMisc = kQf + 128 * 4;       // tmem base, abort flag
+    static constexpr int kQ = 0;                      // [2 tiles][2 blocks][128 rows][128 B]
+    static constexpr int kK = 65536;                  // [2 stages][2 blocks][64 keys][128 B]
+    static constexpr int kV = kK + 32768;             // [2 stages][2 blocks][64 keys][128 B]
+    static constexpr int kP = kV + 32768;             // [2 buffers][2 tiles][128 rows][128 B]
+    static constexpr int kBars = kP + 65536;          // mbarriers
+    static constexpr int kQf = kBars + 256;           // float [256]
+    static constexpr int kMisc = kQf + 256 * 4;       // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static_assert(kBytes <= 232448, "shared memory per CTA");
 };
+// mbarrier slots
+enum { kBarQ = 0, kBarKV = 1, kBarS = 3, kBarP = 7, kBarPV = 11, kBarO = 15, kBarDrain = 16, kNumBars = 17 };
 
-// byte offset of row r, 16-byte chunk c (0..15 over 128 columns of fp16) in a
-// two-block 128-byte-swizzled operand
-__device__ __forceinline__ uint32_t tc_swz(int r, int c) {
-    return (uint32_t)(c >> 3) * TcSmem::kBlk + (uint32_t)r * 128u + (uint32_t)(((c ^ r) & 7) * 16);
+// byte offset of row r, 16-byte chunk c (0..15: 8 fp16 each) in a two-block
+// 128-byte-swizzled operand whose blocks are `blk` bytes apart
+__device__ __forceinline__ uint32_t tc_swz(int r, int c, uint32_t blk) {
+    return (uint32_t)(c >> 3) * blk + (uint32_t)r * 128u + (uint32_t)(((c ^ r) & 7) * 16);
 }
 
-struct TcRaw {
-    uint4 k[8];  // K codes of the key
-    uint4 v[4];  // V nibbles
-    uint2 vs;    // 4 V scales
-    uint32_t ks; // K scale (low half)
-    int ok;      // key inside the sequence
+struct TcRawK {
+    uint4 k[8];   // K codes of the key
+    uint32_t ks;  // K scale (low half)
+    int ok;       // key inside the sequence
+};
+struct TcRawV {
+    uint4 v[4];   // V nibbles
+    uint2 vs;     // 4 V scales
+    int ok;
 };
 
-__device__ __forceinline__ void tc_load(const PrefillParams &p, const int32_t *bt, int L, int h, int tile, int t,
-                                        TcRaw &r) {
-    const int pos = tile * kTcKeys + t;
-    const int blk = bt[(tile * kTcKeys) >> 8];  // a tile lies in one block whose entry exists
-    r.ok = pos < L;
-    if (blk < 0 || blk >= p.num_blocks) {
-        if (t == 0) report(NF_DEVERR_BLOCK_ID);
+// a tile lies in one 256-key block, and its first key is < L, so the table
+// entry of that block exists; a bad entry reads as zeros (and is reported)
+__device__ __forceinline__ size_t tc_slot(const PrefillParams &p, const int32_t *bt, int h, int pos, bool &good) {
+    const int blk = bt[pos >> 8];
+    good = blk >= 0 && blk < p.num_blocks;
+    if (!good) {
+        report(NF_DEVERR_BLOCK_ID);
+        return 0;
+    }
+    return ((size_t)blk * p.num_kv_heads + h) * kBlock + (pos & (kBlock - 1));
+}
+__device__ __forceinline__ void tc_load_k(const PrefillParams &p, const int32_t *bt, int L, int h, int tile, int key,
+                                          TcRawK &r) {
+    const int pos = tile * kTcKeys + key;
+    bool good;
+    const size_t si = tc_slot(p, bt, h, pos, good);
+    r.ok = good && pos < L;
+    if (!good) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) r.k[u] = make_uint4(0, 0, 0, 0);
+        r.ks = 0;
+        return;
+    }
+    const unsigned char *kp = reinterpret_cast<const unsigned char *>(p.k_codes) + si * kHeadDim;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) r.k[u] = ldg16(kp + 16 * u);
+    r.ks = __ldg(reinterpret_cast<const unsigned short *>(p.k_scales + si));
+}
+__device__ __forceinline__ void tc_load_v(const PrefillParams &p, const int32_t *bt, int L, int h, int tile, int key,
+                                          TcRawV &r) {
+    const int pos = tile * kTcKeys + key;
+    bool good;
+    const size_t si = tc_slot(p, bt, h, pos, good);
+    r.ok = good && pos < L;
+    if (!good) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) r.v[u] = make_uint4(0, 0, 0, 0);
         r.vs = make_uint2(0, 0);
-        r.ks = 0;
-        r.ok = 0;
         return;
     }
-    const size_t si = ((size_t)blk * p.num_kv_heads + h) * kBlock + (pos & (kBlock - 1));
-    const unsigned char *kp = reinterpret_cast<const unsigned char *>(p.k_codes) + si * kHeadDim;
     const unsigned char *vp = p.v_codes + si * (kHeadDim / 2);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) r.k[u] = ldg16(kp + 16 * u);
 #pragma unroll
     for (int u = 0; u < 4; ++u) r.v[u] = ldg16(vp + 16 * u);
     r.vs = __ldg(reinterpret_cast<const uint2 *>(p.v_scales + si * (kHeadDim / kVGroup)));
-    r.ks = __ldg(reinterpret_cast<const unsigned short *>(p.k_scales + si));
 }
-
-// key t's dequantised fp16 K row (code x K scale) and V row (code x V scale;
-// 0 past the end) into stage buffers kb, vb
-__device__ __forceinline__ void tc_convert(const TcRaw &r, int t, unsigned char *kb, unsigned char *vb) {
-    const uint32_t ks2 = r.ok ? (r.ks & 0xFFFFu) * 0x10001u : 0u;
-    const __half2 sk = u32_h2(ks2);
+// key's dequantised fp16 K row (code x K scale)
+__device__ __forceinline__ void tc_convert_k(const TcRawK &r, int key, unsigned char *kb) {
+    const __half2 sk = u32_h2(r.ok ? (r.ks & 0xFFFFu) * 0x10001u : 0u);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         uint4 a, c;
@@ -146,10 +172,12 @@ __device__ __forceinline__ void tc_convert(const TcRaw &r, int t, unsigned char 
         a.z = h2_u32(__hmul2(u32_h2(a.z), sk)); a.w = h2_u32(__hmul2(u32_h2(a.w), sk));
         c.x = h2_u32(__hmul2(u32_h2(c.x), sk)); c.y = h2_u32(__hmul2(u32_h2(c.y), sk));
         c.z = h2_u32(__hmul2(u32_h2(c.z), sk)); c.w = h2_u32(__hmul2(u32_h2(c.w), sk));
-        *reinterpret_cast<uint4 *>(kb + tc_swz(t, 2 * u)) = a;
-        *reinterpret_cast<uint4 *>(kb + tc_swz(t, 2 * u + 1)) = c;
+        *reinterpret_cast<uint4 *>(kb + tc_swz(key, 2 * u, 8192u)) = a;
+        *reinterpret_cast<uint4 *>(kb + tc_swz(key, 2 * u + 1, 8192u)) = c;
     }
-    // the 4 V scales (one per 32-channel group) as fp16 pairs; 0 past the end
+}
+// key's dequantised fp16 V row (code x V scale; 0 past the end)
+__device__ __forceinline__ void tc_convert_v(const TcRawV &r, int key, unsigned char *vb) {
     const uint32_t keep = r.ok ? 0xFFFFFFFFu : 0u;
     const uint32_t vsg[4] = {prmt(r.vs.x, 0, 0x1010) & keep, prmt(r.vs.x, 0, 0x3232) & keep,
                              prmt(r.vs.y, 0, 0x1010) & keep, prmt(r.vs.y, 0, 0x3232) & keep};
@@ -163,7 +191,7 @@ __device__ __forceinline__ void tc_convert(const TcRaw &r, int t, unsigned char 
         o.y = h2_u32(__hmul2(nib_odd(w), sv));
         o.z = h2_u32(__hmul2(nib_even(w >> 8), sv));
         o.w = h2_u32(__hmul2(nib_odd(w >> 8), sv));
-        *reinterpret_cast<uint4 *>(vb + tc_swz(t, i)) = o;
+        *reinterpret_cast<uint4 *>(vb + tc_swz(key, i, 8192u)) = o;
     }
 }
 
@@ -185,24 +213,29 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TcSmem::kBars);
-    uint64_t *q_full = bars + 0, *kv_full = bars + 1, *s_full = bars + 3, *p_full = bars + 5, *pv_done = bars + 7,
-             *o_full = bars + 9, *drain = bars + 10;
+    uint64_t *q_full = bars + kBarQ, *kv_full = bars + kBarKV, *o_full = bars + kBarO, *drain = bars + kBarDrain;
+    // [tile][buffer]
+    auto s_full = [&](int x, int b) { return bars + kBarS + 2 * x + b; };
+    auto p_full = [&](int x, int b) { return bars + kBarP + 2 * x + b; };
+    auto pv_done = [&](int x, int b) { return bars + kBarPV + 2 * x + b; };
     float *qfs = reinterpret_cast<float *>(smem + TcSmem::kQf);
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + TcSmem::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcSmem::kMisc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.z, h = blockIdx.y;
     const int rt = p.row_tiles - 1 - (int)blockIdx.x;  // late positions first
-    const int r0 = rt * 128;
+    const int r0 = rt * kTcRows;
     const int G = p.group;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 128);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&kv_full[i], 128);
-            mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 128);
-            mbar_init(&pv_done[i], 1);
+            for (int x = 0; x < 2; ++x) {
+                mbar_init(s_full(x, i), 1);
+                mbar_init(p_full(x, i), 128);
+                mbar_init(pv_done(x, i), 1);
+            }
         }
         mbar_init(o_full, 1);
         mbar_init(drain, 1);
@@ -214,7 +247,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         }
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == 12) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
@@ -231,24 +264,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         return ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * G + gq;
     };
     const bool bad_len = L < p.n_q || L > p.max_seqlen;
-    const int last_row = min(r0 + 128, p.rows) - 1;
+    const int last_row = min(r0 + kTcRows, p.rows) - 1;
     const int n_keys = bad_len ? 0 : (p.causal ? L - p.n_q + last_row / G + 1 : L);
     const int T = (n_keys + kTcKeys - 1) / kTcKeys;
     const int32_t *bt = p.block_table + (size_t)b * p.max_blocks;
 
     if (bad_len) {
         if (threadIdx.x == 0 && rt == p.row_tiles - 1 && h == 0) report(NF_DEVERR_SEQLEN);
-        for (int idx = threadIdx.x; idx < 128 * kHeadDim; idx += kTcThreads) {
+        for (int idx = threadIdx.x; idx < kTcRows * kHeadDim; idx += kTcThreads) {
             const int r = r0 + idx / kHeadDim, ch = idx % kHeadDim;
             if (r >= p.rows) continue;
             p.out[out_row(r) * kHeadDim + ch] = 0.f;
             if (ch == 0 && p.out_lse) p.out_lse[out_row(r)] = -INFINITY;
         }
-    } else if (warp >= 4 && warp < 8 && !*abort_flag) {
+    } else if (warp >= 8 && warp < 12 && !*abort_flag) {
         // ================================================== converters
-        const int t = threadIdx.x - 128;
-        {
-            const int r = r0 + t;
+        const int t = threadIdx.x - 256;
+        for (int x = 0; x < 2; ++x) {
+            const int r = r0 + 128 * x + t;
             uint4 qw[16];  // the row as packed bf16
             if (r < p.rows) {
                 const uint4 *qp = reinterpret_cast<const uint4 *>(p.q + out_row(r) * kHeadDim);
@@ -275,53 +308,65 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     o4[e] = pack_f16(__uint_as_float(ww[e] << 16) * inv, __uint_as_float(ww[e] & 0xFFFF0000u) * inv);
-                *reinterpret_cast<uint4 *>(smem + TcSmem::kQ + tc_swz(t, c)) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                *reinterpret_cast<uint4 *>(smem + TcSmem::kQ + x * 32768 + tc_swz(t, c, 16384u)) =
+                    make_uint4(o4[0], o4[1], o4[2], o4[3]);
             }
-            qfs[t] = amax * p.scale_log2;
-            fence_async_smem();
-            mbar_arrive(q_full);
+            qfs[128 * x + t] = amax * p.scale_log2;
         }
-        TcRaw ra, rb;
-        if (T > 0) tc_load(p, bt, L, h, 0, t, ra);
-        auto stage_tile = [&](int j, TcRaw &cur, TcRaw &nxt) -> bool {
-            if (j + 1 < T) tc_load(p, bt, L, h, j + 1, t, nxt);
-            const int s = j & 1;
-            if (j >= 2 && !tc_wait(&pv_done[s], ((j - 2) >> 1) & 1, abort_flag)) return false;
-            tc_convert(cur, t, smem + TcSmem::kK + s * 2 * TcSmem::kBlk, smem + TcSmem::kV + s * 2 * TcSmem::kBlk);
-            fence_async_smem();
-            mbar_arrive(&kv_full[s]);
-            return true;
+        fence_async_smem();
+        mbar_arrive(q_full);
+        // K/V rows: warps 8-9 the K rows of keys 0..63, warps 10-11 the V rows
+        auto ring = [&](auto &ra, auto &rb, auto load, auto convert, int key, int region) {
+            if (T > 0) load(0, ra);
+            auto stage_tile = [&](int j, auto &cur, auto &nxt) -> bool {
+                if (j + 1 < T) load(j + 1, nxt);
+                const int s = j & 1;
+                // the stage was last read by S and O of tile j - 2 (tile b's O group is the later)
+                if (j >= 2 && !tc_wait(pv_done(1, s), ((j - 2) >> 1) & 1, abort_flag)) return false;
+                convert(cur, key, smem + region + s * 16384);
+                fence_async_smem();
+                mbar_arrive(&kv_full[s]);
+                return true;
+            };
+            for (int j = 0; j < T; j += 2) {
+                if (!stage_tile(j, ra, rb)) break;
+                if (j + 1 < T && !stage_tile(j + 1, rb, ra)) break;
+            }
         };
-        for (int j = 0; j < T; j += 2) {
-            if (!stage_tile(j, ra, rb)) break;
-            if (j + 1 < T && !stage_tile(j + 1, rb, ra)) break;
+        if (t < 64) {
+            TcRawK ra, rb;
+            ring(ra, rb, [&](int tile, TcRawK &r) { tc_load_k(p, bt, L, h, tile, t, r); },
+                 [&](const TcRawK &r, int key, unsigned char *dst) { tc_convert_k(r, key, dst); }, t, TcSmem::kK);
+        } else {
+            TcRawV ra, rb;
+            ring(ra, rb, [&](int tile, TcRawV &r) { tc_load_v(p, bt, L, h, tile, t - 64, r); },
+                 [&](const TcRawV &r, int key, unsigned char *dst) { tc_convert_v(r, key, dst); }, t - 64, TcSmem::kV);
         }
-    } else if (warp < 4 && !*abort_flag) {
-        // ================================================== softmax
-        const int r = threadIdx.x;
-        const int row = r0 + r;
+    } else if (warp < 8 && !*abort_flag) {
+        // ================================================== softmax (tile x)
+        const int x = warp >> 2;
+        const int r = threadIdx.x & 127;
+        const int row = r0 + 128 * x + r;
         const int lim = row < p.rows ? (p.causal ? L - p.n_q + row / G : L - 1) : -1;
-        const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const uint32_t s_col = 128u * x, o_col = 256u + 128u * x;
         float m_run = -INFINITY, l_run = 0.f;
         // every wait's outcome is made warp-uniform: the tcgen05 loads and
         // stores below are warp-collective
         bool ok = __all_sync(0xffffffffu, tc_wait(q_full, 0, abort_flag));
-        const float qf = ok ? qfs[r] : 0.f;
+        const float qf = ok ? qfs[128 * x + r] : 0.f;
         for (int j = 0; ok && j < T; ++j) {
             const int sb = j & 1;
-            if (!__all_sync(0xffffffffu, tc_wait(&s_full[sb], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, tc_wait(s_full(x, sb), (j >> 1) & 1, abort_flag))) { ok = false; break; }
             tc_fence_after();
-            uint32_t sa[32], sbv[32], sc[32], sd[32];
-            tmem_ld32(t_lane + (uint32_t)(sb * 128), sa);
-            tmem_ld32(t_lane + (uint32_t)(sb * 128 + 32), sbv);
-            tmem_ld32(t_lane + (uint32_t)(sb * 128 + 64), sc);
-            tmem_ld32(t_lane + (uint32_t)(sb * 128 + 96), sd);
+            uint32_t sa[32], sbv[32];
+            tmem_ld32(t_lane + s_col + 64u * sb, sa);
+            tmem_ld32(t_lane + s_col + 64u * sb + 32u, sbv);
             tmem_wait_ld();
-#define SV(i) ((i) < 32 ? sa[(i)] : (i) < 64 ? sbv[(i) - 32] : (i) < 96 ? sc[(i) - 64] : sd[(i) - 96])
+#define SV(i) ((i) < 32 ? sa[(i)] : sbv[(i) - 32])
             const int key0 = j * kTcKeys;
             const int nvis = min(kTcKeys, lim - key0 + 1);  // keys of the tile this row sees (may be <= 0)
-            const bool full = nvis >= kTcKeys;  // the row sees the whole tile: no mask
-            if (!full) {
+            if (nvis < kTcKeys) {
 #pragma unroll
                 for (int i = 0; i < kTcKeys; ++i)
                     if (i >= nvis) SV(i) = __float_as_uint(-INFINITY);
@@ -347,16 +392,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             // weights 2^(x - m) <= 2^kTcLazy: inside fp16, and the flat-attention
             // bulk (a few units below the max) stays in its normal range
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            // the P buffer was last read by P_{j-2} . V_{j-2}
-            if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(&pv_done[sb], ((j - 2) >> 1) & 1, abort_flag))) {
+            // the P buffer was last read by O of tile j - 2
+            if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(pv_done(x, sb), ((j - 2) >> 1) & 1, abort_flag))) {
                 ok = false;
                 break;
             }
-            unsigned char *pb = smem + TcSmem::kP + sb * 2 * TcSmem::kBlk;
+            unsigned char *pb = smem + TcSmem::kP + sb * 32768 + x * 16384;
             // P = 2^(s qf - m), two at a time in fp16 (masked keys hold -inf: 0)
             float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 uint32_t ph[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -364,7 +409,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
                     const float x1 = fmaf(__uint_as_float(SV(8 * c + 2 * e + 1)), qf, -mu);
                     ph[e] = ex2_h2(pack_f16(x0, x1));
                 }
-                *reinterpret_cast<uint4 *>(pb + tc_swz(r, c)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+                *reinterpret_cast<uint4 *>(pb + tc_swz(r, c, 0u)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
                 // the row sum from the stored fp16 weights, in fp32
                 const __half2 s01 = __hadd2(u32_h2(ph[0]), u32_h2(ph[1]));
                 const __half2 s23 = __hadd2(u32_h2(ph[2]), u32_h2(ph[3]));
@@ -374,9 +419,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             l_run += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
 #undef SV
             if (rescale_o) {
-                // O holds P_{j-1} . V_{j-1} once that MMA group has completed;
-                // P_j . V_j is issued only after this thread's arrival below
-                if (!__all_sync(0xffffffffu, tc_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
+                // O holds the products up to tile j - 1 once that group has
+                // completed; tile j's is issued only after this thread's arrival
+                if (!__all_sync(0xffffffffu, tc_wait(pv_done(x, (j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag))) {
                     ok = false;
                     break;
                 }
@@ -384,17 +429,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
-                    tmem_ld32(t_lane + 256u + 32u * c, o);
+                    tmem_ld32(t_lane + o_col + 32u * c, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(t_lane + 256u + 32u * c, o);
+                    tmem_st32(t_lane + o_col + 32u * c, o);
                 }
                 tmem_wait_st();
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(&p_full[sb]);
+            mbar_arrive(p_full(x, sb));
         }
         if (ok && __all_sync(0xffffffffu, tc_wait(o_full, 0, abort_flag))) {
             tc_fence_after();
@@ -403,7 +448,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                tmem_ld32(t_lane + 256u + 32u * c, o);
+                tmem_ld32(t_lane + o_col + 32u * c, o);
                 tmem_wait_ld();
                 if (dst) {
                     // column 8g + e holds channel 8g + (0, 4, 1, 5, 2, 6, 3, 7)[e]
@@ -421,25 +466,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
                 }
             }
             if (dst && p.out_lse)
-                p.out_lse[out_row(row)] =
-                    l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                p.out_lse[out_row(row)] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
         }
-    } else if (warp == 8 && lane == 0 && !*abort_flag) {
+    } else if (warp == 12 && lane == 0 && !*abort_flag) {
         // ================================================== MMA issue
         const uint32_t sQ = smem_addr(smem + TcSmem::kQ), sK = smem_addr(smem + TcSmem::kK);
         const uint32_t sV = smem_addr(smem + TcSmem::kV), sP = smem_addr(smem + TcSmem::kP);
+        // O_x += P_x . V for K/V tile i
         auto pv = [&](int i) -> bool {
             const int s = i & 1;
-            if (!tc_wait(&p_full[s], (i >> 1) & 1, abort_flag)) return false;
-            tc_fence_after();
+            for (int x = 0; x < 2; ++x) {
+                if (!tc_wait(p_full(x, s), (i >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = umma_desc_sw128(sP + s * 2 * TcSmem::kBlk + (kk >> 2) * TcSmem::kBlk + (kk & 3) * 32,
-                                                    16, 1024);
-                const uint64_t bd = umma_desc_sw128(sV + s * 2 * TcSmem::kBlk + kk * 2048, TcSmem::kBlk, 1024);
-                umma_f16(tmem + 256u, ad, bd, kTcIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = umma_desc_sw128(sP + s * 32768 + x * 16384 + kk * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(sV + s * 16384 + kk * 2048, 8192, 1024);
+                    umma_f16(tmem + 256u + 128u * x, ad, bd, kTcIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(pv_done(x, s));
             }
-            umma_commit(&pv_done[s]);
             return true;
         };
         bool ok = tc_wait(q_full, 0, abort_flag);
@@ -447,14 +493,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             const int s = j & 1;
             if (!tc_wait(&kv_full[s], (j >> 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
+            for (int x = 0; x < 2; ++x) {
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = umma_desc_sw128(sQ + (ks >> 2) * TcSmem::kBlk + (ks & 3) * 32, 16, 1024);
-                const uint64_t bd =
-                    umma_desc_sw128(sK + s * 2 * TcSmem::kBlk + (ks >> 2) * TcSmem::kBlk + (ks & 3) * 32, 16, 1024);
-                umma_f16(tmem + (uint32_t)(s * 128), ad, bd, kTcIdescQK, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t ad = umma_desc_sw128(sQ + x * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(sK + s * 16384 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    umma_f16(tmem + 128u * x + 64u * s, ad, bd, kTcIdescQK, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(s_full(x, s));
             }
-            umma_commit(&s_full[s]);
             if (j >= 1 && !pv(j - 1)) { ok = false; break; }
         }
         if (ok && T > 0) ok = pv(T - 1);
@@ -470,7 +517,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
