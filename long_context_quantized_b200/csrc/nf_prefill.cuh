@@ -54,7 +54,7 @@ struct PrefillParams {
 //              max |q| = 1, fp16) once; then for every 64-key tile thread t
 //              loads key t's K codes (t < 64) or key t - 64's V nibbles and
 //              scales (prefetched a tile ahead in registers) and writes that
-//              dequantised fp16 row into a two-stage ring;
+//              dequantised fp16 row into a three-stage ring;
 //   warp 12    tensor memory allocation and, on one thread, the MMAs: per K/V
 //              tile j, S_x = Q_x . K_j^T (x = a, b) into one of two S buffers
 //              of tile x, then O_x += P_x . V for tile j - 1, each group
@@ -66,7 +66,7 @@ struct PrefillParams {
 // 128-byte-swizzled canonical layouts (rows of 128 bytes = 64 fp16, 8-row
 // groups of 1024 bytes):
 //   Q_x    A of S, K-major: [2 blocks of 64 channels][128 rows][128 bytes];
-//   K      B of S, K-major: [2 blocks of 64 channels][64 keys][128 bytes];
+//   K      B of S, K-major: [2 blocks of 64 channels][64 keys][128 bytes] (x 3 stages);
 //   P_x    A of O, K-major: [128 rows][64 keys x 2 bytes];
 //   V      B of O, MN-major: [2 blocks of 64 channels][64 keys][128 bytes],
 //          channels inside each 8-channel chunk in the nibble-unpacking order.
@@ -84,9 +84,10 @@ constexpr uint32_t kTcIdescPV = umma_idesc_f16(128, 128, true);   // B = V rows,
 
 struct TcSmem {
     static constexpr int kQ = 0;                      // [2 tiles][2 blocks][128 rows][128 B]
-    static constexpr int kK = 65536;                  // [2 stages][2 blocks][64 keys][128 B]
-    static constexpr int kV = kK + 32768;             // [2 stages][2 blocks][64 keys][128 B]
-    static constexpr int kP = kV + 32768;             // [2 buffers][2 tiles][128 rows][128 B]
+    static constexpr int kStages = 3;                 // K/V ring depth
+    static constexpr int kK = 65536;                  // [3 stages][2 blocks][64 keys][128 B]
+    static constexpr int kV = kK + kStages * 16384;   // [3 stages][2 blocks][64 keys][128 B]
+    static constexpr int kP = kV + kStages * 16384;   // [2 buffers][2 tiles][128 rows][128 B]
     static constexpr int kBars = kP + 65536;          // mbarriers
     static constexpr int kQf = kBars + 256;           // float [256]
     static constexpr int kMisc = kQf + 256 * 4;       // tmem base, abort flag
@@ -94,7 +95,8 @@ struct TcSmem {
     static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 // mbarrier slots
-enum { kBarQ = 0, kBarKV = 1, kBarS = 3, kBarP = 7, kBarPV = 11, kBarO = 15, kBarDrain = 16, kNumBars = 17 };
+enum { kBarQ = 0, kBarKV = 1, kBarFree = 4, kBarS = 7, kBarP = 11, kBarPV = 15, kBarO = 19, kBarDrain = 20, kNumBars = 21 };
+static_assert(kNumBars * 8 <= 256, "mbarrier slots");
 
 // byte offset of row r, 16-byte chunk c (0..15: 8 fp16 each) in a two-block
 // 128-byte-swizzled operand whose blocks are `blk` bytes apart
@@ -213,7 +215,8 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, uint32_t parity, volatile
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TcSmem::kBars);
-    uint64_t *q_full = bars + kBarQ, *kv_full = bars + kBarKV, *o_full = bars + kBarO, *drain = bars + kBarDrain;
+    uint64_t *q_full = bars + kBarQ, *kv_full = bars + kBarKV, *kv_free = bars + kBarFree, *o_full = bars + kBarO,
+             *drain = bars + kBarDrain;
     // [tile][buffer]
     auto s_full = [&](int x, int b) { return bars + kBarS + 2 * x + b; };
     auto p_full = [&](int x, int b) { return bars + kBarP + 2 * x + b; };
@@ -229,8 +232,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 128);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < TcSmem::kStages; ++i) {
             mbar_init(&kv_full[i], 128);
+            mbar_init(&kv_free[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             for (int x = 0; x < 2; ++x) {
                 mbar_init(s_full(x, i), 1);
                 mbar_init(p_full(x, i), 128);
@@ -320,9 +326,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             if (T > 0) load(0, ra);
             auto stage_tile = [&](int j, auto &cur, auto &nxt) -> bool {
                 if (j + 1 < T) load(j + 1, nxt);
-                const int s = j & 1;
-                // the stage was last read by S and O of tile j - 2 (tile b's O group is the later)
-                if (j >= 2 && !tc_wait(pv_done(1, s), ((j - 2) >> 1) & 1, abort_flag)) return false;
+                const int s = j % TcSmem::kStages;
+                // the stage is free once every MMA of tile j - 3 has completed
+                if (j >= TcSmem::kStages &&
+                    !tc_wait(&kv_free[s], (j / TcSmem::kStages - 1) & 1, abort_flag))
+                    return false;
                 convert(cur, key, smem + region + s * 16384);
                 fence_async_smem();
                 mbar_arrive(&kv_full[s]);
@@ -472,32 +480,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         // ================================================== MMA issue
         const uint32_t sQ = smem_addr(smem + TcSmem::kQ), sK = smem_addr(smem + TcSmem::kK);
         const uint32_t sV = smem_addr(smem + TcSmem::kV), sP = smem_addr(smem + TcSmem::kP);
-        // O_x += P_x . V for K/V tile i
+        // O_x += P_x . V for K/V tile i (P buffer i & 1, K/V stage i % 3)
         auto pv = [&](int i) -> bool {
-            const int s = i & 1;
+            const int s = i & 1, st = i % TcSmem::kStages;
             for (int x = 0; x < 2; ++x) {
                 if (!tc_wait(p_full(x, s), (i >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t ad = umma_desc_sw128(sP + s * 32768 + x * 16384 + kk * 32, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(sV + s * 16384 + kk * 2048, 8192, 1024);
+                    const uint64_t bd = umma_desc_sw128(sV + st * 16384 + kk * 2048, 8192, 1024);
                     umma_f16(tmem + 256u + 128u * x, ad, bd, kTcIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(pv_done(x, s));
             }
+            umma_commit(&kv_free[st]);  // every MMA that reads stage st for tile i is done
             return true;
         };
         bool ok = tc_wait(q_full, 0, abort_flag);
         for (int j = 0; ok && j < T; ++j) {
-            const int s = j & 1;
-            if (!tc_wait(&kv_full[s], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            const int s = j & 1, st = j % TcSmem::kStages;
+            if (!tc_wait(&kv_full[st], (j / TcSmem::kStages) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             for (int x = 0; x < 2; ++x) {
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t ad = umma_desc_sw128(sQ + x * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(sK + s * 16384 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(sK + st * 16384 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
                     umma_f16(tmem + 128u * x + 64u * s, ad, bd, kTcIdescQK, ks > 0 ? 1u : 0u);
                 }
                 umma_commit(s_full(x, s));
