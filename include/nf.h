@@ -298,7 +298,7 @@ nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_
  * Numerics: each query row is scaled to max |q| = 1 and rounded to fp16 once;
  *   K and V are dequantised to fp16 (code x scale, one rounding each); the
  *   softmax weights are rounded to fp16; products accumulate in fp32 on the
- *   5th-generation tensor cores (tcgen05.mma kind::f16, M = N = 128).
+ *   5th-generation tensor cores (tcgen05.mma kind::f16, M = 128).
  *   The dequantised K values must lie inside the fp16 range as well.
  * Device errors: NF_DEVERR_SEQLEN (the sequence's rows come out o = 0,
  *   lse = -inf), NF_DEVERR_BLOCK_ID (that tile's keys read as zeros).
