@@ -20,6 +20,11 @@
  *         channel in the low nibble;
  *      scale = fp16_rne_saturating(fp32(absmax / 127 or 7));
  *      code  = clamp(round_half_even(fp32(x / float(scale)))), 0 if scale == 0.
+ *  - The same section lists the --kv-dtype options int8 and fp8, by name only.
+ *    Read here as: int8 -- K and V both by the K rule above; fp8 -- K and V as
+ *    OCP E4M3FN codes of x / scale with scale = absmax / 448 per (token,
+ *    kv-head), rounded half to even and saturated at +-448 (formats 2 and 3
+ *    of the pool below).
  *  - The cache is segmented (page "標籤: vLLM", section 2 "C++/CUDA 層的 kernel
  *    fusion 與 KV cache 策略": KV managed as segments rather than one buffer);
  *    here a segment is a 256-token block found through a per-sequence block
