@@ -336,9 +336,14 @@ int nfref_append(int fmt, int num_blocks, int H, int d,
                  const int32_t *block_table, int max_blocks, const int32_t *seqlens_before)
 {
     int status = 0;
+    /* Tokens of one (sequence, kv-head) pair are taken in order; different
+     * pairs write disjoint slots (unless two sequences' tables name the same
+     * block, which is outside the contract), so the pairs may run in parallel
+     * without changing any byte of the result. */
+#pragma omp parallel for collapse(2) schedule(dynamic, 1) reduction(min : status) if ((int64_t)batch * n_new * H > 65536)
     for (int b = 0; b < batch; ++b)
-        for (int i = 0; i < n_new; ++i)
-            for (int h = 0; h < H; ++h) {
+        for (int h = 0; h < H; ++h)
+            for (int i = 0; i < n_new; ++i) {
                 int pos = seqlens_before[b] + i;
                 int bi = pos / NFREF_BLOCK;
                 if (pos < 0 || bi >= max_blocks) {
