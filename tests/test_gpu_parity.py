@@ -174,19 +174,8 @@ def _full_size(name, fmt, heads, layer=0):
     return check_attention(select_heads(g["out"], w, hs), select_heads(g["lse"], w, hs), ref_o, ref_l)
 
 
-def test_workload_tiny_all_heads():
-    _full_size("tiny", K8, heads=None)
-
-
-@pytest.mark.parametrize("name,heads,layer", [
-    ("ctx32k_append", [0, 3], 0),
-    ("ctx32k_append", [1], 15),
-    ("ragged_c2", [0, 3], 0),
-    ("mtp_verify", [2], 0),
-    ("longest", [0, 7], 0),
-])
-def test_workload_full_size_sampled_heads(name, heads, layer):
-    _full_size(name, K8, heads=heads, layer=layer)
+# K8/V4 at full size: every layer's codes and every kv-head's attention of three
+# layers per workload are in test_gpu_full_size.py.
 
 
 def test_workload_longest_bf16_cache_sampled_head():
