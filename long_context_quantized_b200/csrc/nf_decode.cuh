@@ -625,6 +625,11 @@ __device__ __forceinline__ void merge_slots(const DecodeParams &p, const float *
             if (tid == 0) {
                 // the ring's last reads (generic proxy) precede the copies' writes
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                // the slots were written with generic stores (by other CTAs, made
+                // visible to this thread by the ticket's release and the acquire
+                // fence, or by this CTA before the barrier that precedes this
+                // round); order them before the bulk copies' async-proxy reads
+                asm volatile("fence.proxy.async.global;" ::: "memory");
                 mbar_arrive_expect_tx(fin_bar, (uint32_t)nr * slot_bytes);
                 if (stride == (size_t)p.slot_floats)
                     bulk_g2s(smem, rsrc, (uint32_t)nr * slot_bytes, fin_bar);
