@@ -67,6 +67,8 @@ typedef int32_t nf_status;
 #define NF_DEVERR_TIMEOUT 4   /* a bounded wait inside a kernel gave up (the kernel returned) */
 #define NF_DEVERR_INTERNAL 5  /* a launch-time invariant of the kernel failed (e.g. shared-memory
                                  alignment); the call did no work */
+#define NF_DEVERR_RANGE 6     /* nf_prefill_attn: a K or V scale whose dequantised codes leave the
+                                 fp16 range the kernel computes in (the results are not finite) */
 
 /* Element types. */
 #define NF_F32 0
@@ -248,7 +250,9 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
  * library routine).
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make that
- *    first call before any stream capture on the device.
+ *    first call before any stream capture on the device.  The cached address
+ *    belongs to the device's primary context: do not reset the device
+ *    (cudaDeviceReset) in a process that keeps calling this entry point.
  *  - Shapes whose nf_decode_attn_workspace_size() exceeds
  *    NF_NOALLOC_SCRATCH_BYTES are refused with NF_ERR_WORKSPACE.
  *  - All calls on a device share the one array and it keeps the last call's
@@ -293,15 +297,19 @@ nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_
  *   kv->fmt must be NF_KV_K8V4 and q_dtype NF_BF16 (else NF_ERR_UNSUPPORTED);
  *   any n_q >= 1 and any GQA group; no workspace (nothing is split across
  *   CTAs); batch <= 65535, num_kv_heads <= 65535.
- *   The dequantised V values (code x scale) must lie inside the fp16 range,
- *   that is every V group's scale <= 65504 / 7: the kernel holds them as fp16.
+ *   The dequantised K and V values (code x scale) must lie inside the fp16
+ *   range the kernel holds them in: K scales <= 515.5 (127 x 515.5 < 65504)
+ *   and V scales <= 9352 (7 x 9352 < 65504), that is K and V inputs of
+ *   magnitude below about 65500.  A larger scale of a key the call reads is
+ *   recorded as NF_DEVERR_RANGE (and the affected outputs are not finite);
+ *   nf_decode_attn has no such limit.
  * Numerics: each query row is scaled to max |q| = 1 and rounded to fp16 once;
  *   K and V are dequantised to fp16 (code x scale, one rounding each); the
  *   softmax weights are rounded to fp16; products accumulate in fp32 on the
  *   5th-generation tensor cores (tcgen05.mma kind::f16, M = 128).
- *   The dequantised K values must lie inside the fp16 range as well.
  * Device errors: NF_DEVERR_SEQLEN (the sequence's rows come out o = 0,
- *   lse = -inf), NF_DEVERR_BLOCK_ID (that tile's keys read as zeros).
+ *   lse = -inf), NF_DEVERR_BLOCK_ID (that tile's keys read as zeros),
+ *   NF_DEVERR_RANGE (see above).
  * Launch: programmatic dependent launch, as nf_decode_attn; the kernel waits
  *   for the previous kernel on `stream` before reading any argument.
  */

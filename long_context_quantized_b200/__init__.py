@@ -30,7 +30,7 @@ _LIB_PATH = os.path.join(_PKG, "libnf.so")
 NF_OK = 0
 NF_ERR_INVALID_ARG, NF_ERR_UNSUPPORTED, NF_ERR_WORKSPACE, NF_ERR_CUDA, NF_ERR_DEVICE_CHECK = 1, 2, 3, 4, 5
 NF_DEVERR_NONE, NF_DEVERR_BLOCK_ID, NF_DEVERR_TABLE, NF_DEVERR_SEQLEN = 0, 1, 2, 3
-NF_DEVERR_TIMEOUT, NF_DEVERR_INTERNAL = 4, 5
+NF_DEVERR_TIMEOUT, NF_DEVERR_INTERNAL, NF_DEVERR_RANGE = 4, 5, 6
 NF_F32, NF_BF16, NF_F16 = 0, 1, 2
 NF_KV_K8V4, NF_KV_BF16, NF_KV_K8V8, NF_KV_F8 = 0, 1, 2, 3
 BLOCK = 256

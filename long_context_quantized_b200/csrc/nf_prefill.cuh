@@ -160,8 +160,14 @@ __device__ __forceinline__ void tc_load_v(const PrefillParams &p, const int32_t 
     for (int u = 0; u < 4; ++u) r.v[u] = ldg16(vp + 16 * u);
     r.vs = __ldg(reinterpret_cast<const uint2 *>(p.v_scales + si * (kHeadDim / kVGroup)));
 }
+// Largest K and V scales (fp16 bits) whose dequantised codes stay finite in
+// fp16: 127 x 515.5 and 7 x 9352 round to finite values, 127 x 516 and 7 x
+// 9360 to infinity.  A larger scale is reported as NF_DEVERR_RANGE.
+constexpr uint32_t kTcMaxKScaleBits = 0x6007u;  // 515.5
+constexpr uint32_t kTcMaxVScaleBits = 0x7091u;  // 9352
 // key's dequantised fp16 K row (code x K scale)
 __device__ __forceinline__ void tc_convert_k(const TcRawK &r, int key, unsigned char *kb) {
+    if (r.ok && (r.ks & 0x7FFFu) > kTcMaxKScaleBits) report(NF_DEVERR_RANGE);
     const __half2 sk = u32_h2(r.ok ? (r.ks & 0xFFFFu) * 0x10001u : 0u);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -181,6 +187,10 @@ __device__ __forceinline__ void tc_convert_k(const TcRawK &r, int key, unsigned 
 // key's dequantised fp16 V row (code x V scale; 0 past the end)
 __device__ __forceinline__ void tc_convert_v(const TcRawV &r, int key, unsigned char *vb) {
     const uint32_t keep = r.ok ? 0xFFFFFFFFu : 0u;
+    if (r.ok) {
+        const uint32_t sb[4] = {r.vs.x & 0x7FFFu, (r.vs.x >> 16) & 0x7FFFu, r.vs.y & 0x7FFFu, (r.vs.y >> 16) & 0x7FFFu};
+        if (max(max(sb[0], sb[1]), max(sb[2], sb[3])) > kTcMaxVScaleBits) report(NF_DEVERR_RANGE);
+    }
     const uint32_t vsg[4] = {prmt(r.vs.x, 0, 0x1010) & keep, prmt(r.vs.x, 0, 0x3232) & keep,
                              prmt(r.vs.y, 0, 0x1010) & keep, prmt(r.vs.y, 0, 0x3232) & keep};
 #pragma unroll

@@ -12,7 +12,7 @@ import torch
 import long_context_quantized_b200 as nf
 import oracle
 import workloads
-from nfcase import check_attention, compare_pool, gpu_layer, oracle_attention, oracle_pool, run_case
+from nfcase import POISON, check_attention, compare_pool, gpu_layer, oracle_attention, oracle_pool, run_case
 
 pytestmark = pytest.mark.gpu
 K8 = nf.NF_KV_K8V4
@@ -103,3 +103,53 @@ def test_prefill_rejects_other_formats_and_fp32_queries():
     with pytest.raises(nf.NfError) as e:
         nf.nf_prefill_attn(kv8, g["q"], bt, sl, 108, w.softmax_scale, True, g["out"], None)
     assert e.value.status == nf.NF_ERR_UNSUPPORTED
+
+
+def _pool_with_scaled_inputs(w, k_mul, v_mul):
+    dev = "cuda"
+    bt_np = workloads.block_table(w)
+    bt = torch.as_tensor(bt_np, device=dev)
+    kv = nf.KVLayer.empty(K8, w.pool_blocks, w.num_kv_heads, device=dev, fill=POISON)
+    k, v = workloads.layer_kv(w, 0, 0, device=dev)
+    k, v = (k.float() * k_mul).contiguous(), (v.float() * v_mul).contiguous()
+    nf.nf_kv_append_quant(kv, k[None], v[None], bt, torch.zeros(1, dtype=torch.int32, device=dev))
+    return kv, bt, bt_np, [(k, v)]
+
+
+def test_prefill_reports_v_outside_fp16_range_where_decode_is_exact():
+    # V inputs of magnitude ~8e4: V scales above 9352, so 7 x scale leaves fp16.
+    # nf_prefill_attn records NF_DEVERR_RANGE; nf_decode_attn (weights x scale
+    # <= 65504) still matches the oracle.
+    mul = 2e4
+    w = workloads.custom("pf_range_v", cached=(0,), n_new=600, n_q=4, num_q_heads=8, num_kv_heads=1,
+                         q_dtype=torch.bfloat16, kv_in_dtype=torch.float32, causal=True)
+    kv, bt, bt_np, kvin = _pool_with_scaled_inputs(w, 1.0, mul)
+    q = workloads.layer_q(w, 0, device="cuda")
+    sl = torch.as_tensor(w.seqlens, dtype=torch.int32, device="cuda")
+    out = torch.empty((1, w.n_q, w.num_q_heads, 128), device="cuda")
+    lse = torch.empty((1, w.n_q, w.num_q_heads), device="cuda")
+    nf.nf_prefill_attn(kv, q, bt, sl, 600, w.softmax_scale, True, out, lse)
+    torch.cuda.synchronize()
+    assert nf.nf_get_device_error() == nf.NF_DEVERR_RANGE
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(1, w.n_q, w.num_q_heads, 1, 600), dtype=torch.uint8,
+                     device="cuda")
+    nf.nf_decode_attn(kv, q, bt, sl, 600, w.softmax_scale, True, out, lse, ws)
+    torch.cuda.synchronize()
+    assert nf.nf_get_device_error() == 0
+    pool, hs = oracle_pool(w, K8, kvin, bt_np)
+    compare_pool(kv, pool, hs)
+    ref_o, ref_l = oracle_attention(w, pool, hs, q, bt_np)
+    # the tolerance is stated for unit-scale values: compare o / mul
+    check_attention(out / mul, lse, ref_o / mul, ref_l)
+
+
+def test_prefill_reports_k_outside_fp16_range():
+    w = workloads.custom("pf_range_k", cached=(0,), n_new=300, n_q=8, num_q_heads=4, num_kv_heads=1,
+                         q_dtype=torch.bfloat16, kv_in_dtype=torch.float32, causal=True)
+    kv, bt, _, _ = _pool_with_scaled_inputs(w, 3e4, 1.0)
+    q = workloads.layer_q(w, 0, device="cuda")
+    out = torch.empty((1, w.n_q, w.num_q_heads, 128), device="cuda")
+    nf.nf_prefill_attn(kv, q, bt, torch.as_tensor(w.seqlens, dtype=torch.int32, device="cuda"), 300,
+                       w.softmax_scale, True, out, None)
+    torch.cuda.synchronize()
+    assert nf.nf_get_device_error() == nf.NF_DEVERR_RANGE
