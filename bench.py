@@ -42,7 +42,10 @@ import workloads  # noqa: E402
 
 METRIC = "KV tokens/s and achieved HBM GB/s (% of B200 peak) for K8/V4 decode attn"
 UNIT = "KV tokens/s"
-DEFAULT_WORKLOAD = "ctx32k_append"
+DEFAULT_WORKLOAD = "longest"
+# The other workloads of >= 64K keys: at N = 1 their decode roofline and step
+# time are measured after the headline and reported beside it (key "others").
+OTHER_WORKLOADS = ["ragged_c2", "mtp_verify"]
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ["long_context_quantized_b200/csrc/nf_decode.cuh",
                   "long_context_quantized_b200/csrc/nf_common.cuh",
@@ -476,7 +479,8 @@ def prefill_main(args, w, ws, rank, local):
     line = {
         "metric": PREFILL_METRIC, "value": value, "unit": PREFILL_UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "s8/s4 KV codes, f16 tensor-core products (mma.sync), f32 softmax/accumulate",
+        "vs_baseline": None,
+        "dtype": "s8/s4 KV codes dequantised to f16, tcgen05 f16 tensor-core products, f32 softmax/accumulate",
         "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seqlens": list(w.seqlens), "n_q": w.n_q,
                    "n_new": w.n_new, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
@@ -547,6 +551,8 @@ def main():
     ap.add_argument("--kv-format", default="k8v4", choices=["k8v4", "k8v8", "f8", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the other >= 64K workloads measured after the headline at N = 1")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling only: run fewer layers than the workload has")
     args = ap.parse_args()
@@ -640,13 +646,22 @@ def main():
         cv, threads, desc, _ = oracle_sample(w, args.kv_format, budget_s=12.0, device=device)
         cpu = {"value": cv, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
 
+    launches = gw.launches_per_step() * args.steps
+    kv_step_bytes = gw.kv_bytes_per_layer() * w.layers
+    step_bytes = gw.step_bytes()
+    others = None
+    if ws == 1 and w.name == DEFAULT_WORKLOAD and not args.no_others and not args.layers:
+        del gw
+        torch.cuda.empty_cache()
+        others = {name: measure_other(workloads.get(name), args, device) for name in OTHER_WORKLOADS}
+
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
-    l2_note = ("KV bytes per step %.1f MB > 126 MB L2: no flush needed" % (gw.kv_bytes_per_layer() * w.layers / 1e6)
-               if gw.kv_bytes_per_layer() * w.layers > 126e6 else "L2-resident (correctness-size workload)")
+    l2_note = ("KV bytes per step %.1f MB > 126 MB L2: no flush needed" % (kv_step_bytes / 1e6)
+               if kv_step_bytes > 126e6 else "L2-resident (correctness-size workload)")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -657,7 +672,7 @@ def main():
                    "layers": w.layers, "kv_format": args.kv_format, "causal": w.causal,
                    "l2": l2_note, "timing": "CUDA graph of one step, CUDA events, max over ranks",
                    "decode_flags": "NF_DECODE_EARLY_KV"},
-        "step_gbs": gw.step_bytes() / (ms / 1e3) / 1e9,
+        "step_gbs": step_bytes / (ms / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "decode_kernel (nf_decode_attn: split-K with fused combine)", "peak_source": peak_kind,
@@ -667,10 +682,59 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(tokens, ws, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": gw.launches_per_step() * args.steps,
+        "gpu_launches": launches,
         "clocks": clk,
     }
+    if others is not None:
+        line["others"] = others
     print(json.dumps(line), flush=True)
+
+
+def measure_other(w, args, device):
+    """The decode step of another workload, measured like the headline (step
+    graph timed with CUDA events, decode launches back to back for the
+    roofline), for the line's "others" key.  Returns a dict."""
+    steps = max(5, min(args.steps, 30))
+    gw = GpuWorkload(w, args.kv_format, device)
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        gw.step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        gw.step()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(device.index or 0)
+    clocks.start()
+    time.sleep(0.3)
+    ms = time_graph(g, steps, 0, stream)
+    dec_ms = time_decode_stream(gw, steps, stream)
+    clk = clocks.stop()
+    err = gw.nf.nf_get_device_error()
+    assert err == 0, f"device error {err}"
+    peak, peak_kind = measured_peaks()
+    dec_bytes = gw.decode_bytes_per_launch()
+    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    res = {
+        "metric": METRIC, "value": w.kv_tokens_per_step() / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+        "steps": steps, "step_gbs": gw.step_bytes() / (ms / 1e3) / 1e9,
+        "config": {"workload": w.name, "batch": w.batch, "seqlens": list(w.seqlens), "n_q": w.n_q,
+                   "n_new": w.n_new, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "layers": w.layers,
+                   "kv_format": args.kv_format, "causal": w.causal},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": recorded_traffic(w.name, args.kv_format), "peak_source": peak_kind,
+                     "bytes_per_launch": dec_bytes, "launch_us": dec_ms * 1e3},
+        # the timed step graph and the timed graph of back-to-back decode launches
+        "gpu_launches": gw.launches_per_step() * steps + w.layers * steps,
+        "clocks": clk,
+    }
+    del g, gw
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
 
 
 if __name__ == "__main__":
