@@ -32,6 +32,7 @@ FMT_K8V4 = 0
 FMT_BF16 = 1
 FMT_K8V8 = 2
 FMT_F8 = 3
+FMT_K4V4 = 4   # the "RK4V4-E8" reading: 4-bit K and V, power-of-two scale per 32 channels
 BLOCK = 256
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
@@ -77,6 +78,10 @@ def _load():
             lib.nfref_quant_f8.restype = None
             lib.nfref_quant_v.argtypes = [P, I, I, P, P]
             lib.nfref_quant_v.restype = None
+            lib.nfref_quant_e8.argtypes = [P, I, P, P]
+            lib.nfref_quant_e8.restype = None
+            lib.nfref_e8_exponent.argtypes = [ctypes.c_float]
+            lib.nfref_e8_exponent.restype = I
             lib.nfref_append.argtypes = [I, I, I, I, P, P, P, P, P, P, I, I, P, I, P]
             lib.nfref_append.restype = I
             lib.nfref_attn_row.argtypes = [I, I, I, P, P, P, P, P, I, I, P, I, ctypes.c_double, P, P]
@@ -156,6 +161,23 @@ def quant_v(x, group: int = 32):
     return scales, packed
 
 
+def quant_e8(x):
+    """One key or value vector of the RK4V4-E8 cache (fp32, d values) ->
+    (exponent bytes uint8[d/32], packed nibbles uint8[d/2])."""
+    lib = _load()
+    x = _c(x, np.float32)
+    d = x.shape[-1]
+    scales = np.zeros(d // 32, np.uint8)
+    packed = np.zeros(d // 2, np.uint8)
+    lib.nfref_quant_e8(_ptr(x), d, _ptr(scales), _ptr(packed))
+    return scales, packed
+
+
+def e8_exponent(s) -> int:
+    """The scale exponent of a group whose fp32 absmax / 7 is s."""
+    return int(_load().nfref_e8_exponent(float(np.float32(s))))
+
+
 def quant_f8(x):
     """One key or value vector of the fp8 cache (fp32, d values) -> (fp16 scale
     bits, e4m3 codes uint8[d])."""
@@ -179,6 +201,11 @@ class Pool:
             self.k_scale = np.zeros((num_blocks, num_kv_heads, BLOCK), np.uint16)
             self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 2), np.uint8)
             self.v_scale = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 32), np.uint16)
+        elif fmt == FMT_K4V4:
+            self.k = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 2), np.uint8)
+            self.k_scale = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 32), np.uint8)
+            self.v = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 2), np.uint8)
+            self.v_scale = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim // 32), np.uint8)
         elif fmt in (FMT_K8V8, FMT_F8):
             code = np.int8 if fmt == FMT_K8V8 else np.uint8
             self.k = np.zeros((num_blocks, num_kv_heads, BLOCK, head_dim), code)

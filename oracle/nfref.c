@@ -25,6 +25,16 @@
  *    OCP E4M3FN codes of x / scale with scale = absmax / 448 per (token,
  *    kv-head), rounded half to even and saturated at +-448 (formats 2 and 3
  *    of the pool below).
+ *  - Page "影片筆記：NInfer + 千问3.8 27b = 1.5倍速@256K上下文(单张4090 24GB)",
+ *    section 三, names "RK4V4-E8" as the KV quantisation that fits a 256K
+ *    context into 24 GB (its own transcription-doubts section questions the
+ *    name; no page gives its bits).  Read here as format 4: K and V both
+ *    symmetric 4-bit codes in [-7, 7] (nibbles packed as the K8/V4 values
+ *    are), every group of 32 channels of a (token, kv-head) with one shared
+ *    power-of-two scale 2^e stored as an 8-bit exponent byte e + 127 ("E8");
+ *    e is the smallest integer with 2^e >= fp32(absmax / 7), clamped to
+ *    [-126, 127]; code = clamp(round_half_even(fp32(x / 2^e)), -7, 7).  The
+ *    "R" is left unread, as for rk8v4: no rotation.
  *  - The cache is segmented (page "標籤: vLLM", section 2 "C++/CUDA 層的 kernel
  *    fusion 與 KV cache 策略": KV managed as segments rather than one buffer);
  *    here a segment is a 256-token block found through a per-sequence block
@@ -272,6 +282,59 @@ void nfref_quant_v(const float *x, int d, int group, uint16_t *scales, uint8_t *
 }
 
 /* ------------------------------------------------------------------ */
+/* Format 4 ("RK4V4-E8"): 4-bit codes, power-of-two scale per 32 ch.  */
+/* ------------------------------------------------------------------ */
+
+/* The exponent e of the group scale 2^e: the smallest integer with
+ * 2^e >= s, clamped to [-126, 127].  frexp writes s = m * 2^E with
+ * 0.5 <= m < 1, so 2^(E - 1) <= s < 2^E, and s is itself a power of two
+ * exactly when m == 0.5. */
+int nfref_e8_exponent(float s)
+{
+    if (!(s > 0.0f))
+        return -126;
+    int E;
+    double m = frexp((double)s, &E);
+    int e = (m == 0.5) ? E - 1 : E;
+    if (e < -126)
+        e = -126;
+    if (e > 127)
+        e = 127;
+    return e;
+}
+
+/* d values -> d/32 scale bytes (e + 127) and d/2 bytes of packed nibbles
+ * (channel 2j in bits 0..3 of byte j, channel 2j+1 in bits 4..7). */
+void nfref_quant_e8(const float *x, int d, uint8_t *scales, uint8_t *packed)
+{
+    int *codes = (int *)malloc(sizeof(int) * (size_t)d);
+    for (int g = 0; g < d / 32; ++g) {
+        const float *xg = x + g * 32;
+        float a = 0.0f;
+        for (int c = 0; c < 32; ++c) {
+            float v = fabsf(xg[c]);
+            if (v > a)
+                a = v;
+        }
+        float s = a / 7.0f;                      /* fp32 division, round-to-nearest */
+        int e = nfref_e8_exponent(s);
+        float scale = ldexpf(1.0f, e);           /* 2^e, a normal fp32 number */
+        for (int c = 0; c < 32; ++c) {
+            float r = nearbyintf(xg[c] / scale); /* exact division, round half to even */
+            if (r > 7.0f)
+                r = 7.0f;
+            if (r < -7.0f)
+                r = -7.0f;
+            codes[g * 32 + c] = (int)r;
+        }
+        scales[g] = (uint8_t)(e + 127);
+    }
+    for (int j = 0; j < d / 2; ++j)
+        packed[j] = (uint8_t)((codes[2 * j] & 0xF) | ((codes[2 * j + 1] & 0xF) << 4));
+    free(codes);
+}
+
+/* ------------------------------------------------------------------ */
 /* Pool layout.                                                        */
 /* ------------------------------------------------------------------ */
 /*
@@ -286,6 +349,9 @@ void nfref_quant_v(const float *x, int d, int group, uint16_t *scales, uint8_t *
  *   per token and kv-head).
  * fmt 3 (fp8 KV): k_plane, v_plane e4m3 bytes [num_blocks][H][256][d]; k_scale,
  *   v_scale fp16 [num_blocks][H][256] (absmax/448 per token and kv-head).
+ * fmt 4 ("RK4V4-E8"): k_plane, v_plane uint8 nibbles [num_blocks][H][256][d/2];
+ *   k_scale, v_scale uint8 exponent bytes [num_blocks][H][256][d/32] (the
+ *   scale arguments point at bytes for this format).
  * Token position p of sequence b lives in block block_table[b][p / 256],
  * slot p % 256.
  */
@@ -296,8 +362,25 @@ static size_t slot_index(int32_t blk, int H, int h, int slot)
 }
 
 /* Dequantised key / value channel c of the token at pool slot `si`. */
+/* Channel c of the packed nibbles of the token at slot si, as an integer. */
+static int nibble_code(const void *plane, size_t si, int d, int c)
+{
+    uint8_t byte = ((const uint8_t *)plane)[si * (size_t)(d / 2) + (size_t)(c / 2)];
+    int nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
+    return nib >= 8 ? nib - 16 : nib;
+}
+
+/* Format 4: code * 2^(byte - 127) for channel c. */
+static double e8_hat(const void *plane, const uint16_t *scale, size_t si, int d, int c)
+{
+    uint8_t byte = ((const uint8_t *)scale)[si * (size_t)(d / 32) + (size_t)(c / 32)];
+    return ldexp((double)nibble_code(plane, si, d, c), (int)byte - 127);
+}
+
 static double k_hat(int fmt, const void *k_plane, const uint16_t *k_scale, size_t si, int d, int c)
 {
+    if (fmt == 4)
+        return e8_hat(k_plane, k_scale, si, d, c);
     if (fmt == 1)
         return (double)nfref_bf16_to_f32(((const uint16_t *)k_plane)[si * d + c]);
     if (fmt == 3)
@@ -308,6 +391,8 @@ static double k_hat(int fmt, const void *k_plane, const uint16_t *k_scale, size_
 
 static double v_hat(int fmt, const void *v_plane, const uint16_t *v_scale, size_t si, int d, int c)
 {
+    if (fmt == 4)
+        return e8_hat(v_plane, v_scale, si, d, c);
     if (fmt == 1)
         return (double)nfref_bf16_to_f32(((const uint16_t *)v_plane)[si * d + c]);
     if (fmt == 2)
@@ -369,6 +454,11 @@ int nfref_append(int fmt, int num_blocks, int H, int d,
                 } else if (fmt == 3) {
                     nfref_quant_f8(kx, d, &k_scale[si], (uint8_t *)k_plane + si * d);
                     nfref_quant_f8(vx, d, &v_scale[si], (uint8_t *)v_plane + si * d);
+                } else if (fmt == 4) {
+                    nfref_quant_e8(kx, d, (uint8_t *)k_scale + si * (size_t)(d / 32),
+                                   (uint8_t *)k_plane + si * (size_t)(d / 2));
+                    nfref_quant_e8(vx, d, (uint8_t *)v_scale + si * (size_t)(d / 32),
+                                   (uint8_t *)v_plane + si * (size_t)(d / 2));
                 } else {
                     nfref_quant_k(kx, d, &k_scale[si], (int8_t *)k_plane + si * d);
                     nfref_quant_v(vx, d, 32, &v_scale[si * (size_t)(d / 32)],

@@ -98,6 +98,12 @@ def np_dequant_pool(pool):
         k = (pool.k.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
         v = (pool.v.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
         return k, v
+    if pool.fmt == oracle.FMT_K4V4:
+        k = np_unpack_v(pool.k).astype(np.float64) * np.repeat(np.ldexp(1.0, pool.k_scale.astype(np.int64) - 127), 32,
+                                                                axis=-1)
+        v = np_unpack_v(pool.v).astype(np.float64) * np.repeat(np.ldexp(1.0, pool.v_scale.astype(np.int64) - 127), 32,
+                                                                axis=-1)
+        return k, v
     ks = pool.k_scale.view(np.float16).astype(np.float64)
     vs = pool.v_scale.view(np.float16).astype(np.float64)
     k = pool.k.astype(np.float64) * ks[..., None]
@@ -448,7 +454,7 @@ def test_append_rejects_out_of_range():
 SCALE = float(np.float32(1 / math.sqrt(128)))
 
 
-@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8, oracle.FMT_F8])
+@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8, oracle.FMT_F8, oracle.FMT_K4V4])
 def test_attention_zero_query_is_mean_of_visible_values(fmt):
     # q = 0 -> all scores 0 -> o = mean of visible v_hat, lse = log(#visible).
     # Causal with n_q = 4: query j sees L - 4 + j + 1 keys.
@@ -547,7 +553,7 @@ def test_attention_split_and_combine_equals_whole():
     assert lse[0] == pytest.approx(lse_w, abs=1e-12)
 
 
-@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8, oracle.FMT_F8])
+@pytest.mark.parametrize("fmt", [oracle.FMT_K8V4, oracle.FMT_BF16, oracle.FMT_K8V8, oracle.FMT_F8, oracle.FMT_K4V4])
 @pytest.mark.parametrize("causal", [False, True])
 def test_attention_matches_numpy_brute_force(fmt, causal):
     cached = [300, 513]
@@ -629,3 +635,112 @@ def test_combine_weights_two_splits():
     wa = 1 / (1 + math.exp(b - a))
     assert np.allclose(out[0], wa * o[0, 0] + (1 - wa) * o[1, 0], rtol=1e-13)
     assert lse[0] == pytest.approx(math.log(math.exp(a) + math.exp(b)), abs=1e-14)
+
+
+# ------------------------------------------------ RK4V4-E8 (format 4)
+GOLDEN_E8 = os.path.join(os.path.dirname(__file__), "golden", "k4v4_e8_cases.txt")
+
+
+def _e8_cases():
+    cases = []
+    with open(GOLDEN_E8) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, tail = line.split("|")
+            parts = head.split()
+            cases.append((parts[0], parts[1:], tail.split()))
+    return cases
+
+
+@pytest.mark.parametrize("case", _e8_cases(), ids=lambda c: c[0] + ":" + " ".join(c[1][:2]))
+def test_quant_e8_golden(case):
+    kind, head, tail = case
+    x = np.zeros(128, np.float32)
+    if kind == "PACK":
+        xs = np.array([_parse_val(t) for t in head], np.float32)
+        x[:len(xs)] = xs
+        _, packed = oracle.quant_e8(x)
+        want = np.array([int(t, 16) for t in tail], np.uint8)
+        assert np.array_equal(packed[:len(want)], want)
+        return
+    xs = np.array([_parse_val(t) for t in head[1:]], np.float32)
+    x[:len(xs)] = xs
+    scales, packed = oracle.quant_e8(x)
+    assert int(scales[0]) == int(head[0])
+    codes = np_unpack_v(packed)
+    want = np.array([int(t) for t in tail], np.int64)
+    assert np.array_equal(codes[:len(want)], want)
+    assert np.all(codes[len(want):32] == 0)
+
+
+def np_quant_e8(x):
+    """Independent statement of the format: the exponent by searching all
+    powers of two 2^-126 .. 2^127 for the smallest one >= fp32(absmax / 7),
+    the codes by numpy fp32 division and rint.  Returns (bytes[4], codes[128])."""
+    x = np.asarray(x, np.float32)
+    pows = 2.0 ** np.arange(-126, 128)
+    bytes_, codes = [], []
+    for g in range(4):
+        xg = x[32 * g:32 * g + 32]
+        s = np.float32(np.max(np.abs(xg))) / np.float32(7.0)
+        e = int(np.arange(-126, 128)[np.argmax(pows >= float(s))]) if s > 0 else -126
+        scale = np.float32(2.0 ** e)
+        c = np.clip(np.rint(xg / scale), -7, 7).astype(np.int64)
+        bytes_.append(e + 127)
+        codes.append(c)
+    return np.array(bytes_), np.concatenate(codes)
+
+
+def _e8_vectors(n):
+    out = list(_random_vectors(n))
+    for i in range(n // 4):  # groups of very different magnitudes in one vector
+        x = RNG.standard_normal(128)
+        for g in range(4):
+            x[32 * g:32 * g + 32] *= 10.0 ** RNG.uniform(-30, 30)
+        out.append(x.astype(np.float32))
+    return out
+
+
+def test_quant_e8_matches_numpy_statement():
+    for x in _e8_vectors(2400):
+        scales, packed = oracle.quant_e8(x)
+        wb, wc = np_quant_e8(x)
+        assert np.array_equal(scales.astype(np.int64), wb)
+        assert np.array_equal(np_unpack_v(packed), wc)
+
+
+def test_quant_e8_roundtrip_and_scale_bounds():
+    for x in _e8_vectors(1200):
+        scales, packed = oracle.quant_e8(x)
+        codes = np_unpack_v(packed)
+        for g in range(4):
+            e = int(scales[g]) - 127
+            xg = x[32 * g:32 * g + 32].astype(np.float64)
+            s = float(np.float32(np.max(np.abs(x[32 * g:32 * g + 32]))) / np.float32(7.0))
+            assert 2.0 ** e >= s                          # no code is clamped ...
+            assert e == -126 or 2.0 ** (e - 1) < s        # ... and the scale is the smallest such
+            err = np.abs(xg - codes[32 * g:32 * g + 32] * 2.0 ** e)
+            assert np.all(err <= 2.0 ** (e - 1))           # half a step
+            assert codes.min() >= -7 and codes.max() <= 7
+
+
+def test_append_k4v4_places_both_planes_through_block_table():
+    H, d = 2, 128
+    rng = np.random.default_rng(41)
+    pool = oracle.Pool(oracle.FMT_K4V4, 3, H, d, poison=0x5A)
+    bt = np.array([[2, 0]], np.int32)
+    k = rng.standard_normal((1, 300, H, d)).astype(np.float32)
+    v = (rng.standard_normal((1, 300, H, d)) * 3).astype(np.float32)
+    assert oracle.append(pool, k, v, bt, np.array([0], np.int32)) == 0
+    for t in (0, 255, 256, 299):
+        blk, slot = bt[0, t // 256], t % 256
+        for h in range(H):
+            ks, kp = oracle.quant_e8(k[0, t, h])
+            vs, vp = oracle.quant_e8(v[0, t, h])
+            assert np.array_equal(pool.k[blk, h, slot], kp) and np.array_equal(pool.k_scale[blk, h, slot], ks)
+            assert np.array_equal(pool.v[blk, h, slot], vp) and np.array_equal(pool.v_scale[blk, h, slot], vs)
+    # slots past the end keep their poison
+    assert np.all(pool.k[0, :, 44:] == 0x5A) and np.all(pool.v_scale[0, :, 44:] == 0x5A)
+    assert np.all(pool.k[1] == 0x5A)
