@@ -7,7 +7,7 @@ appends) followed by split-K decode attention and the LSE combine, all through
 the C ABI.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                  [--kv-format k8v4|k8v8|f8|bf16] [--impl ours|reference]
+                  [--kv-format k8v4|k8v8|f8|k4v4|bf16] [--impl ours|reference]
 
 --workload prefill_chunk measures chunked-prefill attention instead: per layer
 the 1024-token chunk's append and nf_prefill_attn, reported as chunk tokens/s
@@ -48,6 +48,8 @@ DEFAULT_WORKLOAD = "longest"
 OTHER_WORKLOADS = ["ragged_c2", "mtp_verify"]
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ["long_context_quantized_b200/csrc/nf_decode.cuh",
+                  "long_context_quantized_b200/csrc/nf_decode_tc.cuh",
+                  "long_context_quantized_b200/csrc/nf_tc.cuh",
                   "long_context_quantized_b200/csrc/nf_common.cuh",
                   "long_context_quantized_b200/csrc/nf_api.cu"]
 
@@ -174,7 +176,8 @@ class GpuWorkload:
         self.w = w
         self.dev = device
         self.fmt_name = fmt_name
-        self.fmt = {"k8v4": nf.NF_KV_K8V4, "k8v8": nf.NF_KV_K8V8, "f8": nf.NF_KV_F8, "bf16": nf.NF_KV_BF16}[fmt_name]
+        self.fmt = {"k8v4": nf.NF_KV_K8V4, "k8v8": nf.NF_KV_K8V8, "f8": nf.NF_KV_F8, "k4v4": nf.NF_KV_K4V4,
+                    "bf16": nf.NF_KV_BF16}[fmt_name]
         self.decode_flags = nf.NF_DECODE_EARLY_KV
         assert w.n_new in (0, w.n_q), "the early-KV guarantee needs n_new == n_q"
         bt = workloads.block_table(w)
@@ -507,7 +510,8 @@ def oracle_sample(w, fmt_name, budget_s=12.0, device="cpu"):
     until about budget_s seconds.  Returns (KV tokens/s, threads, description).
     KV tokens counts each key once per kv-head processed, scaled by 1 / H_kv."""
     import oracle
-    fmt = {"k8v4": oracle.FMT_K8V4, "k8v8": oracle.FMT_K8V8, "f8": oracle.FMT_F8, "bf16": oracle.FMT_BF16}[fmt_name]
+    fmt = {"k8v4": oracle.FMT_K8V4, "k8v8": oracle.FMT_K8V8, "f8": oracle.FMT_F8, "k4v4": oracle.FMT_K4V4,
+           "bf16": oracle.FMT_BF16}[fmt_name]
     bt = workloads.block_table(w)
     pool = oracle.Pool(fmt, w.pool_blocks, 1, 128, poison=0)
     for b in range(w.batch):
@@ -538,6 +542,7 @@ DTYPES = {
     "k8v4": "s8/s4 KV codes, f16 tensor-core products, f32 softmax/accumulate",
     "k8v8": "s8/s8 KV codes, f16 tensor-core products, f32 softmax/accumulate",
     "f8": "e4m3 KV codes, f16 tensor-core products, f32 softmax/accumulate",
+    "k4v4": "s4/s4 KV codes with power-of-two scales, s8 and f16 tensor-core products, f32 softmax/accumulate",
     "bf16": "bf16 KV, bf16 tensor-core products, f32 softmax/accumulate",
 }
 
@@ -548,7 +553,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=workloads.ORDER + list(workloads.PREFILL))
-    ap.add_argument("--kv-format", default="k8v4", choices=["k8v4", "k8v8", "f8", "bf16"])
+    ap.add_argument("--kv-format", default="k8v4", choices=["k8v4", "k8v8", "f8", "k4v4", "bf16"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-others", action="store_true",

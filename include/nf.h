@@ -80,6 +80,7 @@ typedef int32_t nf_status;
 #define NF_KV_BF16 1 /* unquantised bf16 K and V (for byte-count comparison) */
 #define NF_KV_K8V8 2 /* the int8 KV dtype defined below (K and V both int8) */
 #define NF_KV_F8 3   /* the fp8 KV dtype defined below (K and V both e4m3) */
+#define NF_KV_K4V4 4 /* the RK4V4-E8 reading defined below (K and V both 4-bit) */
 
 /*
  * One layer's view of the caller-owned KV pool.
@@ -116,6 +117,20 @@ typedef int32_t nf_status;
  *   scale = fp16(fp32(max|x| / 448)) as above; code = e4m3(fp32(x / float(scale)))
  *   rounded half to even and saturated at +-448 (a zero result keeps the sign
  *   of x), or 0x00 when scale is 0.  Dequantised value = e4m3 value * scale.
+ * fmt NF_KV_K4V4 (the "RK4V4-E8" KV quantisation of page "影片筆記：NInfer +
+ *   千问3.8 27b = 1.5倍速@256K上下文(单张4090 24GB)", section 三, which gives no bit
+ *   format; this is the reading defined here; 136 bytes per token per kv-head):
+ *   k_codes  uint8 [num_blocks][num_kv_heads][256][64]  K codes in [-7, 7] as
+ *            nibbles, packed as the K8/V4 V codes
+ *   k_scales uint8 [num_blocks][num_kv_heads][256][4]   one scale byte per 32 channels
+ *   v_codes, v_scales: the same for V
+ *   Quantisation of one 32-channel group x (K or V):
+ *     e = the smallest integer with 2^e >= fp32(max|x| / 7), clamped to
+ *         [-126, 127]; stored as the byte e + 127 (an 8-bit exponent);
+ *     code = clamp(round_half_even(fp32(x / 2^e)), -7, 7).
+ *   Dequantised value = code * 2^e (exact).  The decoder reads scale bytes 1 ..
+ *   254 (the quantiser writes no other); within one sequence the V scales
+ *   should span fewer than 2^100 (their exponents are folded into fp32 sums).
  * fmt NF_KV_BF16 (512 bytes per token per kv-head):
  *   k_codes  bf16 [num_blocks][num_kv_heads][256][128]  (keys)
  *   v_codes  bf16 [num_blocks][num_kv_heads][256][128]  (values)
@@ -123,7 +138,7 @@ typedef int32_t nf_status;
  * Every plane must be 16-byte aligned.
  */
 typedef struct {
-    int32_t fmt;          /* NF_KV_K8V4, NF_KV_K8V8, NF_KV_F8 or NF_KV_BF16 */
+    int32_t fmt;          /* NF_KV_K8V4, NF_KV_K8V8, NF_KV_F8, NF_KV_K4V4 or NF_KV_BF16 */
     int32_t num_blocks;   /* pool capacity in blocks (>= 1) */
     int32_t block_size;   /* must be 256 */
     int32_t num_kv_heads; /* >= 1 */
@@ -282,6 +297,21 @@ nf_status nf_decode_attn_noalloc(const nf_kv_layer *kv, const void *q, int32_t q
 nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_splits,
                           int32_t rows, int32_t head_dim, float *out, float *out_lse,
                           nf_stream_t stream);
+
+/*
+ * nf_attn_combine_packed -- nf_attn_combine of splits stored packed, one slot
+ * per split: parts is fp32 [n_splits][slot], slot = nf_attn_packed_slot_floats(
+ * rows, head_dim) = rows * (head_dim + 1) rounded up to a multiple of 4, each
+ * slot holding o [rows][head_dim] followed by lse [rows] (the layout the decode
+ * kernel gives its own split partials).  A context-sharded decode writes each
+ * rank's partial into one such slot (out = the slot, out_lse = slot + rows *
+ * head_dim), exchanges the slots in one all-gather and merges them with this
+ * call.  parts and out 16-byte aligned; other arguments and results as for
+ * nf_attn_combine.
+ */
+size_t nf_attn_packed_slot_floats(int32_t rows, int32_t head_dim);
+nf_status nf_attn_combine_packed(const float *parts, int32_t n_splits, int32_t rows, int32_t head_dim,
+                                 float *out, float *out_lse, nf_stream_t stream);
 
 /*
  * nf_prefill_attn -- chunked-prefill attention over a K8/V4 pool (page "3090

@@ -14,7 +14,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libnf.so")
 SOURCES = ["nf_api.cu"]
-HEADERS = ["nf_common.cuh", "nf_append.cuh", "nf_decode.cuh", "nf_combine.cuh", "nf_prefill.cuh", "nf_tc.cuh"]
+HEADERS = ["nf_common.cuh", "nf_append.cuh", "nf_decode.cuh", "nf_decode_tc.cuh", "nf_combine.cuh", "nf_prefill.cuh",
+           "nf_tc.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17",

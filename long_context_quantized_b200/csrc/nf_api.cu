@@ -14,6 +14,7 @@
 #include "nf_combine.cuh"
 #include "nf_common.cuh"
 #include "nf_decode.cuh"
+#include "nf_decode_tc.cuh"
 #include "nf_prefill.cuh"
 
 namespace nf {
@@ -51,9 +52,10 @@ nf_status after_launch(const char *what) {
 
 nf_status check_layer(const nf_kv_layer *kv) {
     if (!kv) return fail(NF_ERR_INVALID_ARG, "kv is NULL");
-    if (kv->fmt != NF_KV_K8V4 && kv->fmt != NF_KV_K8V8 && kv->fmt != NF_KV_F8 && kv->fmt != NF_KV_BF16)
-        return fail(NF_ERR_UNSUPPORTED, "kv->fmt %d is not NF_KV_K8V4, NF_KV_K8V8, NF_KV_F8 or NF_KV_BF16",
-                    kv->fmt);
+    if (kv->fmt != NF_KV_K8V4 && kv->fmt != NF_KV_K8V8 && kv->fmt != NF_KV_F8 && kv->fmt != NF_KV_K4V4 &&
+        kv->fmt != NF_KV_BF16)
+        return fail(NF_ERR_UNSUPPORTED,
+                    "kv->fmt %d is not NF_KV_K8V4, NF_KV_K8V8, NF_KV_F8, NF_KV_K4V4 or NF_KV_BF16", kv->fmt);
     const bool scaled = kv->fmt != NF_KV_BF16;
     if (kv->block_size != nf::kBlock)
         return fail(NF_ERR_UNSUPPORTED, "kv->block_size %d (only 256)", kv->block_size);
@@ -112,11 +114,12 @@ bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sm
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 std::once_flag g_encode_once;
 
-// Tensor map of a quantised layer's V codes for the decode kernel: the plane as
-// [num_blocks * H_kv * 256 rows][row bytes], 32-row boxes, the swizzle as wide
-// as a row -- K8/V4 nibbles 64 bytes (64-byte swizzle), K8V8 and fp8 codes
-// 128 bytes (128-byte swizzle).
-nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map) {
+// Tensor map of a quantised layer's V codes (or, k_plane, of its int8 K codes)
+// for the decode kernels: the plane as [num_blocks * H_kv * 256 rows][row
+// bytes], 32-row boxes, the swizzle as wide as a row -- K8/V4 nibbles 64 bytes
+// (64-byte swizzle), K8V8 and fp8 V codes and int8 K codes 128 bytes (128-byte
+// swizzle).
+nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map, bool k_plane = false) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
@@ -128,13 +131,15 @@ nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map) {
     const cuuint64_t rows = (cuuint64_t)kv->num_blocks * (cuuint64_t)kv->num_kv_heads * nf::kBlock;
     if (rows > 0x7fffffffull)
         return fail(NF_ERR_UNSUPPORTED, "pool of %llu token rows per plane (at most 2^31 - 1)", (unsigned long long)rows);
-    const bool v8 = kv->fmt == NF_KV_K8V8 || kv->fmt == NF_KV_F8;
+    // 128-byte rows: int8 K codes, int8 / e4m3 V codes; 64-byte rows: nibbles
+    const bool v8 = k_plane ? kv->fmt != NF_KV_K4V4 : (kv->fmt == NF_KV_K8V8 || kv->fmt == NF_KV_F8);
     const cuuint64_t row_bytes = v8 ? 128 : 64;
     const cuuint64_t dims[2] = {row_bytes, rows};
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)nf::kChunk};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->v_codes, dims, strides, box, estr,
+    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_plane ? kv->k_codes : kv->v_codes,
+                                      dims, strides, box, estr,
                                       CU_TENSOR_MAP_INTERLEAVE_NONE,
                                       v8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -184,6 +189,26 @@ cudaError_t launch_decode(const nf::DecodeParams &p, int ctas, cudaStream_t s) {
     return launch_pdl(nf::decode_kernel<NT, QF32, FMT>, (unsigned)ctas, nf::kDecodeThreads, smem, s, p);
 }
 
+// The tensor-core decode of many rows (K8/V4, 9 to 32 query rows per kv-head),
+// rows padded to RP = 16 or 32.
+template <int RP, bool QF32>
+cudaError_t launch_decode_tc(const nf::DecodeParams &p, int ctas, cudaStream_t s) {
+    constexpr int smem = nf::DtSmem::kBytes;
+    static std::atomic<uint64_t> opted{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+    if (!bit || !(opted.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(nf::decode_tc_kernel<RP, QF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        opted.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    return launch_pdl(nf::decode_tc_kernel<RP, QF32>, (unsigned)ctas, nf::kDtThreads, smem, s, p);
+}
+
+bool uses_decode_tc(int fmt, int rows) { return fmt == NF_KV_K8V4 && rows > 8 && rows <= nf::kDtMaxRows; }
+
 template <int NT>
 cudaError_t dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, int ctas, cudaStream_t s) {
     if (fmt == NF_KV_K8V4)
@@ -192,12 +217,15 @@ cudaError_t dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, int c
         return qf32 ? launch_decode<NT, true, NF_KV_K8V8>(p, ctas, s) : launch_decode<NT, false, NF_KV_K8V8>(p, ctas, s);
     if (fmt == NF_KV_F8)
         return qf32 ? launch_decode<NT, true, NF_KV_F8>(p, ctas, s) : launch_decode<NT, false, NF_KV_F8>(p, ctas, s);
+    if (fmt == NF_KV_K4V4)
+        return qf32 ? launch_decode<NT, true, NF_KV_K4V4>(p, ctas, s) : launch_decode<NT, false, NF_KV_K4V4>(p, ctas, s);
     return qf32 ? launch_decode<NT, true, NF_KV_BF16>(p, ctas, s) : launch_decode<NT, false, NF_KV_BF16>(p, ctas, s);
 }
 
 nf_status launch_combine(const float *part_o, const float *part_lse, int n_splits, int rows,
-                         int head_dim, float *out, float *out_lse, cudaStream_t s) {
-    nf::CombineParams c{part_o, part_lse, n_splits, rows, head_dim, out, out_lse};
+                         int head_dim, size_t o_stride, size_t lse_stride, float *out, float *out_lse,
+                         cudaStream_t s) {
+    nf::CombineParams c{part_o, part_lse, n_splits, rows, head_dim, o_stride, lse_stride, out, out_lse};
     const cudaError_t e = launch_pdl(nf::combine_kernel, (unsigned)rows, nf::kCombineWarps * 32, 0, s, c);
     if (e != cudaSuccess) return fail(NF_ERR_CUDA, "combine kernel launch: %s", cudaGetErrorString(e));
     return after_launch("combine kernel launch");
@@ -337,8 +365,13 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
         return fail(NF_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
 
     nf::DecodeParams p{};
+    const bool tc = uses_decode_tc(kv->fmt, pl.rows);
     if (kv->fmt != NF_KV_BF16) {
         st = encode_v_map(kv, &p.vmap);
+        if (st != NF_OK) return st;
+    }
+    if (tc || kv->fmt == NF_KV_K4V4) {
+        st = encode_v_map(kv, &p.kmap, true);
         if (st != NF_OK) return st;
     }
     p.k_codes = kv->k_codes;
@@ -369,8 +402,12 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
     p.slot_floats = pl.slot_floats;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = pl.nt == 1 ? dispatch_decode<1>(p, q_dtype == NF_F32, kv->fmt, pl.ctas, s)
-                                     : dispatch_decode<2>(p, q_dtype == NF_F32, kv->fmt, pl.ctas, s);
+    const bool qf32 = q_dtype == NF_F32;
+    const cudaError_t e =
+        tc ? (pl.rows <= 16 ? (qf32 ? launch_decode_tc<16, true>(p, pl.ctas, s) : launch_decode_tc<16, false>(p, pl.ctas, s))
+                            : (qf32 ? launch_decode_tc<32, true>(p, pl.ctas, s) : launch_decode_tc<32, false>(p, pl.ctas, s)))
+        : pl.nt == 1 ? dispatch_decode<1>(p, qf32, kv->fmt, pl.ctas, s)
+                     : dispatch_decode<2>(p, qf32, kv->fmt, pl.ctas, s);
     if (e != cudaSuccess) {
         (void)cudaGetLastError();
         return fail(NF_ERR_CUDA, "decode kernel set-up: %s", cudaGetErrorString(e));
@@ -420,7 +457,29 @@ nf_status nf_attn_combine(const float *part_o, const float *part_lse, int32_t n_
     if (!part_o || !part_lse || !out) return fail(NF_ERR_INVALID_ARG, "a device pointer is NULL");
     if ((reinterpret_cast<uintptr_t>(part_o) | reinterpret_cast<uintptr_t>(out)) & 15)
         return fail(NF_ERR_INVALID_ARG, "part_o / out must be 16-byte aligned");
-    return launch_combine(part_o, part_lse, n_splits, rows, head_dim, out, out_lse,
+    return launch_combine(part_o, part_lse, n_splits, rows, head_dim, (size_t)rows * head_dim, (size_t)rows, out,
+                          out_lse, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t nf_attn_packed_slot_floats(int32_t rows, int32_t head_dim) {
+    if (rows < 1 || head_dim < 1) return 0;
+    return ((size_t)rows * (size_t)(head_dim + 1) + 3) / 4 * 4;
+}
+
+nf_status nf_attn_combine_packed(const float *parts, int32_t n_splits, int32_t rows, int32_t head_dim, float *out,
+                                 float *out_lse, nf_stream_t stream) {
+    if (n_splits < 1 || rows < 0) return fail(NF_ERR_INVALID_ARG, "n_splits %d / rows %d", n_splits, rows);
+    if (head_dim < 4 || head_dim > 1024 || head_dim % 4 != 0)
+        return fail(NF_ERR_UNSUPPORTED, "head_dim %d (multiple of 4 in [4, 1024])", head_dim);
+    if (rows == 0) {
+        g_msg[0] = '\0';
+        return NF_OK;
+    }
+    if (!parts || !out) return fail(NF_ERR_INVALID_ARG, "a device pointer is NULL");
+    if ((reinterpret_cast<uintptr_t>(parts) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return fail(NF_ERR_INVALID_ARG, "parts / out must be 16-byte aligned");
+    const size_t slot = nf_attn_packed_slot_floats(rows, head_dim);
+    return launch_combine(parts, parts + (size_t)rows * head_dim, n_splits, rows, head_dim, slot, slot, out, out_lse,
                           reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -135,6 +135,28 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, 
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return mbar_wait_limit(bar, parity, kWaitLimitNs);
 }
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// The same wait without the sleeping form: try_wait (which holds the thread for
+// a short, hardware-defined time) in a loop, for waits on short pipeline steps
+// where waking from a long sleep would cost more than the step.  Bounded by
+// kWaitLimitNs like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
 // 1-D bulk copy global -> shared on the TMA engine, completing on `bar`
 // (16-byte aligned addresses, size a multiple of 16).  No multicast.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -169,6 +191,13 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r
 }
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return __byte_perm(a, b, sel);
+}
+// prmt with the full 4-bit selectors: a selector nibble with its top bit set
+// fills its byte with the sign of the selected byte (0x00 for bytes < 0x80).
+__device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
 }
 // Programmatic dependent launch.  pdl_wait: block until the grids this one
 // depends on have completed and their memory operations are visible (at once

@@ -111,6 +111,20 @@ struct Stage<NF_KV_K8V8, NT> {
     static constexpr int kStages = 4;
     static constexpr int kUnitTiles = 1;  // 8 units of 16 keys per stage: one per consumer warp
 };
+// RK4V4-E8: 136 bytes per key; K and V nibble rows of 64 bytes (both through
+// tensor maps with the 64-byte swizzle), one exponent byte per 32 channels.
+template <int NT>
+struct Stage<NF_KV_K4V4, NT> {
+    static constexpr int kTok = 256;
+    static constexpr int kK = 0;                      // uint8 [kTok][64] (swizzled)
+    static constexpr int kV = kTok * 64;              // uint8 [kTok][64] (swizzled)
+    static constexpr int kKs = kV + kTok * 64;        // uint8 [kTok][4]
+    static constexpr int kVs = kKs + kTok * 4;        // uint8 [kTok][4]
+    static constexpr int kBytesPerTok = 136;
+    static constexpr int kStride = (kTok * kBytesPerTok + 1023) / 1024 * 1024;
+    static constexpr int kStages = 4;
+    static constexpr int kUnitTiles = NT == 1 ? 2 : 1;
+};
 // fp8 KV: the same bytes per key and layout as K8V8 (e4m3 codes for int8 ones).
 template <int NT>
 struct Stage<NF_KV_F8, NT> : Stage<NF_KV_K8V8, NT> {};
@@ -129,6 +143,8 @@ struct Stage<NF_KV_BF16, NT> {
 struct DecodeParams {
     CUtensorMap vmap;  // v_codes as [num_blocks * H_kv * 256 rows][64 (K8/V4) or 128 (K8V8) bytes],
                        // 32-row boxes, swizzle as wide as a row (unused for bf16)
+    CUtensorMap kmap;  // k_codes as [num_blocks * H_kv * 256 rows][128 bytes], 32-row boxes,
+                       // 128-byte swizzle (the tensor-core decode of many rows only)
     const void *k_codes;
     const __half *k_scales;
     const void *v_codes;
@@ -245,7 +261,7 @@ __device__ __forceinline__ int owner_cta(long long x, long long W, int P) {
 // product yields both parts.
 template <int NT, bool QF32, int FMT>
 struct WarpState {
-    static constexpr bool K8 = FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8;  // int8 K
+    static constexpr bool K8 = FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8 || FMT == NF_KV_K4V4;  // int8 products
     uint32_t qa[NT][K8 ? 4 : 8][4];  // A fragments per k-step (32 channels int8 K, 16 channels fp16 / bf16)
     float qw[NT];                    // int8 K: s / 254, fp8 K: s, bf16: 1; times softmax scale x log2(e)
     float m_run[NT], l_run[NT];      // running max (log2 units) and weight sum of row g (lane's keys)
@@ -267,6 +283,7 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
                                             int tok0, int L, int lane, const LaneOffsets &lo) {
     using ST = Stage<FMT, NT>;
     constexpr bool K8 = FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8;  // int8 K codes
+    constexpr bool K4 = FMT == NF_KV_K4V4;                         // 4-bit K and V, exponent-byte scales
     constexpr bool F8 = FMT == NF_KV_F8;                           // e4m3 K and V codes
     constexpr bool PF16 = FMT != NF_KV_BF16;                       // fp16 weights and V codes
     const int g = lane >> 2, t = lane & 3;
@@ -274,13 +291,44 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
     // ---- S = Q . K^T: per m-tile two n-tiles j of 8 keys; the lane's results are
     // row g x keys tb + 8j + 2t + e (e = 0, 1) -> x[mt][nt][2j + e]
     float xv[MT][NT][4];
+    float rl[MT][4];  // K4: 2^-E of the lane's keys 2t, 2t+1, 2t+8, 2t+9 (E: the key's largest V exponent)
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
         const int tb = ub + 16 * mt;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             // K^T B fragments: the lane's column is key tb + 8j + g
-            if (F8) {
+            if (K4) {
+                // word t of 16-byte column i (group i: channels 32i + 8t .. + 7) of key
+                // tb + 8j + g; its even nibbles shifted up and its odd nibbles masked
+                // are 16 x the codes as int8, in the B pairs of k-step i (the query
+                // digits were laid out for that channel order)
+                uint32_t w[4];
+                ldsm_x4(smem_addr(st + ST::kK + (tb + 8 * j) * 64) + lo.k, w[0], w[1], w[2], w[3]);
+                // exponent bytes of the lane's two result keys 2t, 2t + 1
+                const uint2 ke = *reinterpret_cast<const uint2 *>(st + ST::kKs + (tb + 8 * j + 2 * t) * 4);
+                // ... and of their V scales: the largest (E) shifts the key's score by E
+                const uint2 ve = *reinterpret_cast<const uint2 *>(st + ST::kVs + (tb + 8 * j + 2 * t) * 4);
+                const uint32_t m0 = __vmaxu4(ve.x, ve.x >> 16), m1 = __vmaxu4(ve.y, ve.y >> 16);
+                const int E0 = (int)(__vmaxu4(m0, m0 >> 8) & 0xFFu), E1 = (int)(__vmaxu4(m1, m1 >> 8) & 0xFFu);
+                rl[mt][2 * j] = E0 == 254 ? 5.877471754e-39f : __int_as_float((254 - E0) << 23);
+                rl[mt][2 * j + 1] = E1 == 254 ? 5.877471754e-39f : __int_as_float((254 - E1) << 23);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        int d[4] = {0, 0, 0, 0};
+                        mma_s8(d, ws.qa[nt][i][0], ws.qa[nt][i][1], ws.qa[nt][i][2], ws.qa[nt][i][3],
+                               (w[i] << 4) & 0xF0F0F0F0u, w[i] & 0xF0F0F0F0u);
+                        // group i's sum times its 2^e (exponent byte e + 127 -> fp32 bits)
+                        x0 = fmaf((float)(d[0] * 254 + d[2]), __int_as_float(((ke.x >> (8 * i)) & 0xFFu) << 23), x0);
+                        x1 = fmaf((float)(d[1] * 254 + d[3]), __int_as_float(((ke.y >> (8 * i)) & 0xFFu) << 23), x1);
+                    }
+                    xv[mt][nt][2 * j] = fmaf(x0, ws.qw[nt], (float)(E0 - 127));
+                    xv[mt][nt][2 * j + 1] = fmaf(x1, ws.qw[nt], (float)(E1 - 127));
+                }
+            } else if (F8) {
                 // e4m3 bytes 32t..32t+31 of the key -> fp16 pairs; k-step ks takes
                 // channels 32t + 4ks + 0, 1 (b0) and + 2, 3 (b1), the order the
                 // query fragments were written in
@@ -352,6 +400,11 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
                     const int pos = tok0 + tb + 8 * (i >> 1) + 2 * t + (i & 1);
                     if (!(pos < L && pos <= ws.lim[nt])) xv[mt][nt][i] = -INFINITY;
                 }
+            if (K4) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (!(tok0 + tb + 8 * (i >> 1) + 2 * t + (i & 1) < L)) rl[mt][i] = 0.f;
+            }
         }
     }
 
@@ -400,7 +453,10 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
         for (int mt = 0; mt < MT; ++mt) {
             const float p0 = ex2(xv[mt][nt][0] - mu), p1 = ex2(xv[mt][nt][1] - mu);
             const float p2 = ex2(xv[mt][nt][2] - mu), p3 = ex2(xv[mt][nt][3] - mu);
-            ws.l_run[nt] += (p0 + p1) + (p2 + p3);
+            if (K4)  // the weights carry each key's 2^E: the row sum takes it out again
+                ws.l_run[nt] += fmaf(p0, rl[mt][0], p1 * rl[mt][1]) + fmaf(p2, rl[mt][2], p3 * rl[mt][3]);
+            else
+                ws.l_run[nt] += (p0 + p1) + (p2 + p3);
             if (PF16) {
                 pb[mt][nt][0] = pack_f16(p0, p1);
                 pb[mt][nt][1] = pack_f16(p2, p3);
@@ -469,7 +525,7 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
                         mma_f16(ws.acc[2 * cp + jc][nt], a[0], a[1], a[2], a[3], b0[nt], b1[nt]);
                 }
             }
-        } else if (K8) {
+        } else if (K8 || K4) {
             // nibbles: matrix cg (lanes 8cg..8cg+7 address its rows) = the 16-byte
             // column cg (channels 32cg..32cg+31) of 8 keys, stored at column
             // position cg ^ (row address bits 7-8) by the swizzled copy
@@ -478,14 +534,33 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
             ldsm_x4_t(va, R[0][0], R[0][1], R[0][2], R[0][3]);            // keys tb + 0..7
             ldsm_x4_t(va + 8 * 64, R[1][0], R[1][1], R[1][2], R[1][3]);   // keys tb + 8..15
             // V scales of keys (2t, 2t+1) and (2t+8, 2t+9) per group, as fp16 pairs
+            // (K4: the factors 2^(e_g - E) <= 1 of the group exponents relative to
+            // the key's largest, whose 2^E the weights already carry; factors below
+            // 2^-14 flush to zero)
             uint32_t sp[2][4];
 #pragma unroll
             for (int kh = 0; kh < 2; ++kh) {
-                const uint4 sv = lds128(st + ST::kVs + (tb + 8 * kh) * 8 + lo.vs);
-                sp[kh][0] = prmt(sv.x, sv.z, 0x5410);
-                sp[kh][1] = prmt(sv.x, sv.z, 0x7632);
-                sp[kh][2] = prmt(sv.y, sv.w, 0x5410);
-                sp[kh][3] = prmt(sv.y, sv.w, 0x7632);
+                if (K4) {
+                    const uint2 ve = *reinterpret_cast<const uint2 *>(st + ST::kVs + (tb + 8 * kh + 2 * t) * 4);
+                    uint32_t dd[2];
+                    const uint32_t vv[2] = {ve.x, ve.y};
+#pragma unroll
+                    for (int k2 = 0; k2 < 2; ++k2) {
+                        const uint32_t m = __vmaxu4(vv[k2], vv[k2] >> 16);
+                        const uint32_t E = (__vmaxu4(m, m >> 8) & 0xFFu) * 0x01010101u;
+                        // 15 - (E - e_g) per byte, at least 0: the fp16 exponent field of 2^(e_g - E)
+                        dd[k2] = __vsubus4(0x0F0F0F0Fu, __vsubus4(E, vv[k2]));
+                    }
+#pragma unroll
+                    for (int cg = 0; cg < 4; ++cg)  // byte cg of key 2t -> half 0, of key 2t + 1 -> half 1
+                        sp[kh][cg] = prmt_sx(dd[0], dd[1], 0x8080u | (uint32_t)cg | ((uint32_t)(cg + 4) << 8)) << 10;
+                } else {
+                    const uint4 sv = lds128(st + ST::kVs + (tb + 8 * kh) * 8 + lo.vs);
+                    sp[kh][0] = prmt(sv.x, sv.z, 0x5410);
+                    sp[kh][1] = prmt(sv.x, sv.z, 0x7632);
+                    sp[kh][2] = prmt(sv.y, sv.w, 0x5410);
+                    sp[kh][3] = prmt(sv.y, sv.w, 0x7632);
+                }
                 if (!FAST) {
                     // keys past the end hold stale bytes: zero their scales
                     const int pa = tok0 + tb + 8 * kh + 2 * t;
@@ -544,11 +619,11 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
 // Piece i is the slot at ps + i * slot_floats: o at [r][128], lse at
 // lse_off + r.  SMEM: plain loads from shared memory; otherwise loads that
 // bypass L1 (the slots were written by other CTAs), kPB in flight at once.
-// The arithmetic is the same for both sources.
-template <bool SMEM>
+// The arithmetic is the same for both sources and any kPB (the pieces are
+// summed in order; kPB only batches the loads).
+template <bool SMEM, int kPB>
 __device__ __forceinline__ void merge_round(const float *ps, size_t slot_floats, int n, int r, int c4, int lse_off,
                                             float &M, float &S, float4 &A) {
-    constexpr int kPB = 16;
     constexpr float kLog2e = 1.4426950408889634f;
     auto ld1 = [&](const float *a) { return SMEM ? *a : __ldcg(a); };
     float Mr = M;
@@ -602,6 +677,7 @@ __device__ __forceinline__ void merge_round(const float *ps, size_t slot_floats,
 // stream from L2.  The rounds, and so the sums, are the same either way.
 // `state` holds the items' running (M, S, A) between rounds (24 bytes per
 // (row, 4 channels) item).
+template <int kPB = 16>
 __device__ __forceinline__ void merge_slots(const DecodeParams &p, const float *src, size_t stride, int n, int rows,
                                          int per_round, bool in_ring, unsigned char *smem, float *state,
                                          int item_cap, uint64_t *fin_bar, uint32_t &fin_phase, volatile int *misc,
@@ -647,9 +723,9 @@ __device__ __forceinline__ void merge_slots(const DecodeParams &p, const float *
             float M = stM[it], S = stS[it];
             float4 A = stA[it];
             if (in_ring)
-                merge_round<true>(reinterpret_cast<const float *>(smem), p.slot_floats, nr, r, c4, lse_off, M, S, A);
+                merge_round<true, kPB>(reinterpret_cast<const float *>(smem), p.slot_floats, nr, r, c4, lse_off, M, S, A);
             else
-                merge_round<false>(rsrc, stride, nr, r, c4, lse_off, M, S, A);
+                merge_round<false, kPB>(rsrc, stride, nr, r, c4, lse_off, M, S, A);
             stM[it] = M;
             stS[it] = S;
             stA[it] = A;
@@ -677,6 +753,63 @@ __device__ __forceinline__ void merge_slots(const DecodeParams &p, const float *
     }
 }
 
+// The end of a piece whose partial (o, lse) is already in its slot, run by the
+// kConsumerWarps * 32 consumer threads (threads 0 .. 255 of the CTA).  The
+// partials of a segment merge in one step when they fit one round of the
+// ring (ring_bytes); else in two: the last piece of each group of gp
+// consecutive pieces merges its group into the group's first slot, and the
+// last group merges the groups.  The grouping is fixed, so the sums do not
+// depend on which CTA finishes last.  in_ring: this was the CTA's last piece,
+// so the ring is idle and the merge may bring the partials into it.
+template <int kPB = 16>
+__device__ __forceinline__ void finish_segment_piece(const DecodeParams &p, int s_id, int first, int n_pieces,
+                                                     int ring_bytes, bool in_ring, unsigned char *ring, float *state,
+                                                     int item_cap, uint64_t *fin_bar, uint32_t &fin_phase,
+                                                     volatile int *misc, int rows, int b, int h) {
+    const uint32_t slot_bytes = (uint32_t)p.slot_floats * 4u;
+    const int gp = (int)((uint32_t)ring_bytes / slot_bytes);  // slots per ring round
+    const bool two_level = n_pieces > gp;
+    const int pi = (int)blockIdx.x - first;  // this piece's index in the segment
+    const int g0 = two_level ? pi / gp * gp : 0;
+    const int gn = two_level ? min(gp, n_pieces - g0) : n_pieces;
+    int *tk = two_level ? &p.gtickets[s_id + first + g0] : &p.tickets[s_id];
+    if (threadIdx.x == 0) {
+        int is_last = 0;
+        if (n_pieces > 1) {
+            // release: the CTA's partial writes (ordered before this thread
+            // by the barrier) become visible no later than the ticket
+            is_last = atomic_add_release(tk, 1) == gn - 1;
+            if (is_last) __threadfence();  // acquire: the other pieces' partials
+        }
+        misc[1] = is_last;
+    }
+    named_sync(1, kConsumerWarps * 32);
+    if (misc[1]) {
+        // This CTA holds the last ticket of the segment (or of a group).
+        float *slot0 = p.partials + (size_t)(s_id + first) * p.slot_floats;
+        merge_slots<kPB>(p, slot0 + (size_t)g0 * p.slot_floats, p.slot_floats, gn, rows, gp, in_ring, ring, state,
+                    item_cap, fin_bar, fin_phase, misc, two_level ? slot0 + (size_t)g0 * p.slot_floats : nullptr,
+                    b, h);
+        if (threadIdx.x == 0) *tk = 0;
+        if (two_level) {
+            const int ng = (n_pieces + gp - 1) / gp;
+            named_sync(1, kConsumerWarps * 32);
+            if (threadIdx.x == 0) {
+                const int is_last = atomic_add_release(&p.tickets[s_id], 1) == ng - 1;
+                if (is_last) __threadfence();
+                misc[1] = is_last;
+            }
+            named_sync(1, kConsumerWarps * 32);
+            if (misc[1]) {
+                merge_slots<kPB>(p, slot0, (size_t)gp * p.slot_floats, ng, rows, gp, in_ring, ring, state, item_cap,
+                            fin_bar, fin_phase, misc, nullptr, b, h);
+                if (threadIdx.x == 0) p.tickets[s_id] = 0;
+            }
+        }
+        named_sync(1, kConsumerWarps * 32);
+    }
+}
+
 template <int NT, bool QF32, int FMT>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_constant__ DecodeParams p) {
     using ST = Stage<FMT, NT>;
@@ -685,6 +818,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     constexpr bool K8 = (FMT != NF_KV_BF16);  // scaled codes through the bulk/tensor-map copies
     constexpr bool V8 = (FMT == NF_KV_K8V8 || FMT == NF_KV_F8);  // 128-byte V rows, one V scale per key
     constexpr bool F8 = (FMT == NF_KV_F8);
+    constexpr bool K4 = (FMT == NF_KV_K4V4);  // nibble K rows (tensor map), exponent-byte scales
     static_assert(SM::kMergeM - SM::kMergeO >= (kMaxRows * 128 + (NT == 1 ? 8 : kMaxRows)) * 4,
                   "fp8 query fragments and factors in the merge buffer");
     constexpr int NS = ST::kStages;
@@ -804,7 +938,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             stage_ok[stage] = 1;
                             const size_t si = ((size_t)blk * H + walk.ph) * kBlock + (tok0 & (kBlock - 1));
                             mbar_arrive_expect_tx(&full[stage], (uint32_t)(ntok * ST::kBytesPerTok));
-                            if (K8) {
+                            if (K4) {
+                                for (int c = 0; c < ntok; c += kChunk) {
+                                    tma_load_2d(st + ST::kK + c * 64, &p.kmap, 0, (int)si + c, &full[stage]);
+                                    tma_load_2d(st + ST::kV + c * 64, &p.vmap, 0, (int)si + c, &full[stage]);
+                                }
+                                bulk_g2s(st + ST::kKs, reinterpret_cast<const uint8_t *>(p.k_scales) + si * 4, ntok * 4,
+                                         &full[stage]);
+                                bulk_g2s(st + ST::kVs, reinterpret_cast<const uint8_t *>(p.v_scales) + si * 4, ntok * 4,
+                                         &full[stage]);
+                            } else if (K8) {
                                 constexpr int vrow = V8 ? 128 : 64, vsc = V8 ? 1 : 4;  // V bytes, V scales per key
                                 bulk_g2s(st + ST::kK, static_cast<const int8_t *>(p.k_codes) + si * 128, ntok * 128, &full[stage]);
                                 for (int c = 0; c < ntok; c += kChunk)
@@ -868,6 +1011,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         // (128-byte swizzle; m-tiles start on 2048-byte boundaries)
         lo.v = (8 * (((uint32_t)lane >> 3) & 1u) + ((uint32_t)lane & 7u)) * 128 +
                ((((uint32_t)lane >> 4) ^ ((uint32_t)lane & 7u)) * 16);
+    } else if (K4) {
+        // ldmatrix row address of lane l: key l & 7 of an n-tile, 16-byte column
+        // l >> 3 (a scale group) at position (l >> 3) ^ ((l & 7) >> 1) (64-byte
+        // swizzle); the V nibbles likewise
+        lo.k = (lane & 7) * 64 + ((((uint32_t)lane >> 3) ^ (((uint32_t)lane & 7) >> 1)) & 3u) * 16;
+        lo.v = lo.k;
+        lo.ks = lo.vs = 0;
     } else if (K8) {
         lo.k = g * 128 + 32 * t;
         lo.ks = 0;
@@ -947,6 +1097,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                     const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
                     d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
                     d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
+                }
+                if (K4) {
+                    // channels 8m .. 8m + 7 (m = lane / 2 = 4i + t) form k-step i of
+                    // lane t: its even channels in the first word of each digit pair,
+                    // its odd ones in the second (the order of the expanded K nibbles)
+                    const uint32_t p1 = __shfl_xor_sync(0xffffffffu, d1w, 1), p2 = __shfl_xor_sync(0xffffffffu, d2w, 1);
+                    const bool odd = lane & 1;
+                    const uint32_t w1 = odd ? prmt(p1, d1w, 0x7531) : prmt(d1w, p1, 0x6420);
+                    const uint32_t w2 = odd ? prmt(p2, d2w, 0x7531) : prmt(d2w, p2, 0x6420);
+                    const int m = lane >> 1;
+                    uint32_t *dst = qsm + (r * 4 + (m & 3)) * 16 + (m >> 2) * 4 + (odd ? 2 : 0);
+                    dst[0] = w1;
+                    dst[1] = w2;
+                    // the expanded K codes are 16 x code
+                    if (lane == 0) qwsm[r] = s1 / 254.0f * p.scale_log2 * 0.0625f;
+                    continue;
                 }
                 uint32_t *dst = qsm + (r * 4 + (lane >> 3)) * 16 + ((lane >> 1) & 3) * 4 + 2 * (lane & 1);
                 dst[0] = d1w;
@@ -1106,55 +1272,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             }
         }
         named_sync(1, kConsumerWarps * 32);
-        // ---- tickets.  The partials of a segment merge in one step when they fit
-        // one ring round; else in two: the last piece of each group of gp
-        // consecutive pieces merges its group into the group's first slot, and
-        // the last group merges the groups.  The grouping is fixed, so the sums
-        // do not depend on which CTA finishes last.
-        const uint32_t slot_bytes = (uint32_t)p.slot_floats * 4u;
-        const int gp = (int)((uint32_t)(NS * ST::kStride) / slot_bytes);  // slots per ring round
-        const bool two_level = n_pieces > gp;
-        const int pi = (int)blockIdx.x - first;  // this piece's index in the segment
-        const int g0 = two_level ? pi / gp * gp : 0;
-        const int gn = two_level ? min(gp, n_pieces - g0) : n_pieces;
-        int *tk = two_level ? &p.gtickets[s_id + first + g0] : &p.tickets[s_id];
-        if (threadIdx.x == 0) {
-            int is_last = 0;
-            if (n_pieces > 1) {
-                // release: the CTA's partial writes (ordered before this thread
-                // by the barrier) become visible no later than the ticket
-                is_last = atomic_add_release(tk, 1) == gn - 1;
-                if (is_last) __threadfence();  // acquire: the other pieces' partials
-            }
-            misc[1] = is_last;
-        }
-        named_sync(1, kConsumerWarps * 32);
-        if (misc[1]) {
-            // This CTA holds the last ticket of the segment (or of a group).  When
-            // this was the CTA's last piece the stage ring is idle.
-            const bool in_ring = walk.x >= walk.end;
-            float *slot0 = p.partials + (size_t)(s_id + first) * p.slot_floats;
-            merge_slots(p, slot0 + (size_t)g0 * p.slot_floats, p.slot_floats, gn, rows_here, gp, in_ring, smem, sm_o,
-                        SM::kMaxItems, fin_bar, fin_phase, misc, two_level ? slot0 + (size_t)g0 * p.slot_floats : nullptr,
-                        b, h);
-            if (threadIdx.x == 0) *tk = 0;
-            if (two_level) {
-                const int ng = (n_pieces + gp - 1) / gp;
-                named_sync(1, kConsumerWarps * 32);
-                if (threadIdx.x == 0) {
-                    const int is_last = atomic_add_release(&p.tickets[s_id], 1) == ng - 1;
-                    if (is_last) __threadfence();
-                    misc[1] = is_last;
-                }
-                named_sync(1, kConsumerWarps * 32);
-                if (misc[1]) {
-                    merge_slots(p, slot0, (size_t)gp * p.slot_floats, ng, rows_here, gp, in_ring, smem, sm_o,
-                                SM::kMaxItems, fin_bar, fin_phase, misc, nullptr, b, h);
-                    if (threadIdx.x == 0) p.tickets[s_id] = 0;
-                }
-            }
-            named_sync(1, kConsumerWarps * 32);
-        }
+        finish_segment_piece(p, s_id, first, n_pieces, NS * ST::kStride, walk.x >= walk.end, smem, sm_o,
+                             SM::kMaxItems, fin_bar, fin_phase, misc, rows_here, b, h);
     }
 }
 

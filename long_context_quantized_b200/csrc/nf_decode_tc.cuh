@@ -1,0 +1,695 @@
+// nf_decode_tc.cuh -- split-K decode attention over the K8/V4 pool for many
+// query rows per kv-head, on the 5th-generation tensor cores (tcgen05).
+//
+// MTP draft verification is the engine's normal decode step: 1 + 3 query
+// tokens per step (page "3090 单卡跑 Qwen3.8-27B：NInfer 上机实测", section
+// 一.3, --spec mtp --draft-tokens 3), each with the G query heads of a GQA
+// group, so a kv-head serves G * n_q = 32 rows (G = 8).  The work per key then
+// grows with the rows (two products of 128 channels per row and key), and on
+// the per-warp mma.sync path it outgrows the HBM time.  Here the products run
+// as whole-tile tcgen05 MMAs issued by one thread, with the accumulators in
+// tensor memory, and the CUDA cores only do the softmax and the V
+// dequantisation.  The work cut, the split partials and the last-ticket merge
+// are those of decode_kernel (nf_decode.cuh); results and workspace layout are
+// the same.
+//
+// Per tile of up to 128 keys (never crossing a 256-key block):
+//   S^T = K . Q^T       kind::i8, M = 128 keys, N = 2 RP (the query rows'
+//                       high int8 digits, then their low digits), K = 128
+//                       channels; A = the int8 K codes as the TMA brought them
+//                       (128-byte swizzle), B = the query digits.
+//   softmax             one thread per key (its tensor-memory lane): x_r =
+//                       (d1_r * 254 + d2_r) * qw_r * kscale for each row r;
+//                       lazy running max per row (raised, and O rescaled, only
+//                       when a tile exceeds it by 2^4); weights p = 2^(x - m - 4)
+//                       <= 1, times the key's power-of-two V factor f_k, as
+//                       fp16 P' [key][row].
+//   V dequantisation    one thread per key: code x (V scale / f_k) as fp16 V'
+//                       [key][channel]; f_k = 2^(E - 15) with E the largest
+//                       exponent of the key's four V scales, so V' < 14 and
+//                       P' <= 2^15 both stay inside fp16 for any fp16 scale, and
+//                       P' x V' = p x code x scale.
+//   O^T += V'^T . P'    kind::f16, M = 128 channels, N = 64 (rows, padded),
+//                       K = 128 keys; A = V' and B = P', both MN-major
+//                       (128-byte swizzle); O^T lives in tensor memory.
+// Roles (18 warps): warps 0-15 are alike -- warp (q, h) = (w % 4, w / 4)
+// takes the keys (and O^T channel lanes) of tensor-memory quadrant q,
+// dequantises their V' channels of scale group h and runs the softmax of a
+// quarter of the rows; it reads its slice of a stage and releases the stage at
+// once.  Four such warps share each SM sub-partition, so one's latency hides
+// behind the others' work.  Warp 16 is the TMA producer; warp 17 holds the
+// tensor memory and, on one thread, issues the MMAs from an event loop that
+// serves whichever of S and P.V is ready.  Warps 0-15 also encode the query
+// digits at each piece's start; warps 0-7 run the piece's merge.  Every
+// mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT and
+// every role runs to its end without further waits.
+#pragma once
+
+#include <cfloat>
+
+#include "nf_decode.cuh"
+#include "nf_tc.cuh"
+
+namespace nf {
+
+constexpr int kDtConsumers = 16;                   // consumer warps
+constexpr int kDtThreads = (kDtConsumers + 2) * 32;  // + producer and MMA warps
+constexpr int kDtProducer = kDtConsumers, kDtMma = kDtConsumers + 1;
+constexpr int kDtStages = 4;
+constexpr int kDtPvN = 64;       // N of the P.V product: the rows, padded
+constexpr int kDtMaxRows = 32;   // rows per kv-head this kernel serves
+constexpr int kDtChunkTiles = kBlock / kChunk;
+// named barriers: 1 the merge (warps 0-7, inside finish_segment_piece), 2..5
+// the four warps of one row quarter, 6 all consumer warps
+constexpr uint32_t kDtBarAll = 6;
+
+struct DtSmem {
+    // one ring stage: K codes [128 keys][128 B] (128-byte swizzle), V nibbles
+    // [128 keys][64 B] (64-byte swizzle), K scales fp16 [128], V scales fp16 [128][4]
+    static constexpr int kStK = 0, kStV = 16384, kStKs = 24576, kStVs = 24832;
+    static constexpr int kStride = 26624;
+    static constexpr int kBytesPerTok = 202;
+    static constexpr int kRingBytes = kDtStages * kStride;
+    static constexpr int kVh = kRingBytes;        // fp16 V' [2 buffers][2 blocks of 64 channels][128 keys][128 B]
+    static constexpr int kP = kVh + 2 * 32768;    // fp16 P' [2 buffers][128 keys][64 rows x 2 B]
+    static constexpr int kQ = kP + 2 * 16384;     // int8 digits [2 buffers][64 digit rows][128 B]
+    static constexpr int kQw = kQ + 2 * 8192;     // float [2][kDtMaxRows]: row factors
+    static constexpr int kRed = kQw + 2 * kDtMaxRows * 4;   // float [4 quadrants][kDtMaxRows]: row maxima
+    static constexpr int kRed2 = kRed + 4 * kDtMaxRows * 4; // float [4 quadrants][kDtMaxRows]: row sums
+    static constexpr int kBars = kRed2 + 4 * kDtMaxRows * 4;
+    static constexpr int kNumBars = 2 * kDtStages + 10 + 2;
+    static constexpr int kStageOk = kBars + kNumBars * 8;   // int [stages]
+    static constexpr int kTmem = kStageOk + kDtStages * 4;  // u32
+    static constexpr int kSeqC = (kTmem + 4 + 15) / 16 * 16;  // int [kMaxBatch]
+    static constexpr int kSeqL = kSeqC + kMaxBatch * 4;       // int [kMaxBatch]
+    static constexpr int kSeqBase = kSeqL + kMaxBatch * 4;    // i64 [kMaxBatch + 1]
+    static constexpr int kMisc = kSeqBase + (kMaxBatch + 1) * 8;  // int [4]
+    static constexpr int kBytes = kMisc + 16;
+    static_assert(kBytes <= 232448, "shared memory per CTA");
+    static_assert(kStride % 1024 == 0 && kVh % 1024 == 0 && kP % 1024 == 0 && kQ % 1024 == 0, "swizzle atoms");
+    static constexpr int kMaxItems = kDtMaxRows * (kHeadDim / 4);  // final-merge items
+    static_assert(kMaxItems * 24 <= 2 * 32768, "final-merge state in the idle V' buffers");
+};
+
+// End (exclusive, in chunks) of the tile that starts at chunk cx: at most 128
+// keys, never crossing a 256-key block.
+__device__ __forceinline__ int dt_tile_end(int cx, int cx_end) {
+    return min(cx_end, min((cx / kDtChunkTiles + 1) * kDtChunkTiles, cx + 128 / kChunk));
+}
+
+// The largest exponent field E (at least 1) of a key's four fp16 V scales:
+// V' = code x scale x 2^(15 - E) and f = 2^(E - 15) (both sides must agree).
+__device__ __forceinline__ int dt_v_exponent(uint2 vs) {
+    const uint32_t a = max(vs.x & 0x7FFFu, (vs.x >> 16) & 0x7FFFu);
+    const uint32_t c = max(vs.y & 0x7FFFu, (vs.y >> 16) & 0x7FFFu);
+    return max((int)(max(a, c) >> 10), 1);
+}
+
+// Barrier with an OR reduction over `count` threads (named barrier `id`).
+__device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+// Output channel of tensor-memory lane m of O^T: each 8-channel chunk of V'
+// holds the nibble-unpacking order (0, 4, 1, 5, 2, 6, 3, 7).
+__device__ __forceinline__ int dt_channel(int m) {
+    const int q = m & 7;
+    return (m & ~7) | ((q >> 1) + 4 * (q & 1));
+}
+
+// bounded waits shared by all roles: skipped once the kernel has aborted
+__device__ __forceinline__ void dt_wait(uint64_t *bar, uint32_t parity, volatile int *misc) {
+    if (!misc[0] && !mbar_wait_spin(bar, parity)) {
+        report(NF_DEVERR_TIMEOUT);
+        misc[0] = 1;
+    }
+}
+
+// HR consecutive tensor-memory columns of the warp's lanes (HR = 4 or 8)
+template <int HR>
+__device__ __forceinline__ void dt_ld(uint32_t taddr, uint32_t (&r)[HR]) {
+    if constexpr (HR == 8) tmem_ld8(taddr, r); else tmem_ld4(taddr, r);
+}
+template <int HR>
+__device__ __forceinline__ void dt_st(uint32_t taddr, const uint32_t (&r)[HR]) {
+    if constexpr (HR == 8) tmem_st8(taddr, r); else tmem_st4(taddr, r);
+}
+
+// One consumer warp's softmax of one tile for its HR rows: scores from the S
+// columns, the lazy running max (a collective step of the four warps of the
+// rows when some score exceeds it by kLazy), the weights times f into P'.
+// FAST: every row sees every key of the tile (no mask).
+// When the max rises and O^T holds earlier tiles of the piece (has_o), the
+// rows' columns of O^T (taddr) are scaled once the last P.V is done (pv_bar).
+template <int HR, bool FAST>
+__device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint32_t (&d2)[HR], const float (&qw)[HR],
+                                           float ksv, int rmin, int R, int r0, float (&thr)[HR], float (&l_part)[HR],
+                                           float *red, int qd, int lane, uint32_t gbar, float f,
+                                           uint32_t (&pk)[HR / 2], bool has_o, uint32_t taddr, uint64_t *pv_bar,
+                                           uint32_t pv_parity, volatile int *misc) {
+    float x[HR];
+#pragma unroll
+    for (int e = 0; e < HR; ++e) {
+        const float v = (float)((int)d1[e] * 254 + (int)d2[e]) * (qw[e] * ksv);
+        x[e] = FAST ? v : ((r0 + e >= rmin && r0 + e < R) ? v : -INFINITY);
+    }
+    bool raise = false;
+#pragma unroll
+    for (int e = 0; e < HR; ++e) raise |= x[e] > thr[e];  // true when no max yet and x finite
+    raise = bar_red_or(gbar, 128, raise);
+    if (raise) {
+        // row maxima of the tile over its 128 keys: the four warps of these rows
+#pragma unroll
+        for (int e = 0; e < HR; ++e) {
+            float mx = x[e];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) red[qd * kDtMaxRows + r0 + e] = mx;
+        }
+        named_sync(gbar, 128);
+        // every thread of the four warps derives the same new maxima
+        float alpha[HR];
+        bool rescale = false;
+#pragma unroll
+        for (int e = 0; e < HR; ++e) {
+            const int r = r0 + e;
+            const float tm = fmaxf(fmaxf(red[r], red[kDtMaxRows + r]), fmaxf(red[2 * kDtMaxRows + r], red[3 * kDtMaxRows + r]));
+            const float m_old = thr[e] - kLazy;  // -inf when none
+            const float m_new = fmaxf(m_old, tm);
+            alpha[e] = m_old == -INFINITY ? 0.f : ex2(m_old - m_new);
+            rescale |= m_new > m_old && m_old != -INFINITY;
+            l_part[e] *= alpha[e];
+            thr[e] = m_new + kLazy;
+        }
+        if (rescale && has_o) {  // the same decision in the four warps of the rows
+            dt_wait(pv_bar, pv_parity, misc);
+            tc_fence_after();
+            uint32_t o[HR];
+            dt_ld<HR>(taddr, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < HR; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha[e]);
+            dt_st<HR>(taddr, o);
+            tmem_wait_st();
+        }
+    }
+    // weights 2^(x - m - kLazy) <= 1 (the row sum), times f into P'; a row
+    // with no max yet has only -inf scores, and the offset -FLT_MAX gives 0
+#pragma unroll
+    for (int e = 0; e < HR; e += 2) {
+        const float p0 = ex2(x[e] - fmaxf(thr[e], -FLT_MAX)), p1 = ex2(x[e + 1] - fmaxf(thr[e + 1], -FLT_MAX));
+        l_part[e] += p0;
+        l_part[e + 1] += p1;
+        pk[e / 2] = pack_f16(p0 * f, p1 * f);
+    }
+}
+
+template <int RP, bool QF32>
+__global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
+    static_assert(RP == 16 || RP == 32, "rows padded to 16 or 32");
+    constexpr int NS = kDtStages;
+    constexpr int HR = RP / 4;                                    // rows per consumer warp
+    constexpr int NSC = 2 * RP;                                   // S columns per buffer
+    constexpr uint32_t kIdescS = umma_idesc_s8(128, NSC);
+    constexpr uint32_t kIdescO = umma_idesc_f16(128, kDtPvN, true, true);
+    constexpr uint32_t kSCol = 64;                                // S buffer b at columns 64 b
+    constexpr uint32_t kOCol = 128;                               // O^T at columns 128 .. 191
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DtSmem::kBars);
+    uint64_t *full = bars, *empty = bars + NS;
+    uint64_t *sfull = bars + 2 * NS, *sfree = sfull + 2, *pfull = sfree + 2;
+    uint64_t *pvdone = pfull + 2, *qfull = pvdone + 2, *fin_bar = qfull + 2, *drain = fin_bar + 1;
+    volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + DtSmem::kStageOk);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + DtSmem::kTmem);
+    int *seqC = reinterpret_cast<int *>(smem + DtSmem::kSeqC);
+    int *seqL = reinterpret_cast<int *>(smem + DtSmem::kSeqL);
+    long long *seqBase = reinterpret_cast<long long *>(smem + DtSmem::kSeqBase);
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + DtSmem::kMisc);  // [0] abort, [1] last ticket
+    float *qw_sm = reinterpret_cast<float *>(smem + DtSmem::kQw);
+    float *red = reinterpret_cast<float *>(smem + DtSmem::kRed);
+    float *red2 = reinterpret_cast<float *>(smem + DtSmem::kRed2);
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = p.num_kv_heads;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1 + kDtConsumers);  // the S MMA's commit and the consumer warps
+            stage_ok[i] = 0;
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sfull[i], 1);
+            mbar_init(&sfree[i], kDtConsumers);
+            mbar_init(&pfull[i], kDtConsumers);  // V' and P' of a tile written
+            mbar_init(&pvdone[i], 1);
+            mbar_init(&qfull[i], 1);
+        }
+        mbar_init(fin_bar, 1);
+        mbar_init(drain, 1);
+        misc[0] = 0;
+        misc[1] = 0;
+        // the swizzled operands need 1024-byte alignment of the shared window
+        if (smem_addr(smem) & 1023u) {
+            if (blockIdx.x == 0) report(NF_DEVERR_INTERNAL);
+            misc[0] = 1;
+        }
+        fence_mbar_init();
+    }
+    // the query-digit buffers' padding rows stay zero
+    for (int i = threadIdx.x; i < 2 * 8192 / 16; i += kDtThreads)
+        reinterpret_cast<uint4 *>(smem + DtSmem::kQ)[i] = make_uint4(0, 0, 0, 0);
+    fence_async_smem();
+    if (warp == kDtMma) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    if (!p.early_kv) pdl_wait();
+    pdl_trigger();
+    if (warp == 0) {
+        for (int b = lane; b < p.batch; b += 32) {
+            const int L = p.seqlens[b];
+            const bool ok = L >= p.n_q && L <= p.max_seqlen;
+            if (!ok && blockIdx.x == 0) report(NF_DEVERR_SEQLEN);
+            seqC[b] = ok ? (L + kChunk - 1) / kChunk : 0;
+            seqL[b] = ok ? L : 0;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            long long acc = 0;
+            for (int b = 0; b < p.batch; ++b) {
+                seqBase[b] = acc;
+                acc += seqC[b] ? (long long)(seqC[b] + kSegPad) * H : 0;
+            }
+            seqBase[p.batch] = acc;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const long long W = seqBase[p.batch];
+    const int P = (int)(W < (long long)gridDim.x ? W : (long long)gridDim.x);
+    const long long c_begin = (int)blockIdx.x < P ? W * blockIdx.x / P : 0;
+    const long long c_end = (int)blockIdx.x < P ? W * (blockIdx.x + 1) / P : 0;
+    PieceWalker walk{seqC, seqBase, H, p.batch, c_begin, c_end};
+
+    if (warp == kDtProducer) {
+        // =============================================================== producer
+        uint32_t kst = 0;
+        bool stop = false;
+        bool waited = !p.early_kv;
+        while (!stop && walk.next()) {
+            const int32_t *bt = p.block_table + (size_t)walk.pb * p.max_blocks;
+            const int nblk = (seqC[walk.pb] * kChunk + kBlock - 1) / kBlock;
+            int win = -1000000, my_blk = 0;
+            const int cx1 = (int)(walk.xe - walk.s0);
+            for (int cx = (int)(walk.xs - walk.s0); cx < cx1; ++kst) {
+                const int ce = dt_tile_end(cx, cx1);
+                const int tok0 = cx * kChunk, ntok = (ce - cx) * kChunk;
+                cx = ce;
+                if (!waited && tok0 + ntok > seqL[walk.pb] - p.n_q) {
+                    pdl_wait();  // the newest rows may come from the kernels before this one
+                    waited = true;
+                }
+                const int bi = tok0 >> 8;
+                if (bi >= win + 32) {
+                    win = bi;
+                    my_blk = win + lane < nblk ? bt[win + lane] : -1;
+                }
+                const int blk = __shfl_sync(0xffffffffu, my_blk, bi - win);
+                if (lane == 0) {
+                    const int stage = (int)(kst % NS);
+                    dt_wait(&empty[stage], ((kst / NS) & 1) ^ 1, misc);
+                    if (!misc[0]) {
+                        unsigned char *st = smem + stage * DtSmem::kStride;
+                        if (blk < 0 || blk >= p.num_blocks) {
+                            report(NF_DEVERR_BLOCK_ID);
+                            stage_ok[stage] = 0;
+                            mbar_arrive(&full[stage]);
+                        } else {
+                            stage_ok[stage] = 1;
+                            const size_t si = ((size_t)blk * H + walk.ph) * kBlock + (tok0 & (kBlock - 1));
+                            mbar_arrive_expect_tx(&full[stage], (uint32_t)(ntok * DtSmem::kBytesPerTok));
+                            for (int c = 0; c < ntok; c += kChunk) {
+                                tma_load_2d(st + DtSmem::kStK + c * 128, &p.kmap, 0, (int)si + c, &full[stage]);
+                                tma_load_2d(st + DtSmem::kStV + c * 64, &p.vmap, 0, (int)si + c, &full[stage]);
+                            }
+                            bulk_g2s(st + DtSmem::kStKs, p.k_scales + si, ntok * 2, &full[stage]);
+                            bulk_g2s(st + DtSmem::kStVs, p.v_scales + si * 4, ntok * 8, &full[stage]);
+                        }
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, misc[0], 0)) {
+                    stop = true;
+                    break;
+                }
+            }
+        }
+        if (lane == 0) {
+            // no copy into this CTA's shared memory may be in flight at exit
+            for (uint32_t kk = kst > (uint32_t)NS ? kst - NS : 0; kk < kst && !misc[0]; ++kk)
+                dt_wait(&full[kk % NS], (kk / NS) & 1, misc);
+        }
+    } else if (warp == kDtMma) {
+        // =============================================================== MMA issue
+        // An event loop over two in-order streams: S of tile kt (once its stage
+        // is full, its S buffer free and, at a piece's first tile, the piece's
+        // query digits written) and P.V of tile j < kt (once V' and P' of j are
+        // written); whichever is ready goes first, so neither waits behind the
+        // other.
+        if (lane == 0) {
+            const uint32_t sRing = smem_addr(smem), sQ = smem_addr(smem + DtSmem::kQ);
+            const uint32_t sVh = smem_addr(smem + DtSmem::kVh), sP = smem_addr(smem + DtSmem::kP);
+            uint32_t kt = 0, pj = 0, pc = 0;
+            uint64_t first_mask = 0;  // bit (tile % 64): the tile opens its piece (its P.V overwrites O)
+            bool have = walk.next(), need_q = true;
+            int cx = have ? (int)(walk.xs - walk.s0) : 0, cx1 = have ? (int)(walk.xe - walk.s0) : 0;
+            bool first_tile = false;
+            uint64_t t_idle = 0;
+            uint32_t spins = 0;
+            while (!misc[0] && (have || pj < kt)) {
+                bool progress = false;
+                if (have) {
+                    if (need_q) {
+                        if (mbar_test(&qfull[pc & 1], (pc >> 1) & 1)) {
+                            need_q = false;
+                            first_tile = true;
+                            progress = true;
+                        }
+                    } else {
+                        const uint32_t stage = kt % NS, sb = kt & 1;
+                        if (mbar_test(&full[stage], (kt / NS) & 1) && mbar_test(&sfree[sb], ((kt >> 1) & 1) ^ 1)) {
+                            tc_fence_after();
+                            const uint32_t kaddr = sRing + stage * DtSmem::kStride + DtSmem::kStK;
+                            const uint32_t qaddr = sQ + (pc & 1) * 8192u;
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                umma_s8(tmem + sb * kSCol, umma_desc_sw128(kaddr + 32 * ks, 16, 1024),
+                                        umma_desc_sw128(qaddr + 32 * ks, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
+                            umma_commit(&sfull[sb]);
+                            umma_commit(&empty[stage]);  // the stage's K codes are consumed
+                            const uint64_t bit = 1ull << (kt & 63);
+                            first_mask = first_tile ? (first_mask | bit) : (first_mask & ~bit);
+                            first_tile = false;
+                            ++kt;
+                            progress = true;
+                            cx = dt_tile_end(cx, cx1);
+                            if (cx >= cx1) {  // the piece is issued: on to the next
+                                ++pc;
+                                have = walk.next();
+                                if (have) {
+                                    cx = (int)(walk.xs - walk.s0);
+                                    cx1 = (int)(walk.xe - walk.s0);
+                                    need_q = true;
+                                }
+                            }
+                        }
+                    }
+                }
+                if (pj < kt) {
+                    const uint32_t b = pj & 1;
+                    if (mbar_test(&pfull[b], (pj >> 1) & 1)) {
+                        tc_fence_after();
+                        const bool ovw = (first_mask >> (pj & 63)) & 1ull;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint64_t ad = umma_desc_sw128(sVh + b * 32768u + kk * 2048u, 16384, 1024);
+                            const uint64_t bd = umma_desc_sw128(sP + b * 16384u + kk * 2048u, 16384, 1024);
+                            umma_f16(tmem + kOCol, ad, bd, kIdescO, (ovw && kk == 0) ? 0u : 1u);
+                        }
+                        umma_commit(&pvdone[b]);
+                        ++pj;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    spins = 0;
+                    t_idle = 0;
+                } else {
+                    __nanosleep(32);
+                    if ((++spins & 255u) == 0) {
+                        // nothing ready for a while: bound the wait like every other
+                        const uint64_t now = global_ns();
+                        if (t_idle == 0) {
+                            t_idle = now;
+                        } else if (now - t_idle > kWaitLimitNs) {
+                            report(NF_DEVERR_TIMEOUT);
+                            misc[0] = 1;
+                        }
+                    }
+                }
+            }
+            // every MMA this thread issued has completed before tensor memory is freed
+            umma_commit(drain);
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait_sleep(drain, 0, 20000u))
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    report(NF_DEVERR_TIMEOUT);
+                    break;
+                }
+        }
+    } else {
+        // =============================================================== warps 0-15
+        // Warp (q, h) = (warp % 4, warp / 4): tensor-memory lane quadrant q, so
+        // key 32 q + lane of each tile (the lane of S) and channel lane 32 q +
+        // lane of O^T; rows h HR .. h HR + HR - 1 of the softmax, P' and O^T; and
+        // the 32 channels of V scale group h in the dequantisation.
+        if (p.early_kv) pdl_wait();
+        // segments of sequences with no valid key: o = 0, lse = -inf
+        for (int s = blockIdx.x; s < p.batch * H; s += gridDim.x) {
+            const int b = s / H, h = s % H;
+            if (seqC[b] != 0) continue;
+            for (int idx = threadIdx.x; idx < p.rows * kHeadDim; idx += kDtConsumers * 32) {
+                const int r = idx / kHeadDim, ch = idx % kHeadDim;
+                const int j = r / p.group, gq = r % p.group;
+                const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+                p.out[row * kHeadDim + ch] = 0.f;
+                if (ch == 0 && p.out_lse) p.out_lse[row] = -INFINITY;
+            }
+        }
+        const int qd = warp & 3, hq = warp >> 2;
+        const int i = 32 * qd + lane;  // key of the tile (lane of S, channel lane of O^T)
+        const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+        const int r0 = hq * HR;        // first row of this warp
+        const uint32_t gbar = 2 + hq;  // named barrier of the 4 warps with these rows
+        const int R = p.rows;
+        uint32_t kt = 0, pc = 0, fin_phase = 0;
+        float l_part[HR], thr[HR], qw[HR];
+        while (walk.next()) {
+            const int b = walk.pb, h = walk.ph;
+            const int L = seqL[b];
+            // ---- query digits of (b, h): q ~= s (d1 + d2 / 254), s = max|q| / 127;
+            // digit row r (d1) and RP + r (d2) of the K-major B operand of S
+            {
+                unsigned char *qb = smem + DtSmem::kQ + (pc & 1) * 8192;
+                for (int r = warp; r < R; r += kDtConsumers) {
+                    const int j = r / p.group, gq = r % p.group;
+                    const size_t qoff =
+                        (((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq) * kHeadDim + 4 * lane;
+                    float x[4];
+                    if (QF32) {
+                        const float4 v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p.q) + qoff);
+                        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.q) + qoff);
+                        x[0] = __uint_as_float(v.x << 16);
+                        x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+                        x[2] = __uint_as_float(v.y << 16);
+                        x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+                    }
+                    float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                    const float s1 = amax / 127.0f;
+                    const float inv = amax > 0.f ? 127.0f / amax : 0.f;
+                    uint32_t d1w = 0, d2w = 0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float d1 = fminf(fmaxf(rintf(x[e] * inv), -127.f), 127.f);
+                        const float r1 = fmaf(-d1, s1, x[e]);
+                        const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
+                        d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
+                        d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
+                    }
+                    // channels 4 lane .. + 3: 16-byte chunk lane / 4 of the row, swizzled
+                    const uint32_t cofs = ((((uint32_t)lane >> 2) ^ ((uint32_t)r & 7u)) << 4) + 4u * (lane & 3);
+                    *reinterpret_cast<uint32_t *>(qb + r * 128 + cofs) = d1w;
+                    const int r2 = RP + r;
+                    *reinterpret_cast<uint32_t *>(qb + r2 * 128 + ((((uint32_t)lane >> 2) ^ ((uint32_t)r2 & 7u)) << 4) +
+                                                  4u * (lane & 3)) = d2w;
+                    if (lane == 0) qw_sm[(pc & 1) * kDtMaxRows + r] = s1 / 254.0f * p.scale_log2;
+                }
+                fence_async_smem();
+                named_sync(kDtBarAll, kDtConsumers * 32);
+                if (threadIdx.x == 0) mbar_arrive(&qfull[pc & 1]);
+            }
+            // this warp's rows: their factors, empty running maxima and sums
+#pragma unroll
+            for (int e = 0; e < HR; ++e) {
+                qw[e] = r0 + e < R ? qw_sm[(pc & 1) * kDtMaxRows + r0 + e] : 0.f;
+                thr[e] = -INFINITY;
+                l_part[e] = 0.f;
+            }
+            // causal: key position pos is seen by rows r >= (pos - (L - n_q)) * G
+            const int causal_base = p.causal ? L - p.n_q : 0x7fffffff;
+            const int all_see = p.causal ? L - p.n_q + 1 : L;  // keys every row sees
+            const uint32_t kfirst = kt;
+            const int cx1 = (int)(walk.xe - walk.s0);
+            for (int cx = (int)(walk.xs - walk.s0); cx < cx1; ++kt) {
+                const int ce = dt_tile_end(cx, cx1);
+                const int tok0 = cx * kChunk, ntok = (ce - cx) * kChunk;
+                cx = ce;
+                const uint32_t stage = kt % NS, sb = kt & 1;
+                const unsigned char *st = smem + stage * DtSmem::kStride;
+                // ---- the stage: this key's V nibbles of group hq, its scales;
+                // then the stage is released
+                dt_wait(&full[stage], (kt / NS) & 1, misc);
+                const int pos = tok0 + i;
+                const bool sok = !misc[0] && stage_ok[stage];
+                const bool kv_ok = sok && i < ntok && pos < L;
+                const bool fast = sok && ntok == 128 && tok0 + 128 <= all_see && R == RP;
+                uint4 nib = make_uint4(0, 0, 0, 0);
+                uint2 vsr = make_uint2(0, 0);
+                float ksv = 0.f;
+                if (kv_ok) {
+                    nib = *reinterpret_cast<const uint4 *>(st + DtSmem::kStV + i * 64 +
+                                                           ((((uint32_t)hq) ^ (((uint32_t)i >> 1) & 3u)) << 4));
+                    vsr = *reinterpret_cast<const uint2 *>(st + DtSmem::kStVs + i * 8);
+                    ksv = __half2float(*reinterpret_cast<const __half *>(st + DtSmem::kStKs + i * 2));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                const int ev = dt_v_exponent(vsr);
+                // ---- V' and P' buffers sb are free once the P.V of tile kt - 2 is done
+                if (kt >= 2) dt_wait(&pvdone[sb], ((kt >> 1) - 1) & 1, misc);
+                {
+                    // V' = code x scale / f: group hq of the key's row (block hq / 2,
+                    // 16-byte chunks 4 (hq % 2) .. + 3)
+                    unsigned char *vd = smem + DtSmem::kVh + sb * 32768 + (hq >> 1) * 16384 + i * 128;
+                    const uint32_t sw = (uint32_t)i & 7u;
+                    const uint32_t sbits = (hq < 2 ? vsr.x : vsr.y) >> (16 * (hq & 1));
+                    const float sg = __half2float(__ushort_as_half((unsigned short)(sbits & 0xFFFFu))) *
+                                     __int_as_float((127 + 15 - ev) << 23);
+                    const __half2 sv = __float2half2_rn(sg);
+                    const uint32_t wd[4] = {nib.x, nib.y, nib.z, nib.w};
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        uint4 o;
+                        o.x = h2_u32(__hmul2(nib_even(wd[w]), sv));
+                        o.y = h2_u32(__hmul2(nib_odd(wd[w]), sv));
+                        o.z = h2_u32(__hmul2(nib_even(wd[w] >> 8), sv));
+                        o.w = h2_u32(__hmul2(nib_odd(wd[w] >> 8), sv));
+                        const uint32_t cc = (uint32_t)(4 * (hq & 1) + w);
+                        *reinterpret_cast<uint4 *>(vd + ((cc ^ sw) << 4)) = o;
+                    }
+                }
+                // ---- softmax of rows r0 .. r0 + HR - 1 for this key
+                dt_wait(&sfull[sb], (kt >> 1) & 1, misc);
+                tc_fence_after();
+                uint32_t d1[HR], d2[HR];
+                {
+                    const uint32_t ta = tmem + lane_base + sb * kSCol + r0;
+                    dt_ld<HR>(ta, d1);
+                    dt_ld<HR>(ta + RP, d2);
+                    tmem_wait_ld();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfree[sb]);
+                const int dpos = pos - causal_base;
+                const int rmin = kv_ok ? (dpos > 0 ? dpos * p.group : 0) : 0x7fffffff;  // rows rmin .. R - 1 see it
+                const float f = __int_as_float((127 + ev - 15) << 23);
+                uint32_t pk[HR / 2];
+                const uint32_t ota = tmem + lane_base + kOCol + r0;
+                if (fast)
+                    dt_softmax<HR, true>(d1, d2, qw, ksv, rmin, R, r0, thr, l_part, red, qd, lane, gbar, f, pk,
+                                         kt > kfirst, ota, &pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
+                else
+                    dt_softmax<HR, false>(d1, d2, qw, ksv, rmin, R, r0, thr, l_part, red, qd, lane, gbar, f, pk,
+                                          kt > kfirst, ota, &pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
+                // P' row of this key, rows r0 .. r0 + HR - 1 (half or all of one 16-byte chunk)
+                {
+                    unsigned char *pr = smem + DtSmem::kP + sb * 16384 + i * 128 +
+                                        ((((uint32_t)r0 >> 3) ^ ((uint32_t)i & 7u)) << 4) + (r0 & 7) * 2;
+                    if constexpr (HR == 8)
+                        *reinterpret_cast<uint4 *>(pr) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    else
+                        *reinterpret_cast<uint2 *>(pr) = make_uint2(pk[0], pk[1]);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pfull[sb]);
+            }
+
+            // ---- end of the piece: O^T / l into out (one piece) or the partial slot
+            const int s_id = b * H + h;
+            const int first = owner_cta(walk.s0, W, P);
+            const int last = owner_cta(walk.s0 + seqC[b] - 1, W, P);
+            const int n_pieces = last - first + 1;
+            {
+                float l_row[HR];
+#pragma unroll
+                for (int e = 0; e < HR; ++e) {
+                    float v = l_part[e];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    if (lane == 0) red2[qd * kDtMaxRows + r0 + e] = v;
+                }
+                named_sync(gbar, 128);
+#pragma unroll
+                for (int e = 0; e < HR; ++e) {
+                    const int r = r0 + e;
+                    l_row[e] = (red2[r] + red2[kDtMaxRows + r]) + (red2[2 * kDtMaxRows + r] + red2[3 * kDtMaxRows + r]);
+                }
+                if (kt > kfirst) dt_wait(&pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
+                tc_fence_after();
+                uint32_t o[HR];
+                dt_ld<HR>(tmem + lane_base + kOCol + r0, o);
+                tmem_wait_ld();
+                tc_fence_before();
+                const int ch = dt_channel(i);
+                float *slotp = p.partials + (size_t)(s_id + blockIdx.x) * p.slot_floats;
+#pragma unroll
+                for (int e = 0; e < HR; ++e) {
+                    const int r = r0 + e;
+                    if (r >= R) break;
+                    const bool any = thr[e] != -INFINITY;  // thr = m + kLazy: the weights were 2^(x - m - kLazy)
+                    const float val = any ? __uint_as_float(o[e]) / l_row[e] : 0.f;
+                    const float lse = any ? (thr[e] + log2f(l_row[e])) * 0.69314718055994531f : -INFINITY;
+                    if (n_pieces == 1) {
+                        const int j = r / p.group, gq = r % p.group;
+                        const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+                        p.out[row * kHeadDim + ch] = val;
+                        if (i == e && p.out_lse) p.out_lse[row] = lse;
+                    } else {
+                        slotp[r * kHeadDim + ch] = val;
+                        if (i == e) slotp[R * kHeadDim + r] = lse;
+                    }
+                }
+            }
+            named_sync(kDtBarAll, kDtConsumers * 32);  // the piece's outputs are written
+            if (warp < kConsumerWarps)
+                finish_segment_piece<8>(p, s_id, first, n_pieces, DtSmem::kRingBytes, walk.x >= walk.end, smem,
+                                     reinterpret_cast<float *>(smem + DtSmem::kVh), DtSmem::kMaxItems, fin_bar,
+                                     fin_phase, misc, R, b, h);
+            named_sync(kDtBarAll, kDtConsumers * 32);  // the merge is done: its buffers are free again
+            ++pc;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kDtMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace nf
