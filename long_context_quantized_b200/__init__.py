@@ -16,9 +16,9 @@ import threading
 import torch
 
 __all__ = [
-    "NF_OK", "NF_KV_K8V4", "NF_KV_BF16", "NF_KV_K8V8", "NF_KV_F8", "NF_F32", "NF_BF16", "NfError", "KVLayer",
+    "NF_OK", "NF_KV_K8V4", "NF_KV_BF16", "NF_KV_K8V8", "NF_KV_F8", "NF_KV_K4V4", "NF_F32", "NF_BF16", "NfError", "KVLayer",
     "nf_kv_append_quant", "nf_decode_attn_workspace_size", "nf_decode_attn", "nf_decode_attn_noalloc",
-    "nf_attn_combine", "nf_prefill_attn",
+    "nf_attn_combine", "nf_attn_packed_slot_floats", "nf_attn_combine_packed", "nf_prefill_attn",
     "nf_get_device_error", "nf_status_string", "library_path", "load_library",
 ]
 
@@ -32,7 +32,7 @@ NF_ERR_INVALID_ARG, NF_ERR_UNSUPPORTED, NF_ERR_WORKSPACE, NF_ERR_CUDA, NF_ERR_DE
 NF_DEVERR_NONE, NF_DEVERR_BLOCK_ID, NF_DEVERR_TABLE, NF_DEVERR_SEQLEN = 0, 1, 2, 3
 NF_DEVERR_TIMEOUT, NF_DEVERR_INTERNAL, NF_DEVERR_RANGE = 4, 5, 6
 NF_F32, NF_BF16, NF_F16 = 0, 1, 2
-NF_KV_K8V4, NF_KV_BF16, NF_KV_K8V8, NF_KV_F8 = 0, 1, 2, 3
+NF_KV_K8V4, NF_KV_BF16, NF_KV_K8V8, NF_KV_F8, NF_KV_K4V4 = 0, 1, 2, 3, 4
 BLOCK = 256
 HEAD_DIM = 128
 
@@ -88,6 +88,10 @@ def load_library():
         lib.nf_selftest_bounded_wait.restype = I
         lib.nf_attn_combine.argtypes = [P, P, I, I, I, P, P, P]
         lib.nf_attn_combine.restype = I
+        lib.nf_attn_packed_slot_floats.argtypes = [I, I]
+        lib.nf_attn_packed_slot_floats.restype = S
+        lib.nf_attn_combine_packed.argtypes = [P, I, I, I, P, P, P]
+        lib.nf_attn_combine_packed.restype = I
         lib.nf_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32)]
         lib.nf_get_device_error.restype = I
         lib.nf_status_string.argtypes = [I]
@@ -160,6 +164,11 @@ class KVLayer:
             ks = torch.empty((num_blocks, num_kv_heads, BLOCK), dtype=torch.float16, **kw)
             v = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 2), dtype=torch.uint8, **kw)
             vs = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 32), dtype=torch.float16, **kw)
+        elif fmt == NF_KV_K4V4:
+            k = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 2), dtype=torch.uint8, **kw)
+            ks = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 32), dtype=torch.uint8, **kw)
+            v = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 2), dtype=torch.uint8, **kw)
+            vs = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM // 32), dtype=torch.uint8, **kw)
         elif fmt in (NF_KV_K8V8, NF_KV_F8):
             code = torch.int8 if fmt == NF_KV_K8V8 else torch.uint8  # fp8: e4m3 bytes
             k = torch.empty((num_blocks, num_kv_heads, BLOCK, HEAD_DIM), dtype=code, **kw)
@@ -289,6 +298,26 @@ def nf_attn_combine(part_o, part_lse, out, out_lse=None, stream=None):
     st = load_library().nf_attn_combine(_dptr(part_o), _dptr(part_lse), S, rows, d, _dptr(out),
                                         _dptr(out_lse), _stream(stream))
     _check(st, "nf_attn_combine")
+
+
+def nf_attn_packed_slot_floats(rows: int, head_dim: int = HEAD_DIM) -> int:
+    """Floats of one packed split slot: o [rows][head_dim] then lse [rows],
+    rounded up to a multiple of 4 (see nf.h)."""
+    return int(load_library().nf_attn_packed_slot_floats(int(rows), int(head_dim)))
+
+
+def nf_attn_combine_packed(parts, rows: int, out, out_lse=None, stream=None):
+    """parts fp32 [S][slot] (packed split slots) -> out [rows][d], out_lse [rows]."""
+    _need(parts, "parts", torch.float32)
+    _need(out, "out", torch.float32)
+    _need(out_lse, "out_lse", torch.float32)
+    S = parts.shape[0]
+    d = out.shape[-1]
+    if parts.numel() != S * nf_attn_packed_slot_floats(rows, d):
+        raise NfError(NF_ERR_INVALID_ARG, "nf_attn_combine_packed", "parts is not [S][slot]")
+    st = load_library().nf_attn_combine_packed(_dptr(parts), S, int(rows), d, _dptr(out), _dptr(out_lse),
+                                               _stream(stream))
+    _check(st, "nf_attn_combine_packed")
 
 
 def nf_get_device_error() -> int:

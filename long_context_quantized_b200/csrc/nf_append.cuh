@@ -7,7 +7,9 @@
 // lane, a coalesced 128-byte row).  V: absmax over each 8-lane group of 32
 // channels -> fp16 scale absmax/7 -> 4 nibbles per lane packed into 2 bytes;
 // for the int8 KV dtype (same section, --kv-dtype int8) V takes the K rule; the
-// fp8 dtype (--kv-dtype fp8) stores e4m3 codes of x / (absmax / 448) for both.
+// fp8 dtype (--kv-dtype fp8) stores e4m3 codes of x / (absmax / 448) for both;
+// the RK4V4-E8 reading (page "影片筆記：NInfer + 千问3.8 27b = 1.5倍速@256K上下文",
+// section 三) stores 4-bit codes of both with a power-of-two scale per 32 channels.
 // Division and rounding are the IEEE fp32 ones (__fdiv_rn, round half to even),
 // subnormals kept, so the codes are bit-identical to the format definition.
 #pragma once
@@ -91,6 +93,31 @@ __device__ __forceinline__ void quant_row_f8(const float (&x)[4], int lane, uint
     if (lane == 0) *scale = h;
 }
 
+// RK4V4-E8 (both K and V): one power-of-two scale 2^e per 32 channels = 8
+// lanes, e the smallest integer with 2^e >= fp32(absmax / 7) (read from the
+// bits of the quotient: an exact power of two keeps its exponent, anything
+// above it takes the next one), clamped to [-126, 127] and stored as the byte
+// e + 127; codes round_half_even(x / 2^e) clamped to [-7, 7], packed two per
+// byte (the even channel in the low nibble).
+__device__ __forceinline__ void quant_row_e8(const float (&x)[4], int lane, uint8_t *codes, uint8_t *scales) {
+    float a = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const uint32_t sb = __float_as_uint(__fdiv_rn(a, 7.0f));
+    const int ef = (int)(sb >> 23);  // biased exponent; 0 for zero and subnormal quotients
+    int e = ef == 0 ? -126 : ef - 127 + ((sb & 0x7FFFFFu) != 0u ? 1 : 0);
+    e = min(max(e, -126), 127);
+    const float scale = __int_as_float((e + 127) << 23);
+    uint32_t c4 = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const int q = min(max(__float2int_rn(__fdiv_rn(x[c], scale)), -7), 7);
+        c4 |= (uint32_t)(q & 0xF) << (4 * c);
+    }
+    *reinterpret_cast<uint16_t *>(codes + 2 * lane) = (uint16_t)c4;
+    if ((lane & 7) == 0) scales[lane >> 3] = (uint8_t)(e + 127);
+}
+
 __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p) {
     pdl_wait();
     pdl_trigger();
@@ -129,6 +156,14 @@ __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p)
         vb.x = pack_bf16(v[0], v[1]); vb.y = pack_bf16(v[2], v[3]);
         *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.k_codes) + si * kHeadDim + 4 * lane) = kb;
         *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.v_codes) + si * kHeadDim + 4 * lane) = vb;
+        return;
+    }
+
+    if (p.fmt == NF_KV_K4V4) {
+        quant_row_e8(k, lane, static_cast<uint8_t *>(p.k_codes) + si * (kHeadDim / 2),
+                     reinterpret_cast<uint8_t *>(p.k_scales) + si * (kHeadDim / 32));
+        quant_row_e8(v, lane, static_cast<uint8_t *>(p.v_codes) + si * (kHeadDim / 2),
+                     reinterpret_cast<uint8_t *>(p.v_scales) + si * (kHeadDim / 32));
         return;
     }
 

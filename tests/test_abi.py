@@ -116,12 +116,13 @@ def test_prefill_rejects_bad_arguments_before_launch(lib):
     assert _prefill(lib, _layer(), batch=70000) == nf.NF_ERR_UNSUPPORTED
 
 
-def test_int8_and_fp8_layers_need_their_scale_planes(lib):
-    for fmt in (nf.NF_KV_K8V8, nf.NF_KV_F8):
+def test_int8_fp8_and_k4v4_layers_need_their_scale_planes(lib):
+    for fmt in (nf.NF_KV_K8V8, nf.NF_KV_F8, nf.NF_KV_K4V4):
         assert _decode(lib, nf.nf_kv_layer(fmt, 4, 256, 2, 128, 0, 256, 0, 256, 256)) == nf.NF_ERR_INVALID_ARG
         assert _decode(lib, nf.nf_kv_layer(fmt, 4, 256, 2, 128, 0, 256, 256, 256, 0)) == nf.NF_ERR_INVALID_ARG
         assert _decode(lib, nf.nf_kv_layer(fmt, 4, 256, 2, 128, 0, 256, 264, 256, 256)) == nf.NF_ERR_INVALID_ARG
         # v_group is not checked for these formats: the next refusal is the shape's
         assert _decode(lib, nf.nf_kv_layer(fmt, 4, 256, 2, 128, 7, 256, 256, 256, 256), H_q=3) \
             == nf.NF_ERR_INVALID_ARG
-    assert _decode(lib, _layer(fmt=4)) == nf.NF_ERR_UNSUPPORTED
+    assert _decode(lib, _layer(fmt=5)) == nf.NF_ERR_UNSUPPORTED
+    assert _prefill(lib, _layer(fmt=nf.NF_KV_K4V4)) == nf.NF_ERR_UNSUPPORTED  # prefill: K8/V4 only

@@ -17,6 +17,8 @@ def test_bytes_per_token_head_by_format():
     # int8 and fp8: 128 + 2 bytes for each of K and V
     assert workloads.kv_bytes_per_token_head("k8v8") == workloads.kv_bytes_per_token_head("f8") == 260
     assert workloads.kv_bytes_per_token_head("bf16") == 512
+    # RK4V4-E8: 64 bytes of nibbles and 4 exponent bytes for each of K and V
+    assert workloads.kv_bytes_per_token_head("k4v4") == 2 * (64 + 4) == 136
     with pytest.raises(ValueError):
         workloads.kv_bytes_per_token_head("int4")
 

@@ -18,7 +18,7 @@ from nfcase import ATOL, REL_L2, run_case, gpu_layer, oracle_pool, compare_pool,
 
 pytestmark = pytest.mark.gpu
 
-K8, BF, I8, F8 = nf.NF_KV_K8V4, nf.NF_KV_BF16, nf.NF_KV_K8V8, nf.NF_KV_F8
+K8, BF, I8, F8, K4 = nf.NF_KV_K8V4, nf.NF_KV_BF16, nf.NF_KV_K8V8, nf.NF_KV_F8, nf.NF_KV_K4V4
 
 
 @pytest.fixture(autouse=True)
@@ -52,7 +52,7 @@ SMALL = [
 ]
 
 
-@pytest.mark.parametrize("fmt", [K8, BF, I8, F8], ids=["k8v4", "bf16", "k8v8", "f8"])
+@pytest.mark.parametrize("fmt", [K8, BF, I8, F8, K4], ids=["k8v4", "bf16", "k8v8", "f8", "k4v4"])
 @pytest.mark.parametrize("qdt", [torch.float32, torch.bfloat16], ids=["qf32", "qbf16"])
 @pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
 def test_small_shapes(case, qdt, fmt):
@@ -192,12 +192,53 @@ def test_workload_fp8_cache_sampled_heads(name, heads):
     _full_size(name, F8, heads=heads)
 
 
+@pytest.mark.parametrize("name,heads", [("ctx32k_append", [3]), ("ragged_c2", [1]), ("mtp_verify", [0]),
+                                        ("longest", [2])])
+def test_workload_k4v4_cache_sampled_heads(name, heads):
+    _full_size(name, K4, heads=heads)
+
+
+def test_k4v4_groups_of_very_different_magnitudes():
+    # V groups of one key 2^20 apart in magnitude and keys whose largest V
+    # exponents differ widely: the per-key exponent shift and the per-group
+    # factors keep every weight inside fp16
+    w = workloads.custom("k4_mag", cached=(900,), n_new=4, n_q=4, num_q_heads=8, num_kv_heads=1,
+                         q_dtype=torch.bfloat16, kv_in_dtype=torch.float32, causal=True)
+    dev = "cuda"
+    bt_np = workloads.block_table(w)
+    bt = torch.as_tensor(bt_np, device=dev)
+    k, v = workloads.layer_kv(w, 0, 0, device=dev)
+    g = torch.Generator(device="cpu").manual_seed(9)
+    vmul = (2.0 ** torch.randint(-12, 13, (904, 1, 4), generator=g).float()).repeat_interleave(32, dim=2).to(dev)
+    v = (v * vmul).contiguous()
+    kv = nf.KVLayer.empty(K4, w.pool_blocks, 1, device=dev, fill=0xA5)
+    nf.nf_kv_append_quant(kv, k[None].contiguous(), v[None], bt, torch.zeros(1, dtype=torch.int32, device=dev))
+    q = workloads.layer_q(w, 0, device=dev)
+    sl = torch.as_tensor(w.seqlens, dtype=torch.int32, device=dev)
+    out = torch.empty((1, 4, 8, 128), device=dev)
+    lse = torch.empty((1, 4, 8), device=dev)
+    ws = torch.zeros(nf.nf_decode_attn_workspace_size(1, 4, 8, 1, 904), dtype=torch.uint8, device=dev)
+    nf.nf_decode_attn(kv, q, bt, sl, 904, w.softmax_scale, True, out, lse, ws)
+    torch.cuda.synchronize()
+    pool, hs = oracle_pool(w, K4, [(k, v)], bt_np)
+    compare_pool(kv, pool, hs)
+    ref_o, ref_l = oracle_attention(w, pool, hs, q, bt_np)
+    # the values span 2^24: compare relative to the output norm per row
+    go = out.cpu().double().numpy().reshape(ref_o.shape)
+    rel = np.linalg.norm(go - ref_o) / np.linalg.norm(ref_o)
+    assert np.all(np.isfinite(go)) and rel <= REL_L2, rel
+    fin = np.isfinite(ref_l)
+    assert np.abs(lse.cpu().double().numpy().reshape(ref_l.shape)[fin] - ref_l[fin]).max() <= 2e-3
+
+
 # ------------------------------------------- early KV streaming (flag path)
 @pytest.mark.parametrize("name,kw,fmt", [
     ("mtp", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True), K8),
     ("ragged", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2), K8),
     ("mtp_int8", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True), I8),
     ("ragged_fp8", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2), F8),
+    ("mtp_k4v4", dict(cached=(700,), n_new=4, n_q=4, num_q_heads=32, num_kv_heads=4, causal=True), K4),
+    ("ragged_k4v4", dict(cached=(1500, 3000), n_new=1, num_q_heads=16, num_kv_heads=2), K4),
 ])
 def test_early_kv_back_to_back_layers(name, kw, fmt):
     # several layers of (append the step's tokens, decode) queued on one stream

@@ -178,11 +178,14 @@ def kv_bytes_per_token_head(fmt: str = "k8v4", d: int = HEAD_DIM) -> int:
     """Bytes one cached key/value pair occupies per kv-head: K8/V4 stores d int8
     K codes, one fp16 K scale, d/2 bytes of V nibbles and d/32 fp16 V scales;
     the int8 (fp8) cache d int8 (e4m3) codes and one fp16 scale for each of K
-    and V."""
+    and V; the RK4V4-E8 cache d/2 bytes of nibbles and d/32 exponent bytes for
+    each of K and V."""
     if fmt == "k8v4":
         return d + 2 + d // 2 + 2 * (d // 32)
     if fmt in ("k8v8", "f8"):
         return 2 * (d + 2)
+    if fmt == "k4v4":  # RK4V4-E8: d/2 bytes of nibbles and d/32 exponent bytes for each of K and V
+        return 2 * (d // 2 + d // 32)
     if fmt == "bf16":
         return 4 * d  # bf16 K and V
     raise ValueError(f"unknown KV format {fmt!r}")
