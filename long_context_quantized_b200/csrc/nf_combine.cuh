@@ -1,5 +1,8 @@
 // nf_combine.cuh -- log-sum-exp merge of split-K attention partials.
 //
+// The splits come either as two arrays (o [splits][rows][d], lse
+// [splits][rows]) or packed, one slot per split holding its o rows and then
+// its lse values (the layout of the decode kernel's split partials).
 // One CTA of 8 warps per output row.  The splits are dealt round-robin to the
 // warps (so the loads of different splits are in flight together instead of
 // one after another); each lane owns 4 consecutive channels per 128 of the
@@ -16,9 +19,10 @@ constexpr int kCombineWarps = 8;
 constexpr int kCombineMaxDim = 1024;
 
 struct CombineParams {
-    const float *part_o;
-    const float *part_lse;
+    const float *part_o;    // split j's row r at part_o + j * o_stride + r * head_dim
+    const float *part_lse;  // split j's row r at part_lse + j * lse_stride + r
     int n_splits, rows, head_dim;
+    size_t o_stride, lse_stride;  // floats between consecutive splits
     float *out;
     float *out_lse;
 };
@@ -31,11 +35,11 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Combi
     pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int row = blockIdx.x;
-    const float *lse_col = p.part_lse + row;  // stride p.rows
+    const float *lse_col = p.part_lse + row;  // stride p.lse_stride
 
     // M = max_j lse_j
     float M = -INFINITY;
-    for (int j = threadIdx.x; j < p.n_splits; j += blockDim.x) M = fmaxf(M, lse_col[(size_t)j * p.rows]);
+    for (int j = threadIdx.x; j < p.n_splits; j += blockDim.x) M = fmaxf(M, lse_col[(size_t)j * p.lse_stride]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if (lane == 0) red[warp] = M;
@@ -60,10 +64,11 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Combi
         float ws = 0.f;
 #pragma unroll 4
         for (int j = warp; j < p.n_splits; j += kCombineWarps) {
-            const float w = ex2((lse_col[(size_t)j * p.rows] - M) * kLog2e);  // -inf -> 0
+            const float w = ex2((lse_col[(size_t)j * p.lse_stride] - M) * kLog2e);  // -inf -> 0
             ws += w;
             if (c < nchunk && w > 0.f) {
-                const float4 o = reinterpret_cast<const float4 *>(p.part_o + ((size_t)j * p.rows + row) * p.head_dim)[c];
+                const float4 o =
+                    reinterpret_cast<const float4 *>(p.part_o + (size_t)j * p.o_stride + (size_t)row * p.head_dim)[c];
                 acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
             }
         }

@@ -3,8 +3,9 @@
 A request's KV cache is split by position across the ranks of a process group.
 Each rank holds whole 256-token blocks of every sequence and computes decode
 attention of the (replicated) queries against its own keys: a partial output
-and log-sum-exp per query row.  One all-gather exchanges the partials, and
-every rank merges them with the log-sum-exp combine (``nf_attn_combine``).
+and log-sum-exp per query row, written into one packed slot (o rows, then the
+lse values).  One all-gather exchanges the slots, and every rank merges them
+with the log-sum-exp combine (``nf_attn_combine_packed``).
 The pages run one request per GPU; this is the multi-GPU form of their
 segment-at-a-time decode (page "標籤: vLLM", section 2: the KV cache is
 managed in segments by context length), with the flash-decoding merge across
@@ -85,58 +86,112 @@ def local_block_table(spec: ShardSpec, block_table: torch.Tensor) -> torch.Tenso
     return out
 
 
-def decode_partial(kv, q, spec: ShardSpec, local_bt: torch.Tensor, softmax_scale: float, workspace=None):
-    """This shard's partial decode attention: (o [B][n_q][H_q][128], lse
-    [B][n_q][H_q]) over its keys.  Sequences with no key here get o = 0 and
-    lse = -inf (they add nothing to the merge) without a kernel call."""
+def packed_views(slot: torch.Tensor, B: int, n_q: int, H_q: int, d: int = 128):
+    """(o [B][n_q][H_q][d], lse [B][n_q][H_q]) views of one packed split slot
+    (o rows first, then the lse values: the layout nf_attn_combine_packed
+    reads)."""
+    rows = B * n_q * H_q
+    return slot[:rows * d].view(B, n_q, H_q, d), slot[rows * d:rows * (d + 1)].view(B, n_q, H_q)
+
+
+def decode_partial_into(kv, q, spec: ShardSpec, local_bt: torch.Tensor, softmax_scale: float, slot: torch.Tensor,
+                        workspace: torch.Tensor):
+    """This shard's partial decode attention written into its packed slot:
+    o and lse over the shard's keys.  Sequences with no key here get o = 0
+    and lse = -inf (they add nothing to the merge)."""
     B, n_q, H_q, d = q.shape
-    dev = q.device
-    o = torch.zeros((B, n_q, H_q, d), dtype=torch.float32, device=dev)
-    lse = torch.full((B, n_q, H_q), float("-inf"), dtype=torch.float32, device=dev)
+    o, lse = packed_views(slot, B, n_q, H_q, d)
     active = [b for b in range(B) if spec.lengths[b] > 0]
+    if len(active) == B:
+        sl = torch.as_tensor(spec.lengths, dtype=torch.int32, device=q.device)
+        nf.nf_decode_attn(kv, q, local_bt, sl, spec.max_length, softmax_scale, spec.causal, o, lse, workspace)
+        return
+    o.zero_()
+    lse.fill_(float("-inf"))
     if not active:
-        return o, lse
-    idx = torch.as_tensor(active, dtype=torch.long, device=dev)
+        return
+    idx = torch.as_tensor(active, dtype=torch.long, device=q.device)
     q_a = q.index_select(0, idx).contiguous()
     bt_a = local_bt.index_select(0, idx).contiguous()
-    sl = torch.as_tensor([spec.lengths[b] for b in active], dtype=torch.int32, device=dev)
-    msl = max(spec.lengths[b] for b in active)
-    o_a = torch.empty((len(active), n_q, H_q, d), dtype=torch.float32, device=dev)
-    lse_a = torch.empty((len(active), n_q, H_q), dtype=torch.float32, device=dev)
-    if workspace is None:
-        ws = nf.nf_decode_attn_workspace_size(len(active), n_q, H_q, kv.num_kv_heads, msl)
-        workspace = torch.zeros(ws, dtype=torch.uint8, device=dev)
-    nf.nf_decode_attn(kv, q_a, bt_a, sl, msl, softmax_scale, spec.causal, o_a, lse_a, workspace)
+    sl = torch.as_tensor([spec.lengths[b] for b in active], dtype=torch.int32, device=q.device)
+    o_a = torch.empty((len(active), n_q, H_q, d), dtype=torch.float32, device=q.device)
+    lse_a = torch.empty((len(active), n_q, H_q), dtype=torch.float32, device=q.device)
+    nf.nf_decode_attn(kv, q_a, bt_a, sl, spec.max_length, softmax_scale, spec.causal, o_a, lse_a, workspace)
     o.index_copy_(0, idx, o_a)
     lse.index_copy_(0, idx, lse_a)
-    return o, lse
 
 
-def gather_partials(o: torch.Tensor, lse: torch.Tensor, group=None):
-    """All-gather every rank's partial: ([W][rows][d], [W][rows]) in rank order."""
+def decode_partial(kv, q, spec: ShardSpec, local_bt: torch.Tensor, softmax_scale: float, workspace=None):
+    """This shard's partial decode attention: (o [B][n_q][H_q][128], lse
+    [B][n_q][H_q]) over its keys (views of a fresh packed slot)."""
+    B, n_q, H_q, d = q.shape
+    slot = torch.empty(nf.nf_attn_packed_slot_floats(B * n_q * H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.zeros(nf.nf_decode_attn_workspace_size(B, n_q, H_q, kv.num_kv_heads,
+                                                                 max(1, spec.max_length)),
+                                dtype=torch.uint8, device=q.device)
+    decode_partial_into(kv, q, spec, local_bt, softmax_scale, slot, workspace)
+    return packed_views(slot, B, n_q, H_q, d)
+
+
+def gather_packed(slot: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather every rank's packed slot in one collective: [W][slot] in
+    rank order."""
     import torch.distributed as dist
     W = dist.get_world_size(group)
-    d = o.shape[-1]
-    o2 = o.reshape(-1, d).contiguous()
-    l2 = lse.reshape(-1).contiguous()
-    # outputs concatenated along dim 0 (the form every backend accepts), viewed per rank
-    part_o = torch.empty((W * o2.shape[0], d), dtype=o2.dtype, device=o2.device)
-    part_l = torch.empty((W * l2.shape[0],), dtype=l2.dtype, device=l2.device)
-    dist.all_gather_into_tensor(part_o, o2, group=group)
-    dist.all_gather_into_tensor(part_l, l2, group=group)
-    return part_o.view(W, -1, d), part_l.view(W, -1)
+    out = torch.empty((W * slot.numel(),), dtype=slot.dtype, device=slot.device)
+    dist.all_gather_into_tensor(out, slot.contiguous(), group=group)
+    return out.view(W, -1)
+
+
+class ShardedDecoder:
+    """Context-sharded decode attention of one shard plan, with its buffers
+    (the rank's packed slot, the gathered slots, the outputs and one decode
+    workspace) allocated once and reused for every layer and step."""
+
+    def __init__(self, spec: ShardSpec, batch: int, n_q: int, num_q_heads: int, num_kv_heads: int,
+                 device, group=None):
+        self.spec, self.group = spec, group
+        self.B, self.n_q, self.H_q = batch, n_q, num_q_heads
+        rows = batch * n_q * num_q_heads
+        self.rows = rows
+        slot = nf.nf_attn_packed_slot_floats(rows, 128)
+        self.slot = torch.empty(slot, dtype=torch.float32, device=device)
+        self.gathered = torch.empty((spec.world_size, slot), dtype=torch.float32, device=device)
+        self.out = torch.empty((batch, n_q, num_q_heads, 128), dtype=torch.float32, device=device)
+        self.out_lse = torch.empty((batch, n_q, num_q_heads), dtype=torch.float32, device=device)
+        ws = nf.nf_decode_attn_workspace_size(batch, n_q, num_q_heads, num_kv_heads, max(n_q, spec.max_length))
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
+
+    def __call__(self, kv, q, local_bt: torch.Tensor, softmax_scale: float):
+        """One layer: the local partial, one all-gather of the packed slots, the
+        merge; returns (out, out_lse) (this object's buffers) on every rank."""
+        decode_partial_into(kv, q, self.spec, local_bt, softmax_scale, self.slot, self.workspace)
+        if self.spec.world_size == 1:
+            o, lse = packed_views(self.slot, self.B, self.n_q, self.H_q)
+            return o, lse
+        import torch.distributed as dist
+        dist.all_gather_into_tensor(self.gathered.view(-1), self.slot, group=self.group)
+        nf.nf_attn_combine_packed(self.gathered, self.rows, self.out.view(self.rows, 128), self.out_lse.view(-1))
+        return self.out, self.out_lse
 
 
 def sharded_decode_attn(kv, q, spec: ShardSpec, local_bt: torch.Tensor, softmax_scale: float, group=None,
                         workspace=None):
     """Decode attention of q against the keys of all ranks' shards: the local
-    partial, one all-gather, and the merge.  Returns (out [B][n_q][H_q][128],
-    lse [B][n_q][H_q]) on every rank."""
-    o, lse = decode_partial(kv, q, spec, local_bt, softmax_scale, workspace)
+    partial, one all-gather of the packed partials, and the merge.  Returns
+    (out [B][n_q][H_q][128], lse [B][n_q][H_q]) on every rank."""
+    B, n_q, H_q, d = q.shape
+    slot = torch.empty(nf.nf_attn_packed_slot_floats(B * n_q * H_q, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.zeros(nf.nf_decode_attn_workspace_size(B, n_q, H_q, kv.num_kv_heads,
+                                                                 max(n_q, spec.max_length)),
+                                dtype=torch.uint8, device=q.device)
+    decode_partial_into(kv, q, spec, local_bt, softmax_scale, slot, workspace)
     if spec.world_size == 1:
-        return o, lse
-    part_o, part_l = gather_partials(o, lse, group)
-    out = torch.empty_like(part_o[0])
-    out_lse = torch.empty_like(part_l[0])
-    nf.nf_attn_combine(part_o, part_l, out, out_lse)
-    return out.reshape(o.shape), out_lse.reshape(lse.shape)
+        return packed_views(slot, B, n_q, H_q, d)
+    parts = gather_packed(slot, group)
+    out = torch.empty((B, n_q, H_q, d), dtype=torch.float32, device=q.device)
+    out_lse = torch.empty((B, n_q, H_q), dtype=torch.float32, device=q.device)
+    nf.nf_attn_combine_packed(parts, B * n_q * H_q, out.view(-1, d), out_lse.view(-1))
+    return out, out_lse

@@ -94,11 +94,19 @@ def _rank_main(rank, world, port, case, results):
                                             spec.causal)
                 o[b] = ob.reshape(w.n_q, w.num_q_heads, 128)
                 lse[b] = lb.reshape(w.n_q, w.num_q_heads)
-        part_o, part_l = sh.gather_partials(torch.from_numpy(o.astype(np.float32)),
-                                            torch.from_numpy(lse.astype(np.float32)))
-        assert part_o.shape == (world, rows, 128) and part_l.shape == (world, rows)
-        # rank order: this rank's own partial sits at its index
-        assert torch.equal(part_o[rank], torch.from_numpy(o.astype(np.float32)).reshape(rows, 128))
+        # the rank's packed slot (o rows, then lse), exchanged in one all-gather
+        import long_context_quantized_b200 as nf
+        slot = torch.zeros(nf.nf_attn_packed_slot_floats(rows, 128), dtype=torch.float32)
+        so, sl = sh.packed_views(slot, w.batch, w.n_q, w.num_q_heads)
+        so.copy_(torch.from_numpy(o.astype(np.float32)))
+        sl.copy_(torch.from_numpy(lse.astype(np.float32)))
+        parts = sh.gather_packed(slot)
+        assert parts.shape == (world, slot.numel())
+        # rank order: this rank's own slot sits at its index
+        assert torch.equal(parts[rank], slot)
+        views = [sh.packed_views(parts[r], w.batch, w.n_q, w.num_q_heads) for r in range(world)]
+        part_o = torch.stack([v[0].reshape(rows, 128) for v in views])
+        part_l = torch.stack([v[1].reshape(rows) for v in views])
         out, out_lse = oracle.combine(part_o.numpy().astype(np.float64), part_l.numpy().astype(np.float64))
         ref, ref_lse = oracle.decode_attn(pool, q, bt, list(w.seqlens), w.softmax_scale, w.causal)
         results[rank] = (float(np.abs(out - ref).max()), float(np.abs(out_lse - ref_lse).max()))
