@@ -8,6 +8,12 @@ the C ABI.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--kv-format k8v4|k8v8|f8|k4v4|bf16] [--impl ours|reference]
+                  [--sharded] [--replicas]
+
+At N > 1 (one process per GPU under torchrun) the step is the decode of one
+request split by context over the ranks (strong scaling: every rank decodes
+its own keys, one NCCL all-gather of packed partials and a merge per layer);
+--replicas runs N independent copies of the request instead.
 
 --workload prefill_chunk measures chunked-prefill attention instead: per layer
 the 1024-token chunk's append and nf_prefill_attn, reported as chunk tokens/s
@@ -342,6 +348,169 @@ def measure_e2e(gw, args, stream, device):
     return e2e_ms, h2d, d2h
 
 
+# ------------------------------------------------ context-sharded decode leg
+class ShardedWorkload:
+    """One rank's shard of the workload (long_context_quantized_b200.sharded):
+    a pool holding only this rank's blocks of every layer, the replicated
+    queries, and one ShardedDecoder (its packed slot, gather buffer and
+    workspace reused by every layer).  The step's appended tokens belong to
+    the last shard (every shard boundary lies at or before L - n_q), so only
+    the last rank appends."""
+
+    def __init__(self, w, fmt_name, device, world, rank, group=None):
+        import long_context_quantized_b200 as nf
+        from long_context_quantized_b200 import sharded
+        self.nf, self.w, self.dev = nf, w, device
+        self.fmt_name = fmt_name
+        fmt = {"k8v4": nf.NF_KV_K8V4, "k8v8": nf.NF_KV_K8V8, "f8": nf.NF_KV_F8, "k4v4": nf.NF_KV_K4V4,
+               "bf16": nf.NF_KV_BF16}[fmt_name]
+        self.spec = sharded.shard_plan(list(w.seqlens), w.n_q, world, w.causal)[rank]
+        self.local_bt = sharded.local_pool_table(self.spec, device)
+        n_local = max(1, sum(self.spec.n_blocks))
+        self.layers, self.q, self.knew, self.vnew = [], [], [], []
+        new_before = []  # local position of the first new token, per sequence (this rank holds them)
+        for b in range(w.batch):
+            pos = sharded.shard_positions(self.spec, b)
+            new_before.append(w.cached[b] - pos.start if (w.n_new and pos.stop > w.cached[b]) else None)
+        self.appends = w.n_new > 0 and all(x is not None for x in new_before)
+        self.before = torch.as_tensor([x or 0 for x in new_before], dtype=torch.int32, device=device)
+        for layer in range(w.layers):
+            kv = nf.KVLayer.empty(fmt, n_local, w.num_kv_heads, device=device, fill=0)
+            kn, vn = [], []
+            for b in range(w.batch):
+                pos = sharded.shard_positions(self.spec, b)
+                if not len(pos):
+                    continue
+                k, v = workloads.layer_kv(w, layer, b, device=device)
+                end = min(pos.stop, w.cached[b])
+                if end > pos.start:
+                    nf.nf_kv_append_quant(kv, k[None, pos.start:end].contiguous(), v[None, pos.start:end].contiguous(),
+                                          self.local_bt[b:b + 1], torch.zeros(1, dtype=torch.int32, device=device))
+                if self.appends:
+                    kn.append(k[w.cached[b]:pos.stop])
+                    vn.append(v[w.cached[b]:pos.stop])
+                del k, v
+            self.layers.append(kv)
+            if self.appends:
+                self.knew.append(torch.stack(kn).contiguous())
+                self.vnew.append(torch.stack(vn).contiguous())
+            self.q.append(workloads.layer_q(w, layer, device=device))
+        self.dec = sharded.ShardedDecoder(self.spec, w.batch, w.n_q, w.num_q_heads, w.num_kv_heads, device, group)
+        self.out_all = torch.empty((w.layers, w.batch, w.n_q, w.num_q_heads, 128), dtype=torch.float32, device=device)
+        self.lse_all = torch.empty((w.layers, w.batch, w.n_q, w.num_q_heads), dtype=torch.float32, device=device)
+        torch.cuda.synchronize()
+        assert nf.nf_get_device_error() == 0
+
+    def layer(self, i):
+        if self.appends:
+            self.nf.nf_kv_append_quant(self.layers[i], self.knew[i], self.vnew[i], self.local_bt, self.before)
+        self.dec(self.layers[i], self.q[i], self.local_bt, self.w.softmax_scale, self.out_all[i], self.lse_all[i])
+
+    def step(self):
+        for i in range(self.w.layers):
+            self.layer(i)
+
+    def local_decode_bytes(self):
+        per = workloads.kv_bytes_per_token_head(self.fmt_name)
+        return sum(self.spec.lengths) * self.w.num_kv_heads * per
+
+
+def sharded_main(args, w, ws, rank, local):
+    """The decode step of one request split by context over the ranks: every
+    rank decodes its own keys, the ranks exchange one packed partial per
+    layer (NCCL all-gather) and merge it.  Total work is fixed as N grows
+    (strong scaling); the step is timed eagerly (no CUDA graph around the
+    collectives) with CUDA events, max over ranks."""
+    import datetime
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    group = None
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    sw = ShardedWorkload(w, args.kv_format, device, ws, rank, group)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(3, args.warmup)):
+        sw.step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        sw.step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
+    if ws > 1:
+        dist.barrier()
+    err = sw.nf.nf_get_device_error()
+    assert err == 0, f"device error {err}"
+    tokens = w.kv_tokens_per_step()  # the whole request: every key once per layer, over all ranks
+    value = tokens / (ms / 1e3)
+    # this rank's decode launch alone (no exchange), back to back: the roofline
+    g = torch.cuda.CUDAGraph()
+    gs = torch.cuda.Stream(device=device)
+    from long_context_quantized_b200 import sharded
+    with torch.cuda.graph(g, stream=gs):
+        for i in range(w.layers):
+            sharded.decode_partial_into(sw.layers[i], sw.q[i], sw.spec, sw.local_bt, w.softmax_scale, sw.dec.slot,
+                                        sw.dec.workspace, sw.dec.seqlens)
+    dec_ms = time_graph(g, max(5, min(args.steps, 30)), 3, gs) / w.layers
+    del g
+    dec_ms = max_over_ranks(dec_ms, device)
+    peak, peak_kind = measured_peaks()
+    dec_bytes = sw.local_decode_bytes()
+    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    # end to end: every layer's q from pinned host memory, every layer's output back
+    h_q = [t.cpu().pin_memory() for t in sw.q]
+    h_out = torch.empty_like(sw.out_all, device="cpu").pin_memory()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        for i in range(w.layers):
+            sw.q[i].copy_(h_q[i], non_blocking=True)
+            sw.layer(i)
+        h_out.copy_(sw.out_all, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, device)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": DTYPES[args.kv_format], "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlens": list(w.seqlens), "n_q": w.n_q,
+                   "n_new": w.n_new, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "layers": w.layers,
+                   "kv_format": args.kv_format, "causal": w.causal,
+                   "parallelism": f"context split over {ws} GPU(s): per layer the local decode, one NCCL "
+                                  "all-gather of packed (o, lse) partials, nf_attn_combine_packed",
+                   "l2": "KV bytes per step %.1f MB > 126 MB L2" % (sw.local_decode_bytes() * ws * w.layers / 1e6),
+                   "timing": "eager step (no CUDA graph around the collectives), CUDA events, max over ranks"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "decode_kernel of one rank's shard (back to back, no exchange)",
+                     "peak_source": peak_kind, "bytes_per_launch": dec_bytes, "launch_us": dec_ms * 1e3},
+        "cpu_baseline": None,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_q),
+                "d2h_bytes_per_step": h_out.numel() * h_out.element_size()},
+        "gpu_launches": (w.layers * ((1 if sw.appends else 0) + 1 + (1 if ws > 1 else 0))) * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------- chunked prefill leg
 PREFILL_METRIC = "prefill chunk tokens/s through chunked-prefill attention over the K8/V4 cache (all layers)"
 PREFILL_UNIT = "tokens/s"
@@ -558,6 +727,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-others", action="store_true",
                     help="skip the other >= 64K workloads measured after the headline at N = 1")
+    ap.add_argument("--sharded", action="store_true",
+                    help="at N = 1: the context-sharded path (the default at N > 1)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="at N > 1: independent replicas of the whole request instead of the context split")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling only: run fewer layers than the workload has")
     args = ap.parse_args()
@@ -593,6 +766,9 @@ def main():
                 "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
+
+    if (ws > 1 and not args.replicas) or args.sharded:
+        return sharded_main(args, w, ws, rank, local)
 
     import long_context_quantized_b200 as nf
     if ws > 1:

@@ -75,6 +75,29 @@ def shard_plan(seqlens, n_q: int, world_size: int, causal: bool) -> list:
     return specs
 
 
+def shard_positions(spec: ShardSpec, b: int) -> range:
+    """Global key positions of sequence b held by this shard."""
+    start = BLOCK * spec.first_block[b]
+    return range(start, start + spec.lengths[b])
+
+
+def local_pool_table(spec: ShardSpec, device=None) -> torch.Tensor:
+    """Block table of a rank that stores only its own shard: sequence b's
+    n_blocks[b] blocks are local blocks off_b .. off_b + n_blocks[b] - 1 (off_b
+    the blocks of the sequences before it), so a pool of sum(n_blocks) blocks
+    holds the shard; local position p of sequence b (global position
+    BLOCK * first_block[b] + p) is in local block off_b + p // BLOCK.  Rows are
+    padded with -1."""
+    width = max(1, max(spec.n_blocks) if spec.n_blocks else 1)
+    out = torch.full((len(spec.n_blocks), width), -1, dtype=torch.int32)
+    off = 0
+    for b, n in enumerate(spec.n_blocks):
+        if n:
+            out[b, :n] = torch.arange(off, off + n, dtype=torch.int32)
+        off += n
+    return out.to(device) if device is not None else out
+
+
 def local_block_table(spec: ShardSpec, block_table: torch.Tensor) -> torch.Tensor:
     """The shard's rows of the block table: row b = block_table[b, first:first + n]
     (padded with -1), in the same block-id space as the given table."""
@@ -95,15 +118,16 @@ def packed_views(slot: torch.Tensor, B: int, n_q: int, H_q: int, d: int = 128):
 
 
 def decode_partial_into(kv, q, spec: ShardSpec, local_bt: torch.Tensor, softmax_scale: float, slot: torch.Tensor,
-                        workspace: torch.Tensor):
+                        workspace: torch.Tensor, seqlens: torch.Tensor = None):
     """This shard's partial decode attention written into its packed slot:
     o and lse over the shard's keys.  Sequences with no key here get o = 0
-    and lse = -inf (they add nothing to the merge)."""
+    and lse = -inf (they add nothing to the merge).  seqlens: the shard's
+    lengths as a device int32 tensor (made from spec.lengths when None)."""
     B, n_q, H_q, d = q.shape
     o, lse = packed_views(slot, B, n_q, H_q, d)
     active = [b for b in range(B) if spec.lengths[b] > 0]
     if len(active) == B:
-        sl = torch.as_tensor(spec.lengths, dtype=torch.int32, device=q.device)
+        sl = torch.as_tensor(spec.lengths, dtype=torch.int32, device=q.device) if seqlens is None else seqlens
         nf.nf_decode_attn(kv, q, local_bt, sl, spec.max_length, softmax_scale, spec.causal, o, lse, workspace)
         return
     o.zero_()
@@ -162,18 +186,30 @@ class ShardedDecoder:
         self.out_lse = torch.empty((batch, n_q, num_q_heads), dtype=torch.float32, device=device)
         ws = nf.nf_decode_attn_workspace_size(batch, n_q, num_q_heads, num_kv_heads, max(n_q, spec.max_length))
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
+        self.seqlens = torch.as_tensor(spec.lengths, dtype=torch.int32, device=device)  # once, not per call
 
-    def __call__(self, kv, q, local_bt: torch.Tensor, softmax_scale: float):
+    def __call__(self, kv, q, local_bt: torch.Tensor, softmax_scale: float, out=None, out_lse=None):
         """One layer: the local partial, one all-gather of the packed slots, the
-        merge; returns (out, out_lse) (this object's buffers) on every rank."""
-        decode_partial_into(kv, q, self.spec, local_bt, softmax_scale, self.slot, self.workspace)
+        merge into out / out_lse (fp32 [B][n_q][H_q][128] / [B][n_q][H_q];
+        this object's buffers when None).  Returns (out, out_lse) on every
+        rank.  With one rank the decode writes out directly."""
+        out = self.out if out is None else out
+        out_lse = self.out_lse if out_lse is None else out_lse
         if self.spec.world_size == 1:
+            if all(n > 0 for n in self.spec.lengths):
+                nf.nf_decode_attn(kv, q, local_bt, self.seqlens, self.spec.max_length, softmax_scale,
+                                  self.spec.causal, out, out_lse, self.workspace)
+                return out, out_lse
+            decode_partial_into(kv, q, self.spec, local_bt, softmax_scale, self.slot, self.workspace, self.seqlens)
             o, lse = packed_views(self.slot, self.B, self.n_q, self.H_q)
-            return o, lse
+            out.copy_(o)
+            out_lse.copy_(lse)
+            return out, out_lse
+        decode_partial_into(kv, q, self.spec, local_bt, softmax_scale, self.slot, self.workspace, self.seqlens)
         import torch.distributed as dist
         dist.all_gather_into_tensor(self.gathered.view(-1), self.slot, group=self.group)
-        nf.nf_attn_combine_packed(self.gathered, self.rows, self.out.view(self.rows, 128), self.out_lse.view(-1))
-        return self.out, self.out_lse
+        nf.nf_attn_combine_packed(self.gathered, self.rows, out.view(self.rows, 128), out_lse.view(-1))
+        return out, out_lse
 
 
 def sharded_decode_attn(kv, q, spec: ShardSpec, local_bt: torch.Tensor, softmax_scale: float, group=None,

@@ -64,3 +64,23 @@ def test_sharded_decoder_single_rank_equals_plain_call():
         o, lse = dec(g["kv"], g["q"], sharded.local_block_table(spec, bt), w.softmax_scale)
         torch.cuda.synchronize()
         assert torch.equal(o, g["out"]) and torch.equal(lse, g["lse"])
+
+
+def test_bench_sharded_path_single_rank_matches_the_oracle():
+    # the bench's shard-local pool (only this rank's blocks, local table) for
+    # one rank holding everything, with the step's appended tokens: the
+    # decoder's output per layer against the oracle
+    import bench
+    w = workloads.custom("bshard", cached=(3000,), n_new=4, n_q=4, num_q_heads=16, num_kv_heads=2, causal=True,
+                         q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, layers=2)
+    sw = bench.ShardedWorkload(w, "k8v4", torch.device("cuda", 0), 1, 0)
+    assert sw.appends
+    sw.step()
+    torch.cuda.synchronize()
+    assert nf.nf_get_device_error() == 0
+    for layer in range(w.layers):
+        kvin = [workloads.layer_kv(w, layer, b, device="cuda") for b in range(w.batch)]
+        bt = sw.local_bt.cpu().numpy()
+        pool, hs = oracle_pool(w, nf.NF_KV_K8V4, kvin, bt)
+        ref_o, ref_l = oracle_attention(w, pool, hs, sw.q[layer], bt)
+        check_attention(sw.out_all[layer], sw.lse_all[layer], ref_o, ref_l)

@@ -128,3 +128,22 @@ def test_sharded_partials_merge_to_the_whole(world, case):
         err_o, err_l = results[r]
         # fp32 exchange of fp64 partials: relative 2^-24 per value
         assert err_o < 1e-6 and err_l < 1e-5
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_local_pool_table_holds_each_shard_in_its_own_pool(world):
+    # a rank storing only its shard: local blocks are numbered from 0, and
+    # local position p of sequence b maps to global position first * 256 + p
+    seqlens = [5, 256, 1000, 4096 + 3]
+    specs = sharded.shard_plan(seqlens, 4, world, causal=True)
+    covered = [set() for _ in seqlens]
+    for s in specs:
+        t = sharded.local_pool_table(s)
+        ids = t[t >= 0].tolist()
+        assert sorted(ids) == list(range(sum(s.n_blocks)))   # every local block used once
+        for b in range(len(seqlens)):
+            pos = sharded.shard_positions(s, b)
+            assert len(pos) == s.lengths[b]
+            assert all(t[b, (p - pos.start) // 256] >= 0 for p in pos)
+            covered[b].update(pos)
+    assert [sorted(c) for c in covered] == [list(range(L)) for L in seqlens]
