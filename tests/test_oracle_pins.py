@@ -700,6 +700,9 @@ def _e8_vectors(n):
         for g in range(4):
             x[32 * g:32 * g + 32] *= 10.0 ** RNG.uniform(-30, 30)
         out.append(x.astype(np.float32))
+    for i in range(n // 8):  # subnormal groups: the exponent clamps at -126
+        x = RNG.standard_normal(128) * 10.0 ** RNG.uniform(-44, -37)
+        out.append(x.astype(np.float32))
     return out
 
 
