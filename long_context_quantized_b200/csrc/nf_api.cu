@@ -99,11 +99,11 @@ bool make_plan(int batch, int n_q, int H_q, int H_kv, int max_seqlen, int num_sm
     pl.nt = rows <= 8 ? 1 : 2;
     pl.n_rg = pl.nt == 1 ? 1 : (int)((rows + 15) / 16);
     if (pl.n_rg == 3) pl.n_rg = 4;  // 8 consumer warps split evenly over 1, 2 or 4 row groups
-    pl.ctas = num_sms;
+    pl.ctas = num_sms < nf::kMaxCtas ? num_sms : nf::kMaxCtas;
     pl.segments = batch * H_kv;
-    // one counter per segment, then one per partial slot (group counters of
-    // the two-step merge, indexed like the slots)
-    pl.ticket_bytes = ((size_t)(pl.segments + pl.ctas + pl.segments) * 4 + 255) / 256 * 256;
+    // per segment a ticket and a done counter, then one share flag per
+    // partial slot (indexed like the slots)
+    pl.ticket_bytes = ((size_t)(2 * pl.segments + pl.ctas + pl.segments) * 4 + 255) / 256 * 256;
     pl.slot_floats = (pl.rows * (nf::kHeadDim + 1) + 3) / 4 * 4;
     pl.partial_bytes = ((size_t)(pl.ctas + pl.segments) * pl.slot_floats * sizeof(float) + 255) / 256 * 256;
     return true;
@@ -397,7 +397,8 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
     p.out = out;
     p.out_lse = out_lse;
     p.tickets = static_cast<int32_t *>(workspace);
-    p.gtickets = p.tickets + pl.segments;
+    p.done = p.tickets + pl.segments;
+    p.claims = p.done + pl.segments;
     p.partials = reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.ticket_bytes);
     p.slot_floats = pl.slot_floats;
 

@@ -119,8 +119,10 @@ __device__ __forceinline__ void quant_row_e8(const float (&x)[4], int lane, uint
 }
 
 __global__ void __launch_bounds__(256) append_quant_kernel(const AppendParams p) {
-    pdl_wait();
+    // let the next kernel place its CTAs at once (it waits for this grid to
+    // complete before it reads what this one writes)
     pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const long long item = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long total = (long long)p.batch * p.n_new * p.num_kv_heads;

@@ -54,10 +54,13 @@
 // Merge: at the end of each piece the consumer warps merge through shared
 //   memory.  A segment owned by one CTA is written straight to out; otherwise
 //   each piece writes an (o, lse) partial and takes a ticket of the segment's
-//   counter; the CTA with the last ticket merges the partials into out and
-//   resets the counter (no CTA ever waits for another).  When that was the
-//   CTA's last piece, one bulk copy brings the segment's partials into the
-//   then idle stage ring.
+//   counter (acquire-release); the CTA with the last ticket merges the
+//   partials into out straight from L2 -- the weights of every (row, piece)
+//   first, then each output item in piece order -- and resets the counter
+//   (no CTA ever waits for another).  The CTAs take the ranges of the cut in
+//   reverse order, so the CTA placed last (on the SM the previous kernel's
+//   merging CTA leaves last) gets range 0, whose segment padding means fewer
+//   keys.
 // Every mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT
 // and the kernel runs to its end without further waits.
 #pragma once
@@ -73,13 +76,16 @@ constexpr int kConsumerWarps = 8;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxBatch = 256;
 constexpr int kMaxRows = 64;  // G * n_q per kv-head
+constexpr int kMaxCtas = 160;  // grid size cap: a segment has at most this many pieces
 // The running max of a row is raised when a tile's max exceeds it by more than
 // kLazy (log2 units); weights are 2^(x - max - kLazy) <= 1.
 constexpr float kLazy = 4.0f;
 // A CTA whose range crosses into a new segment pays an extra piece set-up and
-// merge; each segment is counted kSegPad chunks longer when the work is cut,
-// so such CTAs get that many fewer keys.
-constexpr int kSegPad = 64;
+// merge (about 5 us measured: the query digits, the piece's merge, its
+// ticket); each segment is counted kSegPad chunks (of about 0.15 us of
+// streaming each) longer when the work is cut, so such CTAs get that many
+// fewer keys.
+constexpr int kSegPad = 32;
 
 template <int FMT, int NT>
 struct Stage;
@@ -162,8 +168,9 @@ struct DecodeParams {
     int early_kv;      // read lengths, tables and older pool rows before the dependency wait
     float *out;      // [batch][n_q][H_q][128]
     float *out_lse;  // [batch][n_q][H_q] or null
-    int32_t *tickets;  // [batch * H_kv], zero between calls
-    int32_t *gtickets; // [gridDim.x + batch * H_kv], indexed like partial slots; zero between calls
+    int32_t *tickets;  // [batch * H_kv] ticket counters, zero between calls
+    int32_t *done;     // [batch * H_kv] done counters of the final merges, zero between calls
+    int32_t *claims;   // [gridDim.x + batch * H_kv] share flags, indexed like the slots; zero between calls
     float *partials;   // [gridDim.x + batch * H_kv] slots of slot_floats
     int slot_floats;   // rows * 128 (o) + rows (lse), rounded up to 4 floats
 };
@@ -176,8 +183,7 @@ struct DecodeSmem {
     static constexpr int kMergeO = kStagesBytes;                               // float [warp][NR][132]
     static constexpr int kMergeM = kMergeO + kConsumerWarps * NR * 132 * 4;    // float [warp][NR]
     static constexpr int kMergeL = kMergeM + kConsumerWarps * NR * 4;          // float [warp][NR]
-    static constexpr int kMergeLse = kMergeL + kConsumerWarps * NR * 4;        // float [kMaxRows]
-    static constexpr int kBars = kMergeLse + kMaxRows * 4;                     // u64 [2][stages] + 1
+    static constexpr int kBars = kMergeL + kConsumerWarps * NR * 4;            // u64 [2][stages] + 1
     static constexpr int kStageOk = kBars + (2 * ST::kStages + 1) * 8;         // int [stages]
     static constexpr int kSeqC = kStageOk + ST::kStages * 4;                   // int [kMaxBatch]
     static constexpr int kSeqL = kSeqC + kMaxBatch * 4;                        // int [kMaxBatch]
@@ -186,8 +192,9 @@ struct DecodeSmem {
     static constexpr int kBytes = kMisc + 16;
     static_assert(kBytes <= 232448, "shared memory per CTA");
     // final merge: (row, 4 channels) items of at most 8 rows (NT = 1) or kMaxRows
-    static constexpr int kMaxItems = (NT == 1 ? 8 : kMaxRows) * (kHeadDim / 4);
-    static_assert(kMergeM - kMergeO >= kMaxItems * 24, "final-merge state in the merge buffer");
+    // the final merge's weights (rows x pieces) in the merge buffer
+    static constexpr int kMergeFloats = (kMergeM - kMergeO) / 4;
+    static_assert(kMergeFloats >= kMaxCtas, "a row of final-merge weights in the merge buffer");
     static_assert(ST::kStride % 128 == 0, "stage alignment");
 };
 
@@ -210,12 +217,12 @@ __device__ __forceinline__ int v_channel_bf16(int m, int rho) {
 }
 // Walks a CTA's chunk range piece by piece (a piece = the part of one segment
 // that falls in the range).  Positions are in "cut" units: segment s spans
-// kSegPad padding units and then its C_b chunks; base[b] is the position of
+// `pad` padding units and then its C_b chunks; base[b] is the position of
 // sequence b's first segment.  Producer and consumers walk it identically.
 struct PieceWalker {
     const int *C;              // chunks per sequence
     const long long *base;     // position of sequence b's first segment
-    int H, batch;
+    int H, batch, pad;
     long long x, end;          // next position, end of the CTA range
     int b = 0;
     // current piece
@@ -224,10 +231,10 @@ struct PieceWalker {
     __device__ bool next() {
         while (x < end) {
             while (b + 1 <= batch && base[b + 1] <= x) ++b;
-            const long long span = kSegPad + (long long)C[b];
+            const long long span = pad + (long long)C[b];
             pb = b;
             ph = (int)((x - base[b]) / span);
-            s0 = base[b] + (long long)ph * span + kSegPad;
+            s0 = base[b] + (long long)ph * span + pad;
             xs = x > s0 ? x : s0;
             xe = min(s0 + C[b], end);
             if (xs < xe) {
@@ -250,6 +257,19 @@ __device__ __forceinline__ int stage_end(int cx, int cx_end) {
 
 __device__ __forceinline__ int owner_cta(long long x, long long W, int P) {
     return (int)(((x + 1) * P - 1) / W);
+}
+
+// Brings the query rows of (sequence b, kv-head h) into L2 -- thread t < rows
+// x lines per row takes one 128-byte line -- so that the piece that reads
+// them later finds them there.  No value is read into the thread.
+template <bool QF32>
+__device__ __forceinline__ void prefetch_q_rows(const DecodeParams &p, int b, int h, int t) {
+    constexpr int rb = kHeadDim * (QF32 ? 4 : 2) / 128;  // 128-byte lines per row
+    if (t < p.rows * rb) {
+        const int r = t / rb, j = r / p.group, gq = r % p.group;
+        const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
+        prefetch_l2(static_cast<const char *>(p.q) + row * kHeadDim * (QF32 ? 4 : 2) + (t % rb) * 128);
+    }
 }
 
 // Per-warp consumer state: the query fragments of the current (sequence,
@@ -612,201 +632,305 @@ __device__ __forceinline__ void decode_unit(WarpState<NT, QF32, FMT> &ws, const 
     }
 }
 
-// One round of the log-sum-exp merge for row r, channels 4c4..4c4+3: folds n
-// pieces' (o, lse) into the running (M, S, A) -- M the max lse so far, S the
-// sum of weights 2^((lse_i - M) log2 e), A the weighted sum of the o_i -- in
-// piece order, first raising M to the round's max (and rescaling S and A).
-// Piece i is the slot at ps + i * slot_floats: o at [r][128], lse at
-// lse_off + r.  SMEM: plain loads from shared memory; otherwise loads that
-// bypass L1 (the slots were written by other CTAs), kPB in flight at once.
-// The arithmetic is the same for both sources and any kPB (the pieces are
-// summed in order; kPB only batches the loads).
-template <bool SMEM, int kPB>
-__device__ __forceinline__ void merge_round(const float *ps, size_t slot_floats, int n, int r, int c4, int lse_off,
-                                            float &M, float &S, float4 &A) {
+// How long a CTA whose piece shares the final merge of its segment waits for
+// the segment's last piece before it leaves its share to the CTA that draws
+// the last ticket.  Far above the spread of the pieces' end times (a few
+// microseconds); it only comes into play when some CTA of the grid could not
+// be placed on an SM while the others wait.
+constexpr uint64_t kCoopWaitNs = 50000ull;
+
+// Share j of m of a segment's final merge: output items [j I / m, (j + 1) I /
+// m) of the I = rows x 32 items (row, 4 channels), each the sum over the n
+// pieces of w_k o_k, w_k = e^(lse_k - M) / sum_i e^(lse_i - M) with M the
+// row's largest lse.  slots: piece k's slot at slots + k * p.slot_floats (its
+// normalised o rows, then their lse), read from L2.  Threads 0 .. NTHR - 1,
+// named barrier BAR; sm: scratch of (NTHR / 32 + 2) kMaxCtas + 4 NTHR floats.
+// The items go in chunks of up to NTHR; in a chunk of c items thread t takes
+// item t % c and the pieces t / c, t / c + Q, ... (Q = NTHR / c), and the Q
+// partial sums are then added in order, so the arithmetic depends only on (n,
+// m, j, rows), not on which CTA merges the share.  A row no piece saw a key
+// of (every lse -inf) comes out as o = 0, lse = -inf.
+template <int NTHR, uint32_t BAR>
+__device__ __noinline__ void merge_share(const DecodeParams &p, const float *slots, int n, int rows, int j, int m,
+                                            float *sm, int b, int h) {
     constexpr float kLog2e = 1.4426950408889634f;
-    auto ld1 = [&](const float *a) { return SMEM ? *a : __ldcg(a); };
-    float Mr = M;
-    for (int i0 = 0; i0 < n; i0 += kPB) {
-        float l[kPB];
-#pragma unroll
-        for (int k = 0; k < kPB; ++k) l[k] = i0 + k < n ? ld1(ps + (size_t)(i0 + k) * slot_floats + lse_off + r) : -INFINITY;
-#pragma unroll
-        for (int k = 0; k < kPB; ++k) Mr = fmaxf(Mr, l[k]);
-    }
-    if (Mr == -INFINITY) return;
-    if (Mr > M && M != -INFINITY) {
-        const float a = ex2((M - Mr) * kLog2e);
-        S *= a;
-        A.x *= a; A.y *= a; A.z *= a; A.w *= a;
-    }
-    M = Mr;
-    for (int i0 = 0; i0 < n; i0 += kPB) {
-        float4 o[kPB];
-        float l[kPB];
-#pragma unroll
-        for (int k = 0; k < kPB; ++k) {
-            const float *sp = ps + (size_t)(i0 + k) * slot_floats;
-            if (i0 + k < n) {
-                const float4 *op = reinterpret_cast<const float4 *>(sp + r * kHeadDim) + c4;
-                o[k] = SMEM ? *op : __ldcg(op);
-                l[k] = ld1(sp + lse_off + r);
-            } else {
-                o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                l[k] = -INFINITY;
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < kPB; ++k) {
-            const float wk = l[k] == -INFINITY ? 0.f : ex2((l[k] - M) * kLog2e);
-            S += wk;
-            A.x = fmaf(wk, o[k].x, A.x);
-            A.y = fmaf(wk, o[k].y, A.y);
-            A.z = fmaf(wk, o[k].z, A.z);
-            A.w = fmaf(wk, o[k].w, A.w);
-        }
-    }
-}
-
-// Merges n partial slots -- slot i at src + i * stride floats -- of `rows`
-// rows, in rounds of `per_round` slots: into the slot dst (normalised o and
-// lse, the format of a piece's partial) when dst is not null, else into the
-// output rows of (sequence b, kv-head h).  Run by all consumer threads of the
-// CTA.  in_ring: the stage ring is idle, and each round's slots come into it
-// with bulk copies (one per slot unless the slots are consecutive); else they
-// stream from L2.  The rounds, and so the sums, are the same either way.
-// `state` holds the items' running (M, S, A) between rounds (24 bytes per
-// (row, 4 channels) item).
-template <int kPB = 16>
-__device__ __forceinline__ void merge_slots(const DecodeParams &p, const float *src, size_t stride, int n, int rows,
-                                         int per_round, bool in_ring, unsigned char *smem, float *state,
-                                         int item_cap, uint64_t *fin_bar, uint32_t &fin_phase, volatile int *misc,
-                                         float *dst, int b, int h) {
-    const int nthr = kConsumerWarps * 32, tid = threadIdx.x;
+    constexpr int NW = NTHR / 32, NJ = kMaxCtas / 32, KB = 4;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t sf = p.slot_floats;
     const int lse_off = rows * kHeadDim;
-    const uint32_t slot_bytes = (uint32_t)p.slot_floats * 4u;
-    const int n_items = rows * (kHeadDim / 4);
-    float4 *stA = reinterpret_cast<float4 *>(state);
-    float *stM = reinterpret_cast<float *>(stA + item_cap);
-    float *stS = stM + item_cap;
-    for (int it = tid; it < n_items; it += nthr) {
-        stA[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-        stM[it] = -INFINITY;
-        stS[it] = 0.f;
-    }
-    for (int i0 = 0; i0 < n; i0 += per_round) {
-        const int nr = min(per_round, n - i0);
-        const float *rsrc = src + (size_t)i0 * stride;
-        if (in_ring) {
-            if (tid == 0) {
-                // the ring's last reads (generic proxy) precede the copies' writes
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                // the slots were written with generic stores (by other CTAs, made
-                // visible to this thread by the ticket's release and the acquire
-                // fence, or by this CTA before the barrier that precedes this
-                // round); order them before the bulk copies' async-proxy reads
-                asm volatile("fence.proxy.async.global;" ::: "memory");
-                mbar_arrive_expect_tx(fin_bar, (uint32_t)nr * slot_bytes);
-                if (stride == (size_t)p.slot_floats)
-                    bulk_g2s(smem, rsrc, (uint32_t)nr * slot_bytes, fin_bar);
-                else
-                    for (int i = 0; i < nr; ++i) bulk_g2s(smem + (size_t)i * slot_bytes, rsrc + (size_t)i * stride, slot_bytes, fin_bar);
+    const int I = rows * (kHeadDim / 4);
+    const int i0 = (int)((long long)I * j / m), i1 = (int)((long long)I * (j + 1) / m);
+    float *wsm = sm;                                                       // [rows of the chunk][n]
+    float4 *red = reinterpret_cast<float4 *>(sm + (NW + 2) * kMaxCtas);  // [Q][c]
+    for (int c0 = i0; c0 < i1; c0 += NTHR) {
+        const int c = min(NTHR, i1 - c0), Q = NTHR / c;
+        const int r_lo = c0 / 32, nrr = (c0 + c - 1) / 32 - r_lo + 1;
+        const bool act = tid < Q * c;
+        const int it = c0 + (act ? tid % c : 0), q = act ? tid / c : 0;
+        const int r = it / 32, c4 = it % 32;
+        const float *src = slots + (size_t)r * kHeadDim + 4 * c4;
+        // the first pieces' o, in flight while the weights are worked out
+        float4 o[KB];
+#pragma unroll
+        for (int u = 0; u < KB; ++u) {
+            const int k = q + Q * u;
+            o[u] = act && k < n ? __ldcg(reinterpret_cast<const float4 *>(src + k * sf)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        // the weights of the chunk's rows: one warp per row, lane l holds pieces l + 32 i
+        for (int rr = warp; rr < nrr; rr += NW) {
+            const int rw = r_lo + rr;
+            float lv[NJ], w[NJ];
+            float mx = -INFINITY, s = 0.f;
+#pragma unroll
+            for (int i = 0; i < NJ; ++i) {
+                const int k = lane + 32 * i;
+                lv[i] = k < n ? __ldcg(slots + k * sf + lse_off + rw) : -INFINITY;
+                mx = fmaxf(mx, lv[i]);
             }
-            if (!misc[0] && !mbar_wait(fin_bar, fin_phase)) {
-                report(NF_DEVERR_TIMEOUT);
-                misc[0] = 1;
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+#pragma unroll
+            for (int i = 0; i < NJ; ++i) {
+                w[i] = lv[i] == -INFINITY ? 0.f : ex2((lv[i] - mx) * kLog2e);
+                s += w[i];
             }
-            fin_phase ^= 1u;
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+            const float inv = mx == -INFINITY ? 0.f : 1.0f / s;
+#pragma unroll
+            for (int i = 0; i < NJ; ++i)
+                if (lane + 32 * i < n) wsm[rr * n + lane + 32 * i] = w[i] * inv;
+            // the row's lse goes with the share that holds the row's first item
+            if (lane == 0 && p.out_lse && rw * 32 >= c0 && rw * 32 < c0 + c) {
+                const int jq = rw / p.group, gq = rw % p.group;
+                const size_t row = ((size_t)b * p.n_q + jq) * p.num_q_heads + (size_t)h * p.group + gq;
+                p.out_lse[row] = mx == -INFINITY ? -INFINITY : mx + logf(s);
+            }
         }
-        for (int it = tid; it < n_items; it += nthr) {
-            const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
-            float M = stM[it], S = stS[it];
-            float4 A = stA[it];
-            if (in_ring)
-                merge_round<true, kPB>(reinterpret_cast<const float *>(smem), p.slot_floats, nr, r, c4, lse_off, M, S, A);
-            else
-                merge_round<false, kPB>(rsrc, stride, nr, r, c4, lse_off, M, S, A);
-            stM[it] = M;
-            stS[it] = S;
-            stA[it] = A;
+        named_sync(BAR, NTHR);
+        // this thread's pieces, KB loads at a time
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *wr = wsm + (r - r_lo) * n;
+        for (int u0 = 0;; u0 += KB) {
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                const int k = q + Q * (u0 + u);
+                const float wk = act && k < n ? wr[k] : 0.f;
+                acc.x = fmaf(wk, o[u].x, acc.x);
+                acc.y = fmaf(wk, o[u].y, acc.y);
+                acc.z = fmaf(wk, o[u].z, acc.z);
+                acc.w = fmaf(wk, o[u].w, acc.w);
+            }
+            if (!act || q + Q * (u0 + KB) >= n) break;
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                const int k = q + Q * (u0 + KB + u);
+                o[u] = k < n ? __ldcg(reinterpret_cast<const float4 *>(src + k * sf)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
-        if (in_ring) named_sync(1, kConsumerWarps * 32);  // the ring is read before the next round's copy
-    }
-    // every read of the sources precedes the writes (dst may be the first source)
-    if (!in_ring) named_sync(1, kConsumerWarps * 32);
-    for (int it = tid; it < n_items; it += nthr) {
-        const int r = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4);
-        const float M = stM[it], S = stS[it];
-        float4 a = stA[it];
-        const float inv = M == -INFINITY ? 0.f : 1.0f / S;
-        a.x *= inv; a.y *= inv; a.z *= inv; a.w *= inv;
-        const float lse = M == -INFINITY ? -INFINITY : M + logf(S);
-        if (dst) {
-            reinterpret_cast<float4 *>(dst + r * kHeadDim)[c4] = a;
-            if (c4 == 0) dst[lse_off + r] = lse;
-        } else {
-            const int j = r / p.group, gq = r % p.group;
-            const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-            reinterpret_cast<float4 *>(p.out + row * kHeadDim)[c4] = a;
-            if (c4 == 0 && p.out_lse) p.out_lse[row] = lse;
+        if (act) red[q * c + tid % c] = acc;
+        named_sync(BAR, NTHR);
+        if (tid < c) {
+            float4 sum = red[tid];
+            for (int qq = 1; qq < Q; ++qq) {
+                const float4 v = red[qq * c + tid];
+                sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+            }
+            const int ri = (c0 + tid) / 32, ci = (c0 + tid) % 32;
+            const int jq = ri / p.group, gq = ri % p.group;
+            const size_t row = ((size_t)b * p.n_q + jq) * p.num_q_heads + (size_t)h * p.group + gq;
+            reinterpret_cast<float4 *>(p.out + row * kHeadDim)[ci] = sum;
         }
+        named_sync(BAR, NTHR);  // the scratch is free again
     }
 }
 
-// The end of a piece whose partial (o, lse) is already in its slot, run by the
-// kConsumerWarps * 32 consumer threads (threads 0 .. 255 of the CTA).  The
-// partials of a segment merge in one step when they fit one round of the
-// ring (ring_bytes); else in two: the last piece of each group of gp
-// consecutive pieces merges its group into the group's first slot, and the
-// last group merges the groups.  The grouping is fixed, so the sums do not
-// depend on which CTA finishes last.  in_ring: this was the CTA's last piece,
-// so the ring is idle and the merge may bring the partials into it.
-template <int kPB = 16>
-__device__ __forceinline__ void finish_segment_piece(const DecodeParams &p, int s_id, int first, int n_pieces,
-                                                     int ring_bytes, bool in_ring, unsigned char *ring, float *state,
-                                                     int item_cap, uint64_t *fin_bar, uint32_t &fin_phase,
-                                                     volatile int *misc, int rows, int b, int h) {
-    const uint32_t slot_bytes = (uint32_t)p.slot_floats * 4u;
-    const int gp = (int)((uint32_t)ring_bytes / slot_bytes);  // slots per ring round
-    const bool two_level = n_pieces > gp;
-    const int pi = (int)blockIdx.x - first;  // this piece's index in the segment
-    const int g0 = two_level ? pi / gp * gp : 0;
-    const int gn = two_level ? min(gp, n_pieces - g0) : n_pieces;
-    int *tk = two_level ? &p.gtickets[s_id + first + g0] : &p.tickets[s_id];
-    if (threadIdx.x == 0) {
-        int is_last = 0;
-        if (n_pieces > 1) {
-            // release: the CTA's partial writes (ordered before this thread
-            // by the barrier) become visible no later than the ticket
-            is_last = atomic_add_release(tk, 1) == gn - 1;
-            if (is_last) __threadfence();  // acquire: the other pieces' partials
-        }
-        misc[1] = is_last;
+// Merges the n partial slots of a segment -- slot k at src + k * sf floats:
+// its normalised o rows [rows][128], then their lse [rows] -- into the output
+// rows (row r of the kv-head's group at out + orow(r) * 128, lse at out_lse +
+// orow(r)), by threads 0 .. NTHR - 1 (named barrier BAR).  SMEM: the slots sit
+// in this CTA's shared memory; else they are read from L2 (the last ticket's
+// acquire made them visible).  Per row the weights w_k = e^(lse_k - M) /
+// sum_i e^(lse_i - M), M the largest lse, go to wsm (room for wcap floats, at
+// least n); then every (row, 4 channels) item sums w_k o_k in piece order:
+// the same arithmetic whichever source.  A row no piece saw a key of comes out
+// as o = 0, lse = -inf.  Rows go in passes of as many as wsm holds.
+struct OutRows {
+    float *out, *out_lse;
+    size_t base;  // row index of (b, query 0, first q-head of the group)
+    int group, n_q, num_q_heads;
+    __device__ size_t operator()(int r) const {
+        return base + (size_t)(r / group) * num_q_heads + r % group;
     }
-    named_sync(1, kConsumerWarps * 32);
-    if (misc[1]) {
-        // This CTA holds the last ticket of the segment (or of a group).
-        float *slot0 = p.partials + (size_t)(s_id + first) * p.slot_floats;
-        merge_slots<kPB>(p, slot0 + (size_t)g0 * p.slot_floats, p.slot_floats, gn, rows, gp, in_ring, ring, state,
-                    item_cap, fin_bar, fin_phase, misc, two_level ? slot0 + (size_t)g0 * p.slot_floats : nullptr,
-                    b, h);
-        if (threadIdx.x == 0) *tk = 0;
-        if (two_level) {
-            const int ng = (n_pieces + gp - 1) / gp;
-            named_sync(1, kConsumerWarps * 32);
-            if (threadIdx.x == 0) {
-                const int is_last = atomic_add_release(&p.tickets[s_id], 1) == ng - 1;
-                if (is_last) __threadfence();
-                misc[1] = is_last;
+};
+
+template <int NTHR, uint32_t BAR, bool SMEM>
+__device__ __noinline__ void merge_slots(const float *src, size_t sf, int n, int rows, float *wsm, int wcap,
+                                            const OutRows orow) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr int NW = NTHR / 32, NJ = kMaxCtas / 32, KB = 8;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lse_off = rows * kHeadDim;
+    const int rpp = min(rows, max(1, wcap / n));
+    for (int r0 = 0; r0 < rows; r0 += rpp) {
+        const int nr = min(rpp, rows - r0);
+        for (int rr = warp; rr < nr; rr += NW) {
+            const int r = r0 + rr;
+            float lv[NJ], w[NJ];
+            float mx = -INFINITY, s = 0.f;
+#pragma unroll
+            for (int i = 0; i < NJ; ++i) {
+                const int k = lane + 32 * i;
+                const float *a = src + k * sf + lse_off + r;
+                lv[i] = k < n ? (SMEM ? *a : __ldcg(a)) : -INFINITY;
+                mx = fmaxf(mx, lv[i]);
             }
-            named_sync(1, kConsumerWarps * 32);
-            if (misc[1]) {
-                merge_slots<kPB>(p, slot0, (size_t)gp * p.slot_floats, ng, rows, gp, in_ring, ring, state, item_cap,
-                            fin_bar, fin_phase, misc, nullptr, b, h);
-                if (threadIdx.x == 0) p.tickets[s_id] = 0;
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+#pragma unroll
+            for (int i = 0; i < NJ; ++i) {
+                w[i] = lv[i] == -INFINITY ? 0.f : ex2((lv[i] - mx) * kLog2e);
+                s += w[i];
             }
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+            const float inv = mx == -INFINITY ? 0.f : 1.0f / s;
+#pragma unroll
+            for (int i = 0; i < NJ; ++i)
+                if (lane + 32 * i < n) wsm[rr * n + lane + 32 * i] = w[i] * inv;
+            if (lane == 0 && orow.out_lse) orow.out_lse[orow(r)] = mx == -INFINITY ? -INFINITY : mx + logf(s);
         }
-        named_sync(1, kConsumerWarps * 32);
+        named_sync(BAR, NTHR);
+        for (int it = tid; it < nr * (kHeadDim / 4); it += NTHR) {
+            const int rr = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4), r = r0 + rr;
+            const float *wr = wsm + rr * n;
+            const float4 *op = reinterpret_cast<const float4 *>(src + (size_t)r * kHeadDim) + c4;
+            const size_t s4 = sf / 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k0 = 0; k0 < n; k0 += KB) {
+                float4 o[KB];
+#pragma unroll
+                for (int j = 0; j < KB; ++j)
+                    o[j] = k0 + j < n ? (SMEM ? op[(k0 + j) * s4] : __ldcg(op + (k0 + j) * s4))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < KB; ++j) {
+                    const float wk = k0 + j < n ? wr[k0 + j] : 0.f;
+                    acc.x = fmaf(wk, o[j].x, acc.x);
+                    acc.y = fmaf(wk, o[j].y, acc.y);
+                    acc.z = fmaf(wk, o[j].z, acc.z);
+                    acc.w = fmaf(wk, o[j].w, acc.w);
+                }
+            }
+            reinterpret_cast<float4 *>(orow.out + orow(r) * kHeadDim)[c4] = acc;
+        }
+        named_sync(BAR, NTHR);  // wsm is free again
+    }
+}
+
+// The end of a piece of a segment split over n > 1 CTAs, its partial already
+// in its slot, run by threads 0 .. NTHR - 1 after a barrier that orders the
+// slot writes before thread 0; no CTA waits for another.  The piece draws a
+// ticket of the segment's counter (acquire-release: it publishes the slot
+// and, for the last ticket, makes every other slot visible); the CTA with the
+// last ticket merges the segment's partials into out and resets the counter.
+// When this was the CTA's last piece (ring_idle: every stage consumed, no copy
+// in flight) and the n slots fit the ring, one bulk copy brings them into it
+// and the merge reads shared memory; else it reads them from L2.
+template <int NTHR, uint32_t BAR>
+__device__ __forceinline__ void finish_piece_single(const DecodeParams &p, int s_id, int first, int n, int rows,
+                                                    int b, int h, bool ring_idle, unsigned char *ring,
+                                                    uint32_t ring_bytes, uint64_t *fin_bar, uint32_t &fin_phase,
+                                                    float *wsm, int wcap, volatile int *misc) {
+    if (n < 2) return;
+    const float *slots = p.partials + (size_t)(s_id + first) * p.slot_floats;
+    const uint32_t bytes = (uint32_t)n * (uint32_t)p.slot_floats * 4u;
+    const bool in_ring = ring_idle && bytes <= ring_bytes;
+    if (threadIdx.x == 0) {
+        const bool last = atomic_add_acq_rel(&p.tickets[s_id], 1) == n - 1;
+        misc[1] = last;
+        if (last && in_ring && !misc[0]) {
+            // the ring's last reads (generic proxy) and the other CTAs' slot
+            // writes (visible through the ticket's acquire) precede the copy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            mbar_arrive_expect_tx(fin_bar, bytes);
+            bulk_g2s(ring, slots, bytes, fin_bar);
+        }
+    }
+    named_sync(BAR, NTHR);
+    if (!misc[1]) return;
+    bool from_ring = in_ring;
+    if (in_ring) {
+        if (!misc[0] && !mbar_wait(fin_bar, fin_phase)) {
+            report(NF_DEVERR_TIMEOUT);
+            misc[0] = 1;
+        }
+        fin_phase ^= 1u;
+        named_sync(BAR, NTHR);
+        from_ring = !misc[0];  // after a timeout the slots are read from L2 instead
+    }
+    const OutRows orow{p.out, p.out_lse, (size_t)b * p.n_q * p.num_q_heads + (size_t)h * p.group, p.group, p.n_q,
+                       p.num_q_heads};
+    if (from_ring)
+        merge_slots<NTHR, BAR, true>(reinterpret_cast<const float *>(ring), p.slot_floats, n, rows, wsm, wcap, orow);
+    else
+        merge_slots<NTHR, BAR, false>(slots, p.slot_floats, n, rows, wsm, wcap, orow);
+    if (threadIdx.x == 0) p.tickets[s_id] = 0;
+}
+
+// The end of a piece of a segment split over n > 1 CTAs, with the final merge
+// shared among the segment's CTAs (decode_tc_kernel, whose 32-row partials
+// are too large for one CTA to read quickly).  The partial (o, lse) is
+// already in its slot -- slot s_id + first + k, k the piece's index in the
+// segment -- and threads 0 .. NTHR - 1 run this after a barrier that orders the
+// slot writes before thread 0.  Each piece draws a ticket of the segment's counter
+// (acquire-release: it publishes the slot and, for the last ticket, makes
+// every other slot visible).  The final merge is cut into m shares, one per
+// participating piece: pieces 0 .. m - 1, whose CTAs have no further work (m
+// = n, or n - 1 when the last piece's CTA goes on into the next segment).
+//  - A participant waits, at most kCoopWaitNs, until all n pieces hold
+//    tickets, then claims its share (compare-and-swap on the share's flag) and
+//    merges it; one that times out leaves its share unclaimed.
+//  - The CTA with the last ticket, after its own share, claims and merges
+//    every share still unclaimed, so each share is merged exactly once
+//    whatever the timing.
+//  - Every piece then counts itself done; the last one returns the ticket,
+//    the done count and the share flags to zero for the next call.
+// No wait is unbounded, and a CTA that stops waiting loses nothing: its share
+// is swept by the last ticket's CTA.
+template <int NTHR, uint32_t BAR>
+__device__ __forceinline__ void finish_piece_coop(const DecodeParams &p, int s_id, int first, int k, int n, int m,
+                                                     float *sm, volatile int *misc, int rows, int b, int h) {
+    constexpr int NW = NTHR / 32;
+    if (n < 2) return;
+    const float *slots = p.partials + (size_t)(s_id + first) * p.slot_floats;
+    int *flag = p.claims + s_id + first;  // flag j: share j claimed
+    if (threadIdx.x == 0) {
+        const bool last = atomic_add_acq_rel(&p.tickets[s_id], 1) == n - 1;
+        bool ready = last;
+        if (!last && k < m) {
+            const uint64_t t0 = global_ns();
+            while (!(ready = ld_acquire(&p.tickets[s_id]) == n) && global_ns() - t0 < kCoopWaitNs) __nanosleep(100);
+        }
+        misc[1] = last;
+        misc[2] = ready && k < m && atomicCAS(&flag[k], 0, 1) == 0;
+    }
+    named_sync(BAR, NTHR);
+    if (misc[2]) merge_share<NTHR, BAR>(p, slots, n, rows, k, m, sm, b, h);
+    if (misc[1]) {
+        // the sweep: the shares nobody has claimed
+        int *won = reinterpret_cast<int *>(sm + (NW + 2) * kMaxCtas + 4 * NTHR);
+        if ((int)threadIdx.x < m) won[threadIdx.x] = atomicCAS(&flag[threadIdx.x], 0, 1) == 0;
+        named_sync(BAR, NTHR);
+        for (int j = 0; j < m; ++j)
+            if (won[j]) merge_share<NTHR, BAR>(p, slots, n, rows, j, m, sm, b, h);
+    }
+    named_sync(BAR, NTHR);  // this CTA's merge reads and writes precede its done count
+    if (threadIdx.x == 0 && atomic_add_acq_rel(&p.done[s_id], 1) == n - 1) {
+        p.tickets[s_id] = 0;
+        p.done[s_id] = 0;
+        for (int j = 0; j < m; ++j) flag[j] = 0;
     }
 }
 
@@ -889,10 +1013,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     // CTAs taking part: never more than there are chunks, so that every CTA
     // between a segment's first and last owner holds a piece of it
     const int P = (int)(W < (long long)gridDim.x ? W : (long long)gridDim.x);
-    const long long c_begin = (int)blockIdx.x < P ? W * blockIdx.x / P : 0;
-    const long long c_end = (int)blockIdx.x < P ? W * (blockIdx.x + 1) / P : 0;
+    // The CTAs take the ranges in reverse order: the highest-numbered CTA is
+    // the last one placed when the previous kernel's CTAs leave the SMs, so it
+    // starts last; range 0 opens a segment with its padding (fewer keys).
+    const int vb = (int)blockIdx.x < P ? P - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    const long long c_begin = vb < P ? W * vb / P : 0;
+    const long long c_end = vb < P ? W * (vb + 1) / P : 0;
 
-    PieceWalker walk{seqC, seqBase, H, p.batch, c_begin, c_end};
+    PieceWalker walk{seqC, seqBase, H, p.batch, kSegPad, c_begin, c_end};
 
     // =================================================================== producer
     // The whole warp walks the stages; its lanes hold a window of 32 block-table
@@ -981,7 +1109,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     }
 
     // =================================================================== consumers
-    if (p.early_kv) pdl_wait();
+    if (p.early_kv) {
+        // the first piece's query rows into L2 while the kernels before this
+        // one finish (no value is read before the wait)
+        PieceWalker w0 = walk;
+        if (w0.next()) prefetch_q_rows<QF32>(p, w0.pb, w0.ph, threadIdx.x);
+        pdl_wait();
+    }
     // segments of sequences with no valid key: o = 0, lse = -inf
     for (int s = blockIdx.x; s < p.batch * H; s += gridDim.x) {
         const int b = s / H, h = s % H;
@@ -999,7 +1133,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     const int rg = warp / CW, slot = warp % CW;
     const int g = lane >> 2, t = lane & 3;
     const int row0 = rg * NR;
-    float *sm_lse = reinterpret_cast<float *>(smem + SM::kMergeLse);
 
     WarpState<NT, QF32, FMT> ws;
     LaneOffsets lo;
@@ -1033,7 +1166,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
 
     int stage = 0;
     uint32_t phase = 0;      // parity of the ring's current round
-    uint32_t fin_phase = 0;  // parity of the final-merge copy barrier
+    uint32_t fin_phase = 0;  // parity of the final merge's copy barrier
     while (walk.next()) {
         const int b = walk.pb, h = walk.ph;
         const int L = seqC[b] ? p.seqlens[b] : 0;
@@ -1120,6 +1253,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                 if (lane == 0) qwsm[r] = s1 / 254.0f * p.scale_log2;
             }
             named_sync(1, kConsumerWarps * 32);
+            {
+                // the next piece's query rows into L2, ahead of its start
+                PieceWalker nx = walk;
+                if (nx.next()) prefetch_q_rows<QF32>(p, nx.pb, nx.ph, threadIdx.x);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int r = row0 + nt * 8 + g;
@@ -1202,64 +1340,59 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
         const int last = owner_cta(walk.s0 + seqC[b] - 1, W, P);
         const int n_pieces = last - first + 1;
         const int rows_here = p.rows;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            float l = ws.l_run[nt];
-            l += __shfl_xor_sync(0xffffffffu, l, 1);
-            l += __shfl_xor_sync(0xffffffffu, l, 2);
-            if (t == 0) {
-                sm_m[warp * NR + nt * 8 + g] = ws.m_run[nt];
-                sm_l[warp * NR + nt * 8 + g] = l;
-            }
-        }
-        named_sync(1, kConsumerWarps * 32);
-        // each lane derives its rows' factor f_w = 2^(m_w - M) / sum_v l_v 2^(m_v - M)
-        // from the group's (m, l) and writes f_w * acc_w to its warp's buffer
+        // every warp's raw accumulators, and its rows' (m, l), into shared memory
         {
             float *buf = sm_o + warp * NR * 132;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt) {
+                float l = ws.l_run[nt];
+                l += __shfl_xor_sync(0xffffffffu, l, 1);
+                l += __shfl_xor_sync(0xffffffffu, l, 2);
+                if (t == 0) {
+                    sm_m[warp * NR + nt * 8 + g] = ws.m_run[nt];
+                    sm_l[warp * NR + nt * 8 + g] = l;
+                }
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int rr = nt * 8 + 2 * t + e;
-                    float M = -INFINITY;
-                    for (int w = 0; w < CW; ++w) M = fmaxf(M, sm_m[(rg * CW + w) * NR + rr]);
-                    float f = 0.f;
-                    if (M != -INFINITY) {
-                        float ls = 0.f;
-                        for (int w = 0; w < CW; ++w)
-                            ls += sm_l[(rg * CW + w) * NR + rr] * ex2(sm_m[(rg * CW + w) * NR + rr] - M);
-                        f = ex2(sm_m[warp * NR + rr] - M) / ls;
-                        // the row's lse: weights were taken relative to m + kLazy
-                        if (slot == 0 && g == 0) sm_lse[row0 + rr] = (M + kLazy + log2f(ls)) * 0.69314718055994531f;
-                    } else if (slot == 0 && g == 0) {
-                        sm_lse[row0 + rr] = -INFINITY;
-                    }
 #pragma unroll
                     for (int m = 0; m < 8; ++m) {
                         const int c0 = V8 ? v_channel_k8v8(m, g) : K8 ? v_channel_k8v4(m, g) : v_channel_bf16(m, g);
                         const int c1 = V8 ? v_channel_k8v8(m, g + 8)
                                           : K8 ? v_channel_k8v4(m, g + 8) : v_channel_bf16(m, g + 8);
-                        buf[rr * 132 + c0] = ws.acc[m][nt][e] * f;
-                        buf[rr * 132 + c1] = ws.acc[m][nt][2 + e] * f;
+                        buf[rr * 132 + c0] = ws.acc[m][nt][e];
+                        buf[rr * 132 + c1] = ws.acc[m][nt][2 + e];
                     }
                 }
+            }
         }
         named_sync(1, kConsumerWarps * 32);
         {
-            // sum the row group's warp buffers, 4 channels per thread
+            // per (row, 4 channels): o = sum_w 2^(m_w - M) acc_w / sum_w 2^(m_w - M) l_w
+            // over the row group's warps (M = max_w m_w; the weights were taken
+            // relative to m + kLazy, so lse = (M + kLazy + log2 of the sum) ln 2)
             const int tid = slot * 32 + lane, nthr = CW * 32;
-            float *slotp = p.partials + (size_t)(s_id + blockIdx.x) * p.slot_floats;
+            float *slotp = p.partials + (size_t)(s_id + vb) * p.slot_floats;
             for (int idx = tid; idx < NR * (kHeadDim / 4); idx += nthr) {
                 const int rr = idx / (kHeadDim / 4), c4 = idx % (kHeadDim / 4);
                 const int r = row0 + rr;
                 if (r >= rows_here) continue;
+                float M = -INFINITY;
+                for (int w = 0; w < CW; ++w) M = fmaxf(M, sm_m[(rg * CW + w) * NR + rr]);
                 float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int w = 0; w < CW; ++w) {
-                    const float4 x = *reinterpret_cast<const float4 *>(sm_o + ((rg * CW + w) * NR + rr) * 132 + 4 * c4);
-                    o.x += x.x; o.y += x.y; o.z += x.z; o.w += x.w;
+                float lse = -INFINITY;
+                if (M != -INFINITY) {
+                    float den = 0.f;
+                    for (int w = 0; w < CW; ++w) {
+                        const float f = ex2(sm_m[(rg * CW + w) * NR + rr] - M);
+                        den = fmaf(f, sm_l[(rg * CW + w) * NR + rr], den);
+                        const float4 x = *reinterpret_cast<const float4 *>(sm_o + ((rg * CW + w) * NR + rr) * 132 + 4 * c4);
+                        o.x = fmaf(f, x.x, o.x); o.y = fmaf(f, x.y, o.y); o.z = fmaf(f, x.z, o.z); o.w = fmaf(f, x.w, o.w);
+                    }
+                    const float inv = 1.0f / den;
+                    o.x *= inv; o.y *= inv; o.z *= inv; o.w *= inv;
+                    lse = (M + kLazy + log2f(den)) * 0.69314718055994531f;
                 }
-                const float lse = sm_lse[r];
                 if (n_pieces == 1) {
                     const int j = r / p.group, gq = r % p.group;
                     const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
@@ -1272,8 +1405,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
             }
         }
         named_sync(1, kConsumerWarps * 32);
-        finish_segment_piece(p, s_id, first, n_pieces, NS * ST::kStride, walk.x >= walk.end, smem, sm_o,
-                             SM::kMaxItems, fin_bar, fin_phase, misc, rows_here, b, h);
+        PieceWalker rest = walk;
+        const bool more = rest.next();  // another piece follows: its stages may be in the ring
+        finish_piece_single<kConsumerWarps * 32, 1>(p, s_id, first, n_pieces, rows_here, b, h, !more, smem,
+                                                    NS * ST::kStride, fin_bar, fin_phase, sm_o, SM::kMergeFloats,
+                                                    misc);
     }
 }
 

@@ -40,7 +40,7 @@
 // behind the others' work.  Warp 16 is the TMA producer; warp 17 holds the
 // tensor memory and, on one thread, issues the MMAs from an event loop that
 // serves whichever of S and P.V is ready.  Warps 0-15 also encode the query
-// digits at each piece's start; warps 0-7 run the piece's merge.  Every
+// digits at each piece's start and run the segment's final merge.  Every
 // mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT and
 // every role runs to its end without further waits.
 #pragma once
@@ -59,8 +59,11 @@ constexpr int kDtStages = 4;
 constexpr int kDtPvN = 64;       // N of the P.V product: the rows, padded
 constexpr int kDtMaxRows = 32;   // rows per kv-head this kernel serves
 constexpr int kDtChunkTiles = kBlock / kChunk;
-// named barriers: 1 the merge (warps 0-7, inside finish_segment_piece), 2..5
-// the four warps of one row quarter, 6 all consumer warps
+// Segment padding of the work cut (see kSegPad): a piece's set-up and merge
+// cost about 4 us here, 12 chunks of this kernel's streaming.
+constexpr int kDtSegPad = 12;
+// named barriers: 2..5 the four warps of one row quarter, 6 all consumer
+// warps (also the final merge's)
 constexpr uint32_t kDtBarAll = 6;
 
 struct DtSmem {
@@ -77,7 +80,7 @@ struct DtSmem {
     static constexpr int kRed = kQw + 2 * kDtMaxRows * 4;   // float [4 quadrants][kDtMaxRows]: row maxima
     static constexpr int kRed2 = kRed + 4 * kDtMaxRows * 4; // float [4 quadrants][kDtMaxRows]: row sums
     static constexpr int kBars = kRed2 + 4 * kDtMaxRows * 4;
-    static constexpr int kNumBars = 2 * kDtStages + 10 + 2;
+    static constexpr int kNumBars = 2 * kDtStages + 10 + 1;
     static constexpr int kStageOk = kBars + kNumBars * 8;   // int [stages]
     static constexpr int kTmem = kStageOk + kDtStages * 4;  // u32
     static constexpr int kSeqC = (kTmem + 4 + 15) / 16 * 16;  // int [kMaxBatch]
@@ -87,8 +90,8 @@ struct DtSmem {
     static constexpr int kBytes = kMisc + 16;
     static_assert(kBytes <= 232448, "shared memory per CTA");
     static_assert(kStride % 1024 == 0 && kVh % 1024 == 0 && kP % 1024 == 0 && kQ % 1024 == 0, "swizzle atoms");
-    static constexpr int kMaxItems = kDtMaxRows * (kHeadDim / 4);  // final-merge items
-    static_assert(kMaxItems * 24 <= 2 * 32768, "final-merge state in the idle V' buffers");
+    // the final merge's scratch in the idle V' buffers
+    static_assert(2 * 32768 / 4 >= (kDtConsumers + 3) * kMaxCtas + 4 * kDtConsumers * 32, "final-merge scratch");
 };
 
 // End (exclusive, in chunks) of the tile that starts at chunk cx: at most 128
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DtSmem::kBars);
     uint64_t *full = bars, *empty = bars + NS;
     uint64_t *sfull = bars + 2 * NS, *sfree = sfull + 2, *pfull = sfree + 2;
-    uint64_t *pvdone = pfull + 2, *qfull = pvdone + 2, *fin_bar = qfull + 2, *drain = fin_bar + 1;
+    uint64_t *pvdone = pfull + 2, *qfull = pvdone + 2, *drain = qfull + 2;
     volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + DtSmem::kStageOk);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + DtSmem::kTmem);
     int *seqC = reinterpret_cast<int *>(smem + DtSmem::kSeqC);
@@ -251,7 +254,6 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             mbar_init(&pvdone[i], 1);
             mbar_init(&qfull[i], 1);
         }
-        mbar_init(fin_bar, 1);
         mbar_init(drain, 1);
         misc[0] = 0;
         misc[1] = 0;
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             long long acc = 0;
             for (int b = 0; b < p.batch; ++b) {
                 seqBase[b] = acc;
-                acc += seqC[b] ? (long long)(seqC[b] + kSegPad) * H : 0;
+                acc += seqC[b] ? (long long)(seqC[b] + kDtSegPad) * H : 0;
             }
             seqBase[p.batch] = acc;
         }
@@ -296,9 +298,11 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
     const uint32_t tmem = *tmem_slot;
     const long long W = seqBase[p.batch];
     const int P = (int)(W < (long long)gridDim.x ? W : (long long)gridDim.x);
-    const long long c_begin = (int)blockIdx.x < P ? W * blockIdx.x / P : 0;
-    const long long c_end = (int)blockIdx.x < P ? W * (blockIdx.x + 1) / P : 0;
-    PieceWalker walk{seqC, seqBase, H, p.batch, c_begin, c_end};
+    // ranges in reverse order of the CTAs (see decode_kernel)
+    const int vb = (int)blockIdx.x < P ? P - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    const long long c_begin = vb < P ? W * vb / P : 0;
+    const long long c_end = vb < P ? W * (vb + 1) / P : 0;
+    PieceWalker walk{seqC, seqBase, H, p.batch, kDtSegPad, c_begin, c_end};
 
     if (warp == kDtProducer) {
         // =============================================================== producer
@@ -461,7 +465,13 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         // key 32 q + lane of each tile (the lane of S) and channel lane 32 q +
         // lane of O^T; rows h HR .. h HR + HR - 1 of the softmax, P' and O^T; and
         // the 32 channels of V scale group h in the dequantisation.
-        if (p.early_kv) pdl_wait();
+        if (p.early_kv) {
+            // the first piece's query rows into L2 while the kernels before
+            // this one finish (no value is read before the wait)
+            PieceWalker w0 = walk;
+            if (w0.next()) prefetch_q_rows<QF32>(p, w0.pb, w0.ph, threadIdx.x);
+            pdl_wait();
+        }
         // segments of sequences with no valid key: o = 0, lse = -inf
         for (int s = blockIdx.x; s < p.batch * H; s += gridDim.x) {
             const int b = s / H, h = s % H;
@@ -480,7 +490,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         const int r0 = hq * HR;        // first row of this warp
         const uint32_t gbar = 2 + hq;  // named barrier of the 4 warps with these rows
         const int R = p.rows;
-        uint32_t kt = 0, pc = 0, fin_phase = 0;
+        uint32_t kt = 0, pc = 0;
         float l_part[HR], thr[HR], qw[HR];
         while (walk.next()) {
             const int b = walk.pb, h = walk.ph;
@@ -529,6 +539,11 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 fence_async_smem();
                 named_sync(kDtBarAll, kDtConsumers * 32);
                 if (threadIdx.x == 0) mbar_arrive(&qfull[pc & 1]);
+                {
+                    // the next piece's query rows into L2, ahead of its start
+                    PieceWalker nx = walk;
+                    if (nx.next()) prefetch_q_rows<QF32>(p, nx.pb, nx.ph, threadIdx.x);
+                }
             }
             // this warp's rows: their factors, empty running maxima and sums
 #pragma unroll
@@ -656,7 +671,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 tmem_wait_ld();
                 tc_fence_before();
                 const int ch = dt_channel(i);
-                float *slotp = p.partials + (size_t)(s_id + blockIdx.x) * p.slot_floats;
+                float *slotp = p.partials + (size_t)(s_id + vb) * p.slot_floats;
 #pragma unroll
                 for (int e = 0; e < HR; ++e) {
                     const int r = r0 + e;
@@ -676,10 +691,11 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 }
             }
             named_sync(kDtBarAll, kDtConsumers * 32);  // the piece's outputs are written
-            if (warp < kConsumerWarps)
-                finish_segment_piece<8>(p, s_id, first, n_pieces, DtSmem::kRingBytes, walk.x >= walk.end, smem,
-                                     reinterpret_cast<float *>(smem + DtSmem::kVh), DtSmem::kMaxItems, fin_bar,
-                                     fin_phase, misc, R, b, h);
+            const bool cont = W * (last + 1) / P > walk.s0 + seqC[b] + kDtSegPad;  // see decode_kernel
+            finish_piece_coop<kDtConsumers * 32, kDtBarAll>(p, s_id, first, vb - first, n_pieces,
+                                                               n_pieces - (cont ? 1 : 0),
+                                                               reinterpret_cast<float *>(smem + DtSmem::kVh), misc, R, b,
+                                                               h);
             named_sync(kDtBarAll, kDtConsumers * 32);  // the merge is done: its buffers are free again
             ++pc;
         }
