@@ -220,6 +220,19 @@ __device__ __forceinline__ int atomic_add_acq_rel(int *p, int v) {
     asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
 }
+// Reciprocal and base-2 logarithm, hardware approximations (relative error
+// about 2^-23 and absolute about 2^-22), for epilogues whose results only need
+// to lie well inside the output tolerance.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 // Load with acquire semantics at GPU scope (sees, and orders after, the
 // writes a release by another CTA published).
 __device__ __forceinline__ int ld_acquire(const int *p) {
@@ -236,6 +249,12 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 __device__ __forceinline__ uint4 lds128(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
+// 16-byte shared-memory load at a shared-window address.
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
 
 // Read-only 16-byte global load.
 __device__ __forceinline__ uint4 ldg16(const void *p) {

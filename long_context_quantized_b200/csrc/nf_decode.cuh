@@ -81,11 +81,11 @@ constexpr int kMaxCtas = 160;  // grid size cap: a segment has at most this many
 // kLazy (log2 units); weights are 2^(x - max - kLazy) <= 1.
 constexpr float kLazy = 4.0f;
 // A CTA whose range crosses into a new segment pays an extra piece set-up and
-// merge (about 5 us measured: the query digits, the piece's merge, its
-// ticket); each segment is counted kSegPad chunks (of about 0.15 us of
+// merge (about 3.5 us measured: the piece's merge, its ticket and the stall
+// of the stream meanwhile); each segment is counted kSegPad chunks (of about 0.15 us of
 // streaming each) longer when the work is cut, so such CTAs get that many
 // fewer keys.
-constexpr int kSegPad = 32;
+constexpr int kSegPad = 24;
 
 template <int FMT, int NT>
 struct Stage;
@@ -651,7 +651,7 @@ constexpr uint64_t kCoopWaitNs = 50000ull;
 // m, j, rows), not on which CTA merges the share.  A row no piece saw a key
 // of (every lse -inf) comes out as o = 0, lse = -inf.
 template <int NTHR, uint32_t BAR>
-__device__ __noinline__ void merge_share(const DecodeParams &p, const float *slots, int n, int rows, int j, int m,
+__device__ __forceinline__ void merge_share(const DecodeParams &p, const float *slots, int n, int rows, int j, int m,
                                             float *sm, int b, int h) {
     constexpr float kLog2e = 1.4426950408889634f;
     constexpr int NW = NTHR / 32, NJ = kMaxCtas / 32, KB = 4;
@@ -745,16 +745,21 @@ __device__ __noinline__ void merge_share(const DecodeParams &p, const float *slo
     }
 }
 
-// Merges the n partial slots of a segment -- slot k at src + k * sf floats:
-// its normalised o rows [rows][128], then their lse [rows] -- into the output
-// rows (row r of the kv-head's group at out + orow(r) * 128, lse at out_lse +
-// orow(r)), by threads 0 .. NTHR - 1 (named barrier BAR).  SMEM: the slots sit
-// in this CTA's shared memory; else they are read from L2 (the last ticket's
-// acquire made them visible).  Per row the weights w_k = e^(lse_k - M) /
-// sum_i e^(lse_i - M), M the largest lse, go to wsm (room for wcap floats, at
-// least n); then every (row, 4 channels) item sums w_k o_k in piece order:
-// the same arithmetic whichever source.  A row no piece saw a key of comes out
-// as o = 0, lse = -inf.  Rows go in passes of as many as wsm holds.
+// The final merge of a segment's n partial slots -- slot k at src + k * sf
+// floats: its normalised o rows [rows][128], then their lse [rows] -- into the
+// output rows (row r of the kv-head's group at out + orow(r) * 128, its lse at
+// out_lse + orow(r)), in two steps run by threads 0 .. NTHR - 1 (named barrier
+// BAR):
+//  merge_weights  per row r in [r0, r0 + nr), one warp per row: w_k = e^(lse_k
+//                 - M) / sum_i e^(lse_i - M) (M the row's largest lse) into
+//                 wsm[(r - r0) n + k], and the row's lse = M + ln sum; the lse
+//                 values come from L2 (the last ticket's acquire made them
+//                 visible);
+//  merge_items    every (row, 4 channels) item of those rows: sum_k w_k o_k in
+//                 piece order, o read from shared memory (SMEM, the slots
+//                 copied into this CTA) or from L2 -- the same arithmetic
+//                 either way.
+// A row no piece saw a key of comes out as o = 0, lse = -inf.
 struct OutRows {
     float *out, *out_lse;
     size_t base;  // row index of (b, query 0, first q-head of the group)
@@ -764,67 +769,68 @@ struct OutRows {
     }
 };
 
-template <int NTHR, uint32_t BAR, bool SMEM>
-__device__ __noinline__ void merge_slots(const float *src, size_t sf, int n, int rows, float *wsm, int wcap,
-                                            const OutRows orow) {
+template <int NTHR>
+__device__ __noinline__ void merge_weights(const float *src, size_t sf, int n, int rows, int r0, int nr, float *wsm,
+                                           const OutRows orow) {
     constexpr float kLog2e = 1.4426950408889634f;
-    constexpr int NW = NTHR / 32, NJ = kMaxCtas / 32, KB = 8;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = NTHR / 32, NJ = kMaxCtas / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int lse_off = rows * kHeadDim;
-    const int rpp = min(rows, max(1, wcap / n));
-    for (int r0 = 0; r0 < rows; r0 += rpp) {
-        const int nr = min(rpp, rows - r0);
-        for (int rr = warp; rr < nr; rr += NW) {
-            const int r = r0 + rr;
-            float lv[NJ], w[NJ];
-            float mx = -INFINITY, s = 0.f;
+    for (int rr = warp; rr < nr; rr += NW) {
+        const int r = r0 + rr;
+        float lv[NJ], w[NJ];
+        float mx = -INFINITY, s = 0.f;
 #pragma unroll
-            for (int i = 0; i < NJ; ++i) {
-                const int k = lane + 32 * i;
-                const float *a = src + k * sf + lse_off + r;
-                lv[i] = k < n ? (SMEM ? *a : __ldcg(a)) : -INFINITY;
-                mx = fmaxf(mx, lv[i]);
-            }
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-#pragma unroll
-            for (int i = 0; i < NJ; ++i) {
-                w[i] = lv[i] == -INFINITY ? 0.f : ex2((lv[i] - mx) * kLog2e);
-                s += w[i];
-            }
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
-            const float inv = mx == -INFINITY ? 0.f : 1.0f / s;
-#pragma unroll
-            for (int i = 0; i < NJ; ++i)
-                if (lane + 32 * i < n) wsm[rr * n + lane + 32 * i] = w[i] * inv;
-            if (lane == 0 && orow.out_lse) orow.out_lse[orow(r)] = mx == -INFINITY ? -INFINITY : mx + logf(s);
+        for (int i = 0; i < NJ; ++i) {
+            const int k = lane + 32 * i;
+            lv[i] = k < n ? __ldcg(src + k * sf + lse_off + r) : -INFINITY;
+            mx = fmaxf(mx, lv[i]);
         }
-        named_sync(BAR, NTHR);
-        for (int it = tid; it < nr * (kHeadDim / 4); it += NTHR) {
-            const int rr = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4), r = r0 + rr;
-            const float *wr = wsm + rr * n;
-            const float4 *op = reinterpret_cast<const float4 *>(src + (size_t)r * kHeadDim) + c4;
-            const size_t s4 = sf / 4;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k0 = 0; k0 < n; k0 += KB) {
-                float4 o[KB];
 #pragma unroll
-                for (int j = 0; j < KB; ++j)
-                    o[j] = k0 + j < n ? (SMEM ? op[(k0 + j) * s4] : __ldcg(op + (k0 + j) * s4))
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int d = 16; d > 0; d >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
 #pragma unroll
-                for (int j = 0; j < KB; ++j) {
-                    const float wk = k0 + j < n ? wr[k0 + j] : 0.f;
-                    acc.x = fmaf(wk, o[j].x, acc.x);
-                    acc.y = fmaf(wk, o[j].y, acc.y);
-                    acc.z = fmaf(wk, o[j].z, acc.z);
-                    acc.w = fmaf(wk, o[j].w, acc.w);
-                }
-            }
-            reinterpret_cast<float4 *>(orow.out + orow(r) * kHeadDim)[c4] = acc;
+        for (int i = 0; i < NJ; ++i) {
+            w[i] = lv[i] == -INFINITY ? 0.f : ex2((lv[i] - mx) * kLog2e);
+            s += w[i];
         }
-        named_sync(BAR, NTHR);  // wsm is free again
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) s += __shfl_xor_sync(0xffffffffu, s, d);
+        const float inv = mx == -INFINITY ? 0.f : 1.0f / s;
+#pragma unroll
+        for (int i = 0; i < NJ; ++i)
+            if (lane + 32 * i < n) wsm[rr * n + lane + 32 * i] = w[i] * inv;
+        if (lane == 0 && orow.out_lse) orow.out_lse[orow(r)] = mx == -INFINITY ? -INFINITY : mx + logf(s);
+    }
+}
+
+template <int NTHR, bool SMEM>
+__device__ __noinline__ void merge_items(const float *src, size_t sf, int n, int r0, int nr, const float *wsm,
+                                         const OutRows orow) {
+    constexpr int KB = 8;
+    const size_t s4 = sf / 4;
+    for (int it = threadIdx.x; it < nr * (kHeadDim / 4); it += NTHR) {
+        const int rr = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4), r = r0 + rr;
+        const float *wr = wsm + rr * n;
+        const float4 *op = reinterpret_cast<const float4 *>(src + (size_t)r * kHeadDim) + c4;
+        const uint32_t sop = SMEM ? smem_addr(op) : 0u;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k0 = 0; k0 < n; k0 += KB) {
+            float4 o[KB];
+#pragma unroll
+            for (int j = 0; j < KB; ++j)
+                o[j] = k0 + j >= n ? make_float4(0.f, 0.f, 0.f, 0.f)
+                       : SMEM      ? lds_f4(sop + (uint32_t)((k0 + j) * s4 * 16))
+                                   : __ldcg(op + (k0 + j) * s4);
+#pragma unroll
+            for (int j = 0; j < KB; ++j) {
+                const float wk = k0 + j < n ? wr[k0 + j] : 0.f;
+                acc.x = fmaf(wk, o[j].x, acc.x);
+                acc.y = fmaf(wk, o[j].y, acc.y);
+                acc.z = fmaf(wk, o[j].z, acc.z);
+                acc.w = fmaf(wk, o[j].w, acc.w);
+            }
+        }
+        reinterpret_cast<float4 *>(orow.out + orow(r) * kHeadDim)[c4] = acc;
     }
 }
 
@@ -835,8 +841,10 @@ __device__ __noinline__ void merge_slots(const float *src, size_t sf, int n, int
 // and, for the last ticket, makes every other slot visible); the CTA with the
 // last ticket merges the segment's partials into out and resets the counter.
 // When this was the CTA's last piece (ring_idle: every stage consumed, no copy
-// in flight) and the n slots fit the ring, one bulk copy brings them into it
-// and the merge reads shared memory; else it reads them from L2.
+// in flight) and the n slots fit the ring and every row's weights fit wsm
+// (wcap floats), one bulk copy brings the slots into the ring while the
+// weights are worked out from L2, and the items read shared memory; else the
+// merge reads L2, in passes of as many rows as wsm holds.
 template <int NTHR, uint32_t BAR>
 __device__ __forceinline__ void finish_piece_single(const DecodeParams &p, int s_id, int first, int n, int rows,
                                                     int b, int h, bool ring_idle, unsigned char *ring,
@@ -844,8 +852,9 @@ __device__ __forceinline__ void finish_piece_single(const DecodeParams &p, int s
                                                     float *wsm, int wcap, volatile int *misc) {
     if (n < 2) return;
     const float *slots = p.partials + (size_t)(s_id + first) * p.slot_floats;
-    const uint32_t bytes = (uint32_t)n * (uint32_t)p.slot_floats * 4u;
-    const bool in_ring = ring_idle && bytes <= ring_bytes;
+    const size_t sf = p.slot_floats;
+    const uint32_t bytes = (uint32_t)n * (uint32_t)sf * 4u;
+    const bool in_ring = ring_idle && bytes <= ring_bytes && rows * n <= wcap;
     if (threadIdx.x == 0) {
         const bool last = atomic_add_acq_rel(&p.tickets[s_id], 1) == n - 1;
         misc[1] = last;
@@ -860,22 +869,30 @@ __device__ __forceinline__ void finish_piece_single(const DecodeParams &p, int s
     }
     named_sync(BAR, NTHR);
     if (!misc[1]) return;
-    bool from_ring = in_ring;
+    const OutRows orow{p.out, p.out_lse, (size_t)b * p.n_q * p.num_q_heads + (size_t)h * p.group, p.group, p.n_q,
+                       p.num_q_heads};
     if (in_ring) {
+        merge_weights<NTHR>(slots, sf, n, rows, 0, rows, wsm, orow);  // while the copy is in flight
         if (!misc[0] && !mbar_wait(fin_bar, fin_phase)) {
             report(NF_DEVERR_TIMEOUT);
             misc[0] = 1;
         }
         fin_phase ^= 1u;
         named_sync(BAR, NTHR);
-        from_ring = !misc[0];  // after a timeout the slots are read from L2 instead
+        if (!misc[0])
+            merge_items<NTHR, true>(reinterpret_cast<const float *>(ring), sf, n, 0, rows, wsm, orow);
+        else  // after a timeout the slots are read from L2 instead
+            merge_items<NTHR, false>(slots, sf, n, 0, rows, wsm, orow);
+    } else {
+        const int rpp = min(rows, max(1, wcap / n));
+        for (int r0 = 0; r0 < rows; r0 += rpp) {
+            const int nr = min(rpp, rows - r0);
+            merge_weights<NTHR>(slots, sf, n, rows, r0, nr, wsm, orow);
+            named_sync(BAR, NTHR);
+            merge_items<NTHR, false>(slots, sf, n, r0, nr, wsm, orow);
+            named_sync(BAR, NTHR);  // wsm is free again
+        }
     }
-    const OutRows orow{p.out, p.out_lse, (size_t)b * p.n_q * p.num_q_heads + (size_t)h * p.group, p.group, p.n_q,
-                       p.num_q_heads};
-    if (from_ring)
-        merge_slots<NTHR, BAR, true>(reinterpret_cast<const float *>(ring), p.slot_floats, n, rows, wsm, wcap, orow);
-    else
-        merge_slots<NTHR, BAR, false>(slots, p.slot_floats, n, rows, wsm, wcap, orow);
     if (threadIdx.x == 0) p.tickets[s_id] = 0;
 }
 
@@ -1389,9 +1406,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                         const float4 x = *reinterpret_cast<const float4 *>(sm_o + ((rg * CW + w) * NR + rr) * 132 + 4 * c4);
                         o.x = fmaf(f, x.x, o.x); o.y = fmaf(f, x.y, o.y); o.z = fmaf(f, x.z, o.z); o.w = fmaf(f, x.w, o.w);
                     }
-                    const float inv = 1.0f / den;
+                    const float inv = __frcp_rn(den);
                     o.x *= inv; o.y *= inv; o.z *= inv; o.w *= inv;
-                    lse = (M + kLazy + log2f(den)) * 0.69314718055994531f;
+                    if (c4 == 0) lse = (M + kLazy + log2f(den)) * 0.69314718055994531f;
                 }
                 if (n_pieces == 1) {
                     const int j = r / p.group, gq = r % p.group;

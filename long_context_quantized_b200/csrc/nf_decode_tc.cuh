@@ -53,6 +53,8 @@
 namespace nf {
 
 constexpr int kDtConsumers = 16;                   // consumer warps
+constexpr int kDtRowGroups = kDtConsumers / 4;     // warps of one tensor-memory quadrant: row groups
+constexpr int kDtVG = 4 / kDtRowGroups;            // V scale groups (32 channels) per consumer warp
 constexpr int kDtThreads = (kDtConsumers + 2) * 32;  // + producer and MMA warps
 constexpr int kDtProducer = kDtConsumers, kDtMma = kDtConsumers + 1;
 constexpr int kDtStages = 4;
@@ -137,11 +139,11 @@ __device__ __forceinline__ void dt_wait(uint64_t *bar, uint32_t parity, volatile
 // HR consecutive tensor-memory columns of the warp's lanes (HR = 4 or 8)
 template <int HR>
 __device__ __forceinline__ void dt_ld(uint32_t taddr, uint32_t (&r)[HR]) {
-    if constexpr (HR == 8) tmem_ld8(taddr, r); else tmem_ld4(taddr, r);
+    if constexpr (HR == 16) tmem_ld16(taddr, r); else if constexpr (HR == 8) tmem_ld8(taddr, r); else tmem_ld4(taddr, r);
 }
 template <int HR>
 __device__ __forceinline__ void dt_st(uint32_t taddr, const uint32_t (&r)[HR]) {
-    if constexpr (HR == 8) tmem_st8(taddr, r); else tmem_st4(taddr, r);
+    if constexpr (HR == 16) tmem_st16(taddr, r); else if constexpr (HR == 8) tmem_st8(taddr, r); else tmem_st4(taddr, r);
 }
 
 // One consumer warp's softmax of one tile for its HR rows: scores from the S
@@ -217,7 +219,7 @@ template <int RP, bool QF32>
 __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
     static_assert(RP == 16 || RP == 32, "rows padded to 16 or 32");
     constexpr int NS = kDtStages;
-    constexpr int HR = RP / 4;                                    // rows per consumer warp
+    constexpr int HR = RP / kDtRowGroups;                         // rows per consumer warp
     constexpr int NSC = 2 * RP;                                   // S columns per buffer
     constexpr uint32_t kIdescS = umma_idesc_s8(128, NSC);
     constexpr uint32_t kIdescO = umma_idesc_f16(128, kDtPvN, true, true);
@@ -464,7 +466,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         // Warp (q, h) = (warp % 4, warp / 4): tensor-memory lane quadrant q, so
         // key 32 q + lane of each tile (the lane of S) and channel lane 32 q +
         // lane of O^T; rows h HR .. h HR + HR - 1 of the softmax, P' and O^T; and
-        // the 32 channels of V scale group h in the dequantisation.
+        // the kDtVG V scale groups h kDtVG .. of 32 channels in the dequantisation.
         if (p.early_kv) {
             // the first piece's query rows into L2 while the kernels before
             // this one finish (no value is read before the wait)
@@ -570,12 +572,17 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 const bool sok = !misc[0] && stage_ok[stage];
                 const bool kv_ok = sok && i < ntok && pos < L;
                 const bool fast = sok && ntok == 128 && tok0 + 128 <= all_see && R == RP;
-                uint4 nib = make_uint4(0, 0, 0, 0);
+                uint4 nib[kDtVG];
                 uint2 vsr = make_uint2(0, 0);
                 float ksv = 0.f;
+#pragma unroll
+                for (int gg = 0; gg < kDtVG; ++gg) nib[gg] = make_uint4(0, 0, 0, 0);
                 if (kv_ok) {
-                    nib = *reinterpret_cast<const uint4 *>(st + DtSmem::kStV + i * 64 +
-                                                           ((((uint32_t)hq) ^ (((uint32_t)i >> 1) & 3u)) << 4));
+#pragma unroll
+                    for (int gg = 0; gg < kDtVG; ++gg)
+                        nib[gg] = *reinterpret_cast<const uint4 *>(
+                            st + DtSmem::kStV + i * 64 +
+                            ((((uint32_t)(hq * kDtVG + gg)) ^ (((uint32_t)i >> 1) & 3u)) << 4));
                     vsr = *reinterpret_cast<const uint2 *>(st + DtSmem::kStVs + i * 8);
                     ksv = __half2float(*reinterpret_cast<const __half *>(st + DtSmem::kStKs + i * 2));
                 }
@@ -584,16 +591,18 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 const int ev = dt_v_exponent(vsr);
                 // ---- V' and P' buffers sb are free once the P.V of tile kt - 2 is done
                 if (kt >= 2) dt_wait(&pvdone[sb], ((kt >> 1) - 1) & 1, misc);
-                {
-                    // V' = code x scale / f: group hq of the key's row (block hq / 2,
-                    // 16-byte chunks 4 (hq % 2) .. + 3)
-                    unsigned char *vd = smem + DtSmem::kVh + sb * 32768 + (hq >> 1) * 16384 + i * 128;
+#pragma unroll
+                for (int gg = 0; gg < kDtVG; ++gg) {
+                    // V' = code x scale / f: group vg of the key's row (block vg / 2,
+                    // 16-byte chunks 4 (vg % 2) .. + 3)
+                    const int vg = hq * kDtVG + gg;
+                    unsigned char *vd = smem + DtSmem::kVh + sb * 32768 + (vg >> 1) * 16384 + i * 128;
                     const uint32_t sw = (uint32_t)i & 7u;
-                    const uint32_t sbits = (hq < 2 ? vsr.x : vsr.y) >> (16 * (hq & 1));
+                    const uint32_t sbits = (vg < 2 ? vsr.x : vsr.y) >> (16 * (vg & 1));
                     const float sg = __half2float(__ushort_as_half((unsigned short)(sbits & 0xFFFFu))) *
                                      __int_as_float((127 + 15 - ev) << 23);
                     const __half2 sv = __float2half2_rn(sg);
-                    const uint32_t wd[4] = {nib.x, nib.y, nib.z, nib.w};
+                    const uint32_t wd[4] = {nib[gg].x, nib[gg].y, nib[gg].z, nib[gg].w};
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         uint4 o;
@@ -601,7 +610,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                         o.y = h2_u32(__hmul2(nib_odd(wd[w]), sv));
                         o.z = h2_u32(__hmul2(nib_even(wd[w] >> 8), sv));
                         o.w = h2_u32(__hmul2(nib_odd(wd[w] >> 8), sv));
-                        const uint32_t cc = (uint32_t)(4 * (hq & 1) + w);
+                        const uint32_t cc = (uint32_t)(4 * (vg & 1) + w);
                         *reinterpret_cast<uint4 *>(vd + ((cc ^ sw) << 4)) = o;
                     }
                 }
@@ -629,14 +638,19 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 else
                     dt_softmax<HR, false>(d1, d2, qw, ksv, rmin, R, r0, thr, l_part, red, qd, lane, gbar, f, pk,
                                           kt > kfirst, ota, &pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
-                // P' row of this key, rows r0 .. r0 + HR - 1 (half or all of one 16-byte chunk)
+                // P' row of this key, rows r0 .. r0 + HR - 1 (half of one, one or two
+                // 16-byte chunks)
                 {
-                    unsigned char *pr = smem + DtSmem::kP + sb * 16384 + i * 128 +
-                                        ((((uint32_t)r0 >> 3) ^ ((uint32_t)i & 7u)) << 4) + (r0 & 7) * 2;
-                    if constexpr (HR == 8)
-                        *reinterpret_cast<uint4 *>(pr) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    else
-                        *reinterpret_cast<uint2 *>(pr) = make_uint2(pk[0], pk[1]);
+                    unsigned char *pr = smem + DtSmem::kP + sb * 16384 + i * 128;
+                    if constexpr (HR >= 8) {
+#pragma unroll
+                        for (int c = 0; c < HR / 8; ++c)
+                            *reinterpret_cast<uint4 *>(pr + (((((uint32_t)r0 >> 3) + c) ^ ((uint32_t)i & 7u)) << 4)) =
+                                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    } else {
+                        *reinterpret_cast<uint2 *>(pr + ((((uint32_t)r0 >> 3) ^ ((uint32_t)i & 7u)) << 4) +
+                                                   (r0 & 7) * 2) = make_uint2(pk[0], pk[1]);
+                    }
                 }
                 fence_async_smem();
                 tc_fence_before();
@@ -650,7 +664,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             const int last = owner_cta(walk.s0 + seqC[b] - 1, W, P);
             const int n_pieces = last - first + 1;
             {
-                float l_row[HR];
+                // row sums: the four warps' partial sums of each row
 #pragma unroll
                 for (int e = 0; e < HR; ++e) {
                     float v = l_part[e];
@@ -659,36 +673,40 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     if (lane == 0) red2[qd * kDtMaxRows + r0 + e] = v;
                 }
                 named_sync(gbar, 128);
-#pragma unroll
-                for (int e = 0; e < HR; ++e) {
-                    const int r = r0 + e;
-                    l_row[e] = (red2[r] + red2[kDtMaxRows + r]) + (red2[2 * kDtMaxRows + r] + red2[3 * kDtMaxRows + r]);
-                }
                 if (kt > kfirst) dt_wait(&pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
                 tc_fence_after();
-                uint32_t o[HR];
-                dt_ld<HR>(tmem + lane_base + kOCol + r0, o);
-                tmem_wait_ld();
-                tc_fence_before();
                 const int ch = dt_channel(i);
                 float *slotp = p.partials + (size_t)(s_id + vb) * p.slot_floats;
+                // O^T / l, four rows at a time (few live registers)
 #pragma unroll
-                for (int e = 0; e < HR; ++e) {
-                    const int r = r0 + e;
-                    if (r >= R) break;
-                    const bool any = thr[e] != -INFINITY;  // thr = m + kLazy: the weights were 2^(x - m - kLazy)
-                    const float val = any ? __uint_as_float(o[e]) / l_row[e] : 0.f;
-                    const float lse = any ? (thr[e] + log2f(l_row[e])) * 0.69314718055994531f : -INFINITY;
-                    if (n_pieces == 1) {
-                        const int j = r / p.group, gq = r % p.group;
-                        const size_t row = ((size_t)b * p.n_q + j) * p.num_q_heads + (size_t)h * p.group + gq;
-                        p.out[row * kHeadDim + ch] = val;
-                        if (i == e && p.out_lse) p.out_lse[row] = lse;
-                    } else {
-                        slotp[r * kHeadDim + ch] = val;
-                        if (i == e) slotp[R * kHeadDim + r] = lse;
+                for (int e0 = 0; e0 < HR; e0 += 4) {
+                    uint32_t o[4];
+                    tmem_ld4(tmem + lane_base + kOCol + r0 + e0, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = r0 + e0 + e;
+                        if (r >= R) break;
+                        const float l = (red2[r] + red2[kDtMaxRows + r]) + (red2[2 * kDtMaxRows + r] + red2[3 * kDtMaxRows + r]);
+                        const bool any = thr[e0 + e] != -INFINITY;  // thr = m + kLazy: the weights were 2^(x - m - kLazy)
+                        const float val = any ? __uint_as_float(o[e]) * rcp_approx(l) : 0.f;
+                        const size_t row = n_pieces == 1 ? ((size_t)b * p.n_q + r / p.group) * p.num_q_heads +
+                                                               (size_t)h * p.group + r % p.group
+                                                         : 0;
+                        if (n_pieces == 1)
+                            p.out[row * kHeadDim + ch] = val;
+                        else
+                            slotp[r * kHeadDim + ch] = val;
+                        if (i == e0 + e) {  // one lane per row: the row's lse
+                            const float lse = any ? (thr[e0 + e] + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
+                            if (n_pieces > 1)
+                                slotp[R * kHeadDim + r] = lse;
+                            else if (p.out_lse)
+                                p.out_lse[row] = lse;
+                        }
                     }
                 }
+                tc_fence_before();
             }
             named_sync(kDtBarAll, kDtConsumers * 32);  // the piece's outputs are written
             const bool cont = W * (last + 1) / P > walk.s0 + seqC[b] + kDtSegPad;  // see decode_kernel
