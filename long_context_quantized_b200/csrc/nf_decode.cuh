@@ -81,11 +81,11 @@ constexpr int kMaxCtas = 160;  // grid size cap: a segment has at most this many
 // kLazy (log2 units); weights are 2^(x - max - kLazy) <= 1.
 constexpr float kLazy = 4.0f;
 // A CTA whose range crosses into a new segment pays an extra piece set-up and
-// merge (about 3.5 us measured: the piece's merge, its ticket and the stall
-// of the stream meanwhile); each segment is counted kSegPad chunks (of about 0.15 us of
+// merge (about 3.5-4.5 us measured: the piece's merge, its ticket and the
+// stall of the stream meanwhile); each segment is counted kSegPad chunks (of about 0.15 us of
 // streaming each) longer when the work is cut, so such CTAs get that many
 // fewer keys.
-constexpr int kSegPad = 24;
+constexpr int kSegPad = 32;
 
 template <int FMT, int NT>
 struct Stage;
@@ -806,7 +806,7 @@ __device__ __noinline__ void merge_weights(const float *src, size_t sf, int n, i
 template <int NTHR, bool SMEM>
 __device__ __noinline__ void merge_items(const float *src, size_t sf, int n, int r0, int nr, const float *wsm,
                                          const OutRows orow) {
-    constexpr int KB = 8;
+    constexpr int KB = 16;
     const size_t s4 = sf / 4;
     for (int it = threadIdx.x; it < nr * (kHeadDim / 4); it += NTHR) {
         const int rr = it / (kHeadDim / 4), c4 = it % (kHeadDim / 4), r = r0 + rr;
