@@ -43,16 +43,25 @@ def _two_calls_match(w):
 
 
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
-    # ragged batch, causal MTP rows: segments split over a few CTAs, one-step merges
+    # ragged batch, causal MTP rows (32 per kv-head: the tcgen05 kernel):
+    # segments split over a few CTAs, their final merges shared among them
     w = workloads.custom("noalloc", cached=(3000, 1200), n_new=4, n_q=4, num_q_heads=16, num_kv_heads=2,
                          q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, causal=True)
     _two_calls_match(w)
 
 
-def test_noalloc_two_level_merge_on_two_calls():
+def test_noalloc_merge_from_the_ring_on_two_calls():
+    # four segments of about 37 pieces each, 8 rows: the partial slots fit the
+    # idle stage ring, so the last ticket's CTA merges them from its bulk copy
+    w = workloads.custom("noalloc_ring", cached=(20000,), n_q=1, num_q_heads=32, num_kv_heads=4,
+                         q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, causal=False)
+    _two_calls_match(w)
+
+
+def test_noalloc_merge_from_l2_on_two_calls():
     # one sequence and one kv-head: every CTA holds a piece of the single
-    # segment, more pieces than one merge round takes, so the group tickets
-    # and the two-step merge run -- the scratch state reused across calls
+    # segment, more partial slots than the stage ring holds, so the last
+    # ticket's CTA merges them from L2 -- the ticket state reused across calls
     w = workloads.custom("noalloc_long", cached=(60000,), n_q=1, num_q_heads=8, num_kv_heads=1,
                          q_dtype=torch.bfloat16, kv_in_dtype=torch.bfloat16, causal=False)
     _two_calls_match(w)
