@@ -89,12 +89,55 @@ struct DtSmem {
     static constexpr int kSeqL = kSeqC + kMaxBatch * 4;       // int [kMaxBatch]
     static constexpr int kSeqBase = kSeqL + kMaxBatch * 4;    // i64 [kMaxBatch + 1]
     static constexpr int kMisc = kSeqBase + (kMaxBatch + 1) * 8;  // int [4]
-    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kPiece = kMisc + 16;                     // DtPiece: the consumers' current piece
+    static constexpr int kWalk = kPiece + 32;                     // DtWalk: the consumers' walker
+    static constexpr int kBytes = kWalk + 144;
     static_assert(kBytes <= 232448, "shared memory per CTA");
     static_assert(kStride % 1024 == 0 && kVh % 1024 == 0 && kP % 1024 == 0 && kQ % 1024 == 0, "swizzle atoms");
     // the final merge's scratch in the idle V' buffers
     static_assert(2 * 32768 / 4 >= (kDtConsumers + 3) * kMaxCtas + 4 * kDtConsumers * 32, "final-merge scratch");
 };
+
+// A piece as the consumer warps see it: read from shared memory at its start,
+// so that the walker over the CTA's range holds no registers in the tile loop.
+struct DtPiece {
+    int valid, b, h, cx0, cx1;  // sequence, kv-head, chunks [cx0, cx1) of the segment
+    int first, n, m;            // the segment's first CTA, its pieces, the final merge's shares
+};
+// The consumers' walker over the CTA's range and the work cut it follows (W
+// chunks, padding included, over P CTAs), in shared memory.
+struct DtWalk {
+    PieceWalker w;
+    long long W;
+    int P;
+};
+static_assert(sizeof(DtWalk) <= 144, "walker slot");
+
+// Advances the consumers' walker (one thread, in shared memory) to the next
+// piece and describes it: n pieces of the segment from CTA `first`, m of them
+// on CTAs with no further work (see finish_piece_coop).
+__device__ __forceinline__ void dt_next_piece(DtWalk *dw, DtPiece *pd) {
+    PieceWalker *wk = &dw->w;
+    const long long W = dw->W;
+    const int P = dw->P;
+    if (!wk->next()) {
+        pd->valid = 0;
+        return;
+    }
+    const long long s0 = wk->s0;
+    const int C = wk->C[wk->pb];
+    const int first = owner_cta(s0, W, P), last = owner_cta(s0 + C - 1, W, P);
+    // the last piece's CTA goes on into the next segment (see decode_kernel)
+    const bool cont = W * (last + 1) / P > s0 + C + kDtSegPad;
+    pd->b = wk->pb;
+    pd->h = wk->ph;
+    pd->cx0 = (int)(wk->xs - s0);
+    pd->cx1 = (int)(wk->xe - s0);
+    pd->first = first;
+    pd->n = last - first + 1;
+    pd->m = last - first + 1 - (cont ? 1 : 0);
+    pd->valid = 1;
+}
 
 // End (exclusive, in chunks) of the tile that starts at chunk cx: at most 128
 // keys, never crossing a 256-key block.
@@ -130,6 +173,7 @@ __device__ __forceinline__ int dt_channel(int m) {
 
 // bounded waits shared by all roles: skipped once the kernel has aborted
 __device__ __forceinline__ void dt_wait(uint64_t *bar, uint32_t parity, volatile int *misc) {
+    if (mbar_try_wait(bar, parity)) return;
     if (!misc[0] && !mbar_wait_spin(bar, parity)) {
         report(NF_DEVERR_TIMEOUT);
         misc[0] = 1;
@@ -149,26 +193,44 @@ __device__ __forceinline__ void dt_st(uint32_t taddr, const uint32_t (&r)[HR]) {
 // One consumer warp's softmax of one tile for its HR rows: scores from the S
 // columns, the lazy running max (a collective step of the four warps of the
 // rows when some score exceeds it by kLazy), the weights times f into P'.
+// Each row keeps nthr = -max(m + kLazy, -FLT_MAX), FLT_MAX while the row has
+// no max yet, so one FMA per score gives the exponent y = x - m - kLazy (a
+// score's x = v c with v its integer dot product and c the row's and key's
+// factors) and y > 0 flags a score above the threshold.
 // FAST: every row sees every key of the tile (no mask).
 // When the max rises and O^T holds earlier tiles of the piece (has_o), the
 // rows' columns of O^T (taddr) are scaled once the last P.V is done (pv_bar).
 template <int HR, bool FAST>
-__device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint32_t (&d2)[HR], const float (&qw)[HR],
-                                           float ksv, int rmin, int R, int r0, float (&thr)[HR], float (&l_part)[HR],
+__device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint32_t (&d2)[HR], const float *qwr,
+                                           float ksv, int rmin, int R, int r0, float (&nthr)[HR], float (&l_part)[HR],
                                            float *red, int qd, int lane, uint32_t gbar, float f,
                                            uint32_t (&pk)[HR / 2], bool has_o, uint32_t taddr, uint64_t *pv_bar,
                                            uint32_t pv_parity, volatile int *misc) {
-    float x[HR];
-#pragma unroll
-    for (int e = 0; e < HR; ++e) {
-        const float v = (float)((int)d1[e] * 254 + (int)d2[e]) * (qw[e] * ksv);
-        x[e] = FAST ? v : ((r0 + e >= rmin && r0 + e < R) ? v : -INFINITY);
-    }
+    float c[HR], y[HR];
     bool raise = false;
 #pragma unroll
-    for (int e = 0; e < HR; ++e) raise |= x[e] > thr[e];  // true when no max yet and x finite
+    for (int e = 0; e < HR; e += 4) {
+        const float4 w = *reinterpret_cast<const float4 *>(qwr + e);  // (rows >= R: never used unmasked)
+        c[e] = w.x * ksv;
+        c[e + 1] = w.y * ksv;
+        c[e + 2] = w.z * ksv;
+        c[e + 3] = w.w * ksv;
+    }
+#pragma unroll
+    for (int e = 0; e < HR; ++e) {
+        const float v = (float)((int)d1[e] * 254 + (int)d2[e]);
+        y[e] = (FAST || (r0 + e >= rmin && r0 + e < R)) ? fmaf(v, c[e], nthr[e]) : -INFINITY;
+        raise |= y[e] > 0.f;  // true when no max yet and the score finite
+    }
     raise = bar_red_or(gbar, 128, raise);
     if (raise) {
+        // the scores themselves (y loses them while a row has no max)
+        float x[HR];
+#pragma unroll
+        for (int e = 0; e < HR; ++e) {
+            const float v = (float)((int)d1[e] * 254 + (int)d2[e]);
+            x[e] = (FAST || (r0 + e >= rmin && r0 + e < R)) ? v * c[e] : -INFINITY;
+        }
         // row maxima of the tile over its 128 keys: the four warps of these rows
 #pragma unroll
         for (int e = 0; e < HR; ++e) {
@@ -185,12 +247,13 @@ __device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint3
         for (int e = 0; e < HR; ++e) {
             const int r = r0 + e;
             const float tm = fmaxf(fmaxf(red[r], red[kDtMaxRows + r]), fmaxf(red[2 * kDtMaxRows + r], red[3 * kDtMaxRows + r]));
-            const float m_old = thr[e] - kLazy;  // -inf when none
+            const float m_old = nthr[e] == FLT_MAX ? -INFINITY : -nthr[e] - kLazy;
             const float m_new = fmaxf(m_old, tm);
             alpha[e] = m_old == -INFINITY ? 0.f : ex2(m_old - m_new);
             rescale |= m_new > m_old && m_old != -INFINITY;
             l_part[e] *= alpha[e];
-            thr[e] = m_new + kLazy;
+            nthr[e] = -fmaxf(m_new + kLazy, -FLT_MAX);
+            y[e] = x[e] + nthr[e];
         }
         if (rescale && has_o) {  // the same decision in the four warps of the rows
             dt_wait(pv_bar, pv_parity, misc);
@@ -204,11 +267,11 @@ __device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint3
             tmem_wait_st();
         }
     }
-    // weights 2^(x - m - kLazy) <= 1 (the row sum), times f into P'; a row
-    // with no max yet has only -inf scores, and the offset -FLT_MAX gives 0
+    // weights 2^y <= 1 (the row sum), times f into P'; a row with no max yet
+    // has only -inf scores, and y = -inf gives 0
 #pragma unroll
     for (int e = 0; e < HR; e += 2) {
-        const float p0 = ex2(x[e] - fmaxf(thr[e], -FLT_MAX)), p1 = ex2(x[e + 1] - fmaxf(thr[e + 1], -FLT_MAX));
+        const float p0 = ex2(y[e]), p1 = ex2(y[e + 1]);
         l_part[e] += p0;
         l_part[e + 1] += p1;
         pk[e / 2] = pack_f16(p0 * f, p1 * f);
@@ -467,11 +530,19 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         // key 32 q + lane of each tile (the lane of S) and channel lane 32 q +
         // lane of O^T; rows h HR .. h HR + HR - 1 of the softmax, P' and O^T; and
         // the kDtVG V scale groups h kDtVG .. of 32 channels in the dequantisation.
+        DtPiece *pd = reinterpret_cast<DtPiece *>(smem + DtSmem::kPiece);
+        DtWalk *wk = reinterpret_cast<DtWalk *>(smem + DtSmem::kWalk);
+        if (threadIdx.x == 0) {
+            wk->w = walk;
+            wk->W = W;
+            wk->P = P;
+            dt_next_piece(wk, pd);
+        }
+        named_sync(kDtBarAll, kDtConsumers * 32);
         if (p.early_kv) {
             // the first piece's query rows into L2 while the kernels before
             // this one finish (no value is read before the wait)
-            PieceWalker w0 = walk;
-            if (w0.next()) prefetch_q_rows<QF32>(p, w0.pb, w0.ph, threadIdx.x);
+            if (pd->valid) prefetch_q_rows<QF32>(p, pd->b, pd->h, threadIdx.x);
             pdl_wait();
         }
         // segments of sequences with no valid key: o = 0, lse = -inf
@@ -493,9 +564,11 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         const uint32_t gbar = 2 + hq;  // named barrier of the 4 warps with these rows
         const int R = p.rows;
         uint32_t kt = 0, pc = 0;
-        float l_part[HR], thr[HR], qw[HR];
-        while (walk.next()) {
-            const int b = walk.pb, h = walk.ph;
+        float l_part[HR], nthr[HR];
+        while (true) {
+            const DtPiece pce = *pd;
+            if (!pce.valid) break;
+            const int b = pce.b, h = pce.h;
             const int L = seqL[b];
             // ---- query digits of (b, h): q ~= s (d1 + d2 / 254), s = max|q| / 127;
             // digit row r (d1) and RP + r (d2) of the K-major B operand of S
@@ -541,25 +614,29 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 fence_async_smem();
                 named_sync(kDtBarAll, kDtConsumers * 32);
                 if (threadIdx.x == 0) mbar_arrive(&qfull[pc & 1]);
-                {
-                    // the next piece's query rows into L2, ahead of its start
-                    PieceWalker nx = walk;
-                    if (nx.next()) prefetch_q_rows<QF32>(p, nx.pb, nx.ph, threadIdx.x);
+                if (warp == 0) {
+                    // the next piece into the slot (every consumer warp has read
+                    // this one), and its query rows into L2 ahead of its start
+                    if (lane == 0) dt_next_piece(wk, pd);
+                    __syncwarp();
+                    if (pd->valid)
+                        for (int t = lane; t < R * 4; t += 32) prefetch_q_rows<QF32>(p, pd->b, pd->h, t);
                 }
             }
-            // this warp's rows: their factors, empty running maxima and sums
+            // this warp's rows: empty running maxima and sums (the rows' factors
+            // are read from qw_sm at each tile)
 #pragma unroll
             for (int e = 0; e < HR; ++e) {
-                qw[e] = r0 + e < R ? qw_sm[(pc & 1) * kDtMaxRows + r0 + e] : 0.f;
-                thr[e] = -INFINITY;
+                nthr[e] = FLT_MAX;
                 l_part[e] = 0.f;
             }
+            const float *qwr = qw_sm + (pc & 1) * kDtMaxRows + r0;
             // causal: key position pos is seen by rows r >= (pos - (L - n_q)) * G
             const int causal_base = p.causal ? L - p.n_q : 0x7fffffff;
             const int all_see = p.causal ? L - p.n_q + 1 : L;  // keys every row sees
             const uint32_t kfirst = kt;
-            const int cx1 = (int)(walk.xe - walk.s0);
-            for (int cx = (int)(walk.xs - walk.s0); cx < cx1; ++kt) {
+            const int cx1 = pce.cx1;
+            for (int cx = pce.cx0; cx < cx1; ++kt) {
                 const int ce = dt_tile_end(cx, cx1);
                 const int tok0 = cx * kChunk, ntok = (ce - cx) * kChunk;
                 cx = ce;
@@ -569,7 +646,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 // then the stage is released
                 dt_wait(&full[stage], (kt / NS) & 1, misc);
                 const int pos = tok0 + i;
-                const bool sok = !misc[0] && stage_ok[stage];
+                const bool sok = stage_ok[stage] != 0;  // (garbage after an abort is never used)
                 const bool kv_ok = sok && i < ntok && pos < L;
                 const bool fast = sok && ntok == 128 && tok0 + 128 <= all_see && R == RP;
                 uint4 nib[kDtVG];
@@ -633,10 +710,10 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 uint32_t pk[HR / 2];
                 const uint32_t ota = tmem + lane_base + kOCol + r0;
                 if (fast)
-                    dt_softmax<HR, true>(d1, d2, qw, ksv, rmin, R, r0, thr, l_part, red, qd, lane, gbar, f, pk,
+                    dt_softmax<HR, true>(d1, d2, qwr, ksv, rmin, R, r0, nthr, l_part, red, qd, lane, gbar, f, pk,
                                          kt > kfirst, ota, &pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
                 else
-                    dt_softmax<HR, false>(d1, d2, qw, ksv, rmin, R, r0, thr, l_part, red, qd, lane, gbar, f, pk,
+                    dt_softmax<HR, false>(d1, d2, qwr, ksv, rmin, R, r0, nthr, l_part, red, qd, lane, gbar, f, pk,
                                           kt > kfirst, ota, &pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
                 // P' row of this key, rows r0 .. r0 + HR - 1 (half of one, one or two
                 // 16-byte chunks)
@@ -660,9 +737,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
 
             // ---- end of the piece: O^T / l into out (one piece) or the partial slot
             const int s_id = b * H + h;
-            const int first = owner_cta(walk.s0, W, P);
-            const int last = owner_cta(walk.s0 + seqC[b] - 1, W, P);
-            const int n_pieces = last - first + 1;
+            const int first = pce.first, n_pieces = pce.n;
             {
                 // row sums: the four warps' partial sums of each row
 #pragma unroll
@@ -688,7 +763,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                         const int r = r0 + e0 + e;
                         if (r >= R) break;
                         const float l = (red2[r] + red2[kDtMaxRows + r]) + (red2[2 * kDtMaxRows + r] + red2[3 * kDtMaxRows + r]);
-                        const bool any = thr[e0 + e] != -INFINITY;  // thr = m + kLazy: the weights were 2^(x - m - kLazy)
+                        const bool any = nthr[e0 + e] != FLT_MAX;  // nthr = -(m + kLazy): the weights were 2^(x - m - kLazy)
                         const float val = any ? __uint_as_float(o[e]) * rcp_approx(l) : 0.f;
                         const size_t row = n_pieces == 1 ? ((size_t)b * p.n_q + r / p.group) * p.num_q_heads +
                                                                (size_t)h * p.group + r % p.group
@@ -698,7 +773,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                         else
                             slotp[r * kHeadDim + ch] = val;
                         if (i == e0 + e) {  // one lane per row: the row's lse
-                            const float lse = any ? (thr[e0 + e] + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
+                            const float lse = any ? (lg2_approx(l) - nthr[e0 + e]) * 0.69314718055994531f : -INFINITY;
                             if (n_pieces > 1)
                                 slotp[R * kHeadDim + r] = lse;
                             else if (p.out_lse)
@@ -709,9 +784,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 tc_fence_before();
             }
             named_sync(kDtBarAll, kDtConsumers * 32);  // the piece's outputs are written
-            const bool cont = W * (last + 1) / P > walk.s0 + seqC[b] + kDtSegPad;  // see decode_kernel
-            finish_piece_coop<kDtConsumers * 32, kDtBarAll>(p, s_id, first, vb - first, n_pieces,
-                                                               n_pieces - (cont ? 1 : 0),
+            finish_piece_coop<kDtConsumers * 32, kDtBarAll>(p, s_id, first, vb - first, n_pieces, pce.m,
                                                                reinterpret_cast<float *>(smem + DtSmem::kVh), misc, R, b,
                                                                h);
             named_sync(kDtBarAll, kDtConsumers * 32);  // the merge is done: its buffers are free again
