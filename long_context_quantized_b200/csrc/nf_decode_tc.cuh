@@ -260,7 +260,7 @@ __device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint3
             tc_fence_after();
             uint32_t o[HR];
             dt_ld<HR>(taddr, o);
-            tmem_wait_ld();
+            tmem_wait_ld_tied<HR>(o);
 #pragma unroll
             for (int e = 0; e < HR; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha[e]);
             dt_st<HR>(taddr, o);
@@ -699,7 +699,9 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     const uint32_t ta = tmem + lane_base + sb * kSCol + r0;
                     dt_ld<HR>(ta, d1);
                     dt_ld<HR>(ta + RP, d2);
-                    tmem_wait_ld();
+                    tmem_wait_ld_tied<HR>(d1);
+#pragma unroll
+                    for (int k = 0; k < HR; ++k) asm volatile("" : "+r"(d2[k]));
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 for (int e0 = 0; e0 < HR; e0 += 4) {
                     uint32_t o[4];
                     tmem_ld4(tmem + lane_base + kOCol + r0 + e0, o);
-                    tmem_wait_ld();
+                    tmem_wait_ld_tied<4>(o);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int r = r0 + e0 + e;

@@ -144,5 +144,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// The wait for this thread's tensor-memory loads, with the loaded registers
+// tied to it: no use of them can be scheduled before the wait.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[N]) {
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < N; ++k) asm volatile("" : "+r"(r[k]));
+}
 
 }  // namespace nf
