@@ -32,14 +32,16 @@
 //   O^T += V'^T . P'    kind::f16, M = 128 channels, N = 64 (rows, padded),
 //                       K = 128 keys; A = V' and B = P', both MN-major
 //                       (128-byte swizzle); O^T lives in tensor memory.
-// Roles (18 warps): warps 0-15 are alike -- warp (q, h) = (w % 4, w / 4)
+// Roles (19 warps): warps 0-15 are alike -- warp (q, h) = (w % 4, w / 4)
 // takes the keys (and O^T channel lanes) of tensor-memory quadrant q,
 // dequantises their V' channels of scale group h and runs the softmax of a
 // quarter of the rows; it reads its slice of a stage and releases the stage at
 // once.  Four such warps share each SM sub-partition, so one's latency hides
 // behind the others' work.  Warp 16 is the TMA producer; warp 17 holds the
-// tensor memory and, on one thread, issues the MMAs from an event loop that
-// serves whichever of S and P.V is ready.  Warps 0-15 also encode the query
+// tensor memory and issues the S MMAs, warp 18 the P.V MMAs, each on one
+// thread: the three issue streams sit on sub-partitions 0, 1 and 2, so that
+// no one sub-partition's consumer warps carry them all (the row-group barrier
+// waits for the slowest of its four warps).  Warps 0-15 also encode the query
 // digits at each piece's start and run the segment's final merge.  Every
 // mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT and
 // every role runs to its end without further waits.
@@ -55,8 +57,9 @@ namespace nf {
 constexpr int kDtConsumers = 16;                   // consumer warps
 constexpr int kDtRowGroups = kDtConsumers / 4;     // warps of one tensor-memory quadrant: row groups
 constexpr int kDtVG = 4 / kDtRowGroups;            // V scale groups (32 channels) per consumer warp
-constexpr int kDtThreads = (kDtConsumers + 2) * 32;  // + producer and MMA warps
-constexpr int kDtProducer = kDtConsumers, kDtMma = kDtConsumers + 1;
+constexpr int kDtThreads = (kDtConsumers + 3) * 32;  // + producer, S-issue and P.V-issue warps
+// one extra warp on each of sub-partitions 0, 1 and 2 (warp w runs on w % 4)
+constexpr int kDtProducer = kDtConsumers, kDtMma = kDtConsumers + 1, kDtPv = kDtConsumers + 2;
 constexpr int kDtStages = 4;
 constexpr int kDtPvN = 64;       // N of the P.V product: the rows, padded
 constexpr int kDtMaxRows = 32;   // rows per kv-head this kernel serves
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             mbar_init(&pvdone[i], 1);
             mbar_init(&qfull[i], 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);  // the S and the P.V issuers' last commits
         misc[0] = 0;
         misc[1] = 0;
         // the swizzled operands need 1024-byte alignment of the shared window
@@ -427,102 +430,64 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 dt_wait(&full[kk % NS], (kk / NS) & 1, misc);
         }
     } else if (warp == kDtMma) {
-        // =============================================================== MMA issue
-        // An event loop over two in-order streams: S of tile kt (once its stage
-        // is full, its S buffer free and, at a piece's first tile, the piece's
-        // query digits written) and P.V of tile j < kt (once V' and P' of j are
-        // written); whichever is ready goes first, so neither waits behind the
-        // other.
+        // =============================================================== S issue
+        // S of tile kt once its stage is full, its S buffer free and, at a
+        // piece's first tile, the piece's query digits written.  The two
+        // streams of MMAs (S here, P.V on warp kDtPv) are issued from different
+        // sub-partitions, as is the producer's TMA work.
         if (lane == 0) {
             const uint32_t sRing = smem_addr(smem), sQ = smem_addr(smem + DtSmem::kQ);
+            uint32_t kt = 0, pc = 0;
+            while (!misc[0] && walk.next()) {
+                dt_wait(&qfull[pc & 1], (pc >> 1) & 1, misc);
+                const uint32_t qaddr = sQ + (pc & 1) * 8192u;
+                const int cx1 = (int)(walk.xe - walk.s0);
+                for (int cx = (int)(walk.xs - walk.s0); cx < cx1 && !misc[0]; ++kt) {
+                    cx = dt_tile_end(cx, cx1);
+                    const uint32_t stage = kt % NS, sb = kt & 1;
+                    dt_wait(&full[stage], (kt / NS) & 1, misc);
+                    dt_wait(&sfree[sb], ((kt >> 1) & 1) ^ 1, misc);
+                    if (misc[0]) break;
+                    tc_fence_after();
+                    const uint32_t kaddr = sRing + stage * DtSmem::kStride + DtSmem::kStK;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_s8(tmem + sb * kSCol, umma_desc_sw128(kaddr + 32 * ks, 16, 1024),
+                                umma_desc_sw128(qaddr + 32 * ks, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
+                    umma_commit(&sfull[sb]);
+                    umma_commit(&empty[stage]);  // the stage's K codes are consumed
+                }
+                ++pc;
+            }
+            umma_commit(drain);  // arrives once every MMA this thread issued has completed
+        }
+    } else if (warp == kDtPv) {
+        // =============================================================== P.V issue
+        // P.V of tile j, in tile order, once V' and P' of j are written; a
+        // piece's first tile overwrites O^T.
+        if (lane == 0) {
             const uint32_t sVh = smem_addr(smem + DtSmem::kVh), sP = smem_addr(smem + DtSmem::kP);
-            uint32_t kt = 0, pj = 0, pc = 0;
-            uint64_t first_mask = 0;  // bit (tile % 64): the tile opens its piece (its P.V overwrites O)
-            bool have = walk.next(), need_q = true;
-            int cx = have ? (int)(walk.xs - walk.s0) : 0, cx1 = have ? (int)(walk.xe - walk.s0) : 0;
-            bool first_tile = false;
-            uint64_t t_idle = 0;
-            uint32_t spins = 0;
-            while (!misc[0] && (have || pj < kt)) {
-                bool progress = false;
-                if (have) {
-                    if (need_q) {
-                        if (mbar_test(&qfull[pc & 1], (pc >> 1) & 1)) {
-                            need_q = false;
-                            first_tile = true;
-                            progress = true;
-                        }
-                    } else {
-                        const uint32_t stage = kt % NS, sb = kt & 1;
-                        if (mbar_test(&full[stage], (kt / NS) & 1) && mbar_test(&sfree[sb], ((kt >> 1) & 1) ^ 1)) {
-                            tc_fence_after();
-                            const uint32_t kaddr = sRing + stage * DtSmem::kStride + DtSmem::kStK;
-                            const uint32_t qaddr = sQ + (pc & 1) * 8192u;
-#pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                umma_s8(tmem + sb * kSCol, umma_desc_sw128(kaddr + 32 * ks, 16, 1024),
-                                        umma_desc_sw128(qaddr + 32 * ks, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
-                            umma_commit(&sfull[sb]);
-                            umma_commit(&empty[stage]);  // the stage's K codes are consumed
-                            const uint64_t bit = 1ull << (kt & 63);
-                            first_mask = first_tile ? (first_mask | bit) : (first_mask & ~bit);
-                            first_tile = false;
-                            ++kt;
-                            progress = true;
-                            cx = dt_tile_end(cx, cx1);
-                            if (cx >= cx1) {  // the piece is issued: on to the next
-                                ++pc;
-                                have = walk.next();
-                                if (have) {
-                                    cx = (int)(walk.xs - walk.s0);
-                                    cx1 = (int)(walk.xe - walk.s0);
-                                    need_q = true;
-                                }
-                            }
-                        }
-                    }
-                }
-                if (pj < kt) {
+            uint32_t pj = 0;
+            while (!misc[0] && walk.next()) {
+                const int cx1 = (int)(walk.xe - walk.s0);
+                bool ovw = true;
+                for (int cx = (int)(walk.xs - walk.s0); cx < cx1 && !misc[0]; ++pj) {
+                    cx = dt_tile_end(cx, cx1);
                     const uint32_t b = pj & 1;
-                    if (mbar_test(&pfull[b], (pj >> 1) & 1)) {
-                        tc_fence_after();
-                        const bool ovw = (first_mask >> (pj & 63)) & 1ull;
+                    dt_wait(&pfull[b], (pj >> 1) & 1, misc);
+                    if (misc[0]) break;
+                    tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint64_t ad = umma_desc_sw128(sVh + b * 32768u + kk * 2048u, 16384, 1024);
-                            const uint64_t bd = umma_desc_sw128(sP + b * 16384u + kk * 2048u, 16384, 1024);
-                            umma_f16(tmem + kOCol, ad, bd, kIdescO, (ovw && kk == 0) ? 0u : 1u);
-                        }
-                        umma_commit(&pvdone[b]);
-                        ++pj;
-                        progress = true;
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t ad = umma_desc_sw128(sVh + b * 32768u + kk * 2048u, 16384, 1024);
+                        const uint64_t bd = umma_desc_sw128(sP + b * 16384u + kk * 2048u, 16384, 1024);
+                        umma_f16(tmem + kOCol, ad, bd, kIdescO, (ovw && kk == 0) ? 0u : 1u);
                     }
-                }
-                if (progress) {
-                    spins = 0;
-                    t_idle = 0;
-                } else {
-                    __nanosleep(32);
-                    if ((++spins & 255u) == 0) {
-                        // nothing ready for a while: bound the wait like every other
-                        const uint64_t now = global_ns();
-                        if (t_idle == 0) {
-                            t_idle = now;
-                        } else if (now - t_idle > kWaitLimitNs) {
-                            report(NF_DEVERR_TIMEOUT);
-                            misc[0] = 1;
-                        }
-                    }
+                    umma_commit(&pvdone[b]);
+                    ovw = false;
                 }
             }
-            // every MMA this thread issued has completed before tensor memory is freed
             umma_commit(drain);
-            const uint64_t t0 = global_ns();
-            while (!mbar_try_wait_sleep(drain, 0, 20000u))
-                if (global_ns() - t0 > kWaitLimitNs) {
-                    report(NF_DEVERR_TIMEOUT);
-                    break;
-                }
         }
     } else {
         // =============================================================== warps 0-15
@@ -796,6 +761,16 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
     tc_fence_before();
     __syncthreads();
     if (warp == kDtMma) {
+        // every MMA of both issuers has completed before tensor memory is freed
+        if (lane == 0) {
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait_sleep(drain, 0, 20000u))
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    report(NF_DEVERR_TIMEOUT);
+                    break;
+                }
+        }
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
