@@ -116,10 +116,12 @@ std::once_flag g_encode_once;
 
 // Tensor map of a quantised layer's V codes (or, k_plane, of its int8 K codes)
 // for the decode kernels: the plane as [num_blocks * H_kv * 256 rows][row
-// bytes], 32-row boxes, the swizzle as wide as a row -- K8/V4 nibbles 64 bytes
-// (64-byte swizzle), K8V8 and fp8 V codes and int8 K codes 128 bytes (128-byte
-// swizzle).
-nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map, bool k_plane = false) {
+// bytes], boxes of box_rows rows (32 for decode_kernel's stages, 128 for
+// decode_tc_kernel's tiles), the swizzle as wide as a row -- K8/V4 nibbles 64
+// bytes (64-byte swizzle), K8V8 and fp8 V codes and int8 K codes 128 bytes
+// (128-byte swizzle).
+nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map, bool k_plane = false,
+                       unsigned box_rows = nf::kChunk) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
@@ -136,7 +138,7 @@ nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map, bool k_plane = f
     const cuuint64_t row_bytes = v8 ? 128 : 64;
     const cuuint64_t dims[2] = {row_bytes, rows};
     const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)nf::kChunk};
+    const cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_plane ? kv->k_codes : kv->v_codes,
                                       dims, strides, box, estr,
@@ -366,12 +368,14 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
 
     nf::DecodeParams p{};
     const bool tc = uses_decode_tc(kv->fmt, pl.rows);
+    // decode_tc_kernel loads a tile's K and V rows with one box each
+    const unsigned box_rows = tc ? (unsigned)nf::kDtTileKeys : (unsigned)nf::kChunk;
     if (kv->fmt != NF_KV_BF16) {
-        st = encode_v_map(kv, &p.vmap);
+        st = encode_v_map(kv, &p.vmap, false, box_rows);
         if (st != NF_OK) return st;
     }
     if (tc || kv->fmt == NF_KV_K4V4) {
-        st = encode_v_map(kv, &p.kmap, true);
+        st = encode_v_map(kv, &p.kmap, true, box_rows);
         if (st != NF_OK) return st;
     }
     p.k_codes = kv->k_codes;

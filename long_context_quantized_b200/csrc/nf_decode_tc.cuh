@@ -32,16 +32,17 @@
 //   O^T += V'^T . P'    kind::f16, M = 128 channels, N = 64 (rows, padded),
 //                       K = 128 keys; A = V' and B = P', both MN-major
 //                       (128-byte swizzle); O^T lives in tensor memory.
-// Roles (19 warps): warps 0-15 are alike -- warp (q, h) = (w % 4, w / 4)
+// Roles (20 warps): warps 0-15 are alike -- warp (q, h) = (w % 4, w / 4)
 // takes the keys (and O^T channel lanes) of tensor-memory quadrant q,
 // dequantises their V' channels of scale group h and runs the softmax of a
 // quarter of the rows; it reads its slice of a stage and releases the stage at
 // once.  Four such warps share each SM sub-partition, so one's latency hides
 // behind the others' work.  Warp 16 is the TMA producer; warp 17 holds the
-// tensor memory and issues the S MMAs, warp 18 the P.V MMAs, each on one
-// thread: the three issue streams sit on sub-partitions 0, 1 and 2, so that
-// no one sub-partition's consumer warps carry them all (the row-group barrier
-// waits for the slowest of its four warps).  Warps 0-15 also encode the query
+// tensor memory and issues the S MMAs; warps 18 and 19 issue the P.V MMAs of
+// the even and the odd tiles, each issuer on one thread.  The issue streams
+// sit one on each sub-partition: issuing an MMA takes issue cycles from the
+// consumer warps beside it, and the row-group barrier waits for the slowest
+// of its four warps, one per sub-partition.  Warps 0-15 also encode the query
 // digits at each piece's start and run the segment's final merge.  Every
 // mbarrier wait is bounded (2 s); a timeout records NF_DEVERR_TIMEOUT and
 // every role runs to its end without further waits.
@@ -57,10 +58,12 @@ namespace nf {
 constexpr int kDtConsumers = 16;                   // consumer warps
 constexpr int kDtRowGroups = kDtConsumers / 4;     // warps of one tensor-memory quadrant: row groups
 constexpr int kDtVG = 4 / kDtRowGroups;            // V scale groups (32 channels) per consumer warp
-constexpr int kDtThreads = (kDtConsumers + 3) * 32;  // + producer, S-issue and P.V-issue warps
-// one extra warp on each of sub-partitions 0, 1 and 2 (warp w runs on w % 4)
+constexpr int kDtThreads = (kDtConsumers + 4) * 32;  // + producer, S-issue and two P.V-issue warps
+// one extra warp on each sub-partition (warp w runs on w % 4); the P.V
+// issuers take the even and the odd tiles
 constexpr int kDtProducer = kDtConsumers, kDtMma = kDtConsumers + 1, kDtPv = kDtConsumers + 2;
 constexpr int kDtStages = 4;
+constexpr int kDtTileKeys = 128;  // keys of a full tile: one TMA box of K and one of V rows
 constexpr int kDtPvN = 64;       // N of the P.V product: the rows, padded
 constexpr int kDtMaxRows = 32;   // rows per kv-head this kernel serves
 constexpr int kDtChunkTiles = kBlock / kChunk;
@@ -322,7 +325,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             mbar_init(&pvdone[i], 1);
             mbar_init(&qfull[i], 1);
         }
-        mbar_init(drain, 2);  // the S and the P.V issuers' last commits
+        mbar_init(drain, 3);  // the S and the two P.V issuers' last commits
         misc[0] = 0;
         misc[1] = 0;
         // the swizzled operands need 1024-byte alignment of the shared window
@@ -408,11 +411,12 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                         } else {
                             stage_ok[stage] = 1;
                             const size_t si = ((size_t)blk * H + walk.ph) * kBlock + (tok0 & (kBlock - 1));
-                            mbar_arrive_expect_tx(&full[stage], (uint32_t)(ntok * DtSmem::kBytesPerTok));
-                            for (int c = 0; c < ntok; c += kChunk) {
-                                tma_load_2d(st + DtSmem::kStK + c * 128, &p.kmap, 0, (int)si + c, &full[stage]);
-                                tma_load_2d(st + DtSmem::kStV + c * 64, &p.vmap, 0, (int)si + c, &full[stage]);
-                            }
+                            // one box of 128 K rows and one of 128 V rows, whatever ntok: a
+                            // shorter tile's extra rows (the next rows of the plane, or the
+                            // fill past its end) are never used unmasked
+                            mbar_arrive_expect_tx(&full[stage], (uint32_t)(kDtTileKeys * (128 + 64) + ntok * (2 + 8)));
+                            tma_load_2d(st + DtSmem::kStK, &p.kmap, 0, (int)si, &full[stage]);
+                            tma_load_2d(st + DtSmem::kStV, &p.vmap, 0, (int)si, &full[stage]);
                             bulk_g2s(st + DtSmem::kStKs, p.k_scales + si, ntok * 2, &full[stage]);
                             bulk_g2s(st + DtSmem::kStVs, p.v_scales + si * 4, ntok * 8, &full[stage]);
                         }
@@ -461,11 +465,14 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             }
             umma_commit(drain);  // arrives once every MMA this thread issued has completed
         }
-    } else if (warp == kDtPv) {
+    } else if (warp == kDtPv || warp == kDtPv + 1) {
         // =============================================================== P.V issue
-        // P.V of tile j, in tile order, once V' and P' of j are written; a
-        // piece's first tile overwrites O^T.
+        // P.V of tile j once V' and P' of j are written, tile j on warp
+        // kDtPv + (j & 1) -- so that buffer b = j & 1 and its pvdone[b] belong
+        // to one issuer -- and only after P.V of tile j - 1 has completed, so
+        // that O^T accumulates in tile order; a piece's first tile overwrites O^T.
         if (lane == 0) {
+            const uint32_t mine = (uint32_t)(warp - kDtPv);
             const uint32_t sVh = smem_addr(smem + DtSmem::kVh), sP = smem_addr(smem + DtSmem::kP);
             uint32_t pj = 0;
             while (!misc[0] && walk.next()) {
@@ -474,16 +481,18 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 for (int cx = (int)(walk.xs - walk.s0); cx < cx1 && !misc[0]; ++pj) {
                     cx = dt_tile_end(cx, cx1);
                     const uint32_t b = pj & 1;
-                    dt_wait(&pfull[b], (pj >> 1) & 1, misc);
-                    if (misc[0]) break;
-                    tc_fence_after();
+                    if (b == mine) {
+                        dt_wait(&pfull[b], (pj >> 1) & 1, misc);
+                        if (pj > 0) dt_wait(&pvdone[b ^ 1], ((pj - 1) >> 1) & 1, misc);
+                        if (misc[0]) break;
+                        tc_fence_after();
+                        const uint64_t ad = umma_desc_sw128(sVh + b * 32768u, 16384, 1024);
+                        const uint64_t bd = umma_desc_sw128(sP + b * 16384u, 16384, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t ad = umma_desc_sw128(sVh + b * 32768u + kk * 2048u, 16384, 1024);
-                        const uint64_t bd = umma_desc_sw128(sP + b * 16384u + kk * 2048u, 16384, 1024);
-                        umma_f16(tmem + kOCol, ad, bd, kIdescO, (ovw && kk == 0) ? 0u : 1u);
+                        for (int kk = 0; kk < 8; ++kk)  // + 2048 bytes along K: + 128 in the address field
+                            umma_f16(tmem + kOCol, ad + 128u * kk, bd + 128u * kk, kIdescO, (ovw && kk == 0) ? 0u : 1u);
+                        umma_commit(&pvdone[b]);
                     }
-                    umma_commit(&pvdone[b]);
                     ovw = false;
                 }
             }
