@@ -315,13 +315,15 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1 + kDtConsumers);  // the S MMA's commit and the consumer warps
+            mbar_init(&empty[i], 1 + kDtConsumers * 32);  // the S MMA's commit and every consumer thread
             stage_ok[i] = 0;
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sfull[i], 1);
-            mbar_init(&sfree[i], kDtConsumers);
-            mbar_init(&pfull[i], kDtConsumers);  // V' and P' of a tile written
+            // every consumer thread arrives on its own (its accesses are ordered
+            // before its arrival): no warp convergence or elected lane per tile
+            mbar_init(&sfree[i], kDtConsumers * 32);
+            mbar_init(&pfull[i], kDtConsumers * 32);  // V' and P' of a tile written
             mbar_init(&pvdone[i], 1);
             mbar_init(&qfull[i], 1);
         }
@@ -637,8 +639,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     vsr = *reinterpret_cast<const uint2 *>(st + DtSmem::kStVs + i * 8);
                     ksv = __half2float(*reinterpret_cast<const __half *>(st + DtSmem::kStKs + i * 2));
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[stage]);
+                mbar_arrive(&empty[stage]);
                 const int ev = dt_v_exponent(vsr);
                 // ---- V' and P' buffers sb are free once the P.V of tile kt - 2 is done
                 if (kt >= 2) dt_wait(&pvdone[sb], ((kt >> 1) - 1) & 1, misc);
@@ -678,8 +679,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     for (int k = 0; k < HR; ++k) asm volatile("" : "+r"(d2[k]));
                 }
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sfree[sb]);
+                mbar_arrive(&sfree[sb]);
                 const int dpos = pos - causal_base;
                 const int rmin = kv_ok ? (dpos > 0 ? dpos * p.group : 0) : 0x7fffffff;  // rows rmin .. R - 1 see it
                 const float f = __int_as_float((127 + ev - 15) << 23);
@@ -707,8 +707,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 }
                 fence_async_smem();
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&pfull[sb]);
+                mbar_arrive(&pfull[sb]);
             }
 
             // ---- end of the piece: O^T / l into out (one piece) or the partial slot
