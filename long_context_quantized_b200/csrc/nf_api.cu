@@ -116,10 +116,10 @@ std::once_flag g_encode_once;
 
 // Tensor map of a quantised layer's V codes (or, k_plane, of its int8 K codes)
 // for the decode kernels: the plane as [num_blocks * H_kv * 256 rows][row
-// bytes], boxes of box_rows rows (32 for decode_kernel's stages, 128 for
-// decode_tc_kernel's tiles), the swizzle as wide as a row -- K8/V4 nibbles 64
-// bytes (64-byte swizzle), K8V8 and fp8 V codes and int8 K codes 128 bytes
-// (128-byte swizzle).
+// bytes], boxes of box_rows rows (32: any chunk of decode_kernel's stages; a
+// whole stage, 128 or 256; 128 for decode_tc_kernel's tiles), the swizzle as
+// wide as a row -- K8/V4 nibbles 64 bytes (64-byte swizzle), K8V8 and fp8 V
+// codes and int8 K codes 128 bytes (128-byte swizzle).
 nf_status encode_v_map(const nf_kv_layer *kv, CUtensorMap *map, bool k_plane = false,
                        unsigned box_rows = nf::kChunk) {
     std::call_once(g_encode_once, [] {
@@ -377,6 +377,16 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
     if (tc || kv->fmt == NF_KV_K4V4) {
         st = encode_v_map(kv, &p.kmap, true, box_rows);
         if (st != NF_OK) return st;
+    }
+    if (!tc && kv->fmt != NF_KV_BF16) {
+        // decode_kernel: a whole stage's V (and RK4V4 K) rows in one box
+        const unsigned stage_rows = (kv->fmt == NF_KV_K8V8 || kv->fmt == NF_KV_F8) ? 128u : 256u;
+        st = encode_v_map(kv, &p.vmap_full, false, stage_rows);
+        if (st != NF_OK) return st;
+        if (kv->fmt == NF_KV_K4V4) {
+            st = encode_v_map(kv, &p.kmap_full, true, stage_rows);
+            if (st != NF_OK) return st;
+        }
     }
     p.k_codes = kv->k_codes;
     p.k_scales = static_cast<const __half *>(kv->k_scales);

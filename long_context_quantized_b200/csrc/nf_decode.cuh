@@ -151,6 +151,8 @@ struct DecodeParams {
                        // 32-row boxes, swizzle as wide as a row (unused for bf16)
     CUtensorMap kmap;  // k_codes as [num_blocks * H_kv * 256 rows][128 bytes], 32-row boxes,
                        // 128-byte swizzle (the tensor-core decode of many rows only)
+    CUtensorMap vmap_full, kmap_full;  // the same planes with boxes of a whole stage (decode_kernel:
+                                       // a full stage's rows in one copy each)
     const void *k_codes;
     const __half *k_scales;
     const void *v_codes;
@@ -1084,9 +1086,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             const size_t si = ((size_t)blk * H + walk.ph) * kBlock + (tok0 & (kBlock - 1));
                             mbar_arrive_expect_tx(&full[stage], (uint32_t)(ntok * ST::kBytesPerTok));
                             if (K4) {
-                                for (int c = 0; c < ntok; c += kChunk) {
-                                    tma_load_2d(st + ST::kK + c * 64, &p.kmap, 0, (int)si + c, &full[stage]);
-                                    tma_load_2d(st + ST::kV + c * 64, &p.vmap, 0, (int)si + c, &full[stage]);
+                                if (ntok == ST::kTok) {  // a whole stage: one box each
+                                    tma_load_2d(st + ST::kK, &p.kmap_full, 0, (int)si, &full[stage]);
+                                    tma_load_2d(st + ST::kV, &p.vmap_full, 0, (int)si, &full[stage]);
+                                } else {
+                                    for (int c = 0; c < ntok; c += kChunk) {
+                                        tma_load_2d(st + ST::kK + c * 64, &p.kmap, 0, (int)si + c, &full[stage]);
+                                        tma_load_2d(st + ST::kV + c * 64, &p.vmap, 0, (int)si + c, &full[stage]);
+                                    }
                                 }
                                 bulk_g2s(st + ST::kKs, reinterpret_cast<const uint8_t *>(p.k_scales) + si * 4, ntok * 4,
                                          &full[stage]);
@@ -1095,8 +1102,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
                             } else if (K8) {
                                 constexpr int vrow = V8 ? 128 : 64, vsc = V8 ? 1 : 4;  // V bytes, V scales per key
                                 bulk_g2s(st + ST::kK, static_cast<const int8_t *>(p.k_codes) + si * 128, ntok * 128, &full[stage]);
-                                for (int c = 0; c < ntok; c += kChunk)
-                                    tma_load_2d(st + ST::kV + c * vrow, &p.vmap, 0, (int)si + c, &full[stage]);
+                                if (ntok == ST::kTok)  // a whole stage: one box
+                                    tma_load_2d(st + ST::kV, &p.vmap_full, 0, (int)si, &full[stage]);
+                                else
+                                    for (int c = 0; c < ntok; c += kChunk)
+                                        tma_load_2d(st + ST::kV + c * vrow, &p.vmap, 0, (int)si + c, &full[stage]);
                                 bulk_g2s(st + ST::kKs, p.k_scales + si, ntok * 2, &full[stage]);
                                 bulk_g2s(st + ST::kVs, p.v_scales + si * vsc, ntok * 2 * vsc, &full[stage]);
                             } else {
