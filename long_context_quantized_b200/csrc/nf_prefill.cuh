@@ -55,10 +55,14 @@ struct PrefillParams {
 //              loads key t's K codes (t < 64) or key t - 64's V nibbles and
 //              scales (prefetched a tile ahead in registers) and writes that
 //              dequantised fp16 row into a three-stage ring;
-//   warp 12    tensor memory allocation and, on one thread, the MMAs: per K/V
-//              tile j, S_x = Q_x . K_j^T (x = a, b) into one of two S buffers
-//              of tile x, then O_x += P_x . V for tile j - 1, each group
-//              committed to an mbarrier.
+//   warps 12-15 the MMAs, each stream on one thread of its own warp: warp
+//              12 (which also holds the tensor memory) S_a = Q_a . K_j^T and
+//              warp 13 S_b, each into one of two S buffers of its tile once
+//              the softmax has read that buffer's last S; warps 14 and 15
+//              O_a += P_a . V_j and O_b += P_b . V_j.  Each group is committed
+//              to an mbarrier.  One issue stream per SM sub-partition: issuing
+//              an MMA takes issue cycles from the warps beside it, and each
+//              softmax tile waits for the slowest of its four warps.
 // The K/V ring is converted once for 256 rows, and each SM sub-partition runs
 // two softmax warps, one of each tile.
 // Tensor memory (512 columns x 128 lanes): S of tile x, buffer b at columns
@@ -75,7 +79,7 @@ struct PrefillParams {
 // Every mbarrier wait is bounded; a timeout records NF_DEVERR_TIMEOUT and
 // every role leaves its loop.
 // ============================================================================
-constexpr int kTcThreads = 416;
+constexpr int kTcThreads = 512;
 constexpr int kTcRows = 256;   // query rows per CTA (two MMA tiles of 128)
 constexpr int kTcKeys = 64;    // keys per K/V tile (N of S = Q.K^T, K of O += P.V)
 constexpr float kTcLazy = 8.0f;
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         mbar_init(q_full, 128);
         for (int i = 0; i < TcSmem::kStages; ++i) {
             mbar_init(&kv_full[i], 128);
-            mbar_init(&kv_free[i], 1);
+            mbar_init(&kv_free[i], 4);  // the four MMA streams' commits for the stage's tile
         }
         for (int i = 0; i < 2; ++i) {
             for (int x = 0; x < 2; ++x) {
@@ -253,8 +257,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
                 mbar_init(pv_done(x, i), 1);
             }
         }
-        mbar_init(o_full, 1);
-        mbar_init(drain, 1);
+        mbar_init(o_full, 2);  // the two P.V streams' last commits
+        mbar_init(drain, 4);
         *abort_flag = 0;
         // the swizzled operands need 1024-byte alignment of the window
         if (smem_addr(smem) & 1023u) {
@@ -486,33 +490,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             if (dst && p.out_lse)
                 p.out_lse[out_row(row)] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
         }
-    } else if (warp == 12 && lane == 0 && !*abort_flag) {
+    } else if (warp >= 12 && lane == 0 && !*abort_flag) {
         // ================================================== MMA issue
+        const int role = warp - 12, x = role & 1;
         const uint32_t sQ = smem_addr(smem + TcSmem::kQ), sK = smem_addr(smem + TcSmem::kK);
         const uint32_t sV = smem_addr(smem + TcSmem::kV), sP = smem_addr(smem + TcSmem::kP);
-        // O_x += P_x . V for K/V tile i (P buffer i & 1, K/V stage i % 3)
-        auto pv = [&](int i) -> bool {
-            const int s = i & 1, st = i % TcSmem::kStages;
-            for (int x = 0; x < 2; ++x) {
-                if (!tc_wait(p_full(x, s), (i >> 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = umma_desc_sw128(sP + s * 32768 + x * 16384 + kk * 32, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(sV + st * 16384 + kk * 2048, 8192, 1024);
-                    umma_f16(tmem + 256u + 128u * x, ad, bd, kTcIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
+        bool ok = true;
+        if (role < 2) {
+            // S_x of tile j once K of tile j is staged and the softmax of tile
+            // x has read S of tile j - 2 (the same buffer)
+            ok = tc_wait(q_full, 0, abort_flag);
+            for (int j = 0; ok && j < T; ++j) {
+                const int s = j & 1, st = j % TcSmem::kStages;
+                if (!tc_wait(&kv_full[st], (j / TcSmem::kStages) & 1, abort_flag) ||
+                    (j >= 2 && !tc_wait(p_full(x, s), ((j - 2) >> 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
                 }
-                umma_commit(pv_done(x, s));
-            }
-            umma_commit(&kv_free[st]);  // every MMA that reads stage st for tile i is done
-            return true;
-        };
-        bool ok = tc_wait(q_full, 0, abort_flag);
-        for (int j = 0; ok && j < T; ++j) {
-            const int s = j & 1, st = j % TcSmem::kStages;
-            if (!tc_wait(&kv_full[st], (j / TcSmem::kStages) & 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            for (int x = 0; x < 2; ++x) {
+                tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t ad = umma_desc_sw128(sQ + x * 32768 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
@@ -520,23 +515,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
                     umma_f16(tmem + 128u * x + 64u * s, ad, bd, kTcIdescQK, ks > 0 ? 1u : 0u);
                 }
                 umma_commit(s_full(x, s));
+                umma_commit(&kv_free[st]);  // this stream's reads of stage st are done
             }
-            if (j >= 1 && !pv(j - 1)) { ok = false; break; }
+        } else {
+            // O_x += P_x . V of tile j once the softmax of tile x has written P
+            for (int j = 0; ok && j < T; ++j) {
+                const int s = j & 1, st = j % TcSmem::kStages;
+                if (!tc_wait(&kv_full[st], (j / TcSmem::kStages) & 1, abort_flag) ||
+                    !tc_wait(p_full(x, s), (j >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = umma_desc_sw128(sP + s * 32768 + x * 16384 + kk * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(sV + st * 16384 + kk * 2048, 8192, 1024);
+                    umma_f16(tmem + 256u + 128u * x, ad, bd, kTcIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(pv_done(x, s));
+                umma_commit(&kv_free[st]);
+            }
+            if (ok) umma_commit(o_full);
         }
-        if (ok && T > 0) ok = pv(T - 1);
-        if (ok) umma_commit(o_full);
-        // every MMA this thread issued has completed before tensor memory is freed
-        umma_commit(drain);
-        const uint64_t t0 = global_ns();
-        while (!mbar_try_wait_sleep(drain, 0, 20000u))
-            if (global_ns() - t0 > kWaitLimitNs) {
-                report(NF_DEVERR_TIMEOUT);
-                break;
-            }
+        umma_commit(drain);  // arrives once every MMA this thread issued has completed
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 12) {
+        // every MMA of the four streams has completed before tensor memory is freed
+        if (lane == 0) {
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait_sleep(drain, 0, 20000u))
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    report(NF_DEVERR_TIMEOUT);
+                    break;
+                }
+        }
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
