@@ -215,7 +215,10 @@ size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_h
  *   the e4m3 codes are exact in fp16; S = Q . K^T uses fp16 products with each
  *   query row split as q = s (hi + lo), s = max|q|, hi and lo fp16.  bf16
  *   cache: bf16 products, the fp32 query and the weights split into bf16 high
- *   and low parts.)
+ *   and low parts.)  With 9 to 32 query rows per kv-head, K8/V4 and K8V8 run on
+ *   the tcgen05 tensor cores instead: the same two-digit Q . K, and P . V as
+ *   V' = code x scale x 2^(15 - E) times P' = weight x 2^(E - 15), each rounded
+ *   to fp16 once (E: the largest exponent field of the key's V scales).
  * Launch: the kernel is launched with programmatic dependent launch, so it may
  *   start while the previous kernel on `stream` finishes; it waits for that
  *   kernel before reading any argument (see nf_decode_attn_ex for a weaker

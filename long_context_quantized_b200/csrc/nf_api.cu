@@ -191,25 +191,32 @@ cudaError_t launch_decode(const nf::DecodeParams &p, int ctas, cudaStream_t s) {
     return launch_pdl(nf::decode_kernel<NT, QF32, FMT>, (unsigned)ctas, nf::kDecodeThreads, smem, s, p);
 }
 
-// The tensor-core decode of many rows (K8/V4, 9 to 32 query rows per kv-head),
-// rows padded to RP = 16 or 32.
-template <int RP, bool QF32>
+// The tensor-core decode of many rows (K8/V4 or K8V8, 9 to 32 query rows per
+// kv-head), rows padded to RP = 16 or 32.
+template <int RP, bool QF32, int FMT>
 cudaError_t launch_decode_tc(const nf::DecodeParams &p, int ctas, cudaStream_t s) {
-    constexpr int smem = nf::DtSmem::kBytes;
+    constexpr int smem = nf::DtSmem<FMT>::kBytes;
     static std::atomic<uint64_t> opted{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
     if (!bit || !(opted.load(std::memory_order_acquire) & bit)) {
-        e = cudaFuncSetAttribute(nf::decode_tc_kernel<RP, QF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(nf::decode_tc_kernel<RP, QF32, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         opted.fetch_or(bit, std::memory_order_acq_rel);
     }
-    return launch_pdl(nf::decode_tc_kernel<RP, QF32>, (unsigned)ctas, nf::kDtThreads, smem, s, p);
+    return launch_pdl(nf::decode_tc_kernel<RP, QF32, FMT>, (unsigned)ctas, nf::kDtThreads, smem, s, p);
+}
+template <int FMT>
+cudaError_t dispatch_decode_tc(const nf::DecodeParams &p, bool qf32, int rows, int ctas, cudaStream_t s) {
+    return rows <= 16 ? (qf32 ? launch_decode_tc<16, true, FMT>(p, ctas, s) : launch_decode_tc<16, false, FMT>(p, ctas, s))
+                      : (qf32 ? launch_decode_tc<32, true, FMT>(p, ctas, s) : launch_decode_tc<32, false, FMT>(p, ctas, s));
 }
 
-bool uses_decode_tc(int fmt, int rows) { return fmt == NF_KV_K8V4 && rows > 8 && rows <= nf::kDtMaxRows; }
+bool uses_decode_tc(int fmt, int rows) {
+    return (fmt == NF_KV_K8V4 || fmt == NF_KV_K8V8) && rows > 8 && rows <= nf::kDtMaxRows;
+}
 
 template <int NT>
 cudaError_t dispatch_decode(const nf::DecodeParams &p, bool qf32, int fmt, int ctas, cudaStream_t s) {
@@ -419,8 +426,8 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool qf32 = q_dtype == NF_F32;
     const cudaError_t e =
-        tc ? (pl.rows <= 16 ? (qf32 ? launch_decode_tc<16, true>(p, pl.ctas, s) : launch_decode_tc<16, false>(p, pl.ctas, s))
-                            : (qf32 ? launch_decode_tc<32, true>(p, pl.ctas, s) : launch_decode_tc<32, false>(p, pl.ctas, s)))
+        tc ? (kv->fmt == NF_KV_K8V8 ? dispatch_decode_tc<NF_KV_K8V8>(p, qf32, pl.rows, pl.ctas, s)
+                                    : dispatch_decode_tc<NF_KV_K8V4>(p, qf32, pl.rows, pl.ctas, s))
         : pl.nt == 1 ? dispatch_decode<1>(p, qf32, kv->fmt, pl.ctas, s)
                      : dispatch_decode<2>(p, qf32, kv->fmt, pl.ctas, s);
     if (e != cudaSuccess) {

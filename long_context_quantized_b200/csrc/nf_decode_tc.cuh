@@ -1,5 +1,8 @@
-// nf_decode_tc.cuh -- split-K decode attention over the K8/V4 pool for many
-// query rows per kv-head, on the 5th-generation tensor cores (tcgen05).
+// nf_decode_tc.cuh -- split-K decode attention over the K8/V4 (or the int8
+// K8V8) pool for many query rows per kv-head, on the 5th-generation tensor
+// cores (tcgen05).  K8V8 differs only in the V side: 128-byte rows of int8
+// codes with one fp16 scale per key, dequantised in channel order, and three
+// ring stages instead of four.
 //
 // MTP draft verification is the engine's normal decode step: 1 + 3 query
 // tokens per step (page "3090 单卡跑 Qwen3.8-27B：NInfer 上机实测", section
@@ -74,13 +77,20 @@ constexpr int kDtSegPad = 12;
 // warps (also the final merge's)
 constexpr uint32_t kDtBarAll = 6;
 
+// Shared-memory layout for the pool format FMT: NF_KV_K8V4 or NF_KV_K8V8.
+template <int FMT>
 struct DtSmem {
-    // one ring stage: K codes [128 keys][128 B] (128-byte swizzle), V nibbles
-    // [128 keys][64 B] (64-byte swizzle), K scales fp16 [128], V scales fp16 [128][4]
-    static constexpr int kStK = 0, kStV = 16384, kStKs = 24576, kStVs = 24832;
-    static constexpr int kStride = 26624;
-    static constexpr int kBytesPerTok = 202;
-    static constexpr int kRingBytes = kDtStages * kStride;
+    // one ring stage: K codes [128 keys][128 B] (128-byte swizzle); V codes
+    // [128 keys][64 B nibbles] (64-byte swizzle, K8/V4) or [128 keys][128 B]
+    // (128-byte swizzle, K8V8); K scales fp16 [128]; V scales fp16 [128][4]
+    // (K8/V4) or [128] (K8V8).  Three K8V8 stages fit beside the other buffers.
+    static constexpr bool kV8 = FMT == NF_KV_K8V8;
+    static constexpr int kVRow = kV8 ? 128 : 64, kVScales = kV8 ? 1 : 4;
+    static constexpr int kStages = kV8 ? 3 : kDtStages;
+    static constexpr int kStK = 0, kStV = 16384, kStKs = kStV + 128 * kVRow, kStVs = kStKs + 256;
+    static constexpr int kStride = (kStVs + 128 * 2 * kVScales + 1023) / 1024 * 1024;
+    static constexpr int kBytesPerTok = 128 + kVRow + 2 + 2 * kVScales;
+    static constexpr int kRingBytes = kStages * kStride;
     static constexpr int kVh = kRingBytes;        // fp16 V' [2 buffers][2 blocks of 64 channels][128 keys][128 B]
     static constexpr int kP = kVh + 2 * 32768;    // fp16 P' [2 buffers][128 keys][64 rows x 2 B]
     static constexpr int kQ = kP + 2 * 16384;     // int8 digits [2 buffers][64 digit rows][128 B]
@@ -88,9 +98,9 @@ struct DtSmem {
     static constexpr int kRed = kQw + 2 * kDtMaxRows * 4;   // float [4 quadrants][kDtMaxRows]: row maxima
     static constexpr int kRed2 = kRed + 4 * kDtMaxRows * 4; // float [4 quadrants][kDtMaxRows]: row sums
     static constexpr int kBars = kRed2 + 4 * kDtMaxRows * 4;
-    static constexpr int kNumBars = 2 * kDtStages + 10 + 1;
+    static constexpr int kNumBars = 2 * kStages + 10 + 1;
     static constexpr int kStageOk = kBars + kNumBars * 8;   // int [stages]
-    static constexpr int kTmem = kStageOk + kDtStages * 4;  // u32
+    static constexpr int kTmem = kStageOk + kStages * 4;    // u32
     static constexpr int kSeqC = (kTmem + 4 + 15) / 16 * 16;  // int [kMaxBatch]
     static constexpr int kSeqL = kSeqC + kMaxBatch * 4;       // int [kMaxBatch]
     static constexpr int kSeqBase = kSeqL + kMaxBatch * 4;    // i64 [kMaxBatch + 1]
@@ -284,10 +294,13 @@ __device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint3
     }
 }
 
-template <int RP, bool QF32>
+template <int RP, bool QF32, int FMT>
 __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
     static_assert(RP == 16 || RP == 32, "rows padded to 16 or 32");
-    constexpr int NS = kDtStages;
+    static_assert(FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8, "int8 K codes");
+    using SM = DtSmem<FMT>;
+    constexpr bool V8 = SM::kV8;  // int8 V codes, one V scale per key
+    constexpr int NS = SM::kStages;
     constexpr int HR = RP / kDtRowGroups;                         // rows per consumer warp
     constexpr int NSC = 2 * RP;                                   // S columns per buffer
     constexpr uint32_t kIdescS = umma_idesc_s8(128, NSC);
@@ -295,19 +308,19 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
     constexpr uint32_t kSCol = 64;                                // S buffer b at columns 64 b
     constexpr uint32_t kOCol = 128;                               // O^T at columns 128 .. 191
     extern __shared__ __align__(1024) unsigned char smem[];
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DtSmem::kBars);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kBars);
     uint64_t *full = bars, *empty = bars + NS;
     uint64_t *sfull = bars + 2 * NS, *sfree = sfull + 2, *pfull = sfree + 2;
     uint64_t *pvdone = pfull + 2, *qfull = pvdone + 2, *drain = qfull + 2;
-    volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + DtSmem::kStageOk);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + DtSmem::kTmem);
-    int *seqC = reinterpret_cast<int *>(smem + DtSmem::kSeqC);
-    int *seqL = reinterpret_cast<int *>(smem + DtSmem::kSeqL);
-    long long *seqBase = reinterpret_cast<long long *>(smem + DtSmem::kSeqBase);
-    volatile int *misc = reinterpret_cast<volatile int *>(smem + DtSmem::kMisc);  // [0] abort, [1] last ticket
-    float *qw_sm = reinterpret_cast<float *>(smem + DtSmem::kQw);
-    float *red = reinterpret_cast<float *>(smem + DtSmem::kRed);
-    float *red2 = reinterpret_cast<float *>(smem + DtSmem::kRed2);
+    volatile int *stage_ok = reinterpret_cast<volatile int *>(smem + SM::kStageOk);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM::kTmem);
+    int *seqC = reinterpret_cast<int *>(smem + SM::kSeqC);
+    int *seqL = reinterpret_cast<int *>(smem + SM::kSeqL);
+    long long *seqBase = reinterpret_cast<long long *>(smem + SM::kSeqBase);
+    volatile int *misc = reinterpret_cast<volatile int *>(smem + SM::kMisc);  // [0] abort, [1] last ticket
+    float *qw_sm = reinterpret_cast<float *>(smem + SM::kQw);
+    float *red = reinterpret_cast<float *>(smem + SM::kRed);
+    float *red2 = reinterpret_cast<float *>(smem + SM::kRed2);
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = p.num_kv_heads;
@@ -339,7 +352,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
     }
     // the query-digit buffers' padding rows stay zero
     for (int i = threadIdx.x; i < 2 * 8192 / 16; i += kDtThreads)
-        reinterpret_cast<uint4 *>(smem + DtSmem::kQ)[i] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4 *>(smem + SM::kQ)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     if (warp == kDtMma) {
         tmem_alloc(tmem_slot, 256);
@@ -405,7 +418,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     const int stage = (int)(kst % NS);
                     dt_wait(&empty[stage], ((kst / NS) & 1) ^ 1, misc);
                     if (!misc[0]) {
-                        unsigned char *st = smem + stage * DtSmem::kStride;
+                        unsigned char *st = smem + stage * SM::kStride;
                         if (blk < 0 || blk >= p.num_blocks) {
                             report(NF_DEVERR_BLOCK_ID);
                             stage_ok[stage] = 0;
@@ -416,11 +429,13 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                             // one box of 128 K rows and one of 128 V rows, whatever ntok: a
                             // shorter tile's extra rows (the next rows of the plane, or the
                             // fill past its end) are never used unmasked
-                            mbar_arrive_expect_tx(&full[stage], (uint32_t)(kDtTileKeys * (128 + 64) + ntok * (2 + 8)));
-                            tma_load_2d(st + DtSmem::kStK, &p.kmap, 0, (int)si, &full[stage]);
-                            tma_load_2d(st + DtSmem::kStV, &p.vmap, 0, (int)si, &full[stage]);
-                            bulk_g2s(st + DtSmem::kStKs, p.k_scales + si, ntok * 2, &full[stage]);
-                            bulk_g2s(st + DtSmem::kStVs, p.v_scales + si * 4, ntok * 8, &full[stage]);
+                            mbar_arrive_expect_tx(&full[stage], (uint32_t)(kDtTileKeys * (128 + SM::kVRow) +
+                                                                           ntok * (2 + 2 * SM::kVScales)));
+                            tma_load_2d(st + SM::kStK, &p.kmap, 0, (int)si, &full[stage]);
+                            tma_load_2d(st + SM::kStV, &p.vmap, 0, (int)si, &full[stage]);
+                            bulk_g2s(st + SM::kStKs, p.k_scales + si, ntok * 2, &full[stage]);
+                            bulk_g2s(st + SM::kStVs, p.v_scales + si * SM::kVScales, ntok * 2 * SM::kVScales,
+                                     &full[stage]);
                         }
                     }
                 }
@@ -442,7 +457,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         // streams of MMAs (S here, P.V on warp kDtPv) are issued from different
         // sub-partitions, as is the producer's TMA work.
         if (lane == 0) {
-            const uint32_t sRing = smem_addr(smem), sQ = smem_addr(smem + DtSmem::kQ);
+            const uint32_t sRing = smem_addr(smem), sQ = smem_addr(smem + SM::kQ);
             uint32_t kt = 0, pc = 0;
             while (!misc[0] && walk.next()) {
                 dt_wait(&qfull[pc & 1], (pc >> 1) & 1, misc);
@@ -455,7 +470,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     dt_wait(&sfree[sb], ((kt >> 1) & 1) ^ 1, misc);
                     if (misc[0]) break;
                     tc_fence_after();
-                    const uint32_t kaddr = sRing + stage * DtSmem::kStride + DtSmem::kStK;
+                    const uint32_t kaddr = sRing + stage * SM::kStride + SM::kStK;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         umma_s8(tmem + sb * kSCol, umma_desc_sw128(kaddr + 32 * ks, 16, 1024),
@@ -475,7 +490,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         // that O^T accumulates in tile order; a piece's first tile overwrites O^T.
         if (lane == 0) {
             const uint32_t mine = (uint32_t)(warp - kDtPv);
-            const uint32_t sVh = smem_addr(smem + DtSmem::kVh), sP = smem_addr(smem + DtSmem::kP);
+            const uint32_t sVh = smem_addr(smem + SM::kVh), sP = smem_addr(smem + SM::kP);
             uint32_t pj = 0;
             while (!misc[0] && walk.next()) {
                 const int cx1 = (int)(walk.xe - walk.s0);
@@ -506,8 +521,8 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         // key 32 q + lane of each tile (the lane of S) and channel lane 32 q +
         // lane of O^T; rows h HR .. h HR + HR - 1 of the softmax, P' and O^T; and
         // the kDtVG V scale groups h kDtVG .. of 32 channels in the dequantisation.
-        DtPiece *pd = reinterpret_cast<DtPiece *>(smem + DtSmem::kPiece);
-        DtWalk *wk = reinterpret_cast<DtWalk *>(smem + DtSmem::kWalk);
+        DtPiece *pd = reinterpret_cast<DtPiece *>(smem + SM::kPiece);
+        DtWalk *wk = reinterpret_cast<DtWalk *>(smem + SM::kWalk);
         if (threadIdx.x == 0) {
             wk->w = walk;
             wk->W = W;
@@ -549,7 +564,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             // ---- query digits of (b, h): q ~= s (d1 + d2 / 254), s = max|q| / 127;
             // digit row r (d1) and RP + r (d2) of the K-major B operand of S
             {
-                unsigned char *qb = smem + DtSmem::kQ + (pc & 1) * 8192;
+                unsigned char *qb = smem + SM::kQ + (pc & 1) * 8192;
                 for (int r = warp; r < R; r += kDtConsumers) {
                     const int j = r / p.group, gq = r % p.group;
                     const size_t qoff =
@@ -617,7 +632,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 const int tok0 = cx * kChunk, ntok = (ce - cx) * kChunk;
                 cx = ce;
                 const uint32_t stage = kt % NS, sb = kt & 1;
-                const unsigned char *st = smem + stage * DtSmem::kStride;
+                const unsigned char *st = smem + stage * SM::kStride;
                 // ---- the stage: this key's V nibbles of group hq, its scales;
                 // then the stage is released
                 dt_wait(&full[stage], (kt / NS) & 1, misc);
@@ -625,22 +640,37 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 const bool sok = stage_ok[stage] != 0;  // (garbage after an abort is never used)
                 const bool kv_ok = sok && i < ntok && pos < L;
                 const bool fast = sok && ntok == 128 && tok0 + 128 <= all_see && R == RP;
-                uint4 nib[kDtVG];
+                // K8/V4: the group's 16 bytes of nibbles; K8V8: its 32 bytes of codes
+                constexpr int VW = V8 ? 2 : 1;
+                uint4 nib[kDtVG][VW];
                 uint2 vsr = make_uint2(0, 0);
                 float ksv = 0.f;
 #pragma unroll
-                for (int gg = 0; gg < kDtVG; ++gg) nib[gg] = make_uint4(0, 0, 0, 0);
+                for (int gg = 0; gg < kDtVG; ++gg)
+#pragma unroll
+                    for (int u = 0; u < VW; ++u) nib[gg][u] = make_uint4(0, 0, 0, 0);
                 if (kv_ok) {
 #pragma unroll
-                    for (int gg = 0; gg < kDtVG; ++gg)
-                        nib[gg] = *reinterpret_cast<const uint4 *>(
-                            st + DtSmem::kStV + i * 64 +
-                            ((((uint32_t)(hq * kDtVG + gg)) ^ (((uint32_t)i >> 1) & 3u)) << 4));
-                    vsr = *reinterpret_cast<const uint2 *>(st + DtSmem::kStVs + i * 8);
-                    ksv = __half2float(*reinterpret_cast<const __half *>(st + DtSmem::kStKs + i * 2));
+                    for (int gg = 0; gg < kDtVG; ++gg) {
+                        const uint32_t g = (uint32_t)(hq * kDtVG + gg);
+                        if constexpr (V8) {
+#pragma unroll
+                            for (int u = 0; u < 2; ++u)
+                                nib[gg][u] = *reinterpret_cast<const uint4 *>(
+                                    st + SM::kStV + i * 128 + (((2 * g + u) ^ ((uint32_t)i & 7u)) << 4));
+                        } else {
+                            nib[gg][0] = *reinterpret_cast<const uint4 *>(st + SM::kStV + i * 64 +
+                                                                           ((g ^ (((uint32_t)i >> 1) & 3u)) << 4));
+                        }
+                    }
+                    if constexpr (V8)
+                        vsr.x = *reinterpret_cast<const unsigned short *>(st + SM::kStVs + i * 2);
+                    else
+                        vsr = *reinterpret_cast<const uint2 *>(st + SM::kStVs + i * 8);
+                    ksv = __half2float(*reinterpret_cast<const __half *>(st + SM::kStKs + i * 2));
                 }
                 mbar_arrive(&empty[stage]);
-                const int ev = dt_v_exponent(vsr);
+                const int ev = dt_v_exponent(vsr);  // (K8V8: the one scale's exponent; the other words are 0)
                 // ---- V' and P' buffers sb are free once the P.V of tile kt - 2 is done
                 if (kt >= 2) dt_wait(&pvdone[sb], ((kt >> 1) - 1) & 1, misc);
 #pragma unroll
@@ -648,20 +678,33 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     // V' = code x scale / f: group vg of the key's row (block vg / 2,
                     // 16-byte chunks 4 (vg % 2) .. + 3)
                     const int vg = hq * kDtVG + gg;
-                    unsigned char *vd = smem + DtSmem::kVh + sb * 32768 + (vg >> 1) * 16384 + i * 128;
+                    unsigned char *vd = smem + SM::kVh + sb * 32768 + (vg >> 1) * 16384 + i * 128;
                     const uint32_t sw = (uint32_t)i & 7u;
-                    const uint32_t sbits = (vg < 2 ? vsr.x : vsr.y) >> (16 * (vg & 1));
+                    const uint32_t sbits = V8 ? vsr.x : (vg < 2 ? vsr.x : vsr.y) >> (16 * (vg & 1));
                     const float sg = __half2float(__ushort_as_half((unsigned short)(sbits & 0xFFFFu))) *
                                      __int_as_float((127 + 15 - ev) << 23);
                     const __half2 sv = __float2half2_rn(sg);
-                    const uint32_t wd[4] = {nib[gg].x, nib[gg].y, nib[gg].z, nib[gg].w};
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         uint4 o;
-                        o.x = h2_u32(__hmul2(nib_even(wd[w]), sv));
-                        o.y = h2_u32(__hmul2(nib_odd(wd[w]), sv));
-                        o.z = h2_u32(__hmul2(nib_even(wd[w] >> 8), sv));
-                        o.w = h2_u32(__hmul2(nib_odd(wd[w] >> 8), sv));
+                        if constexpr (V8) {
+                            // channels 8w .. 8w + 7 of the group in order: codes of words 2w, 2w + 1
+                            const uint4 q = nib[gg][w >> 1];
+                            const uint32_t w0 = (w & 1) ? q.z : q.x, w1 = (w & 1) ? q.w : q.y;
+                            uint32_t lo0, hi0, lo1, hi1;
+                            i8x4_to_f16(w0, lo0, hi0);
+                            i8x4_to_f16(w1, lo1, hi1);
+                            o.x = h2_u32(__hmul2(u32_h2(lo0), sv));
+                            o.y = h2_u32(__hmul2(u32_h2(hi0), sv));
+                            o.z = h2_u32(__hmul2(u32_h2(lo1), sv));
+                            o.w = h2_u32(__hmul2(u32_h2(hi1), sv));
+                        } else {
+                            const uint32_t wd[4] = {nib[gg][0].x, nib[gg][0].y, nib[gg][0].z, nib[gg][0].w};
+                            o.x = h2_u32(__hmul2(nib_even(wd[w]), sv));
+                            o.y = h2_u32(__hmul2(nib_odd(wd[w]), sv));
+                            o.z = h2_u32(__hmul2(nib_even(wd[w] >> 8), sv));
+                            o.w = h2_u32(__hmul2(nib_odd(wd[w] >> 8), sv));
+                        }
                         const uint32_t cc = (uint32_t)(4 * (vg & 1) + w);
                         *reinterpret_cast<uint4 *>(vd + ((cc ^ sw) << 4)) = o;
                     }
@@ -694,7 +737,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 // P' row of this key, rows r0 .. r0 + HR - 1 (half of one, one or two
                 // 16-byte chunks)
                 {
-                    unsigned char *pr = smem + DtSmem::kP + sb * 16384 + i * 128;
+                    unsigned char *pr = smem + SM::kP + sb * 16384 + i * 128;
                     if constexpr (HR >= 8) {
 #pragma unroll
                         for (int c = 0; c < HR / 8; ++c)
@@ -725,7 +768,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 named_sync(gbar, 128);
                 if (kt > kfirst) dt_wait(&pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
                 tc_fence_after();
-                const int ch = dt_channel(i);
+                const int ch = V8 ? i : dt_channel(i);  // K8V8: channels in order
                 float *slotp = p.partials + (size_t)(s_id + vb) * p.slot_floats;
                 // O^T / l, four rows at a time (few live registers)
 #pragma unroll
@@ -760,7 +803,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             }
             named_sync(kDtBarAll, kDtConsumers * 32);  // the piece's outputs are written
             finish_piece_coop<kDtConsumers * 32, kDtBarAll>(p, s_id, first, vb - first, n_pieces, pce.m,
-                                                               reinterpret_cast<float *>(smem + DtSmem::kVh), misc, R, b,
+                                                               reinterpret_cast<float *>(smem + SM::kVh), misc, R, b,
                                                                h);
             named_sync(kDtBarAll, kDtConsumers * 32);  // the merge is done: its buffers are free again
             ++pc;
