@@ -1196,7 +1196,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const __grid_
     uint32_t fin_phase = 0;  // parity of the final merge's copy barrier
     while (walk.next()) {
         const int b = walk.pb, h = walk.ph;
-        const int L = seqC[b] ? p.seqlens[b] : 0;
+        const int L = seqL[b];  // (read once at the start; 0 for a sequence with no valid key)
         // query fragments of this (sequence, kv-head): lane (g, t) holds row g of
         // tile nt, channels 32t..32t+31 (int8 K: k-step ks takes channels 32t + 8ks
         // + 0..3 and + 4..7; fp8 K: 32t + 4ks + 0..3) or 32u + 8t + 4h + 0..3
