@@ -10,9 +10,9 @@
 // group, so a kv-head serves G * n_q = 32 rows (G = 8).  The work per key then
 // grows with the rows (two products of 128 channels per row and key), and on
 // the per-warp mma.sync path it outgrows the HBM time.  Here the products run
-// as whole-tile tcgen05 MMAs issued by one thread, with the accumulators in
-// tensor memory, and the CUDA cores only do the softmax and the V
-// dequantisation.  The work cut, the split partials and the last-ticket merge
+// as whole-tile tcgen05 MMAs, each stream issued by one thread of its own
+// warp, with the accumulators in tensor memory, and the CUDA cores only do
+// the softmax and the V dequantisation.  The work cut, the split partials and the last-ticket merge
 // are those of decode_kernel (nf_decode.cuh); results and workspace layout are
 // the same.
 //
@@ -29,9 +29,10 @@
 //                       fp16 P' [key][row].
 //   V dequantisation    one thread per key: code x (V scale / f_k) as fp16 V'
 //                       [key][channel]; f_k = 2^(E - 15) with E the largest
-//                       exponent of the key's four V scales, so V' < 14 and
-//                       P' <= 2^15 both stay inside fp16 for any fp16 scale, and
-//                       P' x V' = p x code x scale.
+//                       exponent of the key's V scales (four, or K8V8's one),
+//                       so V' < 16 (K8V8: < 256) and P' <= 2^15 both stay
+//                       inside fp16 for any fp16 scale, and P' x V' = p x code
+//                       x scale.
 //   O^T += V'^T . P'    kind::f16, M = 128 channels, N = 64 (rows, padded),
 //                       K = 128 keys; A = V' and B = P', both MN-major
 //                       (128-byte swizzle); O^T lives in tensor memory.
