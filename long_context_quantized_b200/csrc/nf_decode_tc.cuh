@@ -30,7 +30,7 @@
 //   V dequantisation    one thread per key: code x (V scale / f_k) as fp16 V'
 //                       [key][channel]; f_k = 2^(E - 15) with E the largest
 //                       exponent of the key's V scales (four, or K8V8's one),
-//                       so V' < 16 (K8V8: < 256) and P' <= 2^15 both stay
+//                       so V' < 14 (K8V8: < 254) and P' <= 2^15 both stay
 //                       inside fp16 for any fp16 scale, and P' x V' = p x code
 //                       x scale.
 //   O^T += V'^T . P'    kind::f16, M = 128 channels, N = 64 (rows, padded),
