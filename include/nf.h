@@ -215,8 +215,11 @@ size_t nf_decode_attn_workspace_size(int32_t batch, int32_t n_q, int32_t num_q_h
  *   the e4m3 codes are exact in fp16; S = Q . K^T uses fp16 products with each
  *   query row split as q = s (hi + lo), s = max|q|, hi and lo fp16.  bf16
  *   cache: bf16 products, the fp32 query and the weights split into bf16 high
- *   and low parts.)  With 9 to 32 query rows per kv-head, K8/V4 and K8V8 run on
- *   the tcgen05 tensor cores instead: the same two-digit Q . K, and P . V as
+ *   and low parts.)  With 9 to 32 query rows per kv-head, K8/V4, K8V8 and fp8
+ *   run on the tcgen05 tensor cores instead: the same two-digit Q . K for
+ *   int8 K; for e4m3 K, the query row scaled to max|q| = 1 in three e4m3 parts
+ *   (q ~= s (p1 + p2 / 16 + p3 / 256), each part the rounding of what the
+ *   earlier ones leave, times 16) against the exact codes, in fp32; and P . V as
  *   V' = code x scale x 2^(15 - E) times P' = weight x 2^(E - 15), each rounded
  *   to fp16 once (E: the largest exponent field of the key's V scales).
  * Launch: the kernel is launched with programmatic dependent launch, so it may

@@ -215,7 +215,7 @@ cudaError_t dispatch_decode_tc(const nf::DecodeParams &p, bool qf32, int rows, i
 }
 
 bool uses_decode_tc(int fmt, int rows) {
-    return (fmt == NF_KV_K8V4 || fmt == NF_KV_K8V8) && rows > 8 && rows <= nf::kDtMaxRows;
+    return (fmt == NF_KV_K8V4 || fmt == NF_KV_K8V8 || fmt == NF_KV_F8) && rows > 8 && rows <= nf::kDtMaxRows;
 }
 
 template <int NT>
@@ -427,6 +427,7 @@ nf_status nf_decode_attn_ex(const nf_kv_layer *kv, const void *q, int32_t q_dtyp
     const bool qf32 = q_dtype == NF_F32;
     const cudaError_t e =
         tc ? (kv->fmt == NF_KV_K8V8 ? dispatch_decode_tc<NF_KV_K8V8>(p, qf32, pl.rows, pl.ctas, s)
+              : kv->fmt == NF_KV_F8 ? dispatch_decode_tc<NF_KV_F8>(p, qf32, pl.rows, pl.ctas, s)
                                     : dispatch_decode_tc<NF_KV_K8V4>(p, qf32, pl.rows, pl.ctas, s))
         : pl.nt == 1 ? dispatch_decode<1>(p, qf32, kv->fmt, pl.ctas, s)
                      : dispatch_decode<2>(p, qf32, kv->fmt, pl.ctas, s);

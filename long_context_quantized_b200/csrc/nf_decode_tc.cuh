@@ -1,8 +1,12 @@
 // nf_decode_tc.cuh -- split-K decode attention over the K8/V4 (or the int8
-// K8V8) pool for many query rows per kv-head, on the 5th-generation tensor
-// cores (tcgen05).  K8V8 differs only in the V side: 128-byte rows of int8
-// codes with one fp16 scale per key, dequantised in channel order, and three
-// ring stages instead of four.
+// K8V8, or the fp8) pool for many query rows per kv-head, on the 5th-generation
+// tensor cores (tcgen05).  K8V8 differs only in the V side: 128-byte rows of
+// int8 codes with one fp16 scale per key, dequantised in channel order, and
+// three ring stages instead of four.  fp8 has the K8V8 layout with e4m3 codes;
+// its S = K . Q^T runs on kind::f8f6f4 against the query row in three e4m3
+// parts, q ~= s (p1 + p2 / 16 + p3 / 256) with s = max|q|, each part the e4m3
+// rounding of what the earlier parts leave (times 16), into three fp32
+// columns per row (2^-12 of max|q| per element and better).
 //
 // MTP draft verification is the engine's normal decode step: 1 + 3 query
 // tokens per step (page "3090 单卡跑 Qwen3.8-27B：NInfer 上机实测", section
@@ -78,14 +82,16 @@ constexpr int kDtSegPad = 12;
 // warps (also the final merge's)
 constexpr uint32_t kDtBarAll = 6;
 
-// Shared-memory layout for the pool format FMT: NF_KV_K8V4 or NF_KV_K8V8.
+// Shared-memory layout for the pool format FMT: NF_KV_K8V4, NF_KV_K8V8 or NF_KV_F8.
 template <int FMT>
 struct DtSmem {
     // one ring stage: K codes [128 keys][128 B] (128-byte swizzle); V codes
     // [128 keys][64 B nibbles] (64-byte swizzle, K8/V4) or [128 keys][128 B]
     // (128-byte swizzle, K8V8); K scales fp16 [128]; V scales fp16 [128][4]
     // (K8/V4) or [128] (K8V8).  Three K8V8 stages fit beside the other buffers.
-    static constexpr bool kV8 = FMT == NF_KV_K8V8;
+    static constexpr bool kF8 = FMT == NF_KV_F8;                // e4m3 K and V codes
+    static constexpr bool kV8 = FMT == NF_KV_K8V8 || kF8;       // 128-byte V rows, one V scale per key
+    static constexpr int kQBuf = kF8 ? 12288 : 8192;            // query operand rows (2 or 3 per row) x 128 B
     static constexpr int kVRow = kV8 ? 128 : 64, kVScales = kV8 ? 1 : 4;
     static constexpr int kStages = kV8 ? 3 : kDtStages;
     static constexpr int kStK = 0, kStV = 16384, kStKs = kStV + 128 * kVRow, kStVs = kStKs + 256;
@@ -94,8 +100,8 @@ struct DtSmem {
     static constexpr int kRingBytes = kStages * kStride;
     static constexpr int kVh = kRingBytes;        // fp16 V' [2 buffers][2 blocks of 64 channels][128 keys][128 B]
     static constexpr int kP = kVh + 2 * 32768;    // fp16 P' [2 buffers][128 keys][64 rows x 2 B]
-    static constexpr int kQ = kP + 2 * 16384;     // int8 digits [2 buffers][64 digit rows][128 B]
-    static constexpr int kQw = kQ + 2 * 8192;     // float [2][kDtMaxRows]: row factors
+    static constexpr int kQ = kP + 2 * 16384;     // query operand [2 buffers][64 int8 digit rows or 96 e4m3 part rows][128 B]
+    static constexpr int kQw = kQ + 2 * kQBuf;    // float [2][kDtMaxRows]: row factors
     static constexpr int kRed = kQw + 2 * kDtMaxRows * 4;   // float [4 quadrants][kDtMaxRows]: row maxima
     static constexpr int kRed2 = kRed + 4 * kDtMaxRows * 4; // float [4 quadrants][kDtMaxRows]: row sums
     static constexpr int kBars = kRed2 + 4 * kDtMaxRows * 4;
@@ -217,8 +223,19 @@ __device__ __forceinline__ void dt_st(uint32_t taddr, const uint32_t (&r)[HR]) {
 // FAST: every row sees every key of the tile (no mask).
 // When the max rises and O^T holds earlier tiles of the piece (has_o), the
 // rows' columns of O^T (taddr) are scaled once the last P.V is done (pv_bar).
-template <int HR, bool FAST>
-__device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint32_t (&d2)[HR], const float *qwr,
+// The raw product of a row and key from the S words: int8 digits S1 * 254 +
+// S2, or e4m3 parts S1 + S2 / 16 + S3 / 256 (fp32 accumulators).
+template <bool F8>
+__device__ __forceinline__ float dt_product(uint32_t w1, uint32_t w2, uint32_t w3) {
+    if constexpr (F8)
+        return fmaf(__uint_as_float(w3), 0.00390625f, fmaf(__uint_as_float(w2), 0.0625f, __uint_as_float(w1)));
+    else
+        return (float)((int)w1 * 254 + (int)w2);
+}
+
+template <int HR, bool FAST, bool F8>
+__device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint32_t (&d2)[HR], const uint32_t (&d3)[HR],
+                                           const float *qwr,
                                            float ksv, int rmin, int R, int r0, float (&nthr)[HR], float (&l_part)[HR],
                                            float *red, int qd, int lane, uint32_t gbar, float f,
                                            uint32_t (&pk)[HR / 2], bool has_o, uint32_t taddr, uint64_t *pv_bar,
@@ -235,7 +252,7 @@ __device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint3
     }
 #pragma unroll
     for (int e = 0; e < HR; ++e) {
-        const float v = (float)((int)d1[e] * 254 + (int)d2[e]);
+        const float v = dt_product<F8>(d1[e], d2[e], d3[e]);
         y[e] = (FAST || (r0 + e >= rmin && r0 + e < R)) ? fmaf(v, c[e], nthr[e]) : -INFINITY;
         raise |= y[e] > 0.f;  // true when no max yet and the score finite
     }
@@ -244,10 +261,8 @@ __device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint3
         // the scores themselves (y loses them while a row has no max)
         float x[HR];
 #pragma unroll
-        for (int e = 0; e < HR; ++e) {
-            const float v = (float)((int)d1[e] * 254 + (int)d2[e]);
-            x[e] = (FAST || (r0 + e >= rmin && r0 + e < R)) ? v * c[e] : -INFINITY;
-        }
+        for (int e = 0; e < HR; ++e)
+            x[e] = (FAST || (r0 + e >= rmin && r0 + e < R)) ? dt_product<F8>(d1[e], d2[e], d3[e]) * c[e] : -INFINITY;
         // row maxima of the tile over its 128 keys: the four warps of these rows
 #pragma unroll
         for (int e = 0; e < HR; ++e) {
@@ -298,16 +313,17 @@ __device__ __forceinline__ void dt_softmax(const uint32_t (&d1)[HR], const uint3
 template <int RP, bool QF32, int FMT>
 __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_constant__ DecodeParams p) {
     static_assert(RP == 16 || RP == 32, "rows padded to 16 or 32");
-    static_assert(FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8, "int8 K codes");
+    static_assert(FMT == NF_KV_K8V4 || FMT == NF_KV_K8V8 || FMT == NF_KV_F8, "int8 or e4m3 K codes");
     using SM = DtSmem<FMT>;
-    constexpr bool V8 = SM::kV8;  // int8 V codes, one V scale per key
+    constexpr bool V8 = SM::kV8;  // int8 or e4m3 V codes, one V scale per key
+    constexpr bool F8 = SM::kF8;  // e4m3 K: S = K . Q^T on kind::f8f6f4 with the query in three e4m3 parts
     constexpr int NS = SM::kStages;
     constexpr int HR = RP / kDtRowGroups;                         // rows per consumer warp
-    constexpr int NSC = 2 * RP;                                   // S columns per buffer
-    constexpr uint32_t kIdescS = umma_idesc_s8(128, NSC);
+    constexpr int NSC = (F8 ? 3 : 2) * RP;                        // S columns per buffer
+    constexpr uint32_t kIdescS = F8 ? umma_idesc_e4m3(128, NSC) : umma_idesc_s8(128, NSC);
     constexpr uint32_t kIdescO = umma_idesc_f16(128, kDtPvN, true, true);
-    constexpr uint32_t kSCol = 64;                                // S buffer b at columns 64 b
-    constexpr uint32_t kOCol = 128;                               // O^T at columns 128 .. 191
+    constexpr uint32_t kSCol = (F8 && RP == 32) ? 96 : 64;        // S buffer b at columns kSCol b
+    constexpr uint32_t kOCol = 2 * kSCol;                         // O^T: 64 columns from kOCol (<= 256)
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kBars);
     uint64_t *full = bars, *empty = bars + NS;
@@ -352,7 +368,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         fence_mbar_init();
     }
     // the query-digit buffers' padding rows stay zero
-    for (int i = threadIdx.x; i < 2 * 8192 / 16; i += kDtThreads)
+    for (int i = threadIdx.x; i < 2 * SM::kQBuf / 16; i += kDtThreads)
         reinterpret_cast<uint4 *>(smem + SM::kQ)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     if (warp == kDtMma) {
@@ -462,7 +478,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             uint32_t kt = 0, pc = 0;
             while (!misc[0] && walk.next()) {
                 dt_wait(&qfull[pc & 1], (pc >> 1) & 1, misc);
-                const uint32_t qaddr = sQ + (pc & 1) * 8192u;
+                const uint32_t qaddr = sQ + (pc & 1) * (uint32_t)SM::kQBuf;
                 const int cx1 = (int)(walk.xe - walk.s0);
                 for (int cx = (int)(walk.xs - walk.s0); cx < cx1 && !misc[0]; ++kt) {
                     cx = dt_tile_end(cx, cx1);
@@ -473,9 +489,14 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     tc_fence_after();
                     const uint32_t kaddr = sRing + stage * SM::kStride + SM::kStK;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_s8(tmem + sb * kSCol, umma_desc_sw128(kaddr + 32 * ks, 16, 1024),
-                                umma_desc_sw128(qaddr + 32 * ks, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        if constexpr (F8)
+                            umma_e4m3(tmem + sb * kSCol, umma_desc_sw128(kaddr + 32 * ks, 16, 1024),
+                                      umma_desc_sw128(qaddr + 32 * ks, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
+                        else
+                            umma_s8(tmem + sb * kSCol, umma_desc_sw128(kaddr + 32 * ks, 16, 1024),
+                                    umma_desc_sw128(qaddr + 32 * ks, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
+                    }
                     umma_commit(&sfull[sb]);
                     umma_commit(&empty[stage]);  // the stage's K codes are consumed
                 }
@@ -565,7 +586,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             // ---- query digits of (b, h): q ~= s (d1 + d2 / 254), s = max|q| / 127;
             // digit row r (d1) and RP + r (d2) of the K-major B operand of S
             {
-                unsigned char *qb = smem + SM::kQ + (pc & 1) * 8192;
+                unsigned char *qb = smem + SM::kQ + (pc & 1) * SM::kQBuf;
                 for (int r = warp; r < R; r += kDtConsumers) {
                     const int j = r / p.group, gq = r % p.group;
                     const size_t qoff =
@@ -584,24 +605,49 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                     float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                    const float s1 = amax / 127.0f;
-                    const float inv = amax > 0.f ? 127.0f / amax : 0.f;
-                    uint32_t d1w = 0, d2w = 0;
+                    // channels 4 lane .. + 3 of operand row rr: 16-byte chunk lane / 4, swizzled
+                    auto put = [&](int rr, uint32_t w) {
+                        *reinterpret_cast<uint32_t *>(qb + rr * 128 + ((((uint32_t)lane >> 2) ^ ((uint32_t)rr & 7u)) << 4) +
+                                                      4u * (lane & 3)) = w;
+                    };
+                    if constexpr (F8) {
+                        // q ~= s (p1 + p2 / 16 + p3 / 256), s = max|q|: each part the
+                        // e4m3 rounding of what the earlier parts leave (times 16)
+                        const float inv = amax > 0.f ? 1.0f / amax : 0.f;
+                        float y[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float d1 = fminf(fmaxf(rintf(x[e] * inv), -127.f), 127.f);
-                        const float r1 = fmaf(-d1, s1, x[e]);
-                        const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
-                        d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
-                        d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
+                        for (int e = 0; e < 4; ++e) y[e] = x[e] * inv;
+#pragma unroll
+                        for (int part = 0; part < 3; ++part) {
+                            const uint32_t w = f32x4_to_e4m3(y[0], y[1], y[2], y[3]);
+                            put(part * RP + r, w);
+                            if (part < 2) {
+                                uint32_t lo, hi;
+                                e4m3x4_to_f16(w, lo, hi);
+                                const float2 a = __half22float2(u32_h2(lo)), c2 = __half22float2(u32_h2(hi));
+                                y[0] = (y[0] - a.x) * 16.f;
+                                y[1] = (y[1] - a.y) * 16.f;
+                                y[2] = (y[2] - c2.x) * 16.f;
+                                y[3] = (y[3] - c2.y) * 16.f;
+                            }
+                        }
+                        if (lane == 0) qw_sm[(pc & 1) * kDtMaxRows + r] = amax * p.scale_log2;
+                    } else {
+                        const float s1 = amax / 127.0f;
+                        const float inv = amax > 0.f ? 127.0f / amax : 0.f;
+                        uint32_t d1w = 0, d2w = 0;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float d1 = fminf(fmaxf(rintf(x[e] * inv), -127.f), 127.f);
+                            const float r1 = fmaf(-d1, s1, x[e]);
+                            const float d2 = fminf(fmaxf(rintf(r1 * inv * 254.0f), -127.f), 127.f);
+                            d1w |= ((uint32_t)(int)d1 & 0xFFu) << (8 * e);
+                            d2w |= ((uint32_t)(int)d2 & 0xFFu) << (8 * e);
+                        }
+                        put(r, d1w);
+                        put(RP + r, d2w);
+                        if (lane == 0) qw_sm[(pc & 1) * kDtMaxRows + r] = s1 / 254.0f * p.scale_log2;
                     }
-                    // channels 4 lane .. + 3: 16-byte chunk lane / 4 of the row, swizzled
-                    const uint32_t cofs = ((((uint32_t)lane >> 2) ^ ((uint32_t)r & 7u)) << 4) + 4u * (lane & 3);
-                    *reinterpret_cast<uint32_t *>(qb + r * 128 + cofs) = d1w;
-                    const int r2 = RP + r;
-                    *reinterpret_cast<uint32_t *>(qb + r2 * 128 + ((((uint32_t)lane >> 2) ^ ((uint32_t)r2 & 7u)) << 4) +
-                                                  4u * (lane & 3)) = d2w;
-                    if (lane == 0) qw_sm[(pc & 1) * kDtMaxRows + r] = s1 / 254.0f * p.scale_log2;
                 }
                 fence_async_smem();
                 named_sync(kDtBarAll, kDtConsumers * 32);
@@ -693,8 +739,13 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                             const uint4 q = nib[gg][w >> 1];
                             const uint32_t w0 = (w & 1) ? q.z : q.x, w1 = (w & 1) ? q.w : q.y;
                             uint32_t lo0, hi0, lo1, hi1;
-                            i8x4_to_f16(w0, lo0, hi0);
-                            i8x4_to_f16(w1, lo1, hi1);
+                            if constexpr (F8) {
+                                e4m3x4_to_f16(w0, lo0, hi0);
+                                e4m3x4_to_f16(w1, lo1, hi1);
+                            } else {
+                                i8x4_to_f16(w0, lo0, hi0);
+                                i8x4_to_f16(w1, lo1, hi1);
+                            }
                             o.x = h2_u32(__hmul2(u32_h2(lo0), sv));
                             o.y = h2_u32(__hmul2(u32_h2(hi0), sv));
                             o.z = h2_u32(__hmul2(u32_h2(lo1), sv));
@@ -713,14 +764,24 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 // ---- softmax of rows r0 .. r0 + HR - 1 for this key
                 dt_wait(&sfull[sb], (kt >> 1) & 1, misc);
                 tc_fence_after();
-                uint32_t d1[HR], d2[HR];
+                // the S words of the rows (int8 digits: two per row; e4m3 parts: three)
+                uint32_t d1[HR], d2[HR], d3[HR];
                 {
                     const uint32_t ta = tmem + lane_base + sb * kSCol + r0;
                     dt_ld<HR>(ta, d1);
                     dt_ld<HR>(ta + RP, d2);
-                    tmem_wait_ld_tied<HR>(d1);
+                    if constexpr (F8) {
+                        dt_ld<HR>(ta + 2 * RP, d3);
+                        tmem_wait_ld_tied<HR>(d3);
 #pragma unroll
-                    for (int k = 0; k < HR; ++k) asm volatile("" : "+r"(d2[k]));
+                        for (int k = 0; k < HR; ++k) asm volatile("" : "+r"(d1[k]), "+r"(d2[k]));
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < HR; ++k) d3[k] = 0u;
+                        tmem_wait_ld_tied<HR>(d1);
+#pragma unroll
+                        for (int k = 0; k < HR; ++k) asm volatile("" : "+r"(d2[k]));
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(&sfree[sb]);
@@ -730,10 +791,10 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 uint32_t pk[HR / 2];
                 const uint32_t ota = tmem + lane_base + kOCol + r0;
                 if (fast)
-                    dt_softmax<HR, true>(d1, d2, qwr, ksv, rmin, R, r0, nthr, l_part, red, qd, lane, gbar, f, pk,
+                    dt_softmax<HR, true, F8>(d1, d2, d3, qwr, ksv, rmin, R, r0, nthr, l_part, red, qd, lane, gbar, f, pk,
                                          kt > kfirst, ota, &pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
                 else
-                    dt_softmax<HR, false>(d1, d2, qwr, ksv, rmin, R, r0, nthr, l_part, red, qd, lane, gbar, f, pk,
+                    dt_softmax<HR, false, F8>(d1, d2, d3, qwr, ksv, rmin, R, r0, nthr, l_part, red, qd, lane, gbar, f, pk,
                                           kt > kfirst, ota, &pvdone[(kt - 1) & 1], ((kt - 1) >> 1) & 1, misc);
                 // P' row of this key, rows r0 .. r0 + HR - 1 (half of one, one or two
                 // 16-byte chunks)
